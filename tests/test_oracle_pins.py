@@ -1,0 +1,361 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+None of these tests re-derives the oracle's own formulas: each checks it
+against a theorem (losslessness of speculative sampling; the acceptance
+probability sum_x min(p, q)), a special case with a closed form, brute force
+on tiny inputs, an independent library routine (torch / scipy / numpy), or a
+worked example printed on the pages (tests/golden).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import scipy.stats
+import torch
+
+from speculative_decoding_verification_94_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _kind(o, x):
+    return o.DRAFT_PROBS if x.draft_kind == "probs" else o.DRAFT_LOGITS
+
+
+# --------------------------------------------------------------------------
+# Softmax normalisation: an independent library routine.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [0.7, 1.0, 2.5])
+def test_softmax_matches_torch_float64(oracle, dtype, T):
+    x = inputs.make_chain(2, 1, 3001, dtype=dtype, temperature=T, seed=3)
+    z = x.target
+    got = oracle.softmax(z, T)
+    Tf = float(np.float32(T))
+    ref = torch.softmax(z.double() / Tf, dim=-1).numpy()
+    lz = torch.logsumexp(z.double() / Tf, dim=-1).numpy()
+    assert np.allclose(got["p"], ref, rtol=1e-12, atol=1e-300)
+    assert np.allclose(got["log_partition"], lz, rtol=1e-13, atol=0)
+
+
+# --------------------------------------------------------------------------
+# Acceptance rule: special cases with closed forms.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,T", [("f32", 1.0), ("bf16", 0.7), ("bf16", 1.3)])
+def test_identical_draft_accepts_every_token(oracle, dtype, T):
+    """q == p: min(1, p/q) = 1, so all k drafts are accepted."""
+    x = inputs.make_chain(16, 4, 777, dtype=dtype, sigma_d=0.0, temperature=T, seed=5)
+    assert torch.equal(x.target[:, :4], x.draft)
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, T)
+    assert (r["accepted_len"] == 4).all()
+    assert (r["out_tokens"][:, :4] == x.draft_tokens.numpy()).all()
+    assert (r["out_tokens"][:, 4] >= 0).all()
+
+
+def test_disjoint_support_rejects_first_and_resamples_target(oracle):
+    """q disjoint from p: p(x) = 0 for every draft, so position 0 always
+    rejects (even for u = 0) and the residual max(0, p - q) is p itself: the
+    emitted token is the inverse-CDF draw from p_0 (numpy searchsorted)."""
+    V, k, B = 64, 3, 256
+    rng = np.random.default_rng(0)
+    zt = rng.normal(0, 2, (k + 1, V)).astype(np.float32)
+    zd = rng.normal(0, 2, (k, V)).astype(np.float32)
+    zt[:, 1::2] = -np.inf
+    zd[:, 0::2] = -np.inf
+    x = inputs.make_chain_fixed(B, zt, zd, draft_kind="logits", temperature=1.0, seed=1)
+    x.uniforms[:4, 0] = 0.0
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 1.0)
+    assert (r["accepted_len"] == 0).all()
+    p0 = torch.softmax(torch.from_numpy(zt[0]).double(), -1).numpy()
+    cdf = np.cumsum(p0)
+    expect = np.searchsorted(cdf / cdf[-1], x.uniforms[:, k].double().numpy(), side="right")
+    assert (r["out_tokens"][:, 0] == expect).all()
+    assert (r["out_tokens"][:, 0] % 2 == 0).all()
+    assert (r["out_tokens"][:, 1:] == -1).all()
+
+
+def test_two_token_disjoint_closed_form(oracle):
+    """V=2, p=(1,0), q=(0,1): the draft is token 1, always rejected, and the
+    residual puts all mass on token 0."""
+    zt = np.array([[0.0, -np.inf]] * 2, np.float32)
+    zd = np.array([[-np.inf, 0.0]], np.float32)
+    x = inputs.make_chain_fixed(64, zt, zd, draft_kind="logits", seed=2)
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 1.0)
+    assert (x.draft_tokens.numpy() == 1).all()
+    assert (r["accepted_len"] == 0).all() and (r["out_tokens"][:, 0] == 0).all()
+
+
+def test_acceptance_fraction_on_a_uniform_grid(oracle):
+    """With u on the grid m/M, the number of accepted draws of a fixed token x
+    is #{m : m/M < p(x)/q(x)} = ceil(M p/q) when p/q < 1: the rule is
+    'accept with probability min(1, p/q)', checked without sampling noise."""
+    V, M = 10, 4096
+    zt = np.linspace(-1, 1, V, dtype=np.float32)[None].repeat(2, 0)
+    q = np.linspace(2, 0.5, V) ** 2
+    q = (q / q.sum()).astype(np.float32)[None]
+    x = inputs.make_chain_fixed(M, zt, q, draft_kind="probs", seed=3)
+    x.draft_tokens[:] = 0
+    x.uniforms[:, 0] = torch.arange(M, dtype=torch.float32) / M
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 1.0,
+                            draft_kind=oracle.DRAFT_PROBS)
+    p = torch.softmax(torch.from_numpy(zt[0]).double(), -1).numpy()
+    ratio = p[0] / float(q[0, 0])
+    assert ratio < 1
+    assert int((r["accepted_len"] == 1).sum()) == math.ceil(M * ratio)
+
+
+# --------------------------------------------------------------------------
+# Losslessness (Leviathan et al.): the emitted token at every position is
+# distributed as the target row, whatever the draft.  Monte-Carlo chi-square.
+# --------------------------------------------------------------------------
+def _chain_mc(oracle, draft_kind, T, seed, plant=0, B=200_000, V=8, k=3):
+    rng = np.random.default_rng(100 + seed)
+    zt = rng.normal(0, 1.5, (k + 1, V)).astype(np.float32)
+    if draft_kind == "probs":
+        d = rng.dirichlet(np.full(V, 0.7), size=k).astype(np.float32)
+        q = d.astype(np.float64)
+    else:
+        d = (zt[:k] + rng.normal(0, 1.0, (k, V))).astype(np.float32)
+        q = torch.softmax(torch.from_numpy(d).double() / float(np.float32(T)), -1).numpy()
+    x = inputs.make_chain_fixed(B, zt, d, draft_kind=draft_kind, temperature=T, seed=seed)
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, T,
+                            draft_kind=_kind(oracle, x), plant=plant)
+    p = torch.softmax(torch.from_numpy(zt).double() / float(np.float32(T)), -1).numpy()
+    return r, p, q
+
+
+def _position_stats(r, p, q, k=3):
+    out = []
+    for i in range(k + 1):
+        reached = r["accepted_len"] >= i
+        tok = r["out_tokens"][reached, i]
+        counts = np.bincount(tok, minlength=p.shape[1])
+        pval = scipy.stats.chisquare(counts, p[i] * reached.sum()).pvalue
+        acc = None
+        if i < k:
+            n = reached.sum()
+            a = (r["accepted_len"][reached] > i).mean()
+            alpha = np.minimum(p[i], q[i]).sum()
+            acc = (a, alpha, math.sqrt(alpha * (1 - alpha) / n))
+        out.append((pval, acc))
+    return out
+
+
+@pytest.mark.parametrize("draft_kind,T,seed", [("probs", 1.0, 0), ("logits", 0.7, 1)])
+def test_losslessness_and_acceptance_rate(oracle, draft_kind, T, seed):
+    r, p, q = _chain_mc(oracle, draft_kind, T, seed)
+    for i, (pval, acc) in enumerate(_position_stats(r, p, q)):
+        assert pval > 1e-3, f"position {i}: emitted tokens are not distributed as p (p={pval})"
+        if acc is not None:
+            a, alpha, sd = acc
+            assert abs(a - alpha) < 4 * sd + 1e-12, (i, a, alpha, sd)
+
+
+@pytest.mark.parametrize("plant", [1, 2])
+def test_planted_mistakes_are_caught(oracle, plant):
+    """A flipped residual sign (plant 1) or an inverted ratio (plant 2),
+    compiled into a copy of the oracle, must fail the losslessness pin."""
+    oracle.build(plant=plant)
+    r, p, q = _chain_mc(oracle, "probs", 1.0, 0, plant=plant)
+    stats = _position_stats(r, p, q)
+    assert min(s[0] for s in stats) < 1e-6
+
+
+# --------------------------------------------------------------------------
+# Greedy verification: brute force.
+# --------------------------------------------------------------------------
+def _quantised_rows(rng, shape, levels=5):
+    return rng.integers(-levels, levels + 1, size=shape).astype(np.float32)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_greedy_chain_bruteforce(oracle, dtype):
+    rng = np.random.default_rng(7)
+    B, k, V = 300, 4, 40
+    z = _quantised_rows(rng, (B, k + 1, V))
+    first_max = z.argmax(-1)  # numpy returns the first maximal index
+    x = np.where(rng.random((B, k)) < 0.75, first_max[:, :k], rng.integers(0, V, (B, k)))
+    zt = inputs._cast(z, dtype)
+    r = oracle.verify_chain(zt, None, torch.from_numpy(x.astype(np.int32)), None, 0.0)
+    for b in range(B):
+        n = 0
+        while n < k and x[b, n] == first_max[b, n]:
+            n += 1
+        assert r["accepted_len"][b] == n
+        assert list(r["out_tokens"][b, :n]) == list(x[b, :n])
+        assert r["out_tokens"][b, n] == first_max[b, n]
+        assert (r["out_tokens"][b, n + 1:] == -1).all()
+
+
+def _enumerate_tree(z, tok, par):
+    """Brute force over all root-to-node paths."""
+    n = len(par)
+    g = z.argmax(-1)
+    best, best_path = 0, [0]
+    for j in range(n):
+        path = [j]
+        while path[-1] != 0:
+            path.append(int(par[path[-1]]))
+        path = path[::-1]
+        ok = all(tok[path[d + 1]] == g[path[d]] for d in range(len(path) - 1))
+        if ok and (len(path) > len(best_path)):
+            best, best_path = j, path
+    return best, best_path, g
+
+
+def test_tree_greedy_bruteforce(oracle):
+    rng = np.random.default_rng(11)
+    B, n, V, s = 40, 24, 30, 6
+    z = _quantised_rows(rng, (B, n, V), levels=3)
+    par = np.full((B, n), -1, np.int32)
+    depth = np.zeros((B, n), np.int32)
+    tok = np.zeros((B, n), np.int32)
+    for b in range(B):
+        for j in range(1, n):
+            while True:
+                pj = int(rng.integers(0, j))
+                if depth[b, pj] < s:
+                    break
+            par[b, j] = pj
+            depth[b, j] = depth[b, pj] + 1
+            g = int(z[b, pj].argmax())
+            tok[b, j] = g if rng.random() < 0.6 else int(rng.integers(0, V))
+    r = oracle.tree_greedy(torch.from_numpy(z), torch.from_numpy(tok), torch.from_numpy(par), s)
+    for b in range(B):
+        best, path, g = _enumerate_tree(z[b], tok[b], par[b])
+        L = len(path) - 1
+        assert r["accepted_len"][b] == L
+        assert list(r["accepted_nodes"][b, :L + 1]) == path
+        assert list(r["out_tokens"][b, :L]) == [int(tok[b, j]) for j in path[1:]]
+        assert r["out_tokens"][b, L] == g[best]
+        assert (r["out_tokens"][b, L + 1:] == -1).all()
+
+
+def test_chain_shaped_tree_equals_greedy_chain(oracle):
+    x = inputs.make_chain(12, 5, 2000, dtype="bf16", sigma_d=0.5, temperature=0.0, seed=4)
+    B, P, V = x.target.shape
+    par = np.tile(np.arange(-1, P - 1, dtype=np.int32), (B, 1))
+    tok = np.concatenate([np.zeros((B, 1), np.int32), x.draft_tokens.numpy()], axis=1)
+    t = oracle.tree_greedy(x.target, torch.from_numpy(tok), torch.from_numpy(par), P - 1)
+    c = oracle.verify_chain(x.target, None, x.draft_tokens, None, 0.0)
+    assert (t["accepted_len"] == c["accepted_len"]).all()
+    assert (t["out_tokens"] == c["out_tokens"]).all()
+    assert (c["accepted_len"] > 0).any()
+
+
+# --------------------------------------------------------------------------
+# Top-K: a full stable sort (numpy lexsort) and scipy's logsumexp.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("K,T", [(1, 1.0), (7, 0.7), (32, 1.0)])
+def test_topk_matches_full_sort(oracle, K, T):
+    rng = np.random.default_rng(K)
+    z = _quantised_rows(rng, (9, 500), levels=20) / 4
+    zt = inputs._cast(z, "bf16")
+    zz = zt.double().numpy()
+    r = oracle.topk(zt, K, T)
+    Tf = float(np.float32(T))
+    for row in range(z.shape[0]):
+        order = np.lexsort((np.arange(z.shape[1]), -zz[row]))[:K]
+        assert list(r["topk_idx"][row]) == list(order)
+        lse = scipy.special.logsumexp(zz[row] / Tf)
+        assert np.allclose(r["lse"][row], lse, rtol=1e-13)
+        assert np.allclose(r["topk_logp"][row], zz[row, order] / Tf - lse, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# KL(p~ || q): Gibbs' inequality, the zero case, scipy's rel_entr, V=2.
+# --------------------------------------------------------------------------
+def test_kl_nonnegative_and_matches_rel_entr(oracle):
+    x = inputs.make_chain(6, 3, 4000, dtype="bf16", sigma_d=1.0, temperature=1.0, seed=8)
+    tk = oracle.topk(x.target, 32, 1.0)
+    d = oracle.kl(tk["topk_logp"], tk["topk_idx"], x.draft, 1.0)
+    assert (d["kl"] >= -1e-12).all() and (d["kl"] > 0).all()
+    q = torch.softmax(x.draft.double(), -1).numpy()
+    for b in range(6):
+        for i in range(3):
+            pt = scipy.special.softmax(tk["topk_logp"][b, i])
+            ref = scipy.special.rel_entr(pt, q[b, i, tk["topk_idx"][b, i]]).sum()
+            assert np.isclose(d["kl"][b, i], ref, rtol=1e-11, atol=1e-14)
+
+
+def test_kl_zero_when_draft_is_renormalised_topk(oracle):
+    """q equal to the renormalised top-K of p (draft logits = target logits on
+    the kept set, -inf elsewhere) gives KL = 0."""
+    x = inputs.make_chain(3, 2, 1000, dtype="f32", sigma_d=0.0, temperature=0.9, seed=9)
+    tk = oracle.topk(x.target, 32, 0.9)
+    dr = torch.full_like(x.draft, -float("inf"))
+    for b in range(3):
+        for i in range(2):
+            ix = torch.from_numpy(tk["topk_idx"][b, i]).long()
+            dr[b, i, ix] = x.target[b, i, ix]
+    d = oracle.kl(tk["topk_logp"], tk["topk_idx"], dr, 0.9)
+    assert np.abs(d["kl"]).max() < 1e-13
+
+
+def test_kl_two_token_closed_form(oracle):
+    a_t, a_d, T = 0.8, -0.3, 1.0
+    zt = torch.tensor([[[a_t, 0.0], [0.0, 0.0]]], dtype=torch.float32)
+    zd = torch.tensor([[[a_d, 0.0]]], dtype=torch.float32)
+    tk = oracle.topk(zt, 2, T)
+    d = oracle.kl(tk["topk_logp"], tk["topk_idx"], zd, T)
+    p1 = 1 / (1 + math.exp(-float(np.float32(a_t))))
+    q1 = 1 / (1 + math.exp(-float(np.float32(a_d))))
+    ref = p1 * math.log(p1 / q1) + (1 - p1) * math.log((1 - p1) / (1 - q1))
+    assert math.isclose(d["kl"][0, 0], ref, rel_tol=1e-13)
+
+
+def test_kl_infinite_when_draft_misses_a_kept_token(oracle):
+    zt = torch.tensor([[[1.0, 0.5, 0.0], [0.0, 0.0, 0.0]]])
+    q = torch.tensor([[[0.0, 0.5, 0.5]]])
+    tk = oracle.topk(zt, 2, 1.0)
+    d = oracle.kl(tk["topk_logp"], tk["topk_idx"], q, 1.0, draft_kind=oracle.DRAFT_PROBS)
+    assert math.isinf(d["kl"][0, 0]) and d["kl"][0, 0] > 0
+
+
+# --------------------------------------------------------------------------
+# Reward weighting: the pages' worked examples.
+# --------------------------------------------------------------------------
+def test_kd_loss_worked_example(oracle):
+    g = json.load(open(os.path.join(GOLDEN, "respec_kd_loss_example.json")))
+    r = oracle.reward_loss(np.array([g["kl"]]), np.array([g["accepted_len"]]),
+                           np.array([g["reward"]]), mode=oracle.W_RAW)
+    assert math.isclose(r["loss"][0], g["loss"], rel_tol=1e-12)
+    assert math.isclose(r["total"], g["loss"], rel_tol=1e-12)
+    # Only accepted positions count: two accepted positions drop the third term.
+    r2 = oracle.reward_loss(np.array([g["kl"]]), np.array([2]), np.array([g["reward"]]))
+    assert math.isclose(r2["loss"][0], g["reward"] * (g["kl"][0] + g["kl"][1]), rel_tol=1e-12)
+
+
+def test_group_weights_worked_example(oracle):
+    g = json.load(open(os.path.join(GOLDEN, "respec_group_weights_example.json")))
+    rw = np.array(g["reward"])
+    B = len(rw)
+    kl = np.full((B, 1), g["kl_each"])
+    r = oracle.reward_loss(kl, np.ones(B, np.int32), rw, mode=oracle.W_GROUP_NORM, group=B)
+    printed = g["printed_weights"]
+    assert np.allclose(np.round(r["w"][:2], g["printed_decimals"]), printed)
+    assert r["w"][-1] == g["zero_reward_weight"] and r["loss"][-1] == 0.0
+    assert math.isclose(r["w"].sum(), 1.0, rel_tol=1e-12)
+    assert np.allclose(r["loss"], r["w"] * g["kl_each"], rtol=1e-12)
+
+
+def test_group_norm_zero_group_and_clip(oracle):
+    rw = np.array([0.0, 0.0, 0.5, 1.5])
+    kl = np.ones((4, 2))
+    acc = np.array([2, 1, 2, 0], np.int32)
+    r = oracle.reward_loss(kl, acc, rw, mode=oracle.W_GROUP_NORM, group=2)
+    assert (r["w"][:2] == 0).all() and math.isclose(r["w"][2], 0.25)
+    assert r["loss"][3] == 0.0
+    rc = oracle.reward_loss(kl, acc, np.array([0.1, 0.7, -2.0, 3.0]), mode=oracle.W_RAW, clip=0.5)
+    assert np.allclose(rc["w"], [0.1, 0.5, -0.5, 0.5])
+
+
+def test_oracle_is_thread_count_invariant(oracle):
+    x = inputs.make_chain(24, 3, 3000, dtype="bf16", temperature=0.7, seed=12)
+    a = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 0.7, threads=1)
+    b = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 0.7, threads=8)
+    for key in ("accepted_len", "out_tokens", "p_x", "cdf_margin"):
+        assert np.array_equal(a[key], b[key], equal_nan=True)
