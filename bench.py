@@ -1,0 +1,404 @@
+"""Benchmark: batched speculative-sampling verification on B200.
+
+Default workload (one step = one sv_verify_chain call): Qwen-vocabulary chain
+verification, B=32 requests x k=3 drafts, V=151936, bf16 logits, T=0.7.
+Metric: verified rows/s (B*(k+1) target rows per step), with the achieved HBM
+bandwidth of the verification kernel against the measured copy bandwidth.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the float64 CPU oracle, same metric
+
+Under torchrun every rank verifies its own batch (weak scaling, no collective
+on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_decoding_verification_94_b200 import inputs  # noqa: E402
+
+METRIC = "verified rows/s"
+UNIT = "rows/s"
+L2_BYTES = 126 * 1024 * 1024
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the chain
+# kernel, from profiles/ (None until a capture of the current kernel exists).
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="qwen_chain",
+                    choices=["qwen_chain", "kd", "tree", "tiny", "sweep"])
+    ap.add_argument("--B", type=int, default=None)
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--sigma", type=float, default=1.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def make_workload(a, rank):
+    seed = 1000 * rank
+    if a.workload == "qwen_chain":
+        B = a.B or 32
+        k = a.k or 3
+        x = inputs.qwen_chain(B=B, k=k, sigma_d=1.0, seed=seed)
+        return "chain", x, dict(workload="qwen_chain_verify", B=B, k=k, V=x.V, input_dtype="bf16",
+                                temperature=0.7, draft_sigma=1.0)
+    if a.workload == "sweep":
+        B = a.B or 8
+        k = a.k or 3
+        x = inputs.qwen_chain(B=B, k=k, sigma_d=a.sigma, seed=seed)
+        return "chain", x, dict(workload="active_batch_sweep_point", B=B, k=k, V=x.V,
+                                input_dtype="bf16", temperature=0.7, draft_sigma=a.sigma)
+    if a.workload == "kd":
+        B = a.B or 256
+        k = a.k or 3
+        x = inputs.kd_chain(B=B, k=k, seed=seed)
+        return "kd", x, dict(workload="fused_verify_kd", B=B, k=k, V=x.V, input_dtype="bf16",
+                             temperature=1.0, K=32, weighting="group_norm", group=16)
+    if a.workload == "tiny":
+        x = inputs.tiny_chain(seed=seed)
+        return "chain", x, dict(workload="tiny_chain_verify", B=4, k=3, V=1024,
+                                input_dtype="f32", temperature=1.0)
+    if a.workload == "tree":
+        t = inputs.make_tree(B=a.B or 8, seed=seed)
+        return "tree", t, dict(workload="greedy_tree_verify", B=t.logits.shape[0],
+                               n=t.logits.shape[1], V=t.logits.shape[2], depth=t.max_depth,
+                               branching=8, input_dtype="bf16", temperature=0.0)
+    raise ValueError(a.workload)
+
+
+def rows_and_bytes(kind, x):
+    """Verified rows per step and algorithmic bytes (each logit read once + I/O)."""
+    if kind == "tree":
+        B, n, V = x.logits.shape
+        es = x.logits.element_size()
+        return B * n, B * n * V * es + B * n * 8 + B * 4 + 2 * B * (x.max_depth + 1) * 4
+    B, P, V = x.target.shape
+    k = P - 1
+    te, de = x.target.element_size(), x.draft.element_size()
+    by = B * P * V * te + B * k * V * de + B * k * 4 + B * P * 4 + B * 4 + B * P * 4
+    if kind == "kd":
+        K = 32
+        by += B * P * K * 8 + B * P * 4 + B * k * 4 + B * 4 * 2 + 4
+    return B * P, by
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [r for (t, r) in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or [r for _, r in self.rows]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def oracle_step_fn(kind, x, threads=0):
+    from oracle import oracle as O  # CPU baseline only
+    if kind == "tree":
+        return lambda: O.tree_greedy(x.logits, x.node_tokens, x.parents, x.max_depth,
+                                     threads=threads)
+    if kind == "kd":
+        return lambda: O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward,
+                                   x.temperature, 32, mode=O.W_GROUP_NORM, group=16,
+                                   threads=threads)
+    return lambda: O.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, x.temperature,
+                                  threads=threads)
+
+
+def cpu_baseline(kind, x, rows, min_seconds=10.0):
+    """The oracle as it stands on this host's cores, on a bounded sample."""
+    from oracle import oracle as O
+    fn = oracle_step_fn(kind, x)
+    fn()  # builds / warms up
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or n >= 1000:
+            break
+    return {"value": rows * n / dt, "unit": UNIT, "cores": O.max_threads(), "kind": "oracle",
+            "sample": f"{n} full batches of the same workload ({rows} rows each) in {dt:.1f} s"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    kind, x, cfg = make_workload(a, 0)
+    rows, _ = rows_and_bytes(kind, x)
+    from oracle import oracle as O
+    fn = oracle_step_fn(kind, x)
+    for _ in range(a.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        fn()
+    dt = time.perf_counter() - t0
+    value = rows * a.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * dt / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.max_threads(),
+                             "kind": "oracle",
+                             "sample": f"{a.steps} timed full batches ({rows} rows each)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return run_reference(a)
+    from speculative_decoding_verification_94_b200 import sv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    sv.lib()
+    assert a.warmup >= 3, "at least 3 warm-up steps"
+
+    kind, x, cfg = make_workload(a, rank)
+    rows, algo_bytes = rows_and_bytes(kind, x)
+    # input copies rotated so that the set exceeds 2x L2: every step reads HBM
+    ncopy = max(2, math.ceil(2.2 * L2_BYTES / algo_bytes))
+    stream = torch.cuda.current_stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if kind == "tree":
+        sets = [dict(logits=x.logits.to(dev), tok=x.node_tokens.to(dev), par=x.parents.to(dev))
+                for _ in range(ncopy)]
+        outs = dict(accepted_len=torch.empty(x.logits.shape[0], dtype=torch.int32, device=dev),
+                    out_tokens=torch.empty(x.logits.shape[0], x.max_depth + 1,
+                                           dtype=torch.int32, device=dev),
+                    accepted_nodes=torch.empty(x.logits.shape[0], x.max_depth + 1,
+                                               dtype=torch.int32, device=dev))
+
+        def step(i, d=None):
+            s = d or sets[i % ncopy]
+            sv.sv_verify_tree_greedy(s["logits"], s["tok"], s["par"], x.max_depth, out=outs,
+                                     device_status=status)
+    else:
+        sets = [dict(t=x.target.to(dev), d=x.draft.to(dev), tok=x.draft_tokens.to(dev),
+                     u=x.uniforms.to(dev), r=x.reward.to(dev)) for _ in range(ncopy)]
+        kdcfg = None
+        if kind == "kd":
+            kdcfg = dict(K=32, wmode="group_norm", group=16)
+        B, P = x.target.shape[0], x.target.shape[1]
+        outs = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=dev),
+                    out_tokens=torch.empty(B, P, dtype=torch.int32, device=dev))
+        if kdcfg:
+            outs.update(topk_logp=torch.empty(B, P, 32, device=dev),
+                        topk_idx=torch.empty(B, P, 32, dtype=torch.int32, device=dev),
+                        lse=torch.empty(B, P, device=dev), kl=torch.empty(B, P - 1, device=dev),
+                        loss=torch.empty(B, device=dev), total=torch.empty(1, device=dev))
+
+        def step(i, d=None):
+            s = d or sets[i % ncopy]
+            kd = None if kdcfg is None else dict(kdcfg, reward=s["r"])
+            sv.sv_verify_chain(s["t"], s["d"], s["tok"], s["u"], x.temperature, kd=kd, out=outs,
+                               device_status=status)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # warm-up: at least W steps and at least ~0.5 s of load before timing
+    for i in range(a.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    t_end = time.time() + 0.5
+    i = a.warmup
+    while time.time() < t_end:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize(dev)
+
+    # The K timed steps are captured once in a CUDA graph (host launch cost
+    # of a Python call exceeds the kernel time) and replayed once untimed,
+    # then once inside the timed region.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for s_ in range(a.steps):
+            step(s_)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    gstream = torch.cuda.current_stream(dev)
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tw0 = time.time()
+    start.record(gstream)
+    graph.replay()
+    end.record(gstream)
+    torch.cuda.synchronize(dev)
+    tw1 = time.time()
+    barrier()
+    ms_total = start.elapsed_time(end)
+    ms_launch = ms_total / a.steps  # one kernel launch per step
+    clk = clocks.stop(tw0, tw1)
+    if dist is not None:
+        tt = torch.tensor([ms_total, ms_launch], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total, ms_launch = float(tt[0]), float(tt[1])
+    st = int(status.item())
+    assert st & sv.SV_DEV_ERROR_MASK == 0, f"device status {st:#x}"
+
+    peak, peak_kind = load_peaks()
+    achieved = algo_bytes / (ms_launch * 1e-3) / 1e9
+    value = rows * world * a.steps / (ms_total * 1e-3)
+
+    # end to end through the public call: pinned host inputs -> device, verify,
+    # results -> pinned host, all inside the timed region.
+    e2e = None
+    if not a.no_e2e:
+        if kind == "tree":
+            host = dict(logits=x.logits.pin_memory(), tok=x.node_tokens.pin_memory(),
+                        par=x.parents.pin_memory())
+        else:
+            host = dict(t=x.target.pin_memory(), d=x.draft.pin_memory(),
+                        tok=x.draft_tokens.pin_memory(), u=x.uniforms.pin_memory(),
+                        r=x.reward.pin_memory())
+        dsts = sets[0]
+        res_h = {k2: torch.empty(v.shape, dtype=v.dtype).pin_memory()
+                 for k2, v in outs.items() if k2 in ("accepted_len", "out_tokens", "total")}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(v.numel() * v.element_size() for v in res_h.values())
+        n_e2e = max(3, min(a.steps, 50))
+
+        def e2e_step():
+            for k2, v in host.items():
+                dsts[k2].copy_(v, non_blocking=True)
+            step(0, dsts)
+            for k2, v in res_h.items():
+                v.copy_(outs[k2], non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = e0.elapsed_time(e1)
+        if dist is not None:
+            tt = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms_e2e = float(tt[0])
+        e2e = {"value": rows * world * n_e2e / (ms_e2e * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and not a.no_cpu:
+        cpu = cpu_baseline(kind, x, rows)
+
+    if rank == 0:
+        traffic = NCU_TRAFFIC.get(cfg["workload"])
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_total / a.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic",
+                "config": dict(cfg, l2=f"{ncopy} rotating input copies "
+                                       f"({ncopy * algo_bytes / 2**20:.0f} MiB > 2x L2)",
+                               parallelism=f"dp{world}" if world > 1 else "single"),
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
+                             "unit": "GB/s", "frac": achieved / peak,
+                             "traffic": traffic, "peak_kind": peak_kind,
+                             "algorithmic_bytes_per_launch": algo_bytes,
+                             "launch_us": ms_launch * 1e3,
+                             "kernel": "tree_greedy_kernel" if kind == "tree"
+                             else "chain_sample_kernel"},
+                "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / 8000.0,
+                "e2e": e2e, "gpu_launches": a.steps, "clocks": clk,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

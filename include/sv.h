@@ -1,0 +1,225 @@
+/*
+ * sv.h -- C ABI of libsv: batched speculative-sampling verification on B200.
+ *
+ * Pages this interface restates (no page gives an API; the operations are
+ * theirs, the signatures are this library's):
+ *  - "基于推测性解码的强化学习训练" (ReSpec blog), section "推测解码
+ *    Speculative Decoding（SD）": the drafter proposes k tokens, the target
+ *    runs one forward over prefix + k, target and draft logits are compared,
+ *    the first bad token is resampled, else one more token is sampled from the
+ *    target.
+ *  - "ReSpec: Towards Optimizing Speculative Decoding in Reinforcement
+ *    Learning Systems" (reading notes): section 2 (acceptance test min(1, p/q),
+ *    residual max(0, p-q) / sum max(0, p-q)); section 3 (EAGLE candidate
+ *    trees with depth s, branching t, n nodes); section 4 (top-K = 32 target
+ *    log-probs of the V = 151936 row kept for distillation, KD target
+ *    KL(softmax(log p) || q)); section 5 (reward weight w(r) = r, normalised
+ *    and clipped).
+ *  - ReSpec blog, section "奖励加权的适应机制": L_KD = w(r) sum_t KL(p~ || q).
+ *
+ * Conventions shared by every entry point
+ *  - Every array argument is caller-owned DEVICE memory on the current CUDA
+ *    device, dense and row-major in the layout given; scalars are host values.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls only enqueue work on it: they never synchronise, never allocate
+ *    device memory, and outputs are valid once the stream reaches the call.
+ *  - Logits are fp32 or bf16 and must be finite or -inf (no NaN / +inf); every
+ *    row needs at least one finite logit.  Temperature T scales target and
+ *    draft logits alike (softmax(z / T)); T == 0 selects greedy verification
+ *    where the call allows it.
+ *  - Ties in argmax and top-K go to the lowest vocabulary index.
+ *  - Host-detectable errors (null or misaligned pointers, bad sizes, a
+ *    workspace that is too small) return a non-OK status and enqueue nothing.
+ *    Data-dependent errors found on the device are OR-ed as SV_DEV_* bits into
+ *    the optional `device_status` word (one int32 in device memory, may be
+ *    NULL); the caller zeroes it when it wants a fresh reading.  No kernel
+ *    traps, asserts or waits without a time limit.
+ *  - Workspace: the calls that take one need `*_workspace_size(...)` bytes of
+ *    device memory, 16-byte aligned, ZERO-FILLED before its first use.  Its
+ *    first 16 + 8*B bytes are counters; the rest is scratch that needs no
+ *    initialisation.  Every call that runs to completion leaves those 16 + 8*B
+ *    bytes zero again, so the workspace can be reused as is by any later call
+ *    with B' <= B; zero it again before a call with a larger B.  One workspace
+ *    must not be used by two calls that can run at the same time.
+ *  - Results are deterministic: the same inputs on the same device give
+ *    bit-identical outputs.
+ */
+#ifndef SV_H_
+#define SV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SV_API __attribute__((visibility("default")))
+#else
+#define SV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sv_status {
+  SV_OK = 0,
+  SV_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, size or mode out of range */
+  SV_ERR_UNSUPPORTED = 2,  /* valid but beyond this build (e.g. V too large for one row plan) */
+  SV_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, attribute, device query) */
+  SV_ERR_DEVICE_CHECK = 4, /* returned by sv_device_status_check() for SV_DEV_* error bits */
+  SV_ERR_TIMEOUT = 5,      /* returned by sv_device_status_check() for SV_DEV_TIMEOUT */
+  SV_ERR_WORKSPACE = 6     /* workspace pointer NULL, misaligned or smaller than required */
+} sv_status;
+
+typedef enum sv_dtype { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
+
+/* The draft distribution is given either as logits (softmax at T) or as
+ * fp32 probabilities used as given (not renormalised, T not applied). */
+typedef enum sv_draft_kind { SV_DRAFT_LOGITS = 0, SV_DRAFT_PROBS = 1 } sv_draft_kind;
+
+/* Reward weight w_b: RAW w = r_b; GROUP_NORM w = r_b / sum of r over the
+ * request's group of `group` consecutive requests (0 when that sum is 0). */
+typedef enum sv_weight_mode { SV_W_RAW = 0, SV_W_GROUP_NORM = 1 } sv_weight_mode;
+
+/* Device status bits (OR-ed into *device_status). */
+#define SV_DEV_BAD_TOKEN 0x1      /* a draft or node token outside [0, V) */
+#define SV_DEV_NO_FINITE 0x2      /* a logit row with no finite value */
+#define SV_DEV_TIMEOUT 0x4        /* a bounded wait for a bulk copy gave up */
+#define SV_DEV_BAD_TREE 0x8       /* parents[] is not a tree in BFS order, or depth > max_depth */
+#define SV_DEV_BAD_INDEX 0x10     /* a top-K index outside [0, V) given to sv_kd_kl_loss */
+#define SV_DEV_ERROR_MASK 0xff
+#define SV_DEV_RESIDUAL_ZERO 0x100 /* info: a rejection met zero residual mass; the target row was sampled */
+#define SV_DEV_TOPK_SLOW 0x200     /* info: massive ties sent a top-K through the slow exact path */
+
+/* KD outputs fused into sv_verify_chain (all device pointers). */
+typedef struct sv_kd_args {
+  int K;                      /* kept entries per row, 1..32 (32 on the pages) */
+  float* topk_logp;           /* [B, k+1, K] out: log p_j = z_j/T - lse, sorted (value desc, index asc) */
+  int32_t* topk_idx;          /* [B, k+1, K] out: vocabulary indices of the kept entries */
+  float* lse;                 /* [B, k+1]    out: log sum_j exp(z_j / T) of each target row */
+  float* kl;                  /* [B, k]      out: KL(p~ || q) of draft row i vs target row i */
+  const float* reward;        /* [B]         in:  scalar reward per request */
+  sv_weight_mode wmode;       /* reward weighting */
+  int group;                  /* GROUP_NORM group size (B % group == 0); ignored for RAW */
+  float clip;                 /* > 0: clamp w to [-clip, clip]; <= 0: no clipping */
+  float* loss;                /* [B]         out: w_b * sum_{i < accepted_len[b]} kl[b, i] (0 if w_b == 0) */
+  float* total;               /* [1]         out: sum_b loss[b], fixed summation order */
+} sv_kd_args;
+
+/* Bytes of zero-filled workspace needed by each call. */
+SV_API size_t sv_verify_chain_workspace_size(int B, int k);
+SV_API size_t sv_verify_tree_workspace_size(int B, int n);
+SV_API size_t sv_kd_kl_loss_workspace_size(int B, int k);
+
+/*
+ * sv_verify_chain -- verify k drafted tokens for each of B requests.
+ *
+ * Operation (ReSpec blog "推测解码" steps; reading notes section 2):
+ *   p_i = softmax(target[b, i, :] / T), q_i = softmax(draft[b, i, :] / T)
+ *   (or the given probabilities).  For i = 0..k-1 in order, draft token
+ *   x_i = draft_tokens[b, i] is accepted iff uniforms[b, i] * q_i(x_i) <
+ *   p_i(x_i) (probability min(1, p/q)).  At the first rejection i* the
+ *   emitted token is drawn from max(0, p_i* - q_i*) by inverse CDF in
+ *   ascending vocabulary order with uniforms[b, k]; if every draft is
+ *   accepted, a bonus token is drawn the same way from p_k.  A zero residual
+ *   mass (impossible when x ~ q) samples p_i* and sets SV_DEV_RESIDUAL_ZERO.
+ *   T == 0: x_i is accepted iff it equals argmax target[b, i, :]; the argmax
+ *   at the first mismatch (or at row k) is emitted; draft and uniforms may be
+ *   NULL and kd must be NULL.
+ *
+ * Arguments
+ *   target_logits [B, k+1, V] (t_dtype); row i is the target distribution for
+ *                 draft slot i, row k the bonus position.
+ *   draft         [B, k, V] logits (d_dtype) or fp32 probabilities (d_kind).
+ *   draft_tokens  [B, k] int32 in [0, V).
+ *   uniforms      [B, k+1] fp32 in [0, 1): column i < k tests draft i,
+ *                 column k drives the single resample-or-bonus draw.
+ *   B >= 0 (0 is a no-op), 1 <= k <= 255, 1 <= V <= 524288, T >= 0 finite.
+ *   accepted_len  [B] int32 out: n = accepted drafts (0..k); -1 marks a
+ *                 request whose inputs failed a device check.
+ *   out_tokens    [B, k+1] int32 out: x_0..x_{n-1}, then the resampled or
+ *                 bonus token, then -1 padding.
+ *   kd            NULL, or the fused KD outputs (T > 0 only): top-K of every
+ *                 target row, KL of every draft row against its target row,
+ *                 reward-weighted loss over the accepted positions.
+ *   workspace     sv_verify_chain_workspace_size(B, k) bytes, see above.
+ *   device_status optional int32 status word (SV_DEV_* bits).
+ */
+SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                          sv_dtype d_dtype, sv_draft_kind d_kind, const int32_t* draft_tokens,
+                          const float* uniforms, int B, int k, int V, float temperature,
+                          int32_t* accepted_len, int32_t* out_tokens, const sv_kd_args* kd,
+                          void* workspace, size_t workspace_bytes, int32_t* device_status,
+                          void* stream);
+
+/*
+ * sv_verify_tree_greedy -- greedy (T = 0) verification of B candidate trees
+ * (reading notes section 3: EAGLE trees of depth s, top-t branching, n nodes).
+ *
+ *   logits      [B, n, V] (dt): row j is the target distribution after node j.
+ *   node_tokens [B, n] int32: token of node j (node 0, the root, is unused).
+ *   parents     [B, n] int32: parents[b, 0] = -1, 0 <= parents[b, j] < j.
+ *   Node j >= 1 is accepted iff its parent is accepted and node_tokens[j] ==
+ *   argmax logits[b, parents[j], :]; the root is always accepted.  The deepest
+ *   accepted node wins (lowest index among equals); its depth d is
+ *   accepted_len[b] (depth must never exceed max_depth).
+ *   accepted_nodes [B, max_depth+1] out: the path root..best, then -1.
+ *   out_tokens     [B, max_depth+1] out: the path's tokens (root excluded),
+ *                  then argmax logits[b, best, :], then -1.
+ *   1 <= n <= 1024, 0 <= max_depth < n, 1 <= V <= 524288.
+ *   Invalid parents, depths or tokens set SV_DEV_BAD_TREE / SV_DEV_BAD_TOKEN
+ *   and accepted_len[b] = -1.
+ */
+SV_API sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* node_tokens,
+                                const int32_t* parents, int B, int n, int V, int max_depth,
+                                int32_t* accepted_len, int32_t* out_tokens,
+                                int32_t* accepted_nodes, void* workspace, size_t workspace_bytes,
+                                int32_t* device_status, void* stream);
+
+/*
+ * sv_extract_topk_kd -- the distillation buffer of the reading notes,
+ * section 4: for each of `rows` rows of V logits, the K largest logits
+ * (value desc, index asc) as full-vocabulary log-probs at temperature T.
+ *   logits [rows, V] (dt); topk_logp [rows, K] fp32 out; topk_idx [rows, K]
+ *   int32 out; lse [rows] fp32 out (log sum_j exp(z_j / T)).
+ *   1 <= K <= min(32, V), T > 0.  A [B, k+1, V] target is rows = B*(k+1).
+ */
+SV_API sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, int K,
+                             float temperature, float* topk_logp, int32_t* topk_idx, float* lse,
+                             int32_t* device_status, void* stream);
+
+/*
+ * sv_kd_kl_loss -- reward-weighted KD loss (ReSpec blog "奖励加权的适应机制";
+ * reading notes sections 4-5).
+ *   topk_logp, topk_idx [B, k+1, K] as produced by sv_extract_topk_kd on the
+ *   [B, k+1, V] target; draft [B, k, V] logits (d_dtype) or fp32 probs.
+ *   For each draft row (b, i < k): p~ = softmax of topk_logp[b, i, :] (the
+ *   renormalised kept target mass), log q_j = log softmax(draft[b, i] / T)_j
+ *   (or log of the given probability) at j = topk_idx[b, i, :],
+ *   kl[b, i] = sum_j p~_j (log p~_j - log q_j) (+inf when q_j = 0 < p~_j).
+ *   loss[b] = w_b * sum_{i < accepted_len[b]} kl[b, i] (0 when w_b == 0),
+ *   total[0] = sum_b loss[b]; w_b as in sv_weight_mode, optionally clipped.
+ *   accepted_len [B] int32 in [0, k]; reward [B] fp32; T > 0.
+ */
+SV_API sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
+                        const void* draft, sv_dtype d_dtype, sv_draft_kind d_kind, int V,
+                        float temperature, const int32_t* accepted_len, const float* reward,
+                        sv_weight_mode wmode, int group, float clip, float* kl, float* loss,
+                        float* total, void* workspace, size_t workspace_bytes,
+                        int32_t* device_status, void* stream);
+
+/* Map a device status word (read back by the caller) to a host status:
+ * SV_OK, SV_ERR_TIMEOUT if SV_DEV_TIMEOUT is set, else SV_ERR_DEVICE_CHECK
+ * if any other error bit is set.  Informational bits are ignored. */
+SV_API sv_status sv_device_status_check(int32_t device_status_word);
+
+/* Static description of a status code. */
+SV_API const char* sv_status_string(sv_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+SV_API int sv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SV_H_ */
