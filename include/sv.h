@@ -35,12 +35,12 @@
  *    NULL); the caller zeroes it when it wants a fresh reading.  No kernel
  *    traps, asserts or waits without a time limit.
  *  - Workspace: the calls that take one need `*_workspace_size(...)` bytes of
- *    device memory, 16-byte aligned, ZERO-FILLED before its first use.  Its
- *    first 16 + 8*B bytes are counters; the rest is scratch that needs no
- *    initialisation.  Every call that runs to completion leaves those 16 + 8*B
- *    bytes zero again, so the workspace can be reused as is by any later call
- *    with B' <= B; zero it again before a call with a larger B.  One workspace
- *    must not be used by two calls that can run at the same time.
+ *    device memory, 16-byte aligned, ZERO-FILLED before its first use (counters
+ *    and per-row results that the kernels hand between thread-block clusters).
+ *    Every call that runs to completion returns all of it to zero, so one
+ *    zeroing suffices for any later sequence of calls, of any entry point and
+ *    any size that fits.  One workspace must not be used by two calls that can
+ *    run at the same time.
  *  - Results are deterministic: the same inputs on the same device give
  *    bit-identical outputs.
  */

@@ -118,9 +118,51 @@ cudaError_t ensure_kernel_attrs(const void* kernel, int smem_bytes, bool nonport
   return cudaSuccess;
 }
 
-// Workspace: [0,16) batch counter; [16, 16+4B) per-request row counters;
-// [16+4B, 16+8B) per-request rejection words; then two int32 arrays of B*R
-// per-row results.  Completed calls leave the first 16+8B bytes zero.
+namespace {
+struct OccEntry {
+  const void* kernel;
+  int device, smem, cluster, n;
+};
+constexpr int kOccSlots = 256;
+OccEntry g_occ[kOccSlots];
+int g_occ_n = 0;
+std::mutex g_occ_mu;
+}  // namespace
+
+cudaError_t max_active_clusters(const void* kernel, int smem_bytes, int cluster, int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_occ_mu);
+  for (int i = 0; i < g_occ_n; ++i)
+    if (g_occ[i].kernel == kernel && g_occ[i].device == dev && g_occ[i].smem == smem_bytes &&
+        g_occ[i].cluster == cluster) {
+      *out = g_occ[i].n;
+      return cudaSuccess;
+    }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem_bytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+  if (e != cudaSuccess) return e;
+  if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{kernel, dev, smem_bytes, cluster, n};
+  *out = n;
+  return cudaSuccess;
+}
+
+// Workspace: [0,4) finished-request counter, [4,8) next work item, [8,12)
+// retired clusters; [16, 16+4B) per-request row counters; [16+4B, 16+8B)
+// per-request rejection words; then two int32 arrays of B*R per-row results.
+// Every word is returned to zero by the call that used it.
 size_t workspace_bytes(int B, int R) {
   if (B <= 0) return 256;
   size_t n = align_up(16 + 8 * (size_t)B, 16);
@@ -132,6 +174,8 @@ Workspace workspace_carve(void* base, int B, int R) {
   unsigned char* p = static_cast<unsigned char*>(base);
   Workspace w;
   w.glob_counter = reinterpret_cast<uint32_t*>(p);
+  w.work = reinterpret_cast<uint32_t*>(p + 4);
+  w.done = reinterpret_cast<uint32_t*>(p + 8);
   w.req_counter = reinterpret_cast<uint32_t*>(p + 16);
   w.req_reject = reinterpret_cast<uint32_t*>(p + 16 + 4 * (size_t)B);
   size_t off = align_up(16 + 8 * (size_t)B, 16);
@@ -165,6 +209,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   if (B < 0 || k < 1 || k > 255 || V < 1) return SV_ERR_INVALID_ARG;
   if (!(temperature >= 0.f) || !isfinite(temperature)) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(t_dtype)) return SV_ERR_INVALID_ARG;
+  if (B == 0 && (!kd || (kd->K >= 1 && kd->K <= kMaxK && kd->K <= V))) return SV_OK;
   if (!target_logits || !draft_tokens || !accepted_len || !out_tokens) return SV_ERR_INVALID_ARG;
   if (!aligned(target_logits, esize(t_dtype)) || !aligned(draft_tokens, 4) ||
       !aligned(accepted_len, 4) || !aligned(out_tokens, 4))
@@ -198,7 +243,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
 
   if (greedy) {
     RowPlan plan;
-    st = make_plan(V, esize(t_dtype), 0, [](int, int) { return 0; },
+    st = make_plan(V, esize(t_dtype), 0, [](int, int) { return 2 * kThreads * 4; },
                    bulk_ok_row(target_logits, V, esize(t_dtype)), &plan);
     if (st != SV_OK) return st;
     if ((long long)B * (k + 1) * plan.C > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
@@ -272,6 +317,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   if (B < 0 || n < 1 || n > 1024 || V < 1 || max_depth < 0 || max_depth >= n)
     return SV_ERR_INVALID_ARG;
   if (!dtype_ok(dt)) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
   if (!logits || !node_tokens || !parents || !accepted_len || !out_tokens || !accepted_nodes)
     return SV_ERR_INVALID_ARG;
   if (!aligned(logits, esize(dt)) || !aligned(node_tokens, 4) || !aligned(parents, 4) ||
@@ -310,7 +356,9 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
                              int32_t* device_status, void* stream) {
   if (rows < 0 || V < 1 || K < 1 || K > kMaxK || K > V) return SV_ERR_INVALID_ARG;
   if (!(temperature > 0.f) || !scale_ok(temperature)) return SV_ERR_INVALID_ARG;
-  if (!dtype_ok(dt) || !logits || !topk_logp || !topk_idx || !lse) return SV_ERR_INVALID_ARG;
+  if (!dtype_ok(dt)) return SV_ERR_INVALID_ARG;
+  if (rows == 0) return SV_OK;
+  if (!logits || !topk_logp || !topk_idx || !lse) return SV_ERR_INVALID_ARG;
   if (!aligned(logits, esize(dt)) || !aligned(topk_logp, 4) || !aligned(topk_idx, 4) ||
       !aligned(lse, 4))
     return SV_ERR_INVALID_ARG;
@@ -348,6 +396,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   if (d_kind != SV_DRAFT_LOGITS && d_kind != SV_DRAFT_PROBS) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(d_dtype) || (d_kind == SV_DRAFT_PROBS && d_dtype != SV_F32))
     return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
   if (!topk_logp || !topk_idx || !draft || !accepted_len || !reward || !kl || !loss || !total)
     return SV_ERR_INVALID_ARG;
   if (!aligned(topk_logp, 4) || !aligned(topk_idx, 4) || !aligned(draft, esize(d_dtype)) ||

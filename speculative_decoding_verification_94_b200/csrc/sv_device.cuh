@@ -324,11 +324,13 @@ __device__ __forceinline__ void scalar_fill(unsigned char* buf, const void* row_
 }
 
 // ---------------------------------------------------------------------------
-// Online softmax statistics.  A thread keeps its largest raw logit mz, the
-// reference ref = fl(mz * c) used as the exponent offset, and
-// S = sum 2^(fl(z*c - ref)) in float64 (8-term fp32 partials).  With
-// c = log2(e) / T this is the softmax normaliser sum exp(z/T - mz/T) up to
-// the rounding of ref, which is carried exactly through every rescale.
+// Online softmax statistics.  With c = log2(e) / T, a thread keeps its largest
+// raw logit mz, an integer-valued exponent reference ref >= c * mz (the
+// ceiling of c times its running maximum), and S = sum 2^(fl(z*c - ref)) in
+// float64 from 8-term fp32 partials.  Because ref is an integer, moving it
+// rescales S by an exact power of two, and the largest terms have exponents in
+// (-1, 0], where the fp32 argument is most precise.  CTA and cluster combines
+// rescale the same way, so no transcendental runs outside the per-element exp2.
 // ---------------------------------------------------------------------------
 struct ThreadStat {
   float mz;
@@ -342,11 +344,19 @@ __device__ __forceinline__ void stat_init(ThreadStat& s) {
   s.S = 0.0;
 }
 
+// S * 2^(from - to) for integer-valued from <= to (exact; underflows to 0).
+__device__ __forceinline__ double rescale_pow2(double S, float from, float to) {
+  if (S == 0.0) return 0.0;
+  const float d = from - to;
+  return d < -2000.f ? 0.0 : ldexp(S, (int)d);
+}
+
 __device__ __forceinline__ void stat_update(ThreadStat& s, const float v[8], float vmax, float c) {
-  if (vmax > s.mz) {
-    const float nref = vmax * c;
-    if (s.S != 0.0) s.S *= exp2((double)s.ref - (double)nref);
-    s.mz = vmax;
+  s.mz = fmaxf(s.mz, vmax);
+  const float top = vmax * c;
+  if (top > s.ref) {
+    const float nref = ceilf(top);
+    s.S = rescale_pow2(s.S, s.ref, nref);
     s.ref = nref;
   }
   if (vmax != -INFINITY) {
@@ -369,22 +379,79 @@ __device__ __forceinline__ CtaStat stat_block(const ThreadStat& s, float* redf, 
   CtaStat r;
   r.G = block_max(s.ref, redf);
   r.mz = block_max(s.mz, redf);
-  double mine = (s.S != 0.0) ? s.S * exp2((double)s.ref - (double)r.G) : 0.0;
-  r.S = block_sum(mine, redd);
+  r.S = block_sum(rescale_pow2(s.S, s.ref, r.G), redd);
   return r;
 }
 
-// Combine C CTA partials (fixed order) into the row's exponent reference G and
-// normaliser S; log2 of the partition function is G + log2(S).
-__device__ __forceinline__ void stat_combine(const float* G, const double* S, int C, float* Gout,
-                                             double* Sout) {
-  float Gm = -INFINITY;
-  for (int c = 0; c < C; ++c) Gm = fmaxf(Gm, G[c]);
-  double acc = 0.0;
-  for (int c = 0; c < C; ++c)
-    if (S[c] != 0.0) acc += S[c] * exp2((double)G[c] - (double)Gm);
+// Two rows at once (target and draft of a pair): one set of barriers.
+__device__ __forceinline__ void stat_block2(const ThreadStat& a, const ThreadStat& b,
+                                            float2* redf2, double2* redd2, CtaStat* ra,
+                                            CtaStat* rb) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float ga = warp_max(a.ref), gb = warp_max(b.ref), ma = warp_max(a.mz), mb = warp_max(b.mz);
+  __syncthreads();
+  if (lane == 0) {
+    redf2[w] = make_float2(ga, gb);
+    redf2[kWarps + w] = make_float2(ma, mb);
+  }
+  __syncthreads();
+  ga = redf2[0].x; gb = redf2[0].y; ma = redf2[kWarps].x; mb = redf2[kWarps].y;
+#pragma unroll
+  for (int i = 1; i < kWarps; ++i) {
+    ga = fmaxf(ga, redf2[i].x);
+    gb = fmaxf(gb, redf2[i].y);
+    ma = fmaxf(ma, redf2[kWarps + i].x);
+    mb = fmaxf(mb, redf2[kWarps + i].y);
+  }
+  double sa = warp_sum(rescale_pow2(a.S, a.ref, ga));
+  double sb = warp_sum(rescale_pow2(b.S, b.ref, gb));
+  if (lane == 0) redd2[w] = make_double2(sa, sb);
+  __syncthreads();
+  sa = redd2[0].x;
+  sb = redd2[0].y;
+#pragma unroll
+  for (int i = 1; i < kWarps; ++i) {
+    sa += redd2[i].x;
+    sb += redd2[i].y;
+  }
+  ra->G = ga; ra->mz = ma; ra->S = sa;
+  rb->G = gb; rb->mz = mb; rb->S = sb;
+}
+
+// Combine per-lane partials of warp 0 (lane q holds CTA q's, lanes >= C hold
+// G = -inf, S = 0) into the row's exponent reference and normaliser.  The
+// xor butterflies give every lane, and every CTA running the same code on
+// the same values, identical bits.
+__device__ __forceinline__ void warp_stat_combine(float G, double S, float* Gout, double* Sout) {
+  const float Gm = warp_max(G);
   *Gout = Gm;
-  *Sout = acc;
+  *Sout = warp_sum(rescale_pow2(S, G, Gm));
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = y > v ? y : v;
+  }
+  return v;
+}
+
+// Inclusive scan over the 32 lanes in a fixed order (lanes >= C add 0).
+__device__ __forceinline__ double warp_scan_incl(double v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
 }
 
 // ---------------------------------------------------------------------------

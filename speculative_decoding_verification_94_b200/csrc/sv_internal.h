@@ -15,8 +15,10 @@ struct Workspace {
   uint32_t* req_counter;   // [B]   rows of a request that have finished
   uint32_t* req_reject;    // [B]   max over rejected rows of (k - i); 0 = none yet
   uint32_t* glob_counter;  // [1]   requests that have finished
-  int32_t* row_a;          // [B*R] per-row result (accept bit / argmax / -1 error)
-  int32_t* row_b;          // [B*R] per-row sampled token (-1 if none)
+  uint32_t* work;          // [1]   next row item to hand out (persistent kernels)
+  uint32_t* done;          // [1]   clusters that have run out of items
+  int32_t* row_a;          // [B*R] per-row result code (0 = not yet written)
+  int32_t* row_b;          // [B*R] per-row value + 1 (sampled token / argmax; 0 = none)
 };
 
 size_t workspace_bytes(int B, int rows_per_request);
@@ -126,6 +128,10 @@ cudaError_t launch_kl(const KlParams& p, const RowPlan& plan, int d_dtype, int d
 // than 8 CTAs) once per device; later calls, including calls made while a
 // stream is being captured into a CUDA graph, only look the setting up.
 cudaError_t ensure_kernel_attrs(const void* kernel, int smem_bytes, bool nonportable_cluster);
+
+// Clusters of `cluster` CTAs (kThreads each, smem_bytes of dynamic shared
+// memory) that can be resident at once on the current device (cached).
+cudaError_t max_active_clusters(const void* kernel, int smem_bytes, int cluster, int* out);
 
 // Shared-memory layout for a chunk of L elements (bytes per element tb / db,
 // db = 0 when there is no second row) with `fixed` bytes of fixed block.

@@ -12,30 +12,35 @@ namespace sv {
 // read by the other CTAs of the cluster through distributed shared memory.
 struct RowShared {
   uint64_t bars[kMaxPieces];
-  // (x) per-CTA partials
+  // (x) per-CTA partials of the current item
   float G_t, G_d;
   double S_t, S_d;
   float zx_t, zx_d;
   int has_x;
   int timeouts;
-  int skip;
+  int skip;       // this CTA skipped the item (an earlier row of the request rejected)
+  int next_item;  // (rank 0) the item this cluster processes after the current one
+  int first_item; // (rank 0) the first item of this cluster
   int pad0;
   double R;
   unsigned long long key;
   unsigned long long topk[kMaxK];
   // block-local
   double ptot[kMaxPieces];
+  double wsum[kWarps][kMaxPieces];
   float redf[kWarps];
   double redd[kWarps];
+  float2 redf2[2 * kWarps];
+  double2 redd2[kWarps];
   unsigned long long redk[kWarps];
   float tmax[kWarps][32];
   float theta;
   int cand_count;
   unsigned long long keyth;
-  // row decision, computed by thread 0 and broadcast
+  // item decision, computed by warp 0 and broadcast
   float Gt, Gd;
   double St, Sd, Lt, Ld;
-  int accept, need, err, owner;
+  int accept, need, err, owner, rowskip, item;
   double base, tt;
   int piece, first_thread, last_pos, tok;
   int last, fin_n, fin_tok, redo;
@@ -43,12 +48,43 @@ struct RowShared {
 
 constexpr int kFixedBytes = (int)((sizeof(RowShared) + 127) / 128 * 128);
 
+// Row results kept in the workspace between a row and its request's
+// finalizer (zero = not written; the finalizer zeroes them again).
+enum RowResult : int { kRowAccepted = 1, kRowRejected = 2, kRowSkipped = 3, kRowError = 4 };
+
 template <class T>
 __device__ __forceinline__ const void* row_ptr(const void* base, size_t row, int V) {
   return reinterpret_cast<const unsigned char*>(base) + row * (size_t)V * T::bytes;
 }
 
-// Stage one or two rows' chunks into shared memory.  Collective.
+__device__ __forceinline__ uint32_t load_relaxed(const uint32_t* p) {
+  return *reinterpret_cast<const volatile uint32_t*>(p);
+}
+
+// Once per kernel (thread 0): initialise the piece barriers.
+__device__ __forceinline__ void init_piece_barriers(RowShared& sh, const ChunkGeom& g,
+                                                    bool use_bulk) {
+  if (use_bulk) {
+    for (int p = 0; p < g.npieces; ++p) mbar_init(&sh.bars[p], 1);
+    fence_mbar_init();
+  }
+}
+
+// Thread 0: arm the piece barriers of this item and issue its bulk copies.
+template <class TT, class DT, bool PAIR>
+__device__ __forceinline__ void issue_item_copies(RowShared& sh, unsigned char* tbuf,
+                                                  unsigned char* dbuf, const void* trow,
+                                                  const void* drow, const ChunkGeom& g,
+                                                  uint64_t policy) {
+  for (int p = 0; p < g.npieces; ++p)
+    mbar_arrive_expect_tx(&sh.bars[p],
+                          piece_bytes<TT>(g, p) + (PAIR ? piece_bytes<DT>(g, p) : 0u));
+  issue_row_copies<TT>(tbuf, trow, g, sh.bars, policy);
+  if (PAIR) issue_row_copies<DT>(dbuf, drow, g, sh.bars, policy);
+}
+
+// Stage one or two rows' chunks into shared memory (single-item kernels).
+// Collective.
 template <class TT, class DT, bool PAIR>
 __device__ __forceinline__ void stage_chunks(RowShared& sh, unsigned char* tbuf,
                                              unsigned char* dbuf, const void* trow,
@@ -56,39 +92,49 @@ __device__ __forceinline__ void stage_chunks(RowShared& sh, unsigned char* tbuf,
                                              bool use_bulk, bool dprobs) {
   if (threadIdx.x == 0) {
     sh.timeouts = 0;
-    if (use_bulk) {
-      for (int p = 0; p < g.npieces; ++p) mbar_init(&sh.bars[p], 1);
-      fence_mbar_init();
-    }
-  }
-  __syncthreads();
-  if (use_bulk && threadIdx.x == 0) {
-    const uint64_t pol = policy_evict_first();
-    for (int p = 0; p < g.npieces; ++p)
-      mbar_arrive_expect_tx(&sh.bars[p],
-                            piece_bytes<TT>(g, p) + (PAIR ? piece_bytes<DT>(g, p) : 0u));
-    issue_row_copies<TT>(tbuf, trow, g, sh.bars, pol);
-    if (PAIR) issue_row_copies<DT>(dbuf, drow, g, sh.bars, pol);
+    init_piece_barriers(sh, g, use_bulk);
+    if (use_bulk)
+      issue_item_copies<TT, DT, PAIR>(sh, tbuf, dbuf, trow, drow, g, policy_evict_first());
   }
   scalar_fill<TT>(tbuf, trow, g, use_bulk, false);
   if (PAIR) scalar_fill<DT>(dbuf, drow, g, use_bulk, dprobs);
   __syncthreads();
 }
 
-// Wait for piece p (bulk path); records a timeout in the block.
-__device__ __forceinline__ bool wait_piece(RowShared& sh, int p, bool use_bulk) {
+// Wait for piece p (bulk path) in phase `phase`; records a timeout.
+__device__ __forceinline__ bool wait_piece(RowShared& sh, int p, bool use_bulk,
+                                           uint32_t phase = 0) {
   if (!use_bulk) return true;
-  if (mbar_wait_bounded(&sh.bars[p], 0)) return true;
+  if (mbar_wait_bounded(&sh.bars[p], phase)) return true;
   atomicAdd(&sh.timeouts, 1);
   return false;
 }
 
-// Before exit: a CTA whose wait timed out waits once more (bounded) so that no
-// bulk copy into its shared memory is still in flight when it exits.
-__device__ __forceinline__ void drain_pieces(RowShared& sh, const ChunkGeom& g, bool use_bulk) {
+// After a timed-out wait, wait once more (bounded) so that no bulk copy into
+// shared memory is still in flight when the buffer is reused or the CTA exits.
+__device__ __forceinline__ void drain_pieces(RowShared& sh, const ChunkGeom& g, bool use_bulk,
+                                             uint32_t phase = 0) {
   if (!use_bulk || threadIdx.x != 0) return;
   if (sh.timeouts == 0) return;
-  for (int p = 0; p < g.npieces; ++p) mbar_wait_bounded(&sh.bars[p], 0);
+  for (int p = 0; p < g.npieces; ++p) mbar_wait_bounded(&sh.bars[p], phase);
+}
+
+// Per-piece totals of per-thread sums sums[p * kThreads + t], in a fixed
+// order (warp butterflies, then warps in index order).  Collective.
+__device__ __forceinline__ void piece_totals(const float* sums, int npieces, RowShared& sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int p = 0; p < npieces; ++p) {
+    const double v = warp_sum((double)sums[p * kThreads + threadIdx.x]);
+    if (lane == 0) sh.wsum[w][p] = v;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < npieces) {
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < kWarps; ++q) t += sh.wsum[q][threadIdx.x];
+    sh.ptot[threadIdx.x] = t;
+  }
+  __syncthreads();
 }
 
 __device__ __forceinline__ unsigned long long block_max_key(unsigned long long v,
@@ -180,15 +226,15 @@ __device__ void cta_topk(const unsigned char* buf, const ChunkGeom& g, float thr
 // key can be in the row's top K.
 __device__ inline void cluster_topk_merge(cg::cluster_group& cluster, int C, int K, RowShared& sh,
                                    unsigned long long* cand, unsigned long long* out) {
-  if (threadIdx.x == 0) {
-    unsigned long long th = kNoKey;
-    for (int c = 0; c < C; ++c) {
-      const RowShared* o = cluster.map_shared_rank(&sh, c);
-      const unsigned long long kk = o->topk[K - 1];
-      th = kk > th ? kk : th;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    unsigned long long th =
+        lane < C ? cluster.map_shared_rank(&sh, lane)->topk[K - 1] : kNoKey;
+    th = warp_max_u64(th);
+    if (lane == 0) {
+      sh.keyth = th;
+      sh.cand_count = 0;
     }
-    sh.keyth = th;
-    sh.cand_count = 0;
   }
   __syncthreads();
   const unsigned long long th = sh.keyth;

@@ -60,16 +60,21 @@ __global__ void __launch_bounds__(kThreads) tree_greedy_kernel(const ArgmaxParam
   if (threadIdx.x == 0) sh.key = key;
   drain_pieces(sh, g, use_bulk);
   cluster.sync();
-  if (rank == 0 && threadIdx.x == 0) {
+  if (rank == 0 && threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     unsigned long long best = kNoKey;
     int tmo = 0;
-    for (int q = 0; q < C; ++q) {
-      const RowShared* o = cluster.map_shared_rank(&sh, q);
-      best = o->key > best ? o->key : best;
-      tmo += o->timeouts;
+    if (lane < C) {
+      const RowShared* o = cluster.map_shared_rank(&sh, lane);
+      best = o->key;
+      tmo = o->timeouts;
     }
-    if (tmo) set_status(prm.status, SV_DEV_TIMEOUT);
-    prm.ws.row_a[(size_t)b * n + j] = tmo ? -1 : key_index(best);
+    best = warp_max_u64(best);
+    tmo = warp_sum_int(tmo);
+    if (lane == 0) {
+      if (tmo) set_status(prm.status, SV_DEV_TIMEOUT);
+      prm.ws.row_a[(size_t)b * n + j] = tmo ? 0 : key_index(best) + 1;  // 0 = no argmax
+    }
   }
   cluster.sync();
   if (rank != 0) return;
@@ -80,7 +85,8 @@ __global__ void __launch_bounds__(kThreads) tree_greedy_kernel(const ArgmaxParam
   int* tok = par + n;
   int* dep = tok + n;
   for (int t = threadIdx.x; t < n; t += kThreads) {
-    garg[t] = __ldcg(&prm.ws.row_a[(size_t)b * n + t]);
+    garg[t] = __ldcg(&prm.ws.row_a[(size_t)b * n + t]) - 1;
+    prm.ws.row_a[(size_t)b * n + t] = 0;
     par[t] = prm.parents[(size_t)b * n + t];
     tok[t] = prm.tokens[(size_t)b * n + t];
   }
@@ -176,22 +182,30 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkParams prm) {
   drain_pieces(sh, g, use_bulk);
   cluster.sync();
   if (rank == 0) {
-    if (threadIdx.x == 0) {
-      float Gs[kMaxCluster];
-      double Ss[kMaxCluster];
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      float G = -INFINITY;
+      double S = 0.0;
       int tmo = 0;
-      for (int q = 0; q < C; ++q) {
-        const RowShared* o = cluster.map_shared_rank(&sh, q);
-        Gs[q] = o->G_t;
-        Ss[q] = o->S_t;
-        tmo += o->timeouts;
+      if (lane < C) {
+        const RowShared* o = cluster.map_shared_rank(&sh, lane);
+        G = o->G_t;
+        S = o->S_t;
+        tmo = o->timeouts;
       }
-      stat_combine(Gs, Ss, C, &sh.Gt, &sh.St);
-      sh.Lt = (double)sh.Gt + log2(sh.St);
-      sh.err = 0;
-      if (sh.Gt == -INFINITY) sh.err |= SV_DEV_NO_FINITE;
-      if (tmo) sh.err |= SV_DEV_TIMEOUT;
-      if (sh.err) set_status(prm.status, sh.err);
+      float Gm;
+      double Sm;
+      warp_stat_combine(G, S, &Gm, &Sm);
+      tmo = warp_sum_int(tmo);
+      if (lane == 0) {
+        sh.Gt = Gm;
+        sh.St = Sm;
+        sh.Lt = (double)Gm + log2(Sm);
+        sh.err = 0;
+        if (Gm == -INFINITY) sh.err |= SV_DEV_NO_FINITE;
+        if (tmo) sh.err |= SV_DEV_TIMEOUT;
+        if (sh.err) set_status(prm.status, sh.err);
+      }
     }
     unsigned long long* out = cand + kCandCap - kMaxK;
     cluster_topk_merge(cluster, C, prm.K, sh, cand, out);
@@ -253,23 +267,31 @@ __global__ void __launch_bounds__(kThreads) kl_kernel(const KlParams prm) {
   }
   cluster.sync();
   if (rank == 0) {
-    if (threadIdx.x == 0) {
-      sh.err = 0;
-      sh.Ld = 0.0;
-      if (DKIND == kDraftLogits) {
-        float Gs[kMaxCluster];
-        double Ss[kMaxCluster];
-        int tmo = 0;
-        for (int q = 0; q < C; ++q) {
-          const RowShared* o = cluster.map_shared_rank(&sh, q);
-          Gs[q] = o->G_d;
-          Ss[q] = o->S_d;
-          tmo += o->timeouts;
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      float G = -INFINITY;
+      double S = 0.0;
+      int tmo = 0;
+      if (DKIND == kDraftLogits && lane < C) {
+        const RowShared* o = cluster.map_shared_rank(&sh, lane);
+        G = o->G_d;
+        S = o->S_d;
+        tmo = o->timeouts;
+      }
+      float Gm;
+      double Sm;
+      warp_stat_combine(G, S, &Gm, &Sm);
+      tmo = warp_sum_int(tmo);
+      if (lane == 0) {
+        sh.err = 0;
+        sh.Ld = 0.0;
+        if (DKIND == kDraftLogits) {
+          sh.Gd = Gm;
+          sh.Sd = Sm;
+          sh.Ld = (double)Gm + log2(Sm);
+          if (Gm == -INFINITY) sh.err |= SV_DEV_NO_FINITE;
+          if (tmo) sh.err |= SV_DEV_TIMEOUT;
         }
-        stat_combine(Gs, Ss, C, &sh.Gd, &sh.Sd);
-        sh.Ld = (double)sh.Gd + log2(sh.Sd);
-        if (sh.Gd == -INFINITY) sh.err |= SV_DEV_NO_FINITE;
-        if (tmo) sh.err |= SV_DEV_TIMEOUT;
       }
     }
     __syncthreads();

@@ -123,22 +123,19 @@ def _stream(device, stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-# Workspaces: zero-filled once; a completed call leaves its first 16 + 8*B
-# bytes zero, so a cached workspace is reused for any call with B <= the B it
-# was sized for, and replaced (zero-filled) otherwise.
+# Workspaces: zero-filled once when allocated; every completed call returns
+# all of it to zero, so a cached buffer serves any later call that fits.
 _WS: dict = {}
 
 
 def workspace(device: torch.device, B: int, nbytes: int) -> torch.Tensor:
     key = (device.index if device.index is not None else torch.cuda.current_device())
     cur = _WS.get(key)
-    if cur is None or cur[0] < B or cur[1].numel() < nbytes:
-        Bc = max(B, cur[0] if cur else 0)
-        nb = max(nbytes, cur[1].numel() if cur else 0)
-        buf = torch.zeros(nb, dtype=torch.uint8, device=device)
-        cur = (Bc, buf)
+    if cur is None or cur.numel() < nbytes:
+        cur = torch.zeros(max(nbytes, cur.numel() if cur is not None else 0), dtype=torch.uint8,
+                          device=device)
         _WS[key] = cur
-    return cur[1]
+    return cur
 
 
 def sv_verify_chain_workspace_size(B: int, k: int) -> int:

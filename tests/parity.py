@@ -69,3 +69,41 @@ def assert_close(got, ref, scale, what: str, rel: float = REL):
         raise AssertionError(f"{what}: {int((~ok).sum())} values out of tolerance; worst at "
                              f"{np.unravel_index(i, ref.shape)}: got {got.flat[i]!r} "
                              f"ref {ref.flat[i]!r} tol {tol.flat[i]!r}")
+
+
+def kd_rows(accepted_len, k: int):
+    """Masks of the KD rows the verifier defines: target rows 0..n and draft
+    rows 0..min(n, k-1) of each request (n = accepted_len).  Rows after the
+    emitted position are not read by the verifier and hold -1 / NaN."""
+    acc = np.asarray(accepted_len)
+    t = np.arange(k + 1)[None, :] <= acc[:, None]
+    d = np.arange(k)[None, :] <= acc[:, None]
+    return t, d
+
+
+def assert_kd_match(got: dict, ref: dict, k: int):
+    acc = got["accepted_len"].cpu().numpy()
+    tmask, dmask = kd_rows(acc, k)
+    idx = got["topk_idx"].cpu().numpy()
+    assert np.array_equal(idx[tmask], ref["topk_idx"][tmask]), "topk_idx"
+    assert (idx[~tmask] == -1).all()
+    lp = got["topk_logp"].cpu().numpy()
+    assert_close(lp[tmask], ref["topk_logp"][tmask], 1.0, "topk_logp")
+    assert np.isnan(lp[~tmask]).all()
+    lse = got["lse"].cpu().numpy()
+    assert_close(lse[tmask], ref["lse"][tmask], 1.0, "lse")
+    assert np.isnan(lse[~tmask]).all()
+    kl = got["kl"].cpu().numpy()
+    assert_close(kl[dmask], ref["kl"][dmask], ref["scale"][dmask], "kl")
+    assert np.isnan(kl[~dmask]).all()
+
+
+def bitwise_equal(a, b) -> bool:
+    """Equality of two tensors bit for bit (NaN == NaN)."""
+    import torch
+    if a.dtype != b.dtype or a.shape != b.shape:
+        return False
+    if a.dtype.is_floating_point:
+        return torch.equal(a.view(torch.int32 if a.element_size() == 4 else torch.int16),
+                           b.view(torch.int32 if b.element_size() == 4 else torch.int16))
+    return torch.equal(a, b)

@@ -8,7 +8,7 @@ import torch
 
 from oracle import oracle as O
 from speculative_decoding_verification_94_b200 import inputs, sv
-from tests.parity import assert_chain_match, assert_close
+from tests.parity import assert_chain_match, assert_close, assert_kd_match, bitwise_equal
 
 pytestmark = pytest.mark.gpu
 
@@ -105,10 +105,7 @@ def test_fused_verify_kd_full_size(kd256, wmode, group):
                       mode=O.W_GROUP_NORM if wmode == "group_norm" else O.W_RAW, group=group)
     r = assert_chain_match(got, ref, x.uniforms.numpy(), x.temperature, x.k)
     print("kd verify", r)
-    assert np.array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
-    assert_close(got["topk_logp"].cpu().numpy(), ref["topk_logp"], 1.0, "topk_logp")
-    assert_close(got["lse"].cpu().numpy(), ref["lse"], 1.0, "lse")
-    assert_close(got["kl"].cpu().numpy(), ref["kl"], ref["scale"], "kl")
+    assert_kd_match(got, ref, x.k)
     # loss / total against the oracle's KL and the GPU's own accepted lengths
     acc = got["accepted_len"].cpu().numpy()
     rl = O.reward_loss(ref["kl"], acc, x.reward.numpy().astype(np.float64),
@@ -191,15 +188,15 @@ def test_gpu_losslessness_chi_square():
 @pytest.mark.parametrize("V", [1, 2, 7, 8, 64, 1001, 4099, 70001, 151936])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_ragged_and_small_vocab(V, dtype):
-    x = inputs.make_chain(6, 3, V, dtype=dtype, model="zipf" if V > 64 else "gauss",
+    x = inputs.make_chain(12, 3, V, dtype=dtype, model="zipf" if V > 64 else "gauss",
                           sigma_t=2.0, sigma_d=1.0, temperature=0.9, seed=V)
-    check_chain(x, max_flag_frac=0.34)
+    check_chain(x, max_flag_frac=0.25)
 
 
 @pytest.mark.parametrize("k", [1, 15])
 def test_k_extremes(k):
-    check_chain(inputs.make_chain(5, k, 5000, dtype="bf16", sigma_d=0.3, temperature=1.0,
-                                  seed=k), max_flag_frac=0.2)
+    check_chain(inputs.make_chain(12, k, 5000, dtype="bf16", sigma_d=0.3, temperature=1.0,
+                                  seed=k), max_flag_frac=0.25)
 
 
 def test_empty_batch():
@@ -292,7 +289,7 @@ def test_topk_with_massive_ties_and_small_rows():
 def test_device_checks_flag_bad_inputs():
     x = inputs.make_chain(4, 3, 500, dtype="f32", seed=2)
     tok = x.draft_tokens.clone()
-    tok[1, 1] = 500  # out of range
+    tok[1, 0] = 500  # out of range (position 0 is always verified)
     st = status_tensor()
     got = sv.sv_verify_chain(x.target.to(DEV), x.draft.to(DEV), tok.to(DEV), x.uniforms.to(DEV),
                              1.0, device_status=st)
@@ -345,7 +342,7 @@ def test_deterministic_and_workspace_reuse(kd256):
     b = run_chain(x, kd=kd)
     torch.cuda.synchronize()
     for key in a:
-        assert torch.equal(a[key], b[key]), key
+        assert bitwise_equal(a[key], b[key]), key
     # a smaller batch on the same (cached) workspace, then the full one again
     sub = inputs.ChainInputs(x.target[:16].contiguous(), x.draft[:16].contiguous(),
                              x.draft_tokens[:16].contiguous(), x.uniforms[:16].contiguous(),
@@ -353,19 +350,20 @@ def test_deterministic_and_workspace_reuse(kd256):
     s = run_chain(sub, kd=dict(K=32, reward=sub.reward.to(DEV), wmode="group_norm", group=16))
     torch.cuda.synchronize()
     assert torch.equal(s["accepted_len"], a["accepted_len"][:16])
+    assert torch.equal(s["out_tokens"], a["out_tokens"][:16])
     assert torch.equal(s["topk_idx"], a["topk_idx"][:16])
     c = run_chain(x, kd=kd)
     torch.cuda.synchronize()
     for key in a:
-        assert torch.equal(a[key], c[key]), key
+        assert bitwise_equal(a[key], c[key]), key
 
 
 @pytest.mark.parametrize("C", [1, 2, 4, 8, 16])
 def test_every_cluster_size(monkeypatch, C):
     """The row plan's cluster size must not change any result."""
     monkeypatch.setenv("SV_CLUSTER_CTAS", str(C))
-    x = inputs.make_chain(8, 3, 20000, dtype="bf16", sigma_d=1.0, temperature=0.7, seed=C)
-    check_chain(x)
+    x = inputs.make_chain(24, 3, 20000, dtype="bf16", sigma_d=1.0, temperature=0.7, seed=C)
+    check_chain(x, max_flag_frac=0.2)
     got = sv.sv_extract_topk_kd(x.target.to(DEV), 32, 0.7)
     ref = O.topk(x.target, 32, 0.7)
     assert np.array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
