@@ -95,8 +95,27 @@ def make_workload(a, rank):
     raise ValueError(a.workload)
 
 
+def needed_bytes(kind, x, accepted_len):
+    """Bytes verification must read: for each request, target and draft rows
+    0..n (n = accepted drafts; draft rows stop at k-1) and the bonus target
+    row when every draft was accepted, plus the small inputs and outputs.
+    Rows after the first rejection are not part of the computation."""
+    if kind == "tree":
+        return rows_and_bytes(kind, x)[1]
+    B, P, V = x.target.shape
+    k = P - 1
+    te, de = x.target.element_size(), x.draft.element_size()
+    n = np.asarray(accepted_len, np.int64)
+    pairs = np.minimum(n, k - 1) + 1
+    by = int(np.sum(pairs) * V * (te + de) + np.sum(n == k) * V * te)
+    by += B * k * 4 + B * P * 4 + B * 4 + B * P * 4
+    if kind == "kd":
+        by += int(np.sum(n + 1)) * (32 * 8 + 4) + B * k * 4 + B * 4 * 2 + 4
+    return by
+
+
 def rows_and_bytes(kind, x):
-    """Verified rows per step and algorithmic bytes (each logit read once + I/O)."""
+    """Verified rows per step and the bytes of reading every logit once + I/O."""
     if kind == "tree":
         B, n, V = x.logits.shape
         es = x.logits.element_size()
@@ -325,6 +344,8 @@ def main():
     assert st & sv.SV_DEV_ERROR_MASK == 0, f"device status {st:#x}"
 
     peak, peak_kind = load_peaks()
+    full_bytes = algo_bytes
+    algo_bytes = needed_bytes(kind, x, outs["accepted_len"].cpu().numpy())
     achieved = algo_bytes / (ms_launch * 1e-3) / 1e9
     value = rows * world * a.steps / (ms_total * 1e-3)
 
@@ -388,6 +409,7 @@ def main():
                              "unit": "GB/s", "frac": achieved / peak,
                              "traffic": traffic, "peak_kind": peak_kind,
                              "algorithmic_bytes_per_launch": algo_bytes,
+                             "full_read_bytes_per_launch": full_bytes,
                              "launch_us": ms_launch * 1e3,
                              "kernel": "tree_greedy_kernel" if kind == "tree"
                              else "chain_sample_kernel"},

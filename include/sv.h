@@ -105,10 +105,14 @@ typedef struct sv_kd_args {
   float* total;               /* [1]         out: sum_b loss[b], fixed summation order */
 } sv_kd_args;
 
-/* Bytes of zero-filled workspace needed by each call. */
-SV_API size_t sv_verify_chain_workspace_size(int B, int k);
-SV_API size_t sv_verify_tree_workspace_size(int B, int n);
-SV_API size_t sv_kd_kl_loss_workspace_size(int B, int k);
+/* Bytes of zero-filled workspace needed by each call (K = 0: no fused KD).
+ * The workspace holds per-row chunk counters, row records and per-chunk
+ * partial results of the streaming pass: O(rows * V / 8192) small records,
+ * plus K keys per chunk when top-K lists are kept. */
+SV_API size_t sv_verify_chain_workspace_size(int B, int k, int V, int K);
+SV_API size_t sv_verify_tree_workspace_size(int B, int n, int V);
+SV_API size_t sv_extract_topk_workspace_size(int rows, int V, int K);
+SV_API size_t sv_kd_kl_loss_workspace_size(int B, int k, int V);
 
 /*
  * sv_verify_chain -- verify k drafted tokens for each of B requests.
@@ -138,10 +142,19 @@ SV_API size_t sv_kd_kl_loss_workspace_size(int B, int k);
  *                 request whose inputs failed a device check.
  *   out_tokens    [B, k+1] int32 out: x_0..x_{n-1}, then the resampled or
  *                 bonus token, then -1 padding.
- *   kd            NULL, or the fused KD outputs (T > 0 only): top-K of every
- *                 target row, KL of every draft row against its target row,
- *                 reward-weighted loss over the accepted positions.
- *   workspace     sv_verify_chain_workspace_size(B, k) bytes, see above.
+ *   kd            NULL, or the fused KD outputs (T > 0 only), for the rows of
+ *                 the emitted sequence: top-K, lse of target rows 0..n and KL
+ *                 of draft rows 0..min(n, k-1) against their target rows
+ *                 (n = accepted_len[b]); the reward-weighted loss over the
+ *                 accepted positions i < n.  Rows after the emitted position
+ *                 are not verified (and not read when the rejection is known
+ *                 in time): their top-K indices are -1 and their floats NaN.
+ *   workspace     sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0) bytes.
+ *
+ * Verification is sequential within a request: a draft after the first
+ * rejection is never tested.  Rows are streamed position-major and a row whose
+ * request has already rejected at an earlier position is skipped before it is
+ * loaded, so the bytes read approach the rows the outcome depends on.
  *   device_status optional int32 status word (SV_DEV_* bits).
  */
 SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
@@ -182,10 +195,12 @@ SV_API sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const in
  *   logits [rows, V] (dt); topk_logp [rows, K] fp32 out; topk_idx [rows, K]
  *   int32 out; lse [rows] fp32 out (log sum_j exp(z_j / T)).
  *   1 <= K <= min(32, V), T > 0.  A [B, k+1, V] target is rows = B*(k+1).
+ *   workspace: sv_extract_topk_workspace_size(rows, V, K) bytes.
  */
 SV_API sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, int K,
-                             float temperature, float* topk_logp, int32_t* topk_idx, float* lse,
-                             int32_t* device_status, void* stream);
+                                    float temperature, float* topk_logp, int32_t* topk_idx,
+                                    float* lse, void* workspace, size_t workspace_bytes,
+                                    int32_t* device_status, void* stream);
 
 /*
  * sv_kd_kl_loss -- reward-weighted KD loss (ReSpec blog "奖励加权的适应机制";

@@ -1,34 +1,37 @@
-// sv_api.cu -- the C ABI of libsv: argument validation, row plans, workspace
-// layout and kernel dispatch.  No entry point synchronises or allocates.
+// sv_api.cu -- the C ABI of libsv: argument validation, plans, workspace
+// layout and dispatch of the streaming pass and the finishing pass.  No entry
+// point synchronises or allocates.
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
 
-#include "sv_rowops.cuh"
+#include "sv_finish.cuh"
 
 namespace sv {
 
 namespace {
 
-constexpr int kMaxV = kMaxChunk * kMaxCluster;  // 524288
-constexpr int kTargetSmem = 48 * 1024;          // preferred per-CTA footprint
+constexpr int kMaxV = kMaxChunk * kMaxCluster;  // 524288: finishing plan limit
+constexpr int kTargetSmem = 48 * 1024;          // preferred per-CTA footprint (finishing)
 constexpr int kMaxSmem = 200 * 1024;            // hard per-CTA limit used by plans
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+int env_int(const char* name) {
+  const char* s = getenv(name);
+  return s ? atoi(s) : 0;
+}
+
 int forced_cluster() {
-  const char* s = getenv("SV_CLUSTER_CTAS");
-  if (!s) return 0;
-  int c = atoi(s);
+  const int c = env_int("SV_CLUSTER_CTAS");
   return (c == 1 || c == 2 || c == 4 || c == 8 || c == 16) ? c : 0;
 }
 
-// Smallest power-of-two cluster whose chunk fits the preferred shared-memory
-// footprint (or the largest cluster that fits at all).  `x_bytes(L, np)`
-// sizes the scratch region.
+// Finishing plan: the smallest power-of-two cluster whose chunk fits the
+// preferred shared-memory footprint (or the largest that fits at all).
 template <class XB>
 sv_status make_plan(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* plan) {
   if (V < 1 || V > kMaxV) return SV_ERR_UNSUPPORTED;
@@ -40,7 +43,11 @@ sv_status make_plan(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* pl
     const int L = (int)align_up((size_t)((V + C - 1) / C), kVec);
     if (L > kMaxChunk) continue;
     const int np = (L + kRound - 1) / kRound;
-    RowLayout lay = row_layout(kFixedBytes, L, tb, db, np, x_bytes(L, np));
+    RowLayout lay;
+    lay.off_t = kFixedBytes;
+    lay.off_d = lay.off_t + (int)align_up((size_t)L * tb, 128);
+    lay.off_x = lay.off_d + (int)align_up((size_t)L * db, 128);
+    lay.bytes = lay.off_x + (int)align_up((size_t)x_bytes(L, np), 128);
     if (lay.bytes > kMaxSmem) continue;
     best = RowPlan{C, L, np, bulk_ok ? 1 : 0, lay};
     have = true;
@@ -65,124 +72,212 @@ bool dtype_ok(int d) { return d == SV_F32 || d == SV_BF16; }
 
 sv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SV_OK : SV_ERR_CUDA; }
 
-}  // namespace
-
-RowLayout row_layout(int fixed, int L, int tb, int db, int npieces, int x_bytes) {
-  (void)npieces;
-  RowLayout l;
-  l.off_t = fixed;
-  l.off_d = l.off_t + (int)align_up((size_t)L * tb, 128);
-  l.off_x = l.off_d + (int)align_up((size_t)L * db, 128);
-  l.bytes = l.off_x + (int)align_up((size_t)x_bytes, 128);
-  return l;
-}
-
-namespace {
+// ---------------------------------------------------------------------------
+// Per-device caches of kernel attributes and occupancy.
+// ---------------------------------------------------------------------------
 struct AttrEntry {
   const void* kernel;
-  int device;
-  int smem;
-  bool nonportable;
+  int device, smem, extra, value;
 };
-constexpr int kAttrSlots = 256;
-AttrEntry g_attr[kAttrSlots];
+constexpr int kSlots = 512;
+AttrEntry g_attr[kSlots];
 int g_attr_n = 0;
-std::mutex g_attr_mu;
+AttrEntry g_occ[kSlots];
+int g_occ_n = 0;
+int g_sms[64];
+std::mutex g_mu;
+
 }  // namespace
 
 cudaError_t ensure_kernel_attrs(const void* kernel, int smem_bytes, bool nonportable) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_attr_mu);
+  std::lock_guard<std::mutex> lock(g_mu);
   AttrEntry* slot = nullptr;
   for (int i = 0; i < g_attr_n; ++i)
     if (g_attr[i].kernel == kernel && g_attr[i].device == dev) slot = &g_attr[i];
-  if (slot && slot->smem >= smem_bytes && (slot->nonportable || !nonportable)) return cudaSuccess;
+  if (slot && slot->smem >= smem_bytes && (slot->extra || !nonportable)) return cudaSuccess;
   const int want = slot && slot->smem > smem_bytes ? slot->smem : smem_bytes;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
   if (e != cudaSuccess) return e;
-  const bool np = nonportable || (slot && slot->nonportable);
+  const bool np = nonportable || (slot && slot->extra);
   if (np) {
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
   if (!slot) {
-    if (g_attr_n == kAttrSlots) return cudaSuccess;  // table full: set every time
+    if (g_attr_n == kSlots) return cudaSuccess;  // table full: set every time
     slot = &g_attr[g_attr_n++];
     slot->kernel = kernel;
     slot->device = dev;
   }
   slot->smem = want;
-  slot->nonportable = np;
+  slot->extra = np ? 1 : 0;
   return cudaSuccess;
 }
 
-namespace {
-struct OccEntry {
-  const void* kernel;
-  int device, smem, cluster, n;
-};
-constexpr int kOccSlots = 256;
-OccEntry g_occ[kOccSlots];
-int g_occ_n = 0;
-std::mutex g_occ_mu;
-}  // namespace
-
-cudaError_t max_active_clusters(const void* kernel, int smem_bytes, int cluster, int* out) {
+static cudaError_t blocks_per_sm(const void* kernel, int threads, int smem, int* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_occ_mu);
+  std::lock_guard<std::mutex> lock(g_mu);
   for (int i = 0; i < g_occ_n; ++i)
-    if (g_occ[i].kernel == kernel && g_occ[i].device == dev && g_occ[i].smem == smem_bytes &&
-        g_occ[i].cluster == cluster) {
-      *out = g_occ[i].n;
+    if (g_occ[i].kernel == kernel && g_occ[i].device == dev && g_occ[i].smem == smem &&
+        g_occ[i].extra == threads) {
+      *out = g_occ[i].value;
       return cudaSuccess;
     }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cluster, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem_bytes;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, (size_t)smem);
   if (e != cudaSuccess) return e;
-  if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{kernel, dev, smem_bytes, cluster, n};
+  if (g_occ_n < kSlots) g_occ[g_occ_n++] = AttrEntry{kernel, dev, smem, threads, n};
   *out = n;
   return cudaSuccess;
 }
 
-// Workspace: [0,4) finished-request counter, [4,8) next work item, [8,12)
-// retired clusters; [16, 16+4B) per-request row counters; [16+4B, 16+8B)
-// per-request rejection words; then two int32 arrays of B*R per-row results.
-// Every word is returned to zero by the call that used it.
-size_t workspace_bytes(int B, int R) {
-  if (B <= 0) return 256;
-  size_t n = align_up(16 + 8 * (size_t)B, 16);
-  n += 2 * align_up(4 * (size_t)B * (size_t)R, 16);
-  return align_up(n, 256);
+static cudaError_t sm_count(int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    g_sms[dev] = n;
+  }
+  *out = g_sms[dev];
+  return cudaSuccess;
 }
 
-Workspace workspace_carve(void* base, int B, int R) {
-  unsigned char* p = static_cast<unsigned char*>(base);
-  Workspace w;
-  w.glob_counter = reinterpret_cast<uint32_t*>(p);
-  w.work = reinterpret_cast<uint32_t*>(p + 4);
-  w.done = reinterpret_cast<uint32_t*>(p + 8);
-  w.req_counter = reinterpret_cast<uint32_t*>(p + 16);
-  w.req_reject = reinterpret_cast<uint32_t*>(p + 16 + 4 * (size_t)B);
-  size_t off = align_up(16 + 8 * (size_t)B, 16);
-  w.row_a = reinterpret_cast<int32_t*>(p + off);
-  off += align_up(4 * (size_t)B * (size_t)R, 16);
-  w.row_b = reinterpret_cast<int32_t*>(p + off);
+// Chunk length of the stream (a multiple of the piece): at most 8 pieces.
+static int stream_chunk(int V) {
+  const int forced = env_int("SV_STREAM_W");
+  if (forced >= kPiece && forced % kPiece == 0) return forced;
+  const int w = (int)align_up((size_t)V, kPiece);
+  return w < 8 * kPiece ? w : 8 * kPiece;
+}
+
+// Workspace: batch counter, per-request rejection words, per-row chunk
+// counters, row records, chunk partials and (top-K) chunk lists.  Every byte
+// is zero between calls.
+static WsLayout ws_layout(int B, int nrows, int nchunk, int K) {
+  WsLayout w;
+  size_t o = 0;
+  w.off_glob = o;
+  o += 16;
+  w.off_reject = o;
+  o = align_up(o + 4 * (size_t)B, 16);
+  w.off_counter = o;
+  o = align_up(o + 4 * (size_t)nrows, 16);
+  w.off_rec = o;
+  o += sizeof(RowRec) * (size_t)nrows;
+  w.off_part = o;
+  o += sizeof(Partial) * (size_t)nrows * nchunk;
+  w.off_cand = o;
+  o += 8 * (size_t)nrows * nchunk * K;
+  w.bytes = align_up(o, 256);
   return w;
+}
+
+struct WsPtrs {
+  uint32_t* glob;
+  uint32_t* reject;
+  uint32_t* counter;
+  RowRec* rec;
+  Partial* part;
+  unsigned long long* cand;
+};
+
+static WsPtrs ws_carve(void* base, const WsLayout& l) {
+  unsigned char* p = static_cast<unsigned char*>(base);
+  return WsPtrs{reinterpret_cast<uint32_t*>(p + l.off_glob),
+                reinterpret_cast<uint32_t*>(p + l.off_reject),
+                reinterpret_cast<uint32_t*>(p + l.off_counter),
+                reinterpret_cast<RowRec*>(p + l.off_rec), reinterpret_cast<Partial*>(p + l.off_part),
+                reinterpret_cast<unsigned long long*>(p + l.off_cand)};
+}
+
+// ---------------------------------------------------------------------------
+// Streaming pass.
+// ---------------------------------------------------------------------------
+struct StreamGeom {
+  int W, nchunk, stage_bytes, stage_off1, smem;
+};
+
+static StreamGeom stream_geom(int V, int te, int de) {
+  StreamGeom g;
+  g.W = stream_chunk(V);
+  g.nchunk = (V + g.W - 1) / g.W;
+  g.stage_off1 = (int)align_up((size_t)kPiece * te, 128);
+  g.stage_bytes = g.stage_off1 + (int)align_up((size_t)kPiece * de, 128);
+  g.smem = kStreamWarps * kStages * g.stage_bytes + kStreamWarps * kStages * 8;
+  return g;
+}
+
+template <class T0, class T1, int FLAGS>
+static cudaError_t launch_stream(StreamParams p, const StreamGeom& g, cudaStream_t s) {
+  auto kernel = stream_kernel<T0, T1, FLAGS>;
+  const void* kp = reinterpret_cast<const void*>(kernel);
+  cudaError_t e = ensure_kernel_attrs(kp, g.smem, false);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0, sms = 0;
+  if ((e = blocks_per_sm(kp, kStreamThreads, g.smem, &per_sm)) != cudaSuccess) return e;
+  if ((e = sm_count(&sms)) != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const long long items = (long long)p.nrows * p.nchunk;
+  long long grid = (long long)per_sm * sms;
+  const long long need = (items + kStreamWarps - 1) / kStreamWarps;
+  if (need < grid) grid = need;
+  if (grid < 1) grid = 1;
+  kernel<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Finishing pass.
+// ---------------------------------------------------------------------------
+template <class K, class Prm>
+static cudaError_t launch_clusters(K kernel, const Prm& prm, const RowPlan& plan, int nclusters,
+                                   cudaStream_t s) {
+  cudaError_t e = ensure_kernel_attrs(reinterpret_cast<const void*>(kernel), plan.lay.bytes,
+                                      plan.C > 8);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nclusters * (unsigned)plan.C, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)plan.lay.bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)plan.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, prm);
+}
+
+template <class K, class Prm>
+static cudaError_t launch_blocks(K kernel, const Prm& prm, int blocks, int smem, cudaStream_t s) {
+  cudaError_t e = ensure_kernel_attrs(reinterpret_cast<const void*>(kernel), smem, false);
+  if (e != cudaSuccess) return e;
+  kernel<<<(unsigned)blocks, kThreads, smem, s>>>(prm);
+  return cudaGetLastError();
+}
+
+template <class TT, class DT, int DKIND>
+static cudaError_t run_chain_sample(const StreamParams& sp, const StreamGeom& sg,
+                                    const FinishParams& fp, const RowPlan& plan, bool kd,
+                                    cudaStream_t s) {
+  constexpr int base = kFStats0 | kFRow1 | kFGather | (DKIND == kDraftLogits ? kFStats1 : 0);
+  cudaError_t e = kd ? launch_stream<TT, DT, base | kFTopk0>(sp, sg, s)
+                     : launch_stream<TT, DT, base>(sp, sg, s);
+  if (e != cudaSuccess) return e;
+  return kd ? launch_clusters(chain_sample_finish<TT, DT, DKIND, true>, fp, plan, fp.B, s)
+            : launch_clusters(chain_sample_finish<TT, DT, DKIND, false>, fp, plan, fp.B, s);
 }
 
 }  // namespace sv
@@ -191,9 +286,26 @@ using namespace sv;
 
 extern "C" {
 
-size_t sv_verify_chain_workspace_size(int B, int k) { return workspace_bytes(B, k + 1); }
-size_t sv_verify_tree_workspace_size(int B, int n) { return workspace_bytes(B, n); }
-size_t sv_kd_kl_loss_workspace_size(int B, int k) { return workspace_bytes(B, 0); }
+size_t sv_verify_chain_workspace_size(int B, int k, int V, int K) {
+  if (B <= 0 || k < 1 || V < 1) return 256;
+  const int W = stream_chunk(V);
+  return ws_layout(B, B * (k + 1), (V + W - 1) / W, K > 0 ? K : 0).bytes;
+}
+size_t sv_verify_tree_workspace_size(int B, int n, int V) {
+  if (B <= 0 || n < 1 || V < 1) return 256;
+  const int W = stream_chunk(V);
+  return ws_layout(B, B * n, (V + W - 1) / W, 0).bytes;
+}
+size_t sv_extract_topk_workspace_size(int rows, int V, int K) {
+  if (rows <= 0 || V < 1) return 256;
+  const int W = stream_chunk(V);
+  return ws_layout(rows, rows, (V + W - 1) / W, K > 0 ? K : 0).bytes;
+}
+size_t sv_kd_kl_loss_workspace_size(int B, int k, int V) {
+  if (B <= 0 || k < 1 || V < 1) return 256;
+  const int W = stream_chunk(V);
+  return ws_layout(B, B * k, (V + W - 1) / W, 0).bytes;
+}
 
 static sv_status check_workspace(void* ws, size_t bytes, size_t need) {
   if (!ws || !aligned(ws, 16) || bytes < need) return SV_ERR_WORKSPACE;
@@ -204,12 +316,13 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
                           sv_dtype d_dtype, sv_draft_kind d_kind, const int32_t* draft_tokens,
                           const float* uniforms, int B, int k, int V, float temperature,
                           int32_t* accepted_len, int32_t* out_tokens, const sv_kd_args* kd,
-                          void* workspace, size_t workspace_bytes_, int32_t* device_status,
+                          void* workspace, size_t workspace_bytes, int32_t* device_status,
                           void* stream) {
   if (B < 0 || k < 1 || k > 255 || V < 1) return SV_ERR_INVALID_ARG;
   if (!(temperature >= 0.f) || !isfinite(temperature)) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(t_dtype)) return SV_ERR_INVALID_ARG;
-  if (B == 0 && (!kd || (kd->K >= 1 && kd->K <= kMaxK && kd->K <= V))) return SV_OK;
+  if (kd && (kd->K < 1 || kd->K > kMaxK || kd->K > V)) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
   if (!target_logits || !draft_tokens || !accepted_len || !out_tokens) return SV_ERR_INVALID_ARG;
   if (!aligned(target_logits, esize(t_dtype)) || !aligned(draft_tokens, 4) ||
       !aligned(accepted_len, 4) || !aligned(out_tokens, 4))
@@ -226,93 +339,122 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
     if (!scale_ok(temperature)) return SV_ERR_INVALID_ARG;
   }
   if (kd) {
-    if (kd->K < 1 || kd->K > kMaxK || kd->K > V) return SV_ERR_INVALID_ARG;
     if (!kd->topk_logp || !kd->topk_idx || !kd->lse || !kd->kl || !kd->reward || !kd->loss ||
         !kd->total)
       return SV_ERR_INVALID_ARG;
     if (kd->wmode != SV_W_RAW && kd->wmode != SV_W_GROUP_NORM) return SV_ERR_INVALID_ARG;
-    if (kd->wmode == SV_W_GROUP_NORM && (kd->group < 1 || (B > 0 && B % kd->group != 0)))
+    if (kd->wmode == SV_W_GROUP_NORM && (kd->group < 1 || B % kd->group != 0))
       return SV_ERR_INVALID_ARG;
     if (!isfinite(kd->clip)) return SV_ERR_INVALID_ARG;
   }
-  if (B == 0) return SV_OK;
-  sv_status st = check_workspace(workspace, workspace_bytes_, workspace_bytes(B, k + 1));
+  if (V > kMaxV) return SV_ERR_UNSUPPORTED;
+  const int P = k + 1;
+  if ((long long)B * P > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
+  const int K = kd ? kd->K : 0;
+  const int te = esize(t_dtype);
+  const int de = greedy ? 0 : (d_kind == SV_DRAFT_PROBS ? 4 : esize(d_dtype));
+  const StreamGeom sg = stream_geom(V, te, de);
+  const WsLayout wl = ws_layout(B, B * P, sg.nchunk, K);
+  sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
+  const WsPtrs w = ws_carve(workspace, wl);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const Workspace ws = workspace_carve(workspace, B, k + 1);
+
+  StreamParams sp = {};
+  sp.rows0 = target_logits;
+  sp.rows1 = greedy ? nullptr : draft;
+  sp.tokens = draft_tokens;
+  sp.u = uniforms;
+  sp.kind = greedy ? kKindChainGreedy : kKindChainSample;
+  sp.B = B;
+  sp.k = k;
+  sp.V = V;
+  sp.nrows = B * P;
+  sp.W = sg.W;
+  sp.nchunk = sg.nchunk;
+  sp.c = greedy ? 0.f : (float)(1.4426950408889634 / (double)temperature);
+  sp.use_bulk = bulk_ok_row(target_logits, V, te) && (greedy || bulk_ok_row(draft, V, de));
+  sp.K = K > 0 ? K : 1;
+  sp.stage_bytes = sg.stage_bytes;
+  sp.stage_off1 = sg.stage_off1;
+  sp.part = w.part;
+  sp.cand = w.cand;
+  sp.rec = w.rec;
+  sp.row_counter = w.counter;
+  sp.req_reject = w.reject;
+  sp.status = device_status;
+
+  FinishParams fp = {};
+  fp.target = target_logits;
+  fp.draft = draft;
+  fp.tokens = draft_tokens;
+  fp.u = uniforms;
+  fp.B = B;
+  fp.k = k;
+  fp.V = V;
+  fp.nchunk = sg.nchunk;
+  fp.K = K;
+  fp.c = sp.c;
+  fp.accepted_len = accepted_len;
+  fp.out_tokens = out_tokens;
+  fp.part = w.part;
+  fp.cand = w.cand;
+  fp.rec = w.rec;
+  fp.req_reject = w.reject;
+  fp.glob_counter = w.glob;
+  fp.status = device_status;
+  if (kd) {
+    fp.topk_logp = kd->topk_logp;
+    fp.topk_idx = kd->topk_idx;
+    fp.lse = kd->lse;
+    fp.kl = kd->kl;
+    fp.reward = kd->reward;
+    fp.wmode = kd->wmode;
+    fp.group = kd->group < 1 ? 1 : kd->group;
+    fp.clip = kd->clip;
+    fp.loss = kd->loss;
+    fp.total = kd->total;
+  }
 
   if (greedy) {
-    RowPlan plan;
-    st = make_plan(V, esize(t_dtype), 0, [](int, int) { return 2 * kThreads * 4; },
-                   bulk_ok_row(target_logits, V, esize(t_dtype)), &plan);
-    if (st != SV_OK) return st;
-    if ((long long)B * (k + 1) * plan.C > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
-    ArgmaxParams p = {};
-    p.logits = target_logits;
-    p.tokens = draft_tokens;
-    p.B = B;
-    p.R = k + 1;
-    p.V = V;
-    p.L = plan.L;
-    p.use_bulk = plan.use_bulk;
-    p.lay = plan.lay;
-    p.accepted_len = accepted_len;
-    p.out_tokens = out_tokens;
-    p.ws = ws;
-    p.status = device_status;
-    return cuda_status(launch_chain_greedy(p, plan, t_dtype, s));
+    cudaError_t e = t_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
+                                       : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
+    if (e != cudaSuccess) return SV_ERR_CUDA;
+    return cuda_status(launch_blocks(chain_greedy_finish, fp, (B + kWarps - 1) / kWarps, 0, s));
   }
 
-  const int db = d_kind == SV_DRAFT_PROBS ? 4 : esize(d_dtype);
-  const bool with_kd = kd != nullptr;
+  const int nchunk = sg.nchunk;
   RowPlan plan;
   st = make_plan(
-      V, esize(t_dtype), db,
-      [with_kd](int, int np) {
+      V, te, de,
+      [K, nchunk](int, int np) {
         int x = np * kThreads * 4 + kThreads * 8;
         if (x < 2 * kThreads * 4) x = 2 * kThreads * 4;
-        if (with_kd && x < kCandCap * 8) x = kCandCap * 8;
-        return x;
+        const int xk = K > 0 ? kWarps * (nchunk * K + 32) * 8 : 0;
+        return x > xk ? x : xk;
       },
-      bulk_ok_row(target_logits, V, esize(t_dtype)) && bulk_ok_row(draft, V, db), &plan);
+      bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de), &plan);
   if (st != SV_OK) return st;
-  if ((long long)B * (k + 1) * plan.C > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
-  ChainParams p = {};
-  p.target = target_logits;
-  p.draft = draft;
-  p.tokens = draft_tokens;
-  p.u = uniforms;
-  p.B = B;
-  p.k = k;
-  p.V = V;
-  p.L = plan.L;
-  p.c = (float)(1.4426950408889634 / (double)temperature);
-  p.use_bulk = plan.use_bulk;
-  p.lay = plan.lay;
-  p.accepted_len = accepted_len;
-  p.out_tokens = out_tokens;
-  if (kd) {
-    p.K = kd->K;
-    p.topk_logp = kd->topk_logp;
-    p.topk_idx = kd->topk_idx;
-    p.lse = kd->lse;
-    p.kl = kd->kl;
-    p.reward = kd->reward;
-    p.wmode = kd->wmode;
-    p.group = kd->group < 1 ? 1 : kd->group;
-    p.clip = kd->clip;
-    p.loss = kd->loss;
-    p.total = kd->total;
-  }
-  p.ws = ws;
-  p.status = device_status;
-  return cuda_status(launch_chain_sample(p, plan, t_dtype, d_dtype, d_kind, with_kd, s));
+  fp.L = plan.L;
+  fp.use_bulk = plan.use_bulk;
+  fp.lay = plan.lay;
+  cudaError_t e;
+  if (d_kind == SV_DRAFT_PROBS)
+    e = t_dtype == SV_BF16 ? run_chain_sample<BF16, F32, kDraftProbs>(sp, sg, fp, plan, kd, s)
+                           : run_chain_sample<F32, F32, kDraftProbs>(sp, sg, fp, plan, kd, s);
+  else if (t_dtype == SV_BF16)
+    e = d_dtype == SV_BF16 ? run_chain_sample<BF16, BF16, kDraftLogits>(sp, sg, fp, plan, kd, s)
+                           : run_chain_sample<BF16, F32, kDraftLogits>(sp, sg, fp, plan, kd, s);
+  else
+    e = d_dtype == SV_BF16 ? run_chain_sample<F32, BF16, kDraftLogits>(sp, sg, fp, plan, kd, s)
+                           : run_chain_sample<F32, F32, kDraftLogits>(sp, sg, fp, plan, kd, s);
+  return cuda_status(e);
 }
 
 sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* node_tokens,
                                 const int32_t* parents, int B, int n, int V, int max_depth,
                                 int32_t* accepted_len, int32_t* out_tokens,
-                                int32_t* accepted_nodes, void* workspace, size_t workspace_bytes_,
+                                int32_t* accepted_nodes, void* workspace, size_t workspace_bytes,
                                 int32_t* device_status, void* stream) {
   if (B < 0 || n < 1 || n > 1024 || V < 1 || max_depth < 0 || max_depth >= n)
     return SV_ERR_INVALID_ARG;
@@ -324,38 +466,59 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
       !aligned(accepted_len, 4) || !aligned(out_tokens, 4) || !aligned(accepted_nodes, 4))
     return SV_ERR_INVALID_ARG;
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
-  if (B == 0) return SV_OK;
-  sv_status st = check_workspace(workspace, workspace_bytes_, workspace_bytes(B, n));
+  if ((long long)B * n > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
+  const StreamGeom sg = stream_geom(V, esize(dt), 0);
+  const WsLayout wl = ws_layout(B, B * n, sg.nchunk, 0);
+  sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
-  RowPlan plan;
-  st = make_plan(V, esize(dt), 0, [n](int, int) { return 4 * n * 4; },
-                 bulk_ok_row(logits, V, esize(dt)), &plan);
-  if (st != SV_OK) return st;
-  if ((long long)B * n * plan.C > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
-  ArgmaxParams p = {};
-  p.logits = logits;
-  p.tokens = node_tokens;
-  p.parents = parents;
-  p.B = B;
-  p.R = n;
-  p.V = V;
-  p.L = plan.L;
-  p.max_depth = max_depth;
-  p.use_bulk = plan.use_bulk;
-  p.lay = plan.lay;
-  p.accepted_len = accepted_len;
-  p.out_tokens = out_tokens;
-  p.accepted_nodes = accepted_nodes;
-  p.ws = workspace_carve(workspace, B, n);
-  p.status = device_status;
-  return cuda_status(launch_tree_greedy(p, plan, dt, reinterpret_cast<cudaStream_t>(stream)));
+  const WsPtrs w = ws_carve(workspace, wl);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  StreamParams sp = {};
+  sp.rows0 = logits;
+  sp.kind = kKindRows;
+  sp.B = B * n;
+  sp.k = 1;
+  sp.V = V;
+  sp.nrows = B * n;
+  sp.W = sg.W;
+  sp.nchunk = sg.nchunk;
+  sp.use_bulk = bulk_ok_row(logits, V, esize(dt));
+  sp.K = 1;
+  sp.stage_bytes = sg.stage_bytes;
+  sp.stage_off1 = sg.stage_off1;
+  sp.part = w.part;
+  sp.cand = w.cand;
+  sp.rec = w.rec;
+  sp.row_counter = w.counter;
+  sp.req_reject = w.reject;
+  sp.status = device_status;
+  cudaError_t e = dt == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
+                                : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
+  if (e != cudaSuccess) return SV_ERR_CUDA;
+  FinishParams fp = {};
+  fp.tokens = node_tokens;
+  fp.parents = parents;
+  fp.B = B;
+  fp.k = n;
+  fp.V = V;
+  fp.nchunk = sg.nchunk;
+  fp.max_depth = max_depth;
+  fp.accepted_len = accepted_len;
+  fp.out_tokens = out_tokens;
+  fp.accepted_nodes = accepted_nodes;
+  fp.part = w.part;
+  fp.rec = w.rec;
+  fp.req_reject = w.reject;
+  fp.status = device_status;
+  return cuda_status(launch_blocks(tree_finish, fp, B, kFixedBytes + 4 * n * 4, s));
 }
 
 sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, int K,
                              float temperature, float* topk_logp, int32_t* topk_idx, float* lse,
-                             int32_t* device_status, void* stream) {
+                             void* workspace, size_t workspace_bytes, int32_t* device_status,
+                             void* stream) {
   if (rows < 0 || V < 1 || K < 1 || K > kMaxK || K > V) return SV_ERR_INVALID_ARG;
-  if (!(temperature > 0.f) || !scale_ok(temperature)) return SV_ERR_INVALID_ARG;
+  if (!scale_ok(temperature)) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(dt)) return SV_ERR_INVALID_ARG;
   if (rows == 0) return SV_OK;
   if (!logits || !topk_logp || !topk_idx || !lse) return SV_ERR_INVALID_ARG;
@@ -363,39 +526,68 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
       !aligned(lse, 4))
     return SV_ERR_INVALID_ARG;
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
-  if (rows == 0) return SV_OK;
-  RowPlan plan;
-  sv_status st = make_plan(V, esize(dt), 0, [](int, int) { return kCandCap * 8; },
-                           bulk_ok_row(logits, V, esize(dt)), &plan);
+  if (rows > 0x7fffffff / 64) return SV_ERR_UNSUPPORTED;
+  const StreamGeom sg = stream_geom(V, esize(dt), 0);
+  const WsLayout wl = ws_layout(rows, rows, sg.nchunk, K);
+  sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
-  if ((long long)rows * plan.C > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
-  TopkParams p = {};
-  p.logits = logits;
-  p.rows = rows;
-  p.V = V;
-  p.L = plan.L;
-  p.K = K;
-  p.c = (float)(1.4426950408889634 / (double)temperature);
-  p.use_bulk = plan.use_bulk;
-  p.lay = plan.lay;
-  p.topk_logp = topk_logp;
-  p.topk_idx = topk_idx;
-  p.lse = lse;
-  p.status = device_status;
-  return cuda_status(launch_topk(p, plan, dt, reinterpret_cast<cudaStream_t>(stream)));
+  const WsPtrs w = ws_carve(workspace, wl);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  StreamParams sp = {};
+  sp.rows0 = logits;
+  sp.kind = kKindRows;
+  sp.B = rows;
+  sp.k = 1;
+  sp.V = V;
+  sp.nrows = rows;
+  sp.W = sg.W;
+  sp.nchunk = sg.nchunk;
+  sp.c = (float)(1.4426950408889634 / (double)temperature);
+  sp.use_bulk = bulk_ok_row(logits, V, esize(dt));
+  sp.K = K;
+  sp.stage_bytes = sg.stage_bytes;
+  sp.stage_off1 = sg.stage_off1;
+  sp.part = w.part;
+  sp.cand = w.cand;
+  sp.rec = w.rec;
+  sp.row_counter = w.counter;
+  sp.req_reject = w.reject;
+  sp.status = device_status;
+  cudaError_t e = dt == SV_BF16 ? launch_stream<BF16, BF16, kFStats0 | kFTopk0>(sp, sg, s)
+                                : launch_stream<F32, F32, kFStats0 | kFTopk0>(sp, sg, s);
+  if (e != cudaSuccess) return SV_ERR_CUDA;
+  FinishParams fp = {};
+  fp.B = rows;
+  fp.V = V;
+  fp.nchunk = sg.nchunk;
+  fp.K = K;
+  fp.c = sp.c;
+  fp.topk_logp = topk_logp;
+  fp.topk_idx = topk_idx;
+  fp.lse = lse;
+  fp.part = w.part;
+  fp.cand = w.cand;
+  fp.rec = w.rec;
+  fp.status = device_status;
+  const int smem = kWarps * (sg.nchunk * K + 32) * 8;
+  return cuda_status(launch_blocks(topk_finish, fp, (rows + kWarps - 1) / kWarps, smem, s));
 }
 
 sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
                         const void* draft, sv_dtype d_dtype, sv_draft_kind d_kind, int V,
                         float temperature, const int32_t* accepted_len, const float* reward,
                         sv_weight_mode wmode, int group, float clip, float* kl, float* loss,
-                        float* total, void* workspace, size_t workspace_bytes_,
+                        float* total, void* workspace, size_t workspace_bytes,
                         int32_t* device_status, void* stream) {
   if (B < 0 || k < 1 || k > 255 || K < 1 || K > kMaxK || V < 1 || K > V) return SV_ERR_INVALID_ARG;
-  if (!(temperature > 0.f) || !scale_ok(temperature)) return SV_ERR_INVALID_ARG;
+  if (!scale_ok(temperature)) return SV_ERR_INVALID_ARG;
   if (d_kind != SV_DRAFT_LOGITS && d_kind != SV_DRAFT_PROBS) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(d_dtype) || (d_kind == SV_DRAFT_PROBS && d_dtype != SV_F32))
     return SV_ERR_INVALID_ARG;
+  if (wmode != SV_W_RAW && wmode != SV_W_GROUP_NORM) return SV_ERR_INVALID_ARG;
+  if (wmode == SV_W_GROUP_NORM && (group < 1 || (B > 0 && B % group != 0)))
+    return SV_ERR_INVALID_ARG;
+  if (!isfinite(clip)) return SV_ERR_INVALID_ARG;
   if (B == 0) return SV_OK;
   if (!topk_logp || !topk_idx || !draft || !accepted_len || !reward || !kl || !loss || !total)
     return SV_ERR_INVALID_ARG;
@@ -403,47 +595,67 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
       !aligned(accepted_len, 4) || !aligned(reward, 4) || !aligned(kl, 4) || !aligned(loss, 4) ||
       !aligned(total, 4))
     return SV_ERR_INVALID_ARG;
-  if (wmode != SV_W_RAW && wmode != SV_W_GROUP_NORM) return SV_ERR_INVALID_ARG;
-  if (wmode == SV_W_GROUP_NORM && (group < 1 || (B > 0 && B % group != 0)))
-    return SV_ERR_INVALID_ARG;
-  if (!isfinite(clip)) return SV_ERR_INVALID_ARG;
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
-  if (B == 0) return SV_OK;
-  sv_status st = check_workspace(workspace, workspace_bytes_, workspace_bytes(B, 0));
+  if ((long long)B * k > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
+  const StreamGeom sg = stream_geom(V, esize(d_dtype), 0);
+  const WsLayout wl = ws_layout(B, B * k, sg.nchunk, 0);
+  sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
-  RowPlan plan;
-  if (d_kind == SV_DRAFT_PROBS) {
-    plan = RowPlan{1, 0, 0, 0, row_layout(kFixedBytes, 0, 0, 0, 0, 0)};
-  } else {
-    st = make_plan(V, esize(d_dtype), 0, [](int, int) { return 0; },
-                   bulk_ok_row(draft, V, esize(d_dtype)), &plan);
-    if (st != SV_OK) return st;
+  const WsPtrs w = ws_carve(workspace, wl);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const float c = (float)(1.4426950408889634 / (double)temperature);
+  if (d_kind == SV_DRAFT_LOGITS) {
+    StreamParams sp = {};
+    sp.rows0 = draft;
+    sp.kind = kKindRows;
+    sp.B = B * k;
+    sp.k = 1;
+    sp.V = V;
+    sp.nrows = B * k;
+    sp.W = sg.W;
+    sp.nchunk = sg.nchunk;
+    sp.c = c;
+    sp.use_bulk = bulk_ok_row(draft, V, esize(d_dtype));
+    sp.K = 1;
+    sp.stage_bytes = sg.stage_bytes;
+    sp.stage_off1 = sg.stage_off1;
+    sp.part = w.part;
+    sp.cand = w.cand;
+    sp.rec = w.rec;
+    sp.row_counter = w.counter;
+    sp.req_reject = w.reject;
+    sp.status = device_status;
+    cudaError_t e = d_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFStats0>(sp, sg, s)
+                                       : launch_stream<F32, F32, kFStats0>(sp, sg, s);
+    if (e != cudaSuccess) return SV_ERR_CUDA;
   }
-  if ((long long)B * k * plan.C > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
-  KlParams p = {};
-  p.topk_logp = topk_logp;
-  p.topk_idx = topk_idx;
-  p.draft = draft;
-  p.B = B;
-  p.k = k;
-  p.K = K;
-  p.V = V;
-  p.L = plan.L;
-  p.c = (float)(1.4426950408889634 / (double)temperature);
-  p.use_bulk = plan.use_bulk;
-  p.lay = plan.lay;
-  p.accepted_len = accepted_len;
-  p.reward = reward;
-  p.wmode = wmode;
-  p.group = group < 1 ? 1 : group;
-  p.clip = clip;
-  p.kl = kl;
-  p.loss = loss;
-  p.total = total;
-  p.ws = workspace_carve(workspace, B, 0);
-  p.status = device_status;
-  return cuda_status(
-      launch_kl(p, plan, d_dtype, d_kind, reinterpret_cast<cudaStream_t>(stream)));
+  FinishParams fp = {};
+  fp.draft = draft;
+  fp.B = B;
+  fp.k = k;
+  fp.K = K;
+  fp.V = V;
+  fp.nchunk = sg.nchunk;
+  fp.c = c;
+  fp.in_topk_logp = topk_logp;
+  fp.in_topk_idx = topk_idx;
+  fp.in_accepted_len = accepted_len;
+  fp.draft_probs = d_kind == SV_DRAFT_PROBS ? 1 : 0;
+  fp.reward = reward;
+  fp.wmode = wmode;
+  fp.group = group < 1 ? 1 : group;
+  fp.clip = clip;
+  fp.kl = kl;
+  fp.loss = loss;
+  fp.total = total;
+  fp.part = w.part;
+  fp.rec = w.rec;
+  fp.req_reject = w.reject;
+  fp.glob_counter = w.glob;
+  fp.status = device_status;
+  cudaError_t e = (d_dtype == SV_BF16) ? launch_blocks(kl_finish<BF16>, fp, B, kFixedBytes, s)
+                                       : launch_blocks(kl_finish<F32>, fp, B, kFixedBytes, s);
+  return cuda_status(e);
 }
 
 sv_status sv_device_status_check(int32_t w) {
@@ -465,6 +677,6 @@ const char* sv_status_string(sv_status s) {
   return "unknown status";
 }
 
-int sv_version(void) { return 100; }
+int sv_version(void) { return 200; }
 
 }  // extern "C"

@@ -1,6 +1,6 @@
-// sv_rowops.cuh -- row-level collectives built on sv_device.cuh: the shared
-// fixed block of every row kernel, chunk staging, CTA and cluster top-K, the
-// inverse-CDF draw over a cluster-resident row, and the request finalizers.
+// sv_rowops.cuh -- block-level pieces of the finishing kernels, built on
+// sv_device.cuh: the fixed shared-memory block, staging of one row pair's
+// chunk, per-piece totals, reward weights and the request/batch finalizers.
 #pragma once
 
 #include "sv_device.cuh"
@@ -47,10 +47,6 @@ struct RowShared {
 };
 
 constexpr int kFixedBytes = (int)((sizeof(RowShared) + 127) / 128 * 128);
-
-// Row results kept in the workspace between a row and its request's
-// finalizer (zero = not written; the finalizer zeroes them again).
-enum RowResult : int { kRowAccepted = 1, kRowRejected = 2, kRowSkipped = 3, kRowError = 4 };
 
 template <class T>
 __device__ __forceinline__ const void* row_ptr(const void* base, size_t row, int V) {
@@ -134,117 +130,6 @@ __device__ __forceinline__ void piece_totals(const float* sums, int npieces, Row
     for (int q = 0; q < kWarps; ++q) t += sh.wsum[q][threadIdx.x];
     sh.ptot[threadIdx.x] = t;
   }
-  __syncthreads();
-}
-
-__device__ __forceinline__ unsigned long long block_max_key(unsigned long long v,
-                                                            unsigned long long* red) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
-    v = y > v ? y : v;
-  }
-  __syncthreads();
-  if (lane == 0) red[w] = v;
-  __syncthreads();
-  unsigned long long r = red[0];
-#pragma unroll
-  for (int i = 1; i < kWarps; ++i) r = red[i] > r ? red[i] : r;
-  return r;
-}
-
-// CTA top-K of a staged chunk, sorted by (value desc, index asc) into sh.topk.
-// A threshold (the K-th largest per-thread maximum) bounds the candidates: at
-// least K elements reach it, so every top-K element does too.  Candidates are
-// ranked exactly.  Massive ties overflow the candidate buffer and take K
-// exact block-wide passes instead.  Collective.
-template <class T>
-__device__ void cta_topk(const unsigned char* buf, const ChunkGeom& g, float thread_max, int K,
-                         RowShared& sh, unsigned long long* cand, int32_t* status) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  float v = warp_sort_desc(thread_max);
-  sh.tmax[w][lane] = v;
-  __syncthreads();
-  if (w == 0) {
-    float a = sh.tmax[0][lane];
-    for (int q = 1; q < kWarps; ++q) a = warp_merge_desc(a, sh.tmax[q][lane]);
-    if (lane == K - 1) sh.theta = a;
-    if (lane == 0) sh.cand_count = 0;
-  }
-  __syncthreads();
-  const float th = sh.theta;
-  for (int p = 0; p < g.npieces; ++p) {
-    const int e = p * kRound + (int)threadIdx.x * kVec;
-    if (e < g.nvec * kVec) {
-      float x[8];
-      const float m = load8_max<T>(buf, e, x);
-      if (m >= th) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (e + q < g.len && x[q] >= th) {
-            const int pos = atomicAdd(&sh.cand_count, 1);
-            if (pos < kCandCap) cand[pos] = topk_key(x[q], g.j0 + e + q);
-          }
-        }
-      }
-    }
-  }
-  __syncthreads();
-  const int n = sh.cand_count;
-  if (n <= kCandCap) {
-    rank_select(cand, n, K, sh.topk);
-  } else {
-    if (threadIdx.x == 0) set_status(status, SV_DEV_TOPK_SLOW);
-    unsigned long long last = ~0ull;
-    for (int r = 0; r < K; ++r) {
-      unsigned long long best = kNoKey;
-      for (int p = 0; p < g.npieces; ++p) {
-        const int e = p * kRound + (int)threadIdx.x * kVec;
-        if (e < g.nvec * kVec) {
-          float x[8];
-          load8<T>(buf, e, x);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (e + q < g.len) {
-              const unsigned long long kk = topk_key(x[q], g.j0 + e + q);
-              if (kk < last && kk > best) best = kk;
-            }
-          }
-        }
-      }
-      best = block_max_key(best, sh.redk);
-      if (threadIdx.x == 0) sh.topk[r] = best;
-      last = best;
-    }
-  }
-  __syncthreads();
-}
-
-// Merge the C CTA lists of a cluster into the row's top-K (rank 0, collective
-// over its block).  Only keys at least as large as the largest per-CTA K-th
-// key can be in the row's top K.
-__device__ inline void cluster_topk_merge(cg::cluster_group& cluster, int C, int K, RowShared& sh,
-                                   unsigned long long* cand, unsigned long long* out) {
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    unsigned long long th =
-        lane < C ? cluster.map_shared_rank(&sh, lane)->topk[K - 1] : kNoKey;
-    th = warp_max_u64(th);
-    if (lane == 0) {
-      sh.keyth = th;
-      sh.cand_count = 0;
-    }
-  }
-  __syncthreads();
-  const unsigned long long th = sh.keyth;
-  for (int t = threadIdx.x; t < C * K; t += kThreads) {
-    const RowShared* o = cluster.map_shared_rank(&sh, t / K);
-    const unsigned long long kk = o->topk[t % K];
-    if (kk != kNoKey && kk >= th) cand[atomicAdd(&sh.cand_count, 1)] = kk;
-  }
-  __syncthreads();
-  rank_select(cand, sh.cand_count, K, out);
   __syncthreads();
 }
 

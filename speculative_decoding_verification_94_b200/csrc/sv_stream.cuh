@@ -1,0 +1,488 @@
+// sv_stream.cuh -- the streaming pass shared by every entry point.
+//
+// Every warp is an independent worker.  Work items are chunks of W vocabulary
+// entries of one row (or of a target/draft row pair, read together); warp g
+// takes items g, g + NW, g + 2NW, ... (NW warps in the grid), so items are
+// processed roughly in index order.  Chain items are numbered position-major
+// (every request's position 0 first): an item whose request has already
+// rejected at an earlier position is skipped before any byte is loaded, so
+// once a request's fate is known its later rows are never read.
+//
+// A warp streams its items through its own ring of kStages pieces of kPiece
+// elements; lane 0 issues bulk copies (cp.async.bulk, no multicast) up to
+// kStages pieces ahead, across item boundaries, and each piece completes on its
+// own mbarrier.  Per item the warp keeps online softmax statistics (sv_device
+// ThreadStat: exact power-of-two rescales), the element at the draft token,
+// the argmax, and a sorted warp list of the K best keys, reduces them with
+// shuffles, writes one partial record and counts the chunk into its row.  The
+// warp that completes a row combines the row's partials in chunk order (so
+// the result does not depend on which warp finished last) and records the
+// row's normaliser and, for chain rows, the acceptance decision.
+//
+// No __syncthreads, no cluster barrier and no shared-memory residency: the
+// only cross-warp communication is the per-row counter and the records.
+#pragma once
+
+#include "sv_device.cuh"
+
+namespace sv {
+
+constexpr int kPiece = 1024;                  // elements per piece
+constexpr int kLaneVecs = kPiece / (32 * kVec);  // 8-element vectors per lane per piece
+constexpr int kStages = 3;                    // ring depth per warp
+constexpr int kStreamWarps = 8;
+constexpr int kStreamThreads = kStreamWarps * 32;
+
+// What an item computes.
+enum StreamFlags : int {
+  kFStats0 = 1,    // softmax statistics of row 0
+  kFStats1 = 2,    // softmax statistics of row 1 (draft logits)
+  kFRow1 = 4,      // row 1 exists (draft logits or probabilities) and is staged
+  kFArgmax0 = 8,   // argmax of row 0
+  kFTopk0 = 16,    // top-K keys of row 0
+  kFGather = 32,   // the two rows' values at the row's draft token
+};
+
+// How items map to rows and what the row decision is.
+enum StreamKind : int {
+  kKindChainSample = 0,  // rows (i, b) position-major; target i [+ draft i]
+  kKindChainGreedy = 1,  // rows (i, b) position-major; target i
+  kKindRows = 2,         // plain rows (top-K, KL draft rows, tree nodes)
+};
+
+struct __align__(16) Partial {
+  float G0, G1;
+  double S0, S1;
+  float zx0, zx1;
+  int flags;  // kPHasX | kPSkipped | kPTimeout
+  int pad;
+  unsigned long long key;  // argmax key of row 0
+};
+enum : int { kPHasX = 1, kPSkipped = 2, kPTimeout = 4 };
+
+// Row record written by the warp that completes a row.
+struct __align__(16) RowRec {
+  int code;    // RowCode
+  int argmax;  // argmax of row 0 (greedy kinds)
+  float G0, G1;
+  double S0, S1;  // normalisers relative to the references G
+  double L0, L1;  // log2 of the partition functions: G + log2(S)
+};
+enum RowCode : int { kRowNone = 0, kRowAccepted = 1, kRowRejected = 2, kRowSkipped = 3,
+                     kRowError = 4 };
+
+struct StreamParams {
+  const void* rows0;      // row-0 array: target logits (chain, rows) or draft logits (KL)
+  const void* rows1;      // row-1 array: draft logits / probabilities (chain sample)
+  const int32_t* tokens;  // chain: draft tokens [B, k]
+  const float* u;         // chain sample: uniforms [B, k+1]
+  int kind;
+  int B, k, V;            // chain: k drafts per request (k+1 rows)
+  int nrows;              // rows streamed
+  int row0_stride_rows;   // chain: rows per request in rows0 (k+1); rows: 1
+  int W, nchunk;          // chunk length (multiple of kPiece) and chunks per row
+  float c;                // log2(e) / T
+  int use_bulk;
+  int K;                  // top-K list length (kFTopk0)
+  int stage_bytes;        // bytes per ring stage (row 0 then row 1), multiple of 128
+  int stage_off1;         // offset of row 1 inside a stage
+  Partial* part;          // [nrows * nchunk]
+  unsigned long long* cand;  // [nrows * nchunk * K]
+  RowRec* rec;            // [nrows]
+  uint32_t* row_counter;  // [nrows]
+  uint32_t* req_reject;   // [B] max over rejected chain rows of (k - i)
+  int32_t* status;
+};
+
+// Where row r of a stream lives.
+struct RowLoc {
+  int b, i;            // chain: request and position; rows: b = r, i = 0
+  const void* row0;
+  const void* row1;
+  int x;               // chain: draft token of this row (-1 for the bonus row / none)
+};
+
+template <class T0, class T1, int FLAGS>
+__device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r) {
+  RowLoc L;
+  if (p.kind == kKindRows) {
+    L.b = r;
+    L.i = 0;
+    L.row0 = reinterpret_cast<const unsigned char*>(p.rows0) + (size_t)r * p.V * T0::bytes;
+    L.row1 = nullptr;
+    L.x = -1;
+    return L;
+  }
+  L.i = r / p.B;
+  L.b = r - L.i * p.B;
+  const int P = p.k + 1;
+  L.row0 = reinterpret_cast<const unsigned char*>(p.rows0) + ((size_t)L.b * P + L.i) * p.V * T0::bytes;
+  L.row1 = nullptr;
+  if ((FLAGS & kFRow1) && L.i < p.k)
+    L.row1 = reinterpret_cast<const unsigned char*>(p.rows1) +
+             ((size_t)L.b * p.k + L.i) * p.V * T1::bytes;
+  L.x = (L.i < p.k) ? p.tokens[(size_t)L.b * p.k + L.i] : -1;
+  return L;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Insert a warp-uniform key into the sorted warp list (lane t holds entry t,
+// best first; only lanes < K are meaningful).
+__device__ __forceinline__ void warp_list_insert(unsigned long long& list, unsigned long long key,
+                                                 unsigned kmask) {
+  const int lane = threadIdx.x & 31;
+  const int pos = __popc(__ballot_sync(0xffffffffu, list > key) & kmask);
+  const unsigned long long up = __shfl_up_sync(0xffffffffu, list, 1);
+  if (lane > pos) list = up;
+  else if (lane == pos) list = key;
+}
+
+__device__ __forceinline__ uint32_t load_relaxed_u32(const uint32_t* p) {
+  return *reinterpret_cast<const volatile uint32_t*>(p);
+}
+
+// The warp that counted a row's last chunk: combine the row's partials in
+// chunk order (lane l takes chunks l, l+32, ...; butterflies across lanes),
+// then record the row and, for chain rows, take the acceptance decision.
+template <class T0, class T1, int FLAGS>
+__device__ __noinline__ void row_complete(const StreamParams& prm, int r, const RowLoc& L) {
+  const int lane = threadIdx.x & 31;
+  const int nchunk = prm.nchunk;
+  const Partial* base = prm.part + (size_t)r * nchunk;
+  float g0 = -INFINITY, g1 = -INFINITY, zx0 = 0.f, zx1 = 0.f;
+  int flags = 0, hx = 0;
+  unsigned long long key = kNoKey;
+  for (int q = lane; q < nchunk; q += 32) {
+    const Partial* pq = base + q;
+    g0 = fmaxf(g0, __ldcg(&pq->G0));
+    g1 = fmaxf(g1, __ldcg(&pq->G1));
+    const int f = __ldcg(&pq->flags);
+    flags |= f;
+    if (f & kPHasX) {
+      hx = 1;
+      zx0 = __ldcg(&pq->zx0);
+      zx1 = __ldcg(&pq->zx1);
+    }
+    const unsigned long long kq = __ldcg(&pq->key);
+    key = kq > key ? kq : key;
+  }
+  const float G0 = warp_max(g0), G1 = warp_max(g1);
+  double s0 = 0.0, s1 = 0.0;
+  for (int q = lane; q < nchunk; q += 32) {
+    const Partial* pq = base + q;
+    s0 += rescale_pow2(__ldcg(&pq->S0), __ldcg(&pq->G0), G0);
+    s1 += rescale_pow2(__ldcg(&pq->S1), __ldcg(&pq->G1), G1);
+  }
+  const double S0 = warp_sum(s0), S1 = warp_sum(s1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) flags |= __shfl_xor_sync(0xffffffffu, flags, o);
+  key = warp_max_u64(key);
+  const unsigned hm = __ballot_sync(0xffffffffu, hx != 0);
+  if (hm) {
+    const int src = __ffs(hm) - 1;
+    zx0 = __shfl_sync(0xffffffffu, zx0, src);
+    zx1 = __shfl_sync(0xffffffffu, zx1, src);
+  }
+  if (lane != 0) return;
+  RowRec rec;
+  rec.G0 = G0;
+  rec.G1 = G1;
+  rec.S0 = S0;
+  rec.S1 = S1;
+  rec.L0 = (double)G0 + log2(S0);
+  rec.L1 = (double)G1 + log2(S1);
+  rec.argmax = key_index(key);
+  int err = 0, code = kRowAccepted;
+  if (flags & kPTimeout) err |= SV_DEV_TIMEOUT;
+  if ((FLAGS & kFStats0) && G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
+  if ((FLAGS & kFStats1) && L.row1 != nullptr && G1 == -INFINITY) err |= SV_DEV_NO_FINITE;
+  if (prm.kind != kKindRows) {
+    const int i = L.i, b = L.b, k = prm.k;
+    if (flags & kPSkipped) {
+      err = 0;
+      code = kRowSkipped;
+    } else if (prm.kind == kKindChainSample) {
+      if (i < k && !hm) err |= SV_DEV_BAD_TOKEN;
+      if (!err && i < k) {
+        const double c = (double)prm.c;
+        const double px = exp2((double)zx0 * c - rec.L0);
+        const double qx = (FLAGS & kFStats1) ? exp2((double)zx1 * c - rec.L1) : (double)zx1;
+        const double u = (double)prm.u[(size_t)b * (k + 1) + i];
+        code = (u * qx < px) ? kRowAccepted : kRowRejected;
+      }
+    } else {  // greedy: accept iff the draft token is the argmax
+      if (i < k && (L.x < 0 || L.x >= prm.V)) err |= SV_DEV_BAD_TOKEN;
+      if (!err && i < k) code = (L.x == rec.argmax) ? kRowAccepted : kRowRejected;
+    }
+    if (code == kRowRejected && !err) atomicMax(&prm.req_reject[b], (uint32_t)(k - i));
+  }
+  if (err) {
+    set_status(prm.status, err);
+    code = kRowError;
+  }
+  rec.code = code;
+  prm.rec[r] = rec;
+  prm.row_counter[r] = 0u;
+}
+
+template <class T0, class T1, int FLAGS>
+__global__ void __launch_bounds__(kStreamThreads) stream_kernel(const StreamParams prm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char* ring = smem + (size_t)warp * kStages * prm.stage_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kStreamWarps * kStages * prm.stage_bytes) +
+                   warp * kStages;
+  const bool use_bulk = prm.use_bulk != 0;
+  const int V = prm.V, W = prm.W, nchunk = prm.nchunk;
+  const int total = prm.nrows * nchunk;
+  const int nwarps = (int)gridDim.x * kStreamWarps;
+  const int gwarp = (int)blockIdx.x * kStreamWarps + warp;
+  const float c = prm.c;
+  const int K = prm.K;
+  const unsigned kmask = K >= 32 ? 0xffffffffu : ((1u << K) - 1u);
+  uint64_t policy = 0;
+  if (lane == 0) {
+    if (use_bulk) {
+      for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+      fence_mbar_init();
+      policy = policy_evict_first();
+    }
+  }
+  __syncwarp();
+
+  // Pieces of an item; 0 when the item is skipped (an earlier position of its
+  // request rejected) or does not exist.
+  auto item_pieces = [&](int item) -> int {
+    if (item >= total) return 0;
+    const int r = item / nchunk, ch = item - r * nchunk;
+    const int len = min(W, V - ch * W);
+    int skip = 0;
+    if (prm.kind != kKindRows && lane == 0) {
+      const int i = r / prm.B, b = r - i * prm.B;
+      skip = load_relaxed_u32(&prm.req_reject[b]) > (uint32_t)(prm.k - i) ? 1 : 0;
+    }
+    skip = __shfl_sync(0xffffffffu, skip, 0);
+    return skip ? 0 : (len + kPiece - 1) / kPiece;
+  };
+
+  // Lane 0: bulk copies of piece p of item into ring stage s.
+  auto issue = [&](int item, int p, int s) {
+    const int r = item / nchunk, ch = item - r * nchunk;
+    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r);
+    const int e0 = ch * W + p * kPiece;
+    const int n = min(kPiece, min(V, ch * W + W) - e0);
+    const uint32_t nb0 = (uint32_t)(n * T0::bytes) & ~15u;
+    const uint32_t nb1 = (L.row1 != nullptr) ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
+    unsigned char* st = ring + (size_t)s * prm.stage_bytes;
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&bars[s], nb0 + nb1);
+    if (nb0)
+      bulk_g2s(st, reinterpret_cast<const unsigned char*>(L.row0) + (size_t)e0 * T0::bytes, nb0,
+               &bars[s], policy);
+    if (nb1)
+      bulk_g2s(st + prm.stage_off1,
+               reinterpret_cast<const unsigned char*>(L.row1) + (size_t)e0 * T1::bytes, nb1,
+               &bars[s], policy);
+  };
+
+  uint32_t n_issued = 0, n_consumed = 0;
+  int cur = gwarp;
+  int cur_np = item_pieces(cur);
+  int nxt = gwarp + nwarps;
+  int nxt_np = item_pieces(nxt);
+  int iss_which = 0, iss_p = 0;
+  int timeouts = 0;
+
+  auto top_up = [&]() {
+    while (n_issued - n_consumed < (uint32_t)kStages) {
+      int it, pp;
+      if (iss_which == 0) {
+        if (iss_p < cur_np) {
+          it = cur;
+          pp = iss_p++;
+        } else {
+          iss_which = 1;
+          iss_p = 0;
+          continue;
+        }
+      } else {
+        if (iss_p < nxt_np) {
+          it = nxt;
+          pp = iss_p++;
+        } else {
+          break;
+        }
+      }
+      if (use_bulk && lane == 0) issue(it, pp, (int)(n_issued % kStages));
+      ++n_issued;
+    }
+  };
+
+  top_up();
+  while (cur < total) {
+    const int r = cur / nchunk, ch = cur - r * nchunk;
+    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r);
+    const int clen = min(W, V - ch * W);
+    ThreadStat st0, st1;
+    stat_init(st0);
+    stat_init(st1);
+    float best = -INFINITY;
+    int bidx = -1;
+    float zx0 = 0.f, zx1 = 0.f;
+    int hx = 0;
+    unsigned long long list = kNoKey;
+    unsigned long long thr_key = kNoKey;
+    float thr_val = -INFINITY;
+
+    for (int p = 0; p < cur_np; ++p) {
+      const int s = (int)(n_consumed % kStages);
+      const uint32_t ph = (n_consumed / kStages) & 1u;
+      unsigned char* st = ring + (size_t)s * prm.stage_bytes;
+      unsigned char* st1p = st + prm.stage_off1;
+      const int e0 = ch * W + p * kPiece;  // row index of the piece's first element
+      const int n = min(kPiece, clen - p * kPiece);
+      if (use_bulk) {
+        if (!mbar_wait_bounded(&bars[s], ph)) ++timeouts;
+      }
+      // Elements the bulk copy does not cover (the unaligned tail, or the whole
+      // piece on the scalar path) and padding of the last vector.
+      {
+        const int a0 = use_bulk ? (int)(((uint32_t)(n * T0::bytes) & ~15u) / T0::bytes) : 0;
+        const typename T0::storage* src = reinterpret_cast<const typename T0::storage*>(L.row0) + e0;
+        for (int e = a0 + lane; e < n; e += 32)
+          reinterpret_cast<typename T0::storage*>(st)[e] = src[e];
+        for (int e = n + lane; e < ((n + kVec - 1) / kVec) * kVec; e += 32) store_pad<T0>(st, e, false);
+        if (L.row1 != nullptr) {
+          const int a1 = use_bulk ? (int)(((uint32_t)(n * T1::bytes) & ~15u) / T1::bytes) : 0;
+          const typename T1::storage* src1 =
+              reinterpret_cast<const typename T1::storage*>(L.row1) + e0;
+          for (int e = a1 + lane; e < n; e += 32)
+            reinterpret_cast<typename T1::storage*>(st1p)[e] = src1[e];
+          for (int e = n + lane; e < ((n + kVec - 1) / kVec) * kVec; e += 32)
+            store_pad<T1>(st1p, e, !(FLAGS & kFStats1));
+        }
+      }
+      __syncwarp();
+      const int nv = (n + kVec - 1) / kVec;
+#pragma unroll
+      for (int v = 0; v < kLaneVecs; ++v) {
+        const int vi = v * 32 + lane;
+        const bool act = vi < nv;
+        const int e = vi * kVec;
+        float x0[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) x0[t] = -INFINITY;
+        float m0 = -INFINITY;
+        if (act) {
+          m0 = load8_max<T0>(st, e, x0);
+          if (FLAGS & kFStats0) stat_update(st0, x0, m0, c);
+          if (FLAGS & kFArgmax0) {
+            if (m0 > best || bidx < 0) {
+              int q = 0;
+#pragma unroll
+              for (int t = 7; t >= 0; --t)
+                if (x0[t] == m0) q = t;
+              best = m0;
+              bidx = e0 + e + q;
+            }
+          }
+          if ((FLAGS & kFRow1) && L.row1 != nullptr && (FLAGS & kFStats1)) {
+            float x1[8];
+            const float m1 = load8_max<T1>(st1p, e, x1);
+            stat_update(st1, x1, m1, c);
+          }
+          if ((FLAGS & kFGather) && L.x >= e0 + e && L.x < e0 + e + kVec && L.x < e0 + n) {
+            hx = 1;
+            zx0 = load1<T0>(st, L.x - e0);
+            if ((FLAGS & kFRow1) && L.row1 != nullptr) zx1 = load1<T1>(st1p, L.x - e0);
+          }
+        }
+        if (FLAGS & kFTopk0) {
+          unsigned m = __ballot_sync(0xffffffffu, act && m0 >= thr_val);
+          while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            const int sbase = e0 + (v * 32 + src) * kVec;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float val = __shfl_sync(0xffffffffu, x0[q], src);
+              const int idx = sbase + q;
+              if (idx < e0 + n) {
+                const unsigned long long key = topk_key(val, idx);
+                if (key > thr_key) {
+                  warp_list_insert(list, key, kmask);
+                  thr_key = __shfl_sync(0xffffffffu, list, K - 1);
+                }
+              }
+            }
+          }
+          thr_val = thr_key == kNoKey ? -INFINITY : key_value(thr_key);
+        }
+      }
+      __syncwarp();
+      ++n_consumed;
+      top_up();
+    }
+
+    // Per-item reduction and partial record.
+    Partial pr;
+    pr.G0 = pr.G1 = -INFINITY;
+    pr.S0 = pr.S1 = 0.0;
+    if (FLAGS & kFStats0) {
+      pr.G0 = warp_max(st0.ref);
+      pr.S0 = warp_sum(rescale_pow2(st0.S, st0.ref, pr.G0));
+    }
+    if (FLAGS & kFStats1) {
+      pr.G1 = warp_max(st1.ref);
+      pr.S1 = warp_sum(rescale_pow2(st1.S, st1.ref, pr.G1));
+    }
+    pr.key = kNoKey;
+    if (FLAGS & kFArgmax0) pr.key = warp_max_u64(bidx < 0 ? kNoKey : topk_key(best, bidx));
+    pr.zx0 = pr.zx1 = 0.f;
+    int flags = 0;
+    if (FLAGS & kFGather) {
+      const unsigned hm = __ballot_sync(0xffffffffu, hx != 0);
+      if (hm) {
+        const int src = __ffs(hm) - 1;
+        pr.zx0 = __shfl_sync(0xffffffffu, zx0, src);
+        pr.zx1 = __shfl_sync(0xffffffffu, zx1, src);
+        flags |= kPHasX;
+      }
+    }
+    if (cur_np == 0) flags |= kPSkipped;
+    if (__any_sync(0xffffffffu, timeouts != 0)) flags |= kPTimeout;
+    pr.flags = flags;
+    pr.pad = 0;
+    if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)cur * K + lane] = list;
+    int last = 0;
+    if (lane == 0) {
+      prm.part[cur] = pr;
+      __threadfence();
+      last = atomicAdd(&prm.row_counter[r], 1u) == (uint32_t)(nchunk - 1) ? 1 : 0;
+      if (last) __threadfence();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) row_complete<T0, T1, FLAGS>(prm, r, L);
+    timeouts = 0;
+
+    // Advance.
+    cur = nxt;
+    cur_np = nxt_np;
+    if (iss_which == 0) iss_p = 0;  // (the issue side normally moved on to nxt already)
+    iss_which = 0;
+    nxt = cur + nwarps;
+    nxt_np = item_pieces(nxt);
+    top_up();
+  }
+  // Any copy still in flight (only after a timed-out wait) completes before exit.
+  if (use_bulk && lane == 0)
+    while (n_consumed < n_issued) {
+      mbar_wait_bounded(&bars[n_consumed % kStages], (n_consumed / kStages) & 1u);
+      ++n_consumed;
+    }
+}
+
+}  // namespace sv

@@ -28,8 +28,8 @@ SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
 EXPORTS = ("sv_verify_chain", "sv_verify_tree_greedy", "sv_extract_topk_kd", "sv_kd_kl_loss",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
-           "sv_kd_kl_loss_workspace_size", "sv_device_status_check", "sv_status_string",
-           "sv_version")
+           "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size",
+           "sv_device_status_check", "sv_status_string", "sv_version")
 
 
 class SVError(RuntimeError):
@@ -68,16 +68,19 @@ def lib() -> ctypes.CDLL:
                                           ctypes.POINTER(sv_kd_args), vp, sz, vp, vp]
             L.sv_verify_tree_greedy.argtypes = [vp, ci, vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, sz,
                                                 vp, vp]
-            L.sv_extract_topk_kd.argtypes = [vp, ci, ci, ci, ci, cf, vp, vp, vp, vp, vp]
+            L.sv_extract_topk_kd.argtypes = [vp, ci, ci, ci, ci, cf, vp, vp, vp, vp, sz, vp, vp]
             L.sv_kd_kl_loss.argtypes = [vp, vp, ci, ci, ci, vp, ci, ci, ci, cf, vp, vp, ci, ci, cf,
                                         vp, vp, vp, vp, sz, vp, vp]
             for f in ("sv_verify_chain", "sv_verify_tree_greedy", "sv_extract_topk_kd",
                       "sv_kd_kl_loss", "sv_device_status_check"):
                 getattr(L, f).restype = ci
             L.sv_device_status_check.argtypes = [ctypes.c_int32]
+            L.sv_verify_chain_workspace_size.argtypes = [ci, ci, ci, ci]
+            L.sv_verify_tree_workspace_size.argtypes = [ci, ci, ci]
+            L.sv_extract_topk_workspace_size.argtypes = [ci, ci, ci]
+            L.sv_kd_kl_loss_workspace_size.argtypes = [ci, ci, ci]
             for f in ("sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
-                      "sv_kd_kl_loss_workspace_size"):
-                getattr(L, f).argtypes = [ci, ci]
+                      "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size"):
                 getattr(L, f).restype = sz
             L.sv_status_string.argtypes = [ci]
             L.sv_status_string.restype = ctypes.c_char_p
@@ -138,16 +141,20 @@ def workspace(device: torch.device, B: int, nbytes: int) -> torch.Tensor:
     return cur
 
 
-def sv_verify_chain_workspace_size(B: int, k: int) -> int:
-    return int(lib().sv_verify_chain_workspace_size(B, k))
+def sv_verify_chain_workspace_size(B: int, k: int, V: int, K: int = 0) -> int:
+    return int(lib().sv_verify_chain_workspace_size(B, k, V, K))
 
 
-def sv_verify_tree_workspace_size(B: int, n: int) -> int:
-    return int(lib().sv_verify_tree_workspace_size(B, n))
+def sv_verify_tree_workspace_size(B: int, n: int, V: int) -> int:
+    return int(lib().sv_verify_tree_workspace_size(B, n, V))
 
 
-def sv_kd_kl_loss_workspace_size(B: int, k: int) -> int:
-    return int(lib().sv_kd_kl_loss_workspace_size(B, k))
+def sv_extract_topk_workspace_size(rows: int, V: int, K: int) -> int:
+    return int(lib().sv_extract_topk_workspace_size(rows, V, K))
+
+
+def sv_kd_kl_loss_workspace_size(B: int, k: int, V: int) -> int:
+    return int(lib().sv_kd_kl_loss_workspace_size(B, k, V))
 
 
 def sv_verify_chain(target: torch.Tensor, draft: torch.Tensor | None, draft_tokens: torch.Tensor,
@@ -193,7 +200,7 @@ def sv_verify_chain(target: torch.Tensor, draft: torch.Tensor | None, draft_toke
                                          reward.data_ptr(), wmode, int(kd.get("group", 1)),
                                          float(kd.get("clip", 0.0)), o["loss"].data_ptr(),
                                          o["total"].data_ptr()))
-    nbytes = sv_verify_chain_workspace_size(B, k)
+    nbytes = sv_verify_chain_workspace_size(B, k, V, int(kd.get("K", 32)) if kd else 0)
     w = ws if ws is not None else workspace(dev, B, nbytes)
     rc = lib().sv_verify_chain(
         _p(target), _dtype_code(target), _p(draft),
@@ -219,7 +226,7 @@ def sv_verify_tree_greedy(logits: torch.Tensor, node_tokens: torch.Tensor,
     o.setdefault("accepted_len", torch.empty(B, dtype=torch.int32, device=dev))
     o.setdefault("out_tokens", torch.empty(B, W, dtype=torch.int32, device=dev))
     o.setdefault("accepted_nodes", torch.empty(B, W, dtype=torch.int32, device=dev))
-    nbytes = sv_verify_tree_workspace_size(B, n)
+    nbytes = sv_verify_tree_workspace_size(B, n, V)
     w = ws if ws is not None else workspace(dev, B, nbytes)
     rc = lib().sv_verify_tree_greedy(_p(logits), _dtype_code(logits), _p(node_tokens),
                                      _p(parents), B, n, V, max_depth, _p(o["accepted_len"]),
@@ -230,8 +237,8 @@ def sv_verify_tree_greedy(logits: torch.Tensor, node_tokens: torch.Tensor,
 
 
 def sv_extract_topk_kd(logits: torch.Tensor, K: int, temperature: float, *,
-                       out: dict | None = None, device_status: torch.Tensor | None = None,
-                       stream=None) -> dict:
+                       out: dict | None = None, ws: torch.Tensor | None = None,
+                       device_status: torch.Tensor | None = None, stream=None) -> dict:
     """Top-K log-probs of every row of logits [..., V]."""
     _dev(logits, "logits")
     V = logits.shape[-1]
@@ -242,9 +249,11 @@ def sv_extract_topk_kd(logits: torch.Tensor, K: int, temperature: float, *,
     o.setdefault("topk_logp", torch.empty(*lead, K, dtype=torch.float32, device=dev))
     o.setdefault("topk_idx", torch.empty(*lead, K, dtype=torch.int32, device=dev))
     o.setdefault("lse", torch.empty(*lead, dtype=torch.float32, device=dev))
+    nbytes = sv_extract_topk_workspace_size(rows, V, K)
+    w = ws if ws is not None else workspace(dev, rows, nbytes)
     rc = lib().sv_extract_topk_kd(_p(logits), _dtype_code(logits), rows, V, K, float(temperature),
-                                  _p(o["topk_logp"]), _p(o["topk_idx"]), _p(o["lse"]),
-                                  _p(device_status), _stream(dev, stream))
+                                  _p(o["topk_logp"]), _p(o["topk_idx"]), _p(o["lse"]), _p(w),
+                                  w.numel(), _p(device_status), _stream(dev, stream))
     _check(rc, "sv_extract_topk_kd")
     return o
 
@@ -269,7 +278,7 @@ def sv_kd_kl_loss(topk_logp: torch.Tensor, topk_idx: torch.Tensor, draft: torch.
     o.setdefault("kl", torch.empty(B, k, dtype=torch.float32, device=dev))
     o.setdefault("loss", torch.empty(B, dtype=torch.float32, device=dev))
     o.setdefault("total", torch.empty(1, dtype=torch.float32, device=dev))
-    nbytes = sv_kd_kl_loss_workspace_size(B, k)
+    nbytes = sv_kd_kl_loss_workspace_size(B, k, V)
     w = ws if ws is not None else workspace(dev, B, nbytes)
     wm = SV_W_GROUP_NORM if wmode == "group_norm" else SV_W_RAW
     rc = lib().sv_kd_kl_loss(_p(topk_logp), _p(topk_idx), B, k, K, _p(draft), _dtype_code(draft),

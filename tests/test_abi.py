@@ -56,11 +56,16 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_sizes(lib):
-    assert sv.sv_verify_chain_workspace_size(0, 3) == 256
-    a = sv.sv_verify_chain_workspace_size(32, 3)
-    assert a % 256 == 0 and a >= 16 + 8 * 32 + 2 * 4 * 32 * 4
-    assert sv.sv_verify_tree_workspace_size(8, 32) >= 16 + 8 * 8 + 2 * 4 * 8 * 32
-    assert sv.sv_kd_kl_loss_workspace_size(256, 3) >= 16 + 8 * 256
+    assert sv.sv_verify_chain_workspace_size(0, 3, 1024) == 256
+    V = 151936
+    a = sv.sv_verify_chain_workspace_size(32, 3, V)
+    nchunk = -(-V // 8192)
+    # records, partials and counters of 128 rows; KD adds K keys per chunk
+    assert a % 256 == 0 and a >= 128 * (48 + 48 * nchunk + 4) + 4 * 32
+    assert sv.sv_verify_chain_workspace_size(32, 3, V, 32) >= a + 128 * nchunk * 32 * 8
+    assert sv.sv_verify_tree_workspace_size(8, 32, V) >= 256 * 48 * nchunk
+    assert sv.sv_extract_topk_workspace_size(10, 1000, 32) >= 10 * (48 + 48 + 32 * 8)
+    assert sv.sv_kd_kl_loss_workspace_size(256, 3, V) >= 768 * 48 * nchunk
 
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation
@@ -108,7 +113,7 @@ def test_chain_validation_rejects_before_any_cuda_call(lib):
     assert _chain(lib, ws=None) == sv.SV_ERR_WORKSPACE
     assert _chain(lib, wsb=16) == sv.SV_ERR_WORKSPACE
     assert _chain(lib, ws=ctypes.c_void_p(0x10004)) == sv.SV_ERR_WORKSPACE
-    assert _chain(lib, V=600000) == sv.SV_ERR_UNSUPPORTED
+    assert _chain(lib, V=600000, wsb=1 << 40) == sv.SV_ERR_UNSUPPORTED
     # empty batch: nothing to do, nothing enqueued
     assert _chain(lib, B=0, ws=None) == sv.SV_OK
     # greedy: draft and uniforms may be NULL (fails only on the workspace here)
@@ -127,10 +132,13 @@ def test_other_entry_points_validate(lib):
     assert lib.sv_verify_tree_greedy(f, 1, f, f, 2, 4, 100, 4, f, f, f, f, 1 << 20, None,
                                      None) == E
     # top-K: K > 32, K > V, T == 0
-    assert lib.sv_extract_topk_kd(f, 1, 4, 1000, 33, 1.0, f, f, f, None, None) == E
-    assert lib.sv_extract_topk_kd(f, 1, 4, 10, 16, 1.0, f, f, f, None, None) == E
-    assert lib.sv_extract_topk_kd(f, 1, 4, 1000, 32, 0.0, f, f, f, None, None) == E
-    assert lib.sv_extract_topk_kd(f, 1, 0, 1000, 32, 1.0, f, f, f, None, None) == sv.SV_OK
+    assert lib.sv_extract_topk_kd(f, 1, 4, 1000, 33, 1.0, f, f, f, f, 1 << 20, None, None) == E
+    assert lib.sv_extract_topk_kd(f, 1, 4, 10, 16, 1.0, f, f, f, f, 1 << 20, None, None) == E
+    assert lib.sv_extract_topk_kd(f, 1, 4, 1000, 32, 0.0, f, f, f, f, 1 << 20, None, None) == E
+    assert lib.sv_extract_topk_kd(f, 1, 0, 1000, 32, 1.0, f, f, f, f, 1 << 20, None,
+                                  None) == sv.SV_OK
+    assert lib.sv_extract_topk_kd(f, 1, 4, 1000, 32, 1.0, f, f, f, f, 16, None,
+                                  None) == sv.SV_ERR_WORKSPACE
     # KL loss: probs must be fp32, group must divide B
     assert lib.sv_kd_kl_loss(f, f, 4, 3, 32, f, sv.SV_BF16, sv.SV_DRAFT_PROBS, 1000, 1.0, f, f,
                              0, 1, 0.0, f, f, f, f, 1 << 20, None, None) == E
