@@ -152,12 +152,17 @@ static cudaError_t sm_count(int* out) {
   return cudaSuccess;
 }
 
-// Chunk length of the stream (a multiple of the piece): at most 8 pieces.
-static int stream_chunk(int V) {
+// Chunk length of the stream (a multiple of the piece, at most 8 pieces):
+// long enough to amortise the per-chunk record, short enough that a batch
+// gives every warp of the device a few chunks (about 8192 in all).  It
+// depends on the sizes only, so workspace sizes are device independent.
+static int stream_chunk(int V, long long nrows) {
   const int forced = env_int("SV_STREAM_W");
   if (forced >= kPiece && forced % kPiece == 0) return forced;
-  const int w = (int)align_up((size_t)V, kPiece);
-  return w < 8 * kPiece ? w : 8 * kPiece;
+  int w = kPiece;
+  while (w < 8 * kPiece && (long long)V * nrows / (2 * w) >= 8192) w *= 2;
+  const int cap = (int)align_up((size_t)V, kPiece);
+  return w < cap ? w : cap;
 }
 
 // Workspace: batch counter, per-request rejection words, per-row chunk
@@ -207,9 +212,9 @@ struct StreamGeom {
   int W, nchunk, stage_bytes, stage_off1, smem;
 };
 
-static StreamGeom stream_geom(int V, int te, int de) {
+static StreamGeom stream_geom(int V, long long nrows, int te, int de) {
   StreamGeom g;
-  g.W = stream_chunk(V);
+  g.W = stream_chunk(V, nrows);
   g.nchunk = (V + g.W - 1) / g.W;
   g.stage_off1 = (int)align_up((size_t)kPiece * te, 128);
   g.stage_bytes = g.stage_off1 + (int)align_up((size_t)kPiece * de, 128);
@@ -288,22 +293,22 @@ extern "C" {
 
 size_t sv_verify_chain_workspace_size(int B, int k, int V, int K) {
   if (B <= 0 || k < 1 || V < 1) return 256;
-  const int W = stream_chunk(V);
+  const int W = stream_chunk(V, (long long)B * (k + 1));
   return ws_layout(B, B * (k + 1), (V + W - 1) / W, K > 0 ? K : 0).bytes;
 }
 size_t sv_verify_tree_workspace_size(int B, int n, int V) {
   if (B <= 0 || n < 1 || V < 1) return 256;
-  const int W = stream_chunk(V);
+  const int W = stream_chunk(V, (long long)B * n);
   return ws_layout(B, B * n, (V + W - 1) / W, 0).bytes;
 }
 size_t sv_extract_topk_workspace_size(int rows, int V, int K) {
   if (rows <= 0 || V < 1) return 256;
-  const int W = stream_chunk(V);
+  const int W = stream_chunk(V, rows);
   return ws_layout(rows, rows, (V + W - 1) / W, K > 0 ? K : 0).bytes;
 }
 size_t sv_kd_kl_loss_workspace_size(int B, int k, int V) {
   if (B <= 0 || k < 1 || V < 1) return 256;
-  const int W = stream_chunk(V);
+  const int W = stream_chunk(V, (long long)B * k);
   return ws_layout(B, B * k, (V + W - 1) / W, 0).bytes;
 }
 
@@ -353,7 +358,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   const int K = kd ? kd->K : 0;
   const int te = esize(t_dtype);
   const int de = greedy ? 0 : (d_kind == SV_DRAFT_PROBS ? 4 : esize(d_dtype));
-  const StreamGeom sg = stream_geom(V, te, de);
+  const StreamGeom sg = stream_geom(V, (long long)B * P, te, de);
   const WsLayout wl = ws_layout(B, B * P, sg.nchunk, K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
@@ -467,7 +472,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
     return SV_ERR_INVALID_ARG;
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if ((long long)B * n > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
-  const StreamGeom sg = stream_geom(V, esize(dt), 0);
+  const StreamGeom sg = stream_geom(V, (long long)B * n, esize(dt), 0);
   const WsLayout wl = ws_layout(B, B * n, sg.nchunk, 0);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
@@ -527,7 +532,7 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
     return SV_ERR_INVALID_ARG;
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if (rows > 0x7fffffff / 64) return SV_ERR_UNSUPPORTED;
-  const StreamGeom sg = stream_geom(V, esize(dt), 0);
+  const StreamGeom sg = stream_geom(V, rows, esize(dt), 0);
   const WsLayout wl = ws_layout(rows, rows, sg.nchunk, K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
@@ -597,7 +602,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
     return SV_ERR_INVALID_ARG;
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if ((long long)B * k > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
-  const StreamGeom sg = stream_geom(V, esize(d_dtype), 0);
+  const StreamGeom sg = stream_geom(V, (long long)B * k, esize(d_dtype), 0);
   const WsLayout wl = ws_layout(B, B * k, sg.nchunk, 0);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;

@@ -101,6 +101,29 @@ __device__ __forceinline__ float load8_max<F32>(const unsigned char* buf, int e,
                fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
 }
 
+// Maximum of eight elements without widening them all.
+template <class T>
+__device__ __forceinline__ float max8(const unsigned char* buf, int e);
+
+template <>
+__device__ __forceinline__ float max8<BF16>(const unsigned char* buf, int e) {
+  uint4 w = *reinterpret_cast<const uint4*>(buf + (size_t)e * 2);
+  __nv_bfloat162 a = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.x),
+                             *reinterpret_cast<__nv_bfloat162*>(&w.y));
+  __nv_bfloat162 c = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&w.z),
+                             *reinterpret_cast<__nv_bfloat162*>(&w.w));
+  a = __hmax2(a, c);
+  const uint32_t m = *reinterpret_cast<uint32_t*>(&a);
+  return fmaxf(bf16_lo(m), bf16_hi(m));
+}
+
+template <>
+__device__ __forceinline__ float max8<F32>(const unsigned char* buf, int e) {
+  const float4 a = *reinterpret_cast<const float4*>(buf + (size_t)e * 4);
+  const float4 b = *reinterpret_cast<const float4*>(buf + (size_t)e * 4 + 16);
+  return fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(b.x, b.y), fmaxf(b.z, b.w)));
+}
+
 // Value of the element that fills the padding of a partial last vector:
 // -inf for logits (no mass, never a maximum), 0 for probabilities.
 template <class T>
@@ -156,6 +179,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
       "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Same, default L2 policy (data that a later pass may read again).
+__device__ __forceinline__ void bulk_g2s_plain(void* dst, const void* src, uint32_t bytes,
+                                               uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -365,6 +398,34 @@ __device__ __forceinline__ void stat_update(ThreadStat& s, const float v[8], flo
     for (int t = 0; t < 8; ++t) e[t] = ex2(fmaf(v[t], c, -s.ref));
     s.S += (double)(((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7])));
   }
+}
+
+// Move a thread's reference to cover a new maximum pm (before its terms).
+__device__ __forceinline__ void stat_cover(ThreadStat& s, float pm, float c) {
+  s.mz = fmaxf(s.mz, pm);
+  const float top = pm * c;
+  if (top > s.ref) {
+    const float nref = ceilf(top);
+    s.S = rescale_pow2(s.S, s.ref, nref);
+    s.ref = nref;
+  }
+}
+
+// Sum of the exp2 terms of NV vectors of 8 (relative to the current
+// reference), by a fixed fp32 tree.
+template <int NV>
+__device__ __forceinline__ float stat_terms(const ThreadStat& s, const float (&x)[NV][8],
+                                            float c) {
+  float e[NV * 8];
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) e[v * 8 + t] = ex2(fmaf(x[v][t], c, -s.ref));
+#pragma unroll
+  for (int w = NV * 8 / 2; w >= 1; w >>= 1)
+#pragma unroll
+    for (int t = 0; t < w; ++t) e[t] = e[t] + e[t + w];
+  return e[0];
 }
 
 // CTA partial: exponent reference G (max over threads of ref) and

@@ -91,20 +91,27 @@ __device__ __forceinline__ float seq_sum8(const float w[8]) {
   return s;
 }
 
-// First rejection of request b from its row records: n, and whether every
-// row that decides the outcome (0..n) was verified.
-__device__ __forceinline__ int first_rejection(const RowRec* rec, int B, int k, int b,
-                                               bool* bad) {
+// First rejection of request b from its row records (one warp, all lanes
+// return the same): n, and whether every row that decides the outcome
+// (0..n) was verified.
+__device__ __forceinline__ int warp_first_rejection(const RowRec* rec, int B, int k, int b,
+                                                    bool* bad) {
+  const int lane = threadIdx.x & 31;
   int n = k;
-  for (int t = 0; t < k; ++t)
-    if (__ldcg(&rec[(size_t)t * B + b].code) == kRowRejected) {
-      n = t;
+  for (int base = 0; base < k; base += 32) {
+    const int t = base + lane;
+    const int code = t < k ? __ldcg(&rec[(size_t)t * B + b].code) : 0;
+    const unsigned m = __ballot_sync(0xffffffffu, t < k && code == kRowRejected);
+    if (m) {
+      n = base + __ffs(m) - 1;
       break;
     }
+  }
   bool bd = false;
-  for (int t = 0; t <= n; ++t) {
-    const int cd = __ldcg(&rec[(size_t)t * B + b].code);
-    bd |= (cd != kRowAccepted && cd != kRowRejected);
+  for (int base = 0; base <= n; base += 32) {
+    const int t = base + lane;
+    const int code = t <= n ? __ldcg(&rec[(size_t)t * B + b].code) : kRowAccepted;
+    bd |= __any_sync(0xffffffffu, code != kRowAccepted && code != kRowRejected);
   }
   *bad = bd;
   return n;
@@ -175,20 +182,22 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const FinishPara
   const float c = prm.c;
   const bool use_bulk = prm.use_bulk != 0;
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     bool bad;
-    const int n = first_rejection(prm.rec, B, k, b, &bad);
-    sh.fin_n = bad ? -1 : n;
-    sh.need = bad ? 0 : 1;
-    sh.err = 0;
-    // cleared before the draw's first cluster barrier; the owning CTA writes it after
-    if (rank == 0 && !bad) prm.out_tokens[(size_t)b * P + n] = -1;
-    const RowRec* rn = &prm.rec[(size_t)n * B + b];
-    sh.Gt = __ldcg(&rn->G0);
-    sh.St = __ldcg(&rn->S0);
-    sh.Gd = __ldcg(&rn->G1);
-    sh.Sd = __ldcg(&rn->S1);
-    sh.tok = -1;
+    const int n = warp_first_rejection(prm.rec, B, k, b, &bad);
+    if (threadIdx.x == 0) {
+      sh.fin_n = bad ? -1 : n;
+      sh.need = bad ? 0 : 1;
+      sh.err = 0;
+      // cleared before the draw's first cluster barrier; the owning CTA writes it after
+      if (rank == 0 && !bad) prm.out_tokens[(size_t)b * P + n] = -1;
+      const RowRec* rn = &prm.rec[(size_t)n * B + b];
+      sh.Gt = __ldcg(&rn->G0);
+      sh.St = __ldcg(&rn->S0);
+      sh.Gd = __ldcg(&rn->G1);
+      sh.Sd = __ldcg(&rn->S1);
+      sh.tok = -1;
+    }
   }
   __syncthreads();
   const int n = sh.fin_n;
@@ -412,16 +421,10 @@ __global__ void __launch_bounds__(kThreads) chain_greedy_finish(const FinishPara
   const int b = (int)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (b >= prm.B) return;
   const int k = prm.k, P = k + 1, B = prm.B;
-  int n = 0, tok = -1;
   bool bad = false;
-  if (lane == 0) {
-    n = first_rejection(prm.rec, B, k, b, &bad);
-    tok = __ldcg(&prm.rec[(size_t)n * B + b].argmax);
-    if (tok < 0 || tok >= prm.V) bad = true;
-  }
-  n = __shfl_sync(0xffffffffu, n, 0);
-  tok = __shfl_sync(0xffffffffu, tok, 0);
-  bad = __shfl_sync(0xffffffffu, bad ? 1 : 0, 0) != 0;
+  const int n = warp_first_rejection(prm.rec, B, k, b, &bad);
+  const int tok = __ldcg(&prm.rec[(size_t)n * B + b].argmax);
+  if (tok < 0 || tok >= prm.V) bad = true;
   for (int t = lane; t < P; t += 32) {
     int v = -1;
     if (!bad) v = (t < n) ? prm.tokens[(size_t)b * k + t] : (t == n ? tok : -1);

@@ -29,7 +29,7 @@ namespace sv {
 
 constexpr int kPiece = 1024;                  // elements per piece
 constexpr int kLaneVecs = kPiece / (32 * kVec);  // 8-element vectors per lane per piece
-constexpr int kStages = 3;                    // ring depth per warp
+constexpr int kStages = 2;                    // ring depth per warp
 constexpr int kStreamWarps = 8;
 constexpr int kStreamThreads = kStreamWarps * 32;
 
@@ -229,7 +229,7 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, const 
 }
 
 template <class T0, class T1, int FLAGS>
-__global__ void __launch_bounds__(kStreamThreads) stream_kernel(const StreamParams prm) {
+__global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* ring = smem + (size_t)warp * kStages * prm.stage_bytes;
@@ -243,12 +243,10 @@ __global__ void __launch_bounds__(kStreamThreads) stream_kernel(const StreamPara
   const float c = prm.c;
   const int K = prm.K;
   const unsigned kmask = K >= 32 ? 0xffffffffu : ((1u << K) - 1u);
-  uint64_t policy = 0;
   if (lane == 0) {
     if (use_bulk) {
       for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
       fence_mbar_init();
-      policy = policy_evict_first();
     }
   }
   __syncwarp();
@@ -280,12 +278,12 @@ __global__ void __launch_bounds__(kStreamThreads) stream_kernel(const StreamPara
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&bars[s], nb0 + nb1);
     if (nb0)
-      bulk_g2s(st, reinterpret_cast<const unsigned char*>(L.row0) + (size_t)e0 * T0::bytes, nb0,
-               &bars[s], policy);
+      bulk_g2s_plain(st, reinterpret_cast<const unsigned char*>(L.row0) + (size_t)e0 * T0::bytes,
+                     nb0, &bars[s]);
     if (nb1)
-      bulk_g2s(st + prm.stage_off1,
-               reinterpret_cast<const unsigned char*>(L.row1) + (size_t)e0 * T1::bytes, nb1,
-               &bars[s], policy);
+      bulk_g2s_plain(st + prm.stage_off1,
+                     reinterpret_cast<const unsigned char*>(L.row1) + (size_t)e0 * T1::bytes, nb1,
+                     &bars[s]);
   };
 
   uint32_t n_issued = 0, n_consumed = 0;
@@ -347,15 +345,16 @@ __global__ void __launch_bounds__(kStreamThreads) stream_kernel(const StreamPara
       if (use_bulk) {
         if (!mbar_wait_bounded(&bars[s], ph)) ++timeouts;
       }
+      const bool has1 = (FLAGS & kFRow1) && L.row1 != nullptr;
       // Elements the bulk copy does not cover (the unaligned tail, or the whole
       // piece on the scalar path) and padding of the last vector.
-      {
+      if (!use_bulk || n < kPiece) {
         const int a0 = use_bulk ? (int)(((uint32_t)(n * T0::bytes) & ~15u) / T0::bytes) : 0;
         const typename T0::storage* src = reinterpret_cast<const typename T0::storage*>(L.row0) + e0;
         for (int e = a0 + lane; e < n; e += 32)
           reinterpret_cast<typename T0::storage*>(st)[e] = src[e];
         for (int e = n + lane; e < ((n + kVec - 1) / kVec) * kVec; e += 32) store_pad<T0>(st, e, false);
-        if (L.row1 != nullptr) {
+        if (has1) {
           const int a1 = use_bulk ? (int)(((uint32_t)(n * T1::bytes) & ~15u) / T1::bytes) : 0;
           const typename T1::storage* src1 =
               reinterpret_cast<const typename T1::storage*>(L.row1) + e0;
@@ -364,62 +363,116 @@ __global__ void __launch_bounds__(kStreamThreads) stream_kernel(const StreamPara
           for (int e = n + lane; e < ((n + kVec - 1) / kVec) * kVec; e += 32)
             store_pad<T1>(st1p, e, !(FLAGS & kFStats1));
         }
+        __syncwarp();
       }
-      __syncwarp();
       const int nv = (n + kVec - 1) / kVec;
+      // The draft token's values, read once per piece by lane 0.
+      if ((FLAGS & kFGather) && L.x >= e0 && L.x < e0 + n) {
+        hx = 1;
+        zx0 = load1<T0>(st, L.x - e0);
+        if (has1) zx1 = load1<T1>(st1p, L.x - e0);
+      }
+      // Row 0: this lane's kLaneVecs vectors (element (v*32 + lane)*8 + t).
+      // First the maxima (packed, straight from shared memory) and one
+      // reference update per piece, then the exp2 terms two vectors at a time.
+      {
+        float vm[kLaneVecs];
+        float pm = -INFINITY;
 #pragma unroll
-      for (int v = 0; v < kLaneVecs; ++v) {
-        const int vi = v * 32 + lane;
-        const bool act = vi < nv;
-        const int e = vi * kVec;
-        float x0[8];
+        for (int v = 0; v < kLaneVecs; ++v) {
+          const int vi = v * 32 + lane;
+          vm[v] = vi < nv ? max8<T0>(st, vi * kVec) : -INFINITY;
+          pm = fmaxf(pm, vm[v]);
+        }
+        if (FLAGS & kFStats0) {
+          stat_cover(st0, pm, c);
+          if (pm != -INFINITY) {
+            float acc = 0.f;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) x0[t] = -INFINITY;
-        float m0 = -INFINITY;
-        if (act) {
-          m0 = load8_max<T0>(st, e, x0);
-          if (FLAGS & kFStats0) stat_update(st0, x0, m0, c);
-          if (FLAGS & kFArgmax0) {
-            if (m0 > best || bidx < 0) {
-              int q = 0;
+            for (int v = 0; v < kLaneVecs; v += 2) {
+              float x[2][8];
 #pragma unroll
-              for (int t = 7; t >= 0; --t)
-                if (x0[t] == m0) q = t;
-              best = m0;
-              bidx = e0 + e + q;
+              for (int h = 0; h < 2; ++h) {
+                const int vi = (v + h) * 32 + lane;
+                if (vi < nv) load8<T0>(st, vi * kVec, x[h]);
+                else
+#pragma unroll
+                  for (int t = 0; t < 8; ++t) x[h][t] = -INFINITY;
+              }
+              acc += stat_terms<2>(st0, x, c);
             }
+            st0.S += (double)acc;
           }
-          if ((FLAGS & kFRow1) && L.row1 != nullptr && (FLAGS & kFStats1)) {
-            float x1[8];
-            const float m1 = load8_max<T1>(st1p, e, x1);
-            stat_update(st1, x1, m1, c);
-          }
-          if ((FLAGS & kFGather) && L.x >= e0 + e && L.x < e0 + e + kVec && L.x < e0 + n) {
-            hx = 1;
-            zx0 = load1<T0>(st, L.x - e0);
-            if ((FLAGS & kFRow1) && L.row1 != nullptr) zx1 = load1<T1>(st1p, L.x - e0);
+        }
+        if (FLAGS & kFArgmax0) {
+          if (pm > best || (bidx < 0 && nv > lane)) {
+            int bi = -1;
+#pragma unroll
+            for (int v = kLaneVecs - 1; v >= 0; --v) {
+              const int vi = v * 32 + lane;
+              if (vi < nv && vm[v] == pm) {
+                float x[8];
+                load8<T0>(st, vi * kVec, x);
+#pragma unroll
+                for (int t = 7; t >= 0; --t)
+                  if (x[t] == pm) bi = vi * kVec + t;
+              }
+            }
+            best = pm;
+            bidx = e0 + bi;
           }
         }
         if (FLAGS & kFTopk0) {
-          unsigned m = __ballot_sync(0xffffffffu, act && m0 >= thr_val);
-          while (m) {
-            const int src = __ffs(m) - 1;
-            m &= m - 1;
-            const int sbase = e0 + (v * 32 + src) * kVec;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float val = __shfl_sync(0xffffffffu, x0[q], src);
-              const int idx = sbase + q;
-              if (idx < e0 + n) {
-                const unsigned long long key = topk_key(val, idx);
-                if (key > thr_key) {
-                  warp_list_insert(list, key, kmask);
-                  thr_key = __shfl_sync(0xffffffffu, list, K - 1);
+          for (int v = 0; v < kLaneVecs; ++v) {
+            const int vi = v * 32 + lane;
+            unsigned m = __ballot_sync(0xffffffffu, vi < nv && vm[v] >= thr_val);
+            while (m) {
+              const int src = __ffs(m) - 1;
+              m &= m - 1;
+              const int sbase = (v * 32 + src) * kVec;
+              float xs[8];
+              load8<T0>(st, sbase, xs);  // every lane reads the source lane's vector
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const int idx = e0 + sbase + q;
+                if (sbase + q < n) {
+                  const unsigned long long key = topk_key(xs[q], idx);
+                  if (key > thr_key) {
+                    warp_list_insert(list, key, kmask);
+                    thr_key = __shfl_sync(0xffffffffu, list, K - 1);
+                  }
                 }
               }
             }
+            thr_val = thr_key == kNoKey ? -INFINITY : key_value(thr_key);
           }
-          thr_val = thr_key == kNoKey ? -INFINITY : key_value(thr_key);
+        }
+      }
+      if ((FLAGS & kFStats1) && has1) {
+        float pm = -INFINITY;
+#pragma unroll
+        for (int v = 0; v < kLaneVecs; ++v) {
+          const int vi = v * 32 + lane;
+          if (vi < nv) pm = fmaxf(pm, max8<T1>(st1p, vi * kVec));
+        }
+        stat_cover(st1, pm, c);
+        if (pm != -INFINITY) {
+          float acc = 0.f;
+#pragma unroll
+          for (int v = 0; v < kLaneVecs; v += 2) {
+            float x[2][8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int vi = (v + h) * 32 + lane;
+              if (vi < nv) load8<T1>(st1p, vi * kVec, x[h]);
+              else
+#pragma unroll
+                for (int t = 0; t < 8; ++t) x[h][t] = -INFINITY;
+            }
+            acc += stat_terms<2>(st1, x, c);
+          }
+          st1.S += (double)acc;
         }
       }
       __syncwarp();
