@@ -14,7 +14,6 @@ namespace sv {
 namespace {
 
 constexpr int kMaxV = kMaxChunk * kMaxCluster;  // 524288: finishing plan limit
-constexpr int kTargetSmem = 48 * 1024;          // preferred per-CTA footprint (finishing)
 constexpr int kMaxSmem = 200 * 1024;            // hard per-CTA limit used by plans
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -30,14 +29,13 @@ int forced_cluster() {
   return (c == 1 || c == 2 || c == 4 || c == 8 || c == 16) ? c : 0;
 }
 
-// Finishing plan: the smallest power-of-two cluster whose chunk fits the
-// preferred shared-memory footprint (or the largest that fits at all).
+// Finishing plans: every power-of-two cluster size C whose chunk of
+// ceil(V / C) elements fits the shared-memory limit, C ascending.
 template <class XB>
-sv_status make_plan(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* plan) {
-  if (V < 1 || V > kMaxV) return SV_ERR_UNSUPPORTED;
+int feasible_plans(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* plans) {
+  if (V < 1 || V > kMaxV) return 0;
   const int forced = forced_cluster();
-  RowPlan best = {};
-  bool have = false;
+  int n = 0;
   for (int C = 1; C <= kMaxCluster; C *= 2) {
     if (forced && C != forced) continue;
     const int L = (int)align_up((size_t)((V + C - 1) / C), kVec);
@@ -49,13 +47,9 @@ sv_status make_plan(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* pl
     lay.off_x = lay.off_d + (int)align_up((size_t)L * db, 128);
     lay.bytes = lay.off_x + (int)align_up((size_t)x_bytes(L, np), 128);
     if (lay.bytes > kMaxSmem) continue;
-    best = RowPlan{C, L, np, bulk_ok ? 1 : 0, lay};
-    have = true;
-    if (lay.bytes <= kTargetSmem) break;
+    plans[n++] = RowPlan{C, L, np, bulk_ok ? 1 : 0, lay};
   }
-  if (!have) return SV_ERR_UNSUPPORTED;
-  *plan = best;
-  return SV_OK;
+  return n;
 }
 
 bool bulk_ok_row(const void* base, int V, int es) {
@@ -273,16 +267,80 @@ static cudaError_t launch_blocks(K kernel, const Prm& prm, int blocks, int smem,
   return cudaGetLastError();
 }
 
-template <class TT, class DT, int DKIND>
-static cudaError_t run_chain_sample(const StreamParams& sp, const StreamGeom& sg,
-                                    const FinishParams& fp, const RowPlan& plan, bool kd,
-                                    cudaStream_t s) {
-  constexpr int base = kFStats0 | kFRow1 | kFGather | (DKIND == kDraftLogits ? kFStats1 : 0);
-  cudaError_t e = kd ? launch_stream<TT, DT, base | kFTopk0>(sp, sg, s)
-                     : launch_stream<TT, DT, base>(sp, sg, s);
+// Clusters of plan.C CTAs of this kernel that the device holds at once.
+template <class K>
+static cudaError_t cluster_capacity(K kernel, const RowPlan& plan, int* out) {
+  const void* kp = reinterpret_cast<const void*>(kernel);
+  cudaError_t e = ensure_kernel_attrs(kp, plan.lay.bytes, plan.C > 8);
   if (e != cudaSuccess) return e;
-  return kd ? launch_clusters(chain_sample_finish<TT, DT, DKIND, true>, fp, plan, fp.B, s)
-            : launch_clusters(chain_sample_finish<TT, DT, DKIND, false>, fp, plan, fp.B, s);
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_occ_n; ++i)
+      if (g_occ[i].kernel == kp && g_occ[i].device == dev && g_occ[i].smem == plan.lay.bytes &&
+          g_occ[i].extra == -plan.C) {
+        *out = g_occ[i].value;
+        return cudaSuccess;
+      }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)plan.C, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)plan.lay.bytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)plan.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if ((e = cudaOccupancyMaxActiveClusters(&n, kp, &cfg)) != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_occ_n < kSlots) g_occ[g_occ_n++] = AttrEntry{kp, dev, plan.lay.bytes, -plan.C, n};
+  *out = n;
+  return cudaSuccess;
+}
+
+// Cluster size for `nclusters` requests: the plan minimising
+// waves * (chunk + a fixed latency worth of elements), where waves is the
+// number of rounds of co-resident clusters the grid needs.  A smaller
+// cluster (longer chunk) wins when it keeps the grid in one wave.
+template <class K>
+static cudaError_t pick_plan(K kernel, const RowPlan* plans, int np, int nclusters,
+                             RowPlan* out) {
+  constexpr long long kLatencyElems = 8192;
+  long long best = -1;
+  for (int i = 0; i < np; ++i) {
+    int cap = 0;
+    cudaError_t e = cluster_capacity(kernel, plans[i], &cap);
+    if (e != cudaSuccess) return e;
+    if (cap < 1) continue;
+    const long long waves = (nclusters + cap - 1) / cap;
+    const long long cost = waves * (plans[i].L + kLatencyElems);
+    if (best < 0 || cost < best) {
+      best = cost;
+      *out = plans[i];
+    }
+  }
+  return best < 0 ? cudaErrorInvalidConfiguration : cudaSuccess;
+}
+
+template <class TT, class DT, int DKIND>
+static cudaError_t run_chain_sample(const StreamParams& sp, const StreamGeom& sg, FinishParams fp,
+                                    const RowPlan* plans, int np, bool kd, cudaStream_t s) {
+  constexpr int base = kFStats0 | kFRow1 | kFGather | (DKIND == kDraftLogits ? kFStats1 : 0);
+  auto fin = kd ? chain_sample_finish<TT, DT, DKIND, true> : chain_sample_finish<TT, DT, DKIND, false>;
+  RowPlan plan;
+  cudaError_t e = pick_plan(fin, plans, np, fp.B, &plan);
+  if (e != cudaSuccess) return e;
+  fp.L = plan.L;
+  fp.use_bulk = plan.use_bulk;
+  fp.lay = plan.lay;
+  e = kd ? launch_stream<TT, DT, base | kFTopk0>(sp, sg, s) : launch_stream<TT, DT, base>(sp, sg, s);
+  if (e != cudaSuccess) return e;
+  return launch_clusters(fin, fp, plan, fp.B, s);
 }
 
 }  // namespace sv
@@ -419,6 +477,10 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
     fp.clip = kd->clip;
     fp.loss = kd->loss;
     fp.total = kd->total;
+    sp.topk_logp = kd->topk_logp;
+    sp.topk_idx = kd->topk_idx;
+    sp.lse = kd->lse;
+    sp.kl = kd->kl;
   }
 
   if (greedy) {
@@ -428,31 +490,27 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
     return cuda_status(launch_blocks(chain_greedy_finish, fp, (B + kWarps - 1) / kWarps, 0, s));
   }
 
-  const int nchunk = sg.nchunk;
-  RowPlan plan;
-  st = make_plan(
+  RowPlan plans[8];
+  const int np = feasible_plans(
       V, te, de,
-      [K, nchunk](int, int np) {
-        int x = np * kThreads * 4 + kThreads * 8;
-        if (x < 2 * kThreads * 4) x = 2 * kThreads * 4;
-        const int xk = K > 0 ? kWarps * (nchunk * K + 32) * 8 : 0;
-        return x > xk ? x : xk;
+      [](int, int npc) {
+        const int x = npc * kThreads * 4 + kThreads * 8;
+        return x < 2 * kThreads * 4 ? 2 * kThreads * 4 : x;
       },
-      bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de), &plan);
-  if (st != SV_OK) return st;
-  fp.L = plan.L;
-  fp.use_bulk = plan.use_bulk;
-  fp.lay = plan.lay;
+      bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de), plans);
+  if (np == 0) return SV_ERR_UNSUPPORTED;
   cudaError_t e;
   if (d_kind == SV_DRAFT_PROBS)
-    e = t_dtype == SV_BF16 ? run_chain_sample<BF16, F32, kDraftProbs>(sp, sg, fp, plan, kd, s)
-                           : run_chain_sample<F32, F32, kDraftProbs>(sp, sg, fp, plan, kd, s);
+    e = t_dtype == SV_BF16 ? run_chain_sample<BF16, F32, kDraftProbs>(sp, sg, fp, plans, np, kd, s)
+                           : run_chain_sample<F32, F32, kDraftProbs>(sp, sg, fp, plans, np, kd, s);
   else if (t_dtype == SV_BF16)
-    e = d_dtype == SV_BF16 ? run_chain_sample<BF16, BF16, kDraftLogits>(sp, sg, fp, plan, kd, s)
-                           : run_chain_sample<BF16, F32, kDraftLogits>(sp, sg, fp, plan, kd, s);
+    e = d_dtype == SV_BF16
+            ? run_chain_sample<BF16, BF16, kDraftLogits>(sp, sg, fp, plans, np, kd, s)
+            : run_chain_sample<BF16, F32, kDraftLogits>(sp, sg, fp, plans, np, kd, s);
   else
-    e = d_dtype == SV_BF16 ? run_chain_sample<F32, BF16, kDraftLogits>(sp, sg, fp, plan, kd, s)
-                           : run_chain_sample<F32, F32, kDraftLogits>(sp, sg, fp, plan, kd, s);
+    e = d_dtype == SV_BF16
+            ? run_chain_sample<F32, BF16, kDraftLogits>(sp, sg, fp, plans, np, kd, s)
+            : run_chain_sample<F32, F32, kDraftLogits>(sp, sg, fp, plans, np, kd, s);
   return cuda_status(e);
 }
 
@@ -558,24 +616,12 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
   sp.status = device_status;
-  cudaError_t e = dt == SV_BF16 ? launch_stream<BF16, BF16, kFStats0 | kFTopk0>(sp, sg, s)
-                                : launch_stream<F32, F32, kFStats0 | kFTopk0>(sp, sg, s);
-  if (e != cudaSuccess) return SV_ERR_CUDA;
-  FinishParams fp = {};
-  fp.B = rows;
-  fp.V = V;
-  fp.nchunk = sg.nchunk;
-  fp.K = K;
-  fp.c = sp.c;
-  fp.topk_logp = topk_logp;
-  fp.topk_idx = topk_idx;
-  fp.lse = lse;
-  fp.part = w.part;
-  fp.cand = w.cand;
-  fp.rec = w.rec;
-  fp.status = device_status;
-  const int smem = kWarps * (sg.nchunk * K + 32) * 8;
-  return cuda_status(launch_blocks(topk_finish, fp, (rows + kWarps - 1) / kWarps, smem, s));
+  sp.topk_logp = topk_logp;
+  sp.topk_idx = topk_idx;
+  sp.lse = lse;
+  // one pass: the warp that completes a row merges its chunk lists and writes it
+  return cuda_status(dt == SV_BF16 ? launch_stream<BF16, BF16, kFStats0 | kFTopk0>(sp, sg, s)
+                                   : launch_stream<F32, F32, kFStats0 | kFTopk0>(sp, sg, s));
 }
 
 sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,

@@ -37,6 +37,7 @@ constexpr int kMaxCluster = 16;
 constexpr int kMaxK = 32;
 constexpr int kCandCap = 1024;              // top-K candidate buffer per CTA
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
+constexpr uint32_t kWaitHintNs = 1000000u;                  // sleep up to 1 ms per try
 
 enum DraftKind { kDraftLogits = 0, kDraftProbs = 1 };
 
@@ -198,14 +199,16 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// try_wait with a suspend-time hint: the waiting warp sleeps in hardware until
+// the phase completes (or the hint expires) instead of spinning.
 __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, P;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
       : "memory");
   return ok;
 }
@@ -537,50 +540,35 @@ __device__ __forceinline__ float key_value(unsigned long long k) {
 }
 constexpr unsigned long long kNoKey = 0ull;  // below every real key (even -inf)
 
-// Bitonic sort of one value per lane, descending (lane 0 largest).
-__device__ __forceinline__ float warp_sort_desc(float v) {
+// Bitonic sort of one key per lane, descending (lane 0 largest).
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long v) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1) {
-      float o = __shfl_xor_sync(0xffffffffu, v, j);
-      bool up = ((lane & k) == 0);        // this half sorts descending
-      bool lower = ((lane & j) == 0);
-      bool take_max = (lower == up);
-      v = take_max ? fmaxf(v, o) : fminf(v, o);
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool take_max = ((lane & j) == 0) == ((lane & k) == 0);
+      v = take_max ? (o > v ? o : v) : (o < v ? o : v);
     }
   }
   return v;
 }
 
-// Merge two descending lists held one value per lane; keeps the 32 largest,
-// descending.
-__device__ __forceinline__ float warp_merge_desc(float a, float b) {
+// Merge two descending lists held one key per lane; keeps the 32 largest,
+// descending (reverse one list, take the lane-wise maxima, which form a
+// bitonic sequence holding the 32 largest, and sort it with a half cleaner).
+__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long a,
+                                                              unsigned long long b) {
   const int lane = threadIdx.x & 31;
-  float br = __shfl_sync(0xffffffffu, b, 31 - lane);
-  float v = fmaxf(a, br);  // bitonic
+  const unsigned long long br = __shfl_sync(0xffffffffu, b, 31 - lane);
+  unsigned long long v = a > br ? a : br;
 #pragma unroll
   for (int j = 16; j > 0; j >>= 1) {
-    float o = __shfl_xor_sync(0xffffffffu, v, j);
-    v = ((lane & j) == 0) ? fmaxf(v, o) : fminf(v, o);
+    const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+    v = ((lane & j) == 0) ? (o > v ? o : v) : (o < v ? o : v);
   }
   return v;
-}
-
-// Exact selection of the K best keys among n keys in shared memory (all keys
-// distinct).  out[r] receives the key of rank r (r < K); ranks >= n get
-// kNoKey.  Collective over the block.
-__device__ __forceinline__ void rank_select(const unsigned long long* keys, int n, int K,
-                                            unsigned long long* out) {
-  for (int r = threadIdx.x; r < K; r += kThreads)
-    if (r >= n) out[r] = kNoKey;
-  for (int c = threadIdx.x; c < n; c += kThreads) {
-    const unsigned long long mine = keys[c];
-    int rank = 0;
-    for (int o = 0; o < n; ++o) rank += (keys[o] > mine);
-    if (rank < K) out[rank] = mine;
-  }
 }
 
 }  // namespace sv

@@ -6,10 +6,11 @@
 // n = k, the bonus row p_k, by inverse CDF in ascending vocabulary order.  The
 // row pair is staged in shared memory (bulk copies), the CTA chunk masses are
 // combined in a fixed order through distributed shared memory and the owning
-// CTA locates the draw.  Fused KD work (top-K merge of the stream's per-chunk
-// lists, lse, KL against the draft row) is spread over the cluster's warps,
-// one row per warp.  Every finisher returns the workspace words it used to
-// zero, so the workspace stays zero between calls.
+// CTA locates the draw.  Fused KD rows were written by the stream; the
+// finisher marks the rows after the emitted position as undefined and forms
+// the reward-weighted losses.  Every finisher returns the row records it read
+// to zero (the stream zeroes the partials), so the workspace stays zero
+// between calls.
 #include "sv_rowops.cuh"
 #include "sv_stream.cuh"
 
@@ -117,53 +118,11 @@ __device__ __forceinline__ int warp_first_rejection(const RowRec* rec, int B, in
   return n;
 }
 
-// One warp: merge the stream's per-chunk top-K lists of one row (nchunk * K
-// keys) into the row's top K, best first.  Keys below the largest per-chunk
-// K-th key cannot be in the row's top K.  `buf` holds nchunk * K keys.
-__device__ inline unsigned long long warp_merge_topk(const unsigned long long* lists, int nchunk,
-                                                     int K, unsigned long long* buf) {
-  const int lane = threadIdx.x & 31;
-  unsigned long long th = kNoKey;
-  for (int q = lane; q < nchunk; q += 32) {
-    const unsigned long long kk = __ldcg(&lists[(size_t)q * K + K - 1]);
-    th = kk > th ? kk : th;
-  }
-  th = warp_max_u64(th);
-  int n = 0;
-  for (int base = 0; base < nchunk * K; base += 32) {
-    const int t = base + lane;
-    unsigned long long kk = kNoKey;
-    if (t < nchunk * K) kk = __ldcg(&lists[t]);
-    const bool keep = kk != kNoKey && kk >= th;
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    if (keep) buf[n + __popc(m & ((1u << lane) - 1u))] = kk;
-    n += __popc(m);
-  }
-  __syncwarp();
-  // rank selection: the key of rank `lane` ends up in lane `lane`
-  unsigned long long mine = kNoKey;
-  for (int t = lane; t < n; t += 32) {
-    const unsigned long long kk = buf[t];
-    int rank = 0;
-    for (int o = 0; o < n; ++o) rank += (buf[o] > kk);
-    if (rank < 32) buf[nchunk * K + rank] = kk;
-  }
-  __syncwarp();
-  if (lane < K && lane < n) mine = buf[nchunk * K + lane];
-  __syncwarp();
-  return mine;
-}
-
-// Zero the stream scratch of rows [r0, r0 + nr) with threads t0, t0 + nt, ...
-__device__ __forceinline__ void zero_rows(const FinishParams& p, size_t r0, int stride_rows,
-                                          int nr, int t0, int nt, bool with_cand) {
-  for (int q = 0; q < nr; ++q) {
-    const size_t r = r0 + (size_t)q * stride_rows;
-    for (int t = t0; t < p.nchunk; t += nt) p.part[r * p.nchunk + t] = Partial{};
-    if (with_cand)
-      for (int t = t0; t < p.nchunk * p.K; t += nt) p.cand[r * p.nchunk * p.K + t] = 0ull;
-    if (t0 == 0) p.rec[r] = RowRec{};
-  }
+// Zero the row records of rows r0, r0 + stride_rows, ... (nr rows) with
+// threads t0, t0 + nt, ...
+__device__ __forceinline__ void zero_recs(const FinishParams& p, size_t r0, int stride_rows,
+                                          int nr, int t0, int nt) {
+  for (int q = t0; q < nr; q += nt) p.rec[r0 + (size_t)q * stride_rows] = RowRec{};
 }
 
 template <class TT, class DT, int DKIND, bool KD>
@@ -325,54 +284,9 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const FinishPara
     }
   }
 
-  // 2. fused KD: rows 0..n, one warp per row across the cluster.
+  // 2. fused KD: the stream wrote rows 0..n; later rows are not verified and
+  // are defined as empty.
   if (KD) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    // merge buffers reuse the sampling scratch: this CTA's draw is complete
-    unsigned long long* buf = reinterpret_cast<unsigned long long*>(smem + prm.lay.off_x) +
-                              (size_t)w * (prm.nchunk * prm.K + 32);
-    const int nrows_kd = n < 0 ? 0 : n + 1;
-    const double ln2 = 0.69314718055994530942;
-    for (int t = rank * kWarps + w; t < nrows_kd; t += C * kWarps) {
-      const size_t r = (size_t)t * B + b;
-      const size_t orow = (size_t)b * P + t;
-      const unsigned long long kk =
-          warp_merge_topk(prm.cand + r * prm.nchunk * prm.K, prm.nchunk, prm.K, buf);
-      const double L0 = __ldcg(&prm.rec[r].L0);
-      double lp = -INFINITY;
-      int j = -1;
-      if (lane < prm.K) {
-        j = key_index(kk);
-        lp = ((double)key_value(kk) * (double)c - L0) * ln2;
-        prm.topk_logp[orow * prm.K + lane] = (float)lp;
-        prm.topk_idx[orow * prm.K + lane] = j;
-      }
-      if (lane == 0) prm.lse[orow] = (float)(L0 * ln2);
-      if (t < k) {
-        double m = lp;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
-        double s = (lane < prm.K) ? exp(lp - m) : 0.0;
-        s = warp_sum(s);
-        const double lse_k = m + log(s);
-        const double L1 = __ldcg(&prm.rec[r].L1);
-        double term = 0.0;
-        if (lane < prm.K && j >= 0 && j < V) {
-          const float zd =
-              (DKIND == kDraftLogits)
-                  ? load1<DT>(reinterpret_cast<const unsigned char*>(
-                                  row_ptr<DT>(prm.draft, (size_t)b * k + t, V)), j)
-                  : reinterpret_cast<const float*>(row_ptr<F32>(prm.draft, (size_t)b * k + t, V))[j];
-          const double log_pt = lp - lse_k;
-          const double pt = exp(log_pt);
-          const double log_q = (DKIND == kDraftLogits) ? ((double)zd * (double)c - L1) * ln2
-                                                       : log((double)zd);
-          term = (pt == 0.0) ? 0.0 : pt * (log_pt - log_q);
-        }
-        term = warp_sum(term);
-        if (lane == 0) prm.kl[(size_t)b * k + t] = (float)term;
-      }
-    }
     // rows after the emitted position: not verified, defined as empty
     if (rank == 0) {
       const int first_undef = n < 0 ? 0 : n + 1;
@@ -390,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const FinishPara
   cluster.sync();  // draw, KD rows and every read of the records are done
 
   // 3. outputs (rank 0) and workspace hygiene (every CTA).
-  zero_rows(prm, (size_t)b, B, P, rank * kThreads + (int)threadIdx.x, C * kThreads, KD);
+  zero_recs(prm, (size_t)b, B, P, rank * kThreads + (int)threadIdx.x, C * kThreads);
   if (rank != 0) return;
   if (threadIdx.x == 0) {
     int nn = n;
@@ -431,7 +345,7 @@ __global__ void __launch_bounds__(kThreads) chain_greedy_finish(const FinishPara
     prm.out_tokens[(size_t)b * P + t] = v;
   }
   __syncwarp();
-  zero_rows(prm, (size_t)b, B, P, lane, 32, false);
+  zero_recs(prm, (size_t)b, B, P, lane, 32);
   if (lane == 0) {
     prm.accepted_len[b] = bad ? -1 : n;
     prm.req_reject[b] = 0u;
@@ -442,7 +356,7 @@ __global__ void __launch_bounds__(kThreads) chain_greedy_finish(const FinishPara
 __global__ void __launch_bounds__(kThreads) tree_finish(const FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
-  const int n = prm.k, B = prm.B, V = prm.V;
+  const int n = prm.k, V = prm.V;
   const int b = (int)blockIdx.x;
   int* garg = reinterpret_cast<int*>(smem + kFixedBytes);
   int* par = garg + n;
@@ -503,33 +417,7 @@ __global__ void __launch_bounds__(kThreads) tree_finish(const FinishParams prm) 
       ot[Lb] = garg[best];
     }
   }
-  zero_rows(prm, (size_t)b * n, 1, n, threadIdx.x, kThreads, false);
-}
-
-// Top-K extraction: one warp per row.
-__global__ void __launch_bounds__(kThreads) topk_finish(const FinishParams prm) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int row = (int)blockIdx.x * kWarps + w;
-  const int rows = prm.B;
-  if (row >= rows) return;
-  unsigned long long* buf =
-      reinterpret_cast<unsigned long long*>(smem) + (size_t)w * (prm.nchunk * prm.K + 32);
-  const unsigned long long kk =
-      warp_merge_topk(prm.cand + (size_t)row * prm.nchunk * prm.K, prm.nchunk, prm.K, buf);
-  const RowRec* r = &prm.rec[row];
-  const int code = __ldcg(&r->code);
-  const double L0 = __ldcg(&r->L0);
-  const double ln2 = 0.69314718055994530942;
-  const bool ok = code == kRowAccepted;
-  if (lane < prm.K) {
-    prm.topk_logp[(size_t)row * prm.K + lane] =
-        ok ? (float)(((double)key_value(kk) * (double)prm.c - L0) * ln2) : NAN;
-    prm.topk_idx[(size_t)row * prm.K + lane] = key_index(kk);
-  }
-  if (lane == 0) prm.lse[row] = ok ? (float)(L0 * ln2) : NAN;
-  __syncwarp();
-  zero_rows(prm, (size_t)row, 1, 1, lane, 32, true);
+  zero_recs(prm, (size_t)b * n, 1, n, threadIdx.x, kThreads);
 }
 
 // KD loss: one block per request, one warp per draft row (b, i < k).  Draft
@@ -594,7 +482,7 @@ __global__ void __launch_bounds__(kThreads) kl_finish(const FinishParams prm) {
     sh.fin_n = n;
   }
   __syncthreads();
-  if (!prm.draft_probs) zero_rows(prm, (size_t)b * k, 1, k, threadIdx.x, kThreads, false);
+  if (!prm.draft_probs) zero_recs(prm, (size_t)b * k, 1, k, threadIdx.x, kThreads);
   kd_finalize(b, sh.fin_n, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
               prm.total, prm.glob_counter, sh);
 }

@@ -88,6 +88,13 @@ struct StreamParams {
   int stage_off1;         // offset of row 1 inside a stage
   Partial* part;          // [nrows * nchunk]
   unsigned long long* cand;  // [nrows * nchunk * K]
+  // kFTopk0 outputs, written by the warp that completes a row: top-K log
+  // probabilities and indices, log-partition (chain: rows b * (k + 1) + i) and,
+  // for chain rows with a draft row, KL(renormalised top-K || draft).
+  float* topk_logp;
+  int32_t* topk_idx;
+  float* lse;
+  float* kl;
   RowRec* rec;            // [nrows]
   uint32_t* row_counter;  // [nrows]
   uint32_t* req_reject;   // [B] max over rejected chain rows of (k - i)
@@ -144,14 +151,55 @@ __device__ __forceinline__ uint32_t load_relaxed_u32(const uint32_t* p) {
   return *reinterpret_cast<const volatile uint32_t*>(p);
 }
 
+// Top K keys of row r from the stream's per-chunk lists (each sorted, best
+// first), best first in lanes 0..K-1.  The chunk heads are merged first; a
+// chunk whose head is not above the K-th best key so far holds nothing that
+// can enter, so only the few chunks with a larger head are read in full.
+__device__ __forceinline__ unsigned long long row_topk_merge(const unsigned long long* lists,
+                                                             int nchunk, int K) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long list = kNoKey;
+  for (int q0 = 0; q0 < nchunk; q0 += 32) {
+    const int q = q0 + lane;
+    const unsigned long long h = q < nchunk ? __ldcg(&lists[(size_t)q * K]) : kNoKey;
+    list = warp_merge_desc(list, warp_sort_desc(h));
+  }
+  unsigned long long thr = __shfl_sync(0xffffffffu, list, K - 1);
+  for (int q0 = 0; q0 < nchunk; q0 += 32) {
+    const int q = q0 + lane;
+    const unsigned long long h = q < nchunk ? __ldcg(&lists[(size_t)q * K]) : kNoKey;
+    unsigned m = __ballot_sync(0xffffffffu, h > thr);
+    while (m) {
+      // up to four chunks at a time: their keys 1..K-1 (the heads are merged)
+      unsigned long long x[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        x[t] = kNoKey;
+        if (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1;
+          if (lane + 1 < K) x[t] = __ldcg(&lists[(size_t)(q0 + src) * K + lane + 1]);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) list = warp_merge_desc(list, x[t]);
+      thr = __shfl_sync(0xffffffffu, list, K - 1);
+      m &= __ballot_sync(0xffffffffu, h > thr);
+    }
+  }
+  return list;
+}
+
 // The warp that counted a row's last chunk: combine the row's partials in
 // chunk order (lane l takes chunks l, l+32, ...; butterflies across lanes),
-// then record the row and, for chain rows, take the acceptance decision.
+// return the row's partials (and chunk lists) to zero, record the row and,
+// for chain rows, take the acceptance decision.  With kFTopk0 it also writes
+// the row's top-K outputs.
 template <class T0, class T1, int FLAGS>
 __device__ __noinline__ void row_complete(const StreamParams& prm, int r, const RowLoc& L) {
   const int lane = threadIdx.x & 31;
   const int nchunk = prm.nchunk;
-  const Partial* base = prm.part + (size_t)r * nchunk;
+  Partial* base = prm.part + (size_t)r * nchunk;
   float g0 = -INFINITY, g1 = -INFINITY, zx0 = 0.f, zx1 = 0.f;
   int flags = 0, hx = 0;
   unsigned long long key = kNoKey;
@@ -176,7 +224,8 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, const 
     s0 += rescale_pow2(__ldcg(&pq->S0), __ldcg(&pq->G0), G0);
     s1 += rescale_pow2(__ldcg(&pq->S1), __ldcg(&pq->G1), G1);
   }
-  const double S0 = warp_sum(s0), S1 = warp_sum(s1);
+  const double S0 = warp_sum(s0), S1 = warp_sum(s1);  // (every lane has read its partials)
+  for (int q = lane; q < nchunk; q += 32) base[q] = Partial{};
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) flags |= __shfl_xor_sync(0xffffffffu, flags, o);
   key = warp_max_u64(key);
@@ -186,30 +235,85 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, const 
     zx0 = __shfl_sync(0xffffffffu, zx0, src);
     zx1 = __shfl_sync(0xffffffffu, zx1, src);
   }
+  const double L0 = (double)G0 + log2(S0);
+  const double L1 = (double)G1 + log2(S1);
+  int err = 0;
+  if (flags & kPTimeout) err |= SV_DEV_TIMEOUT;
+  if ((FLAGS & kFStats0) && G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
+  if ((FLAGS & kFStats1) && L.row1 != nullptr && G1 == -INFINITY) err |= SV_DEV_NO_FINITE;
+  const bool skipped = prm.kind != kKindRows && (flags & kPSkipped);
+
+  if (FLAGS & kFTopk0) {
+    const int K = prm.K;
+    unsigned long long* lists = prm.cand + (size_t)r * nchunk * K;
+    const unsigned long long kk = row_topk_merge(lists, nchunk, K);
+    __syncwarp();
+    for (int t = lane; t < nchunk * K; t += 32) lists[t] = 0ull;
+    if (!skipped) {
+      const double ln2 = 0.69314718055994530942;
+      const bool rows = prm.kind == kKindRows;
+      const size_t orow = rows ? (size_t)r : (size_t)L.b * (prm.k + 1) + L.i;
+      // a failed row of a plain top-K call reads as NaN; chain rows are
+      // judged by the caller of the chain (accepted_len -1)
+      const bool nan_out = rows && err != 0;
+      double lp = -INFINITY;
+      int j = -1;
+      if (lane < K) {
+        j = key_index(kk);
+        lp = ((double)key_value(kk) * (double)prm.c - L0) * ln2;
+        prm.topk_logp[orow * K + lane] = nan_out ? NAN : (float)lp;
+        prm.topk_idx[orow * K + lane] = j;
+      }
+      if (lane == 0) prm.lse[orow] = nan_out ? NAN : (float)(L0 * ln2);
+      if (!rows && L.row1 != nullptr) {
+        // KL(p~ || q) over the renormalised top-K of the target row
+        double m = lp;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        double s = (lane < K) ? exp(lp - m) : 0.0;
+        s = warp_sum(s);
+        const double lse_k = m + log(s);
+        double term = 0.0;
+        if (lane < K && j >= 0 && j < prm.V) {
+          const float zd = load1<T1>(reinterpret_cast<const unsigned char*>(L.row1), j);
+          const double log_pt = lp - lse_k;
+          const double pt = exp(log_pt);
+          const double log_q = (FLAGS & kFStats1) ? ((double)zd * (double)prm.c - L1) * ln2
+                                                  : log((double)zd);
+          term = (pt == 0.0) ? 0.0 : pt * (log_pt - log_q);
+        }
+        term = warp_sum(term);
+        if (lane == 0) prm.kl[(size_t)L.b * prm.k + L.i] = (float)term;
+      }
+    }
+  }
   if (lane != 0) return;
+  if (prm.kind == kKindRows && (FLAGS & kFTopk0)) {
+    // a plain top-K call has no second pass: no record
+    if (err) set_status(prm.status, err);
+    prm.row_counter[r] = 0u;
+    return;
+  }
   RowRec rec;
   rec.G0 = G0;
   rec.G1 = G1;
   rec.S0 = S0;
   rec.S1 = S1;
-  rec.L0 = (double)G0 + log2(S0);
-  rec.L1 = (double)G1 + log2(S1);
+  rec.L0 = L0;
+  rec.L1 = L1;
   rec.argmax = key_index(key);
-  int err = 0, code = kRowAccepted;
-  if (flags & kPTimeout) err |= SV_DEV_TIMEOUT;
-  if ((FLAGS & kFStats0) && G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
-  if ((FLAGS & kFStats1) && L.row1 != nullptr && G1 == -INFINITY) err |= SV_DEV_NO_FINITE;
+  int code = kRowAccepted;
   if (prm.kind != kKindRows) {
     const int i = L.i, b = L.b, k = prm.k;
-    if (flags & kPSkipped) {
+    if (skipped) {
       err = 0;
       code = kRowSkipped;
     } else if (prm.kind == kKindChainSample) {
       if (i < k && !hm) err |= SV_DEV_BAD_TOKEN;
       if (!err && i < k) {
         const double c = (double)prm.c;
-        const double px = exp2((double)zx0 * c - rec.L0);
-        const double qx = (FLAGS & kFStats1) ? exp2((double)zx1 * c - rec.L1) : (double)zx1;
+        const double px = exp2((double)zx0 * c - L0);
+        const double qx = (FLAGS & kFStats1) ? exp2((double)zx1 * c - L1) : (double)zx1;
         const double u = (double)prm.u[(size_t)b * (k + 1) + i];
         code = (u * qx < px) ? kRowAccepted : kRowRejected;
       }
