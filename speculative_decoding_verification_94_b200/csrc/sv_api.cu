@@ -330,7 +330,8 @@ static cudaError_t pick_plan(K kernel, const RowPlan* plans, int np, int ncluste
 template <class TT, class DT, int DKIND>
 static cudaError_t run_chain_sample(const StreamParams& sp, const StreamGeom& sg, FinishParams fp,
                                     const RowPlan* plans, int np, bool kd, cudaStream_t s) {
-  constexpr int base = kFStats0 | kFRow1 | kFGather | (DKIND == kDraftLogits ? kFStats1 : 0);
+  // probability drafts are not streamed: q(x) is read directly
+  constexpr int base = kFStats0 | kFGather | (DKIND == kDraftLogits ? (kFRow1 | kFStats1) : 0);
   auto fin = kd ? chain_sample_finish<TT, DT, DKIND, true> : chain_sample_finish<TT, DT, DKIND, false>;
   RowPlan plan;
   cudaError_t e = pick_plan(fin, plans, np, fp.B, &plan);
@@ -416,7 +417,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   const int K = kd ? kd->K : 0;
   const int te = esize(t_dtype);
   const int de = greedy ? 0 : (d_kind == SV_DRAFT_PROBS ? 4 : esize(d_dtype));
-  const StreamGeom sg = stream_geom(V, (long long)B * P, te, de);
+  const StreamGeom sg = stream_geom(V, (long long)B * P, te, d_kind == SV_DRAFT_PROBS ? 0 : de);
   const WsLayout wl = ws_layout(B, B * P, sg.nchunk, K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
@@ -435,6 +436,8 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   sp.nrows = B * P;
   sp.W = sg.W;
   sp.nchunk = sg.nchunk;
+  sp.div_nchunk = make_fastdiv(sg.nchunk);
+  sp.div_B = make_fastdiv(sp.B);
   sp.c = greedy ? 0.f : (float)(1.4426950408889634 / (double)temperature);
   sp.use_bulk = bulk_ok_row(target_logits, V, te) && (greedy || bulk_ok_row(draft, V, de));
   sp.K = K > 0 ? K : 1;
@@ -445,6 +448,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   sp.rec = w.rec;
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
+  sp.sched = w.glob + 1;
   sp.status = device_status;
 
   FinishParams fp = {};
@@ -545,6 +549,8 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   sp.nrows = B * n;
   sp.W = sg.W;
   sp.nchunk = sg.nchunk;
+  sp.div_nchunk = make_fastdiv(sg.nchunk);
+  sp.div_B = make_fastdiv(sp.B);
   sp.use_bulk = bulk_ok_row(logits, V, esize(dt));
   sp.K = 1;
   sp.stage_bytes = sg.stage_bytes;
@@ -554,6 +560,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   sp.rec = w.rec;
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
+  sp.sched = w.glob + 1;
   sp.status = device_status;
   cudaError_t e = dt == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
                                 : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
@@ -605,6 +612,8 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   sp.nrows = rows;
   sp.W = sg.W;
   sp.nchunk = sg.nchunk;
+  sp.div_nchunk = make_fastdiv(sg.nchunk);
+  sp.div_B = make_fastdiv(sp.B);
   sp.c = (float)(1.4426950408889634 / (double)temperature);
   sp.use_bulk = bulk_ok_row(logits, V, esize(dt));
   sp.K = K;
@@ -615,6 +624,7 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   sp.rec = w.rec;
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
+  sp.sched = w.glob + 1;
   sp.status = device_status;
   sp.topk_logp = topk_logp;
   sp.topk_idx = topk_idx;
@@ -665,6 +675,8 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
     sp.nrows = B * k;
     sp.W = sg.W;
     sp.nchunk = sg.nchunk;
+  sp.div_nchunk = make_fastdiv(sg.nchunk);
+  sp.div_B = make_fastdiv(sp.B);
     sp.c = c;
     sp.use_bulk = bulk_ok_row(draft, V, esize(d_dtype));
     sp.K = 1;
@@ -675,6 +687,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
     sp.rec = w.rec;
     sp.row_counter = w.counter;
     sp.req_reject = w.reject;
+  sp.sched = w.glob + 1;
     sp.status = device_status;
     cudaError_t e = d_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFStats0>(sp, sg, s)
                                        : launch_stream<F32, F32, kFStats0>(sp, sg, s);

@@ -48,6 +48,27 @@ struct F32 {
   using storage = float;
   static constexpr int bytes = 4;
 };
+// Division by a runtime divisor 1 <= d < 2^31 for dividends 0 <= n < 2^31:
+// floor(n / d) = (n * m) >> (32 + s) with 2^s >= d and m = ceil(2^(32+s) / d)
+// (m < 2^33, so the product fits 64 bits; the rounding excess of m adds less
+// than n / 2^(32+s) < 1/(2d), which never crosses the next multiple of 1/d).
+struct FastDiv {
+  unsigned long long m;
+  int s;
+};
+inline FastDiv make_fastdiv(int d) {
+  int s = 0;
+  while ((1LL << s) < d) ++s;
+  const unsigned __int128 num = (unsigned __int128)1 << (32 + s);
+  FastDiv f;
+  f.m = (unsigned long long)((num + (unsigned)d - 1) / (unsigned)d);
+  f.s = s;
+  return f;
+}
+__device__ __forceinline__ int fast_div(int n, const FastDiv& f) {
+  return (int)(((unsigned long long)(unsigned)n * f.m) >> (32 + f.s));
+}
+
 struct BF16 {
   using storage = uint16_t;
   static constexpr int bytes = 2;
@@ -229,6 +250,28 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Packed pairs of fp32 in one 64-bit register (sm_100 f32x2 arithmetic: one
+// instruction for two lanes of a pair).
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long d, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // 2^x on the special-function unit (ex2.approx.ftz.f32).
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -380,11 +423,24 @@ __device__ __forceinline__ void stat_init(ThreadStat& s) {
   s.S = 0.0;
 }
 
-// S * 2^(from - to) for integer-valued from <= to (exact; underflows to 0).
+// 2^e as a binary64 for integer e in [-1022, 1023], built from the exponent field.
+__device__ __forceinline__ double pow2i(int e) {
+  return __longlong_as_double((long long)(e + 1023) << 52);
+}
+
+// S * 2^(from - to) for integer-valued from <= to: exact for normal results,
+// in two steps below 2^-1022, 0 below 2^-2000.
 __device__ __forceinline__ double rescale_pow2(double S, float from, float to) {
   if (S == 0.0) return 0.0;
   const float d = from - to;
-  return d < -2000.f ? 0.0 : ldexp(S, (int)d);
+  if (d < -2000.f) return 0.0;
+  int e = (int)d;
+  if (e > 1023) e = 1023;
+  if (e < -1022) {
+    S *= pow2i(-1022);
+    e += 1022;
+  }
+  return S * pow2i(e);
 }
 
 __device__ __forceinline__ void stat_update(ThreadStat& s, const float v[8], float vmax, float c) {

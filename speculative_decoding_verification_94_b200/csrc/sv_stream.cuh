@@ -99,6 +99,9 @@ struct StreamParams {
   uint32_t* row_counter;  // [nrows]
   uint32_t* req_reject;   // [B] max over rejected chain rows of (k - i)
   int32_t* status;
+  FastDiv div_nchunk;     // item -> row
+  FastDiv div_B;          // chain row -> position
+  uint32_t* sched;        // [2]: dynamic item counter, exited warps (zero between calls)
 };
 
 // Where row r of a stream lives.
@@ -120,12 +123,12 @@ __device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r) {
     L.x = -1;
     return L;
   }
-  L.i = r / p.B;
+  L.i = fast_div(r, p.div_B);
   L.b = r - L.i * p.B;
   const int P = p.k + 1;
   L.row0 = reinterpret_cast<const unsigned char*>(p.rows0) + ((size_t)L.b * P + L.i) * p.V * T0::bytes;
   L.row1 = nullptr;
-  if ((FLAGS & kFRow1) && L.i < p.k)
+  if (p.rows1 != nullptr && L.i < p.k)
     L.row1 = reinterpret_cast<const unsigned char*>(p.rows1) +
              ((size_t)L.b * p.k + L.i) * p.V * T1::bytes;
   L.x = (L.i < p.k) ? p.tokens[(size_t)L.b * p.k + L.i] : -1;
@@ -234,6 +237,9 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, const 
     const int src = __ffs(hm) - 1;
     zx0 = __shfl_sync(0xffffffffu, zx0, src);
     zx1 = __shfl_sync(0xffffffffu, zx1, src);
+    // a draft row that is not streamed (probabilities): q(x) read directly
+    if (!(FLAGS & kFRow1) && L.row1 != nullptr)
+      zx1 = load1<T1>(reinterpret_cast<const unsigned char*>(L.row1), L.x);
   }
   const double L0 = (double)G0 + log2(S0);
   const double L1 = (double)G1 + log2(S1);
@@ -332,8 +338,150 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, const 
   prm.row_counter[r] = 0u;
 }
 
+// ---------------------------------------------------------------------------
+// One lane's share of one row of a piece: kLaneVecs vectors of 8 elements,
+// vector v holding piece elements (v * 32 + lane) * 8 .. + 7, in registers.
+// Vectors past the end of the piece read as -inf (no mass, never a maximum).
+// ---------------------------------------------------------------------------
+template <class T>
+struct LaneRow;
+template <>
+struct LaneRow<BF16> {
+  uint4 w[kLaneVecs];
+};
+template <>
+struct LaneRow<F32> {
+  float4 w[2 * kLaneVecs];
+};
+
+__device__ __forceinline__ void lane_load(const unsigned char* st, int nv, LaneRow<BF16>& R) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int v = 0; v < kLaneVecs; ++v) {
+    const int vi = v * 32 + lane;
+    R.w[v] = vi < nv ? *reinterpret_cast<const uint4*>(st + (size_t)vi * 16)
+                     : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  }
+}
+__device__ __forceinline__ void lane_load(const unsigned char* st, int nv, LaneRow<F32>& R) {
+  const int lane = threadIdx.x & 31;
+  const float ni = -INFINITY;
+#pragma unroll
+  for (int v = 0; v < kLaneVecs; ++v) {
+    const int vi = v * 32 + lane;
+    if (vi < nv) {
+      R.w[2 * v] = *reinterpret_cast<const float4*>(st + (size_t)vi * 32);
+      R.w[2 * v + 1] = *reinterpret_cast<const float4*>(st + (size_t)vi * 32 + 16);
+    } else {
+      R.w[2 * v] = R.w[2 * v + 1] = make_float4(ni, ni, ni, ni);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Maximum of vector v, and of all the lane's vectors.
+__device__ __forceinline__ float vec_max(const LaneRow<BF16>& R, int v) {
+  const uint32_t m = bmax2(bmax2(R.w[v].x, R.w[v].y), bmax2(R.w[v].z, R.w[v].w));
+  return fmaxf(bf16_lo(m), bf16_hi(m));
+}
+__device__ __forceinline__ float vec_max(const LaneRow<F32>& R, int v) {
+  const float4 a = R.w[2 * v], b = R.w[2 * v + 1];
+  return fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(b.x, b.y), fmaxf(b.z, b.w)));
+}
+__device__ __forceinline__ float lane_max(const LaneRow<BF16>& R) {
+  uint32_t m = bmax2(bmax2(R.w[0].x, R.w[0].y), bmax2(R.w[0].z, R.w[0].w));
+#pragma unroll
+  for (int v = 1; v < kLaneVecs; ++v)
+    m = bmax2(m, bmax2(bmax2(R.w[v].x, R.w[v].y), bmax2(R.w[v].z, R.w[v].w)));
+  return fmaxf(bf16_lo(m), bf16_hi(m));
+}
+__device__ __forceinline__ float lane_max(const LaneRow<F32>& R) {
+  float m = vec_max(R, 0);
+#pragma unroll
+  for (int v = 1; v < kLaneVecs; ++v) m = fmaxf(m, vec_max(R, v));
+  return m;
+}
+
+// Element t (0..7) of vector v.
+__device__ __forceinline__ float lane_elem(const LaneRow<BF16>& R, int v, int t) {
+  const uint32_t w = (t >> 1) == 0 ? R.w[v].x : (t >> 1) == 1 ? R.w[v].y : (t >> 1) == 2 ? R.w[v].z
+                                                                                       : R.w[v].w;
+  return (t & 1) ? bf16_hi(w) : bf16_lo(w);
+}
+__device__ __forceinline__ float lane_elem(const LaneRow<F32>& R, int v, int t) {
+  const float4 q = R.w[2 * v + (t >> 2)];
+  const int u = t & 3;
+  return u == 0 ? q.x : u == 1 ? q.y : u == 2 ? q.z : q.w;
+}
+
+// 2^(x c - ref) for the pair (lo, hi): one packed fma, two exp2.
+__device__ __forceinline__ unsigned long long term2(float lo, float hi, unsigned long long cc,
+                                                    unsigned long long nr) {
+  float a, b;
+  f2_unpack(f2_fma(f2_pack(lo, hi), cc, nr), a, b);
+  return f2_pack(ex2(a), ex2(b));
+}
+
+// Sum over the lane's elements of 2^(x c - ref), by a fixed tree of packed adds.
+__device__ __forceinline__ float lane_terms(const LaneRow<BF16>& R, float c, float ref) {
+  const unsigned long long cc = f2_pack(c, c), nr = f2_pack(-ref, -ref);
+  unsigned long long e[4 * kLaneVecs];
+#pragma unroll
+  for (int v = 0; v < kLaneVecs; ++v) {
+    e[4 * v + 0] = term2(bf16_lo(R.w[v].x), bf16_hi(R.w[v].x), cc, nr);
+    e[4 * v + 1] = term2(bf16_lo(R.w[v].y), bf16_hi(R.w[v].y), cc, nr);
+    e[4 * v + 2] = term2(bf16_lo(R.w[v].z), bf16_hi(R.w[v].z), cc, nr);
+    e[4 * v + 3] = term2(bf16_lo(R.w[v].w), bf16_hi(R.w[v].w), cc, nr);
+  }
+#pragma unroll
+  for (int w = 2 * kLaneVecs; w >= 1; w >>= 1)
+#pragma unroll
+    for (int t = 0; t < w; ++t) e[t] = f2_add(e[t], e[t + w]);
+  float lo, hi;
+  f2_unpack(e[0], lo, hi);
+  return lo + hi;
+}
+__device__ __forceinline__ float lane_terms(const LaneRow<F32>& R, float c, float ref) {
+  const unsigned long long cc = f2_pack(c, c), nr = f2_pack(-ref, -ref);
+  unsigned long long e[4 * kLaneVecs];
+#pragma unroll
+  for (int v = 0; v < 2 * kLaneVecs; ++v) {
+    e[2 * v + 0] = term2(R.w[v].x, R.w[v].y, cc, nr);
+    e[2 * v + 1] = term2(R.w[v].z, R.w[v].w, cc, nr);
+  }
+#pragma unroll
+  for (int w = 2 * kLaneVecs; w >= 1; w >>= 1)
+#pragma unroll
+    for (int t = 0; t < w; ++t) e[t] = f2_add(e[t], e[t + w]);
+  float lo, hi;
+  f2_unpack(e[0], lo, hi);
+  return lo + hi;
+}
+
+// Fold one row of a piece into a lane's statistics (reference moved first).
+template <class T>
+__device__ __forceinline__ void lane_stats(ThreadStat& st, const LaneRow<T>& R, float pm, float c) {
+  stat_cover(st, pm, c);
+  if (pm != -INFINITY) st.S += (double)lane_terms(R, c, st.ref);
+}
+
+// ---------------------------------------------------------------------------
+// The streaming kernel.
+//
+// Work distribution: warp g takes items g and g + NW first, then items
+// 2 NW + t in the order of a device-wide counter t, so the items run roughly
+// in index order (position-major for chains) and no warp waits on a slow
+// neighbour.  The counter of the item after next is fetched when an item
+// starts and that item's skip test is read when its first copy is issued.
+// The last warp to leave returns the counters to zero.
+// ---------------------------------------------------------------------------
 template <class T0, class T1, int FLAGS>
-__global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamParams prm) {
+__global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_constant__ StreamParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* ring = smem + (size_t)warp * kStages * prm.stage_bytes;
@@ -347,37 +495,42 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
   const float c = prm.c;
   const int K = prm.K;
   const unsigned kmask = K >= 32 ? 0xffffffffu : ((1u << K) - 1u);
-  if (lane == 0) {
-    if (use_bulk) {
-      for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-      fence_mbar_init();
-    }
+  if (lane == 0 && use_bulk) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
   }
   __syncwarp();
 
-  // Pieces of an item; 0 when the item is skipped (an earlier position of its
-  // request rejected) or does not exist.
-  auto item_pieces = [&](int item) -> int {
+  // Lane 0: the request-rejection word of an item's row (chain kinds); an
+  // item is skipped when an earlier position of its request rejected.
+  auto reject_word = [&](int item) -> uint32_t {
+    if (prm.kind == kKindRows || item >= total) return 0u;
+    const int r = fast_div(item, prm.div_nchunk);
+    const int i = fast_div(r, prm.div_B);
+    return load_relaxed_u32(&prm.req_reject[r - i * prm.B]);
+  };
+  auto pieces_of = [&](int item, uint32_t rj) -> int {  // lane-uniform
     if (item >= total) return 0;
-    const int r = item / nchunk, ch = item - r * nchunk;
-    const int len = min(W, V - ch * W);
+    const int r = fast_div(item, prm.div_nchunk);
+    const int ch = item - r * nchunk;
     int skip = 0;
-    if (prm.kind != kKindRows && lane == 0) {
-      const int i = r / prm.B, b = r - i * prm.B;
-      skip = load_relaxed_u32(&prm.req_reject[b]) > (uint32_t)(prm.k - i) ? 1 : 0;
+    if (prm.kind != kKindRows) {
+      const int i = fast_div(r, prm.div_B);
+      skip = __shfl_sync(0xffffffffu, rj > (uint32_t)(prm.k - i) ? 1 : 0, 0);
     }
-    skip = __shfl_sync(0xffffffffu, skip, 0);
+    const int len = min(W, V - ch * W);
     return skip ? 0 : (len + kPiece - 1) / kPiece;
   };
 
-  // Lane 0: bulk copies of piece p of item into ring stage s.
+  // Lane 0: bulk copies of piece p of an item into ring stage s.
   auto issue = [&](int item, int p, int s) {
-    const int r = item / nchunk, ch = item - r * nchunk;
+    const int r = fast_div(item, prm.div_nchunk);
+    const int ch = item - r * nchunk;
     const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r);
     const int e0 = ch * W + p * kPiece;
     const int n = min(kPiece, min(V, ch * W + W) - e0);
     const uint32_t nb0 = (uint32_t)(n * T0::bytes) & ~15u;
-    const uint32_t nb1 = (L.row1 != nullptr) ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
+    const uint32_t nb1 = ((FLAGS & kFRow1) && L.row1 != nullptr) ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
     unsigned char* st = ring + (size_t)s * prm.stage_bytes;
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&bars[s], nb0 + nb1);
@@ -392,9 +545,15 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
 
   uint32_t n_issued = 0, n_consumed = 0;
   int cur = gwarp;
-  int cur_np = item_pieces(cur);
+  uint32_t rj = 0;
+  if (lane == 0) rj = reject_word(cur);
+  int cur_np = pieces_of(cur, rj);
   int nxt = gwarp + nwarps;
-  int nxt_np = item_pieces(nxt);
+  uint32_t nxt_rj = 0;
+  if (lane == 0) nxt_rj = reject_word(nxt);
+  int nxt_np = -1;  // resolved when its first copy is due
+  uint32_t pend = 0;  // lane 0: counter value of the item after nxt
+  if (lane == 0 && nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
   int iss_which = 0, iss_p = 0;
   int timeouts = 0;
 
@@ -411,6 +570,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
           continue;
         }
       } else {
+        if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj);
         if (iss_p < nxt_np) {
           it = nxt;
           pp = iss_p++;
@@ -425,7 +585,8 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
 
   top_up();
   while (cur < total) {
-    const int r = cur / nchunk, ch = cur - r * nchunk;
+    const int r = fast_div(cur, prm.div_nchunk);
+    const int ch = cur - r * nchunk;
     const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r);
     const int clen = min(W, V - ch * W);
     ThreadStat st0, st1;
@@ -465,63 +626,30 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
           for (int e = a1 + lane; e < n; e += 32)
             reinterpret_cast<typename T1::storage*>(st1p)[e] = src1[e];
           for (int e = n + lane; e < ((n + kVec - 1) / kVec) * kVec; e += 32)
-            store_pad<T1>(st1p, e, !(FLAGS & kFStats1));
+            store_pad<T1>(st1p, e, false);
         }
         __syncwarp();
       }
       const int nv = (n + kVec - 1) / kVec;
-      // The draft token's values, read once per piece by lane 0.
+      // The draft token's values.
       if ((FLAGS & kFGather) && L.x >= e0 && L.x < e0 + n) {
         hx = 1;
         zx0 = load1<T0>(st, L.x - e0);
         if (has1) zx1 = load1<T1>(st1p, L.x - e0);
       }
-      // Row 0: this lane's kLaneVecs vectors (element (v*32 + lane)*8 + t).
-      // First the maxima (packed, straight from shared memory) and one
-      // reference update per piece, then the exp2 terms two vectors at a time.
       {
-        float vm[kLaneVecs];
-        float pm = -INFINITY;
-#pragma unroll
-        for (int v = 0; v < kLaneVecs; ++v) {
-          const int vi = v * 32 + lane;
-          vm[v] = vi < nv ? max8<T0>(st, vi * kVec) : -INFINITY;
-          pm = fmaxf(pm, vm[v]);
-        }
-        if (FLAGS & kFStats0) {
-          stat_cover(st0, pm, c);
-          if (pm != -INFINITY) {
-            float acc = 0.f;
-#pragma unroll
-            for (int v = 0; v < kLaneVecs; v += 2) {
-              float x[2][8];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int vi = (v + h) * 32 + lane;
-                if (vi < nv) load8<T0>(st, vi * kVec, x[h]);
-                else
-#pragma unroll
-                  for (int t = 0; t < 8; ++t) x[h][t] = -INFINITY;
-              }
-              acc += stat_terms<2>(st0, x, c);
-            }
-            st0.S += (double)acc;
-          }
-        }
+        LaneRow<T0> R;
+        lane_load(st, nv, R);
+        const float pm = lane_max(R);
+        if (FLAGS & kFStats0) lane_stats(st0, R, pm, c);
         if (FLAGS & kFArgmax0) {
           if (pm > best || (bidx < 0 && nv > lane)) {
             int bi = -1;
 #pragma unroll
-            for (int v = kLaneVecs - 1; v >= 0; --v) {
-              const int vi = v * 32 + lane;
-              if (vi < nv && vm[v] == pm) {
-                float x[8];
-                load8<T0>(st, vi * kVec, x);
+            for (int v = kLaneVecs - 1; v >= 0; --v)
 #pragma unroll
-                for (int t = 7; t >= 0; --t)
-                  if (x[t] == pm) bi = vi * kVec + t;
-              }
-            }
+              for (int t = 7; t >= 0; --t)
+                if (lane_elem(R, v, t) == pm) bi = (v * 32 + lane) * kVec + t;
             best = pm;
             bidx = e0 + bi;
           }
@@ -530,7 +658,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
 #pragma unroll
           for (int v = 0; v < kLaneVecs; ++v) {
             const int vi = v * 32 + lane;
-            unsigned m = __ballot_sync(0xffffffffu, vi < nv && vm[v] >= thr_val);
+            unsigned m = __ballot_sync(0xffffffffu, vi < nv && vec_max(R, v) >= thr_val);
             while (m) {
               const int src = __ffs(m) - 1;
               m &= m - 1;
@@ -539,9 +667,8 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
               load8<T0>(st, sbase, xs);  // every lane reads the source lane's vector
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
-                const int idx = e0 + sbase + q;
                 if (sbase + q < n) {
-                  const unsigned long long key = topk_key(xs[q], idx);
+                  const unsigned long long key = topk_key(xs[q], e0 + sbase + q);
                   if (key > thr_key) {
                     warp_list_insert(list, key, kmask);
                     thr_key = __shfl_sync(0xffffffffu, list, K - 1);
@@ -554,30 +681,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
         }
       }
       if ((FLAGS & kFStats1) && has1) {
-        float pm = -INFINITY;
-#pragma unroll
-        for (int v = 0; v < kLaneVecs; ++v) {
-          const int vi = v * 32 + lane;
-          if (vi < nv) pm = fmaxf(pm, max8<T1>(st1p, vi * kVec));
-        }
-        stat_cover(st1, pm, c);
-        if (pm != -INFINITY) {
-          float acc = 0.f;
-#pragma unroll
-          for (int v = 0; v < kLaneVecs; v += 2) {
-            float x[2][8];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int vi = (v + h) * 32 + lane;
-              if (vi < nv) load8<T1>(st1p, vi * kVec, x[h]);
-              else
-#pragma unroll
-                for (int t = 0; t < 8; ++t) x[h][t] = -INFINITY;
-            }
-            acc += stat_terms<2>(st1, x, c);
-          }
-          st1.S += (double)acc;
-        }
+        LaneRow<T1> R;
+        lane_load(st1p, nv, R);
+        lane_stats(st1, R, lane_max(R), c);
       }
       __syncwarp();
       ++n_consumed;
@@ -614,10 +720,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
     pr.flags = flags;
     pr.pad = 0;
     if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)cur * K + lane] = list;
+    if (lane == 0) prm.part[cur] = pr;
+    __syncwarp();
+    __threadfence();  // this item's partial and list before its count
     int last = 0;
     if (lane == 0) {
-      prm.part[cur] = pr;
-      __threadfence();
       last = atomicAdd(&prm.row_counter[r], 1u) == (uint32_t)(nchunk - 1) ? 1 : 0;
       if (last) __threadfence();
     }
@@ -625,13 +732,23 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
     if (last) row_complete<T0, T1, FLAGS>(prm, r, L);
     timeouts = 0;
 
-    // Advance.
+    // Advance: nxt becomes current; the item after it comes from the counter.
     cur = nxt;
+    if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj);
     cur_np = nxt_np;
-    if (iss_which == 0) iss_p = 0;  // (the issue side normally moved on to nxt already)
+    if (iss_which == 0) iss_p = 0;
     iss_which = 0;
-    nxt = cur + nwarps;
-    nxt_np = item_pieces(nxt);
+    if (cur < total) {
+      const int t = __shfl_sync(0xffffffffu, (int)pend, 0);
+      nxt = 2 * nwarps + t;
+    } else {
+      nxt = total;
+    }
+    nxt_np = -1;
+    if (lane == 0) {
+      nxt_rj = reject_word(nxt);
+      if (nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
+    }
     top_up();
   }
   // Any copy still in flight (only after a timed-out wait) completes before exit.
@@ -640,6 +757,15 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const StreamP
       mbar_wait_bounded(&bars[n_consumed % kStages], (n_consumed / kStages) & 1u);
       ++n_consumed;
     }
+  // The last warp to leave returns the scheduling counters to zero.
+  if (lane == 0) {
+    __threadfence();
+    if (atomicAdd(&prm.sched[1], 1u) == (uint32_t)(nwarps - 1)) {
+      __threadfence();
+      prm.sched[0] = 0u;
+      prm.sched[1] = 0u;
+    }
+  }
 }
 
 }  // namespace sv
