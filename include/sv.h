@@ -107,7 +107,7 @@ typedef struct sv_kd_args {
 
 /* Bytes of zero-filled workspace needed by each call (K = 0: no fused KD).
  * The workspace holds per-row chunk counters, row records and per-chunk
- * partial results of the streaming pass: O(rows * V / 8192) small records,
+ * partial results of the streaming pass: at most rows * ceil(V / 1024) small records,
  * plus K keys per chunk when top-K lists are kept. */
 SV_API size_t sv_verify_chain_workspace_size(int B, int k, int V, int K);
 SV_API size_t sv_verify_tree_workspace_size(int B, int n, int V);

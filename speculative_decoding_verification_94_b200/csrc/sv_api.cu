@@ -148,13 +148,14 @@ static cudaError_t sm_count(int* out) {
 
 // Chunk length of the stream (a multiple of the piece, at most 8 pieces):
 // long enough to amortise the per-chunk record, short enough that a batch
-// gives every warp of the device a few chunks (about 8192 in all).  It
+// gives every warp of the device several chunks (about 16384 in all), which
+// keeps the tail of the dynamic schedule short.  It
 // depends on the sizes only, so workspace sizes are device independent.
 static int stream_chunk(int V, long long nrows) {
   const int forced = env_int("SV_STREAM_W");
   if (forced >= kPiece && forced % kPiece == 0) return forced;
   int w = kPiece;
-  while (w < 8 * kPiece && (long long)V * nrows / (2 * w) >= 8192) w *= 2;
+  while (w < 8 * kPiece && (long long)V * nrows / (2 * w) >= 16384) w *= 2;
   const int cap = (int)align_up((size_t)V, kPiece);
   return w < cap ? w : cap;
 }

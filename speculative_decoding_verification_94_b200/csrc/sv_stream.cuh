@@ -107,20 +107,21 @@ struct StreamParams {
 // Where row r of a stream lives.
 struct RowLoc {
   int b, i;            // chain: request and position; rows: b = r, i = 0
-  const void* row0;
-  const void* row1;
+  const unsigned char* row0;
+  const unsigned char* row1;
   int x;               // chain: draft token of this row (-1 for the bonus row / none)
 };
 
+// Row pointers of row r (the draft token is supplied separately).
 template <class T0, class T1, int FLAGS>
-__device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r) {
+__device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r, int x) {
   RowLoc L;
+  L.x = x;
   if (p.kind == kKindRows) {
     L.b = r;
     L.i = 0;
     L.row0 = reinterpret_cast<const unsigned char*>(p.rows0) + (size_t)r * p.V * T0::bytes;
     L.row1 = nullptr;
-    L.x = -1;
     return L;
   }
   L.i = fast_div(r, p.div_B);
@@ -131,8 +132,19 @@ __device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r) {
   if (p.rows1 != nullptr && L.i < p.k)
     L.row1 = reinterpret_cast<const unsigned char*>(p.rows1) +
              ((size_t)L.b * p.k + L.i) * p.V * T1::bytes;
-  L.x = (L.i < p.k) ? p.tokens[(size_t)L.b * p.k + L.i] : -1;
   return L;
+}
+
+// Add with acquire-release semantics at device scope (global memory).
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Warp maximum of a float through the integer reduction unit.
+__device__ __forceinline__ float warp_max_redux(float v) {
+  return order_float(__reduce_max_sync(0xffffffffu, float_order(v)));
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -356,6 +368,12 @@ struct LaneRow<F32> {
 
 __device__ __forceinline__ void lane_load(const unsigned char* st, int nv, LaneRow<BF16>& R) {
   const int lane = threadIdx.x & 31;
+  if (nv == kLaneVecs * 32) {  // full piece (warp-uniform)
+#pragma unroll
+    for (int v = 0; v < kLaneVecs; ++v)
+      R.w[v] = *reinterpret_cast<const uint4*>(st + (size_t)(v * 32 + lane) * 16);
+    return;
+  }
 #pragma unroll
   for (int v = 0; v < kLaneVecs; ++v) {
     const int vi = v * 32 + lane;
@@ -365,6 +383,14 @@ __device__ __forceinline__ void lane_load(const unsigned char* st, int nv, LaneR
 }
 __device__ __forceinline__ void lane_load(const unsigned char* st, int nv, LaneRow<F32>& R) {
   const int lane = threadIdx.x & 31;
+  if (nv == kLaneVecs * 32) {  // full piece (warp-uniform)
+#pragma unroll
+    for (int v = 0; v < kLaneVecs; ++v) {
+      R.w[2 * v] = *reinterpret_cast<const float4*>(st + (size_t)(v * 32 + lane) * 32);
+      R.w[2 * v + 1] = *reinterpret_cast<const float4*>(st + (size_t)(v * 32 + lane) * 32 + 16);
+    }
+    return;
+  }
   const float ni = -INFINITY;
 #pragma unroll
   for (int v = 0; v < kLaneVecs; ++v) {
@@ -476,9 +502,9 @@ __device__ __forceinline__ void lane_stats(ThreadStat& st, const LaneRow<T>& R, 
 // Work distribution: warp g takes items g and g + NW first, then items
 // 2 NW + t in the order of a device-wide counter t, so the items run roughly
 // in index order (position-major for chains) and no warp waits on a slow
-// neighbour.  The counter of the item after next is fetched when an item
-// starts and that item's skip test is read when its first copy is issued.
-// The last warp to leave returns the counters to zero.
+// neighbour.  Lane 0 fetches the counter value of the item after next, and
+// that item's rejection word and draft token, when an item starts.  The last
+// warp to leave returns the counters to zero.
 // ---------------------------------------------------------------------------
 template <class T0, class T1, int FLAGS>
 __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_constant__ StreamParams prm) {
@@ -488,6 +514,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kStreamWarps * kStages * prm.stage_bytes) +
                    warp * kStages;
   const bool use_bulk = prm.use_bulk != 0;
+  const bool chain = prm.kind != kKindRows;
   const int V = prm.V, W = prm.W, nchunk = prm.nchunk;
   const int total = prm.nrows * nchunk;
   const int nwarps = (int)gridDim.x * kStreamWarps;
@@ -501,20 +528,24 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   }
   __syncwarp();
 
-  // Lane 0: the request-rejection word of an item's row (chain kinds); an
-  // item is skipped when an earlier position of its request rejected.
-  auto reject_word = [&](int item) -> uint32_t {
-    if (prm.kind == kKindRows || item >= total) return 0u;
+  // Lane 0: an item's request-rejection word and draft token (chain kinds).
+  auto prefetch = [&](int item, uint32_t& rj, int& x) {
+    rj = 0u;
+    x = -1;
+    if (!chain || item >= total) return;
     const int r = fast_div(item, prm.div_nchunk);
-    const int i = fast_div(r, prm.div_B);
-    return load_relaxed_u32(&prm.req_reject[r - i * prm.B]);
+    const int i = fast_div(r, prm.div_B), b = r - i * prm.B;
+    rj = load_relaxed_u32(&prm.req_reject[b]);
+    if (i < prm.k) x = prm.tokens[(size_t)b * prm.k + i];
   };
-  auto pieces_of = [&](int item, uint32_t rj) -> int {  // lane-uniform
+  // Pieces of an item (lane-uniform); 0 when skipped: an earlier position of
+  // its request rejected.
+  auto pieces_of = [&](int item, uint32_t rj) -> int {
     if (item >= total) return 0;
     const int r = fast_div(item, prm.div_nchunk);
     const int ch = item - r * nchunk;
     int skip = 0;
-    if (prm.kind != kKindRows) {
+    if (chain) {
       const int i = fast_div(r, prm.div_B);
       skip = __shfl_sync(0xffffffffu, rj > (uint32_t)(prm.k - i) ? 1 : 0, 0);
     }
@@ -526,34 +557,37 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   auto issue = [&](int item, int p, int s) {
     const int r = fast_div(item, prm.div_nchunk);
     const int ch = item - r * nchunk;
-    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r);
+    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, -1);
     const int e0 = ch * W + p * kPiece;
     const int n = min(kPiece, min(V, ch * W + W) - e0);
     const uint32_t nb0 = (uint32_t)(n * T0::bytes) & ~15u;
-    const uint32_t nb1 = ((FLAGS & kFRow1) && L.row1 != nullptr) ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
+    const uint32_t nb1 =
+        ((FLAGS & kFRow1) && L.row1 != nullptr) ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
     unsigned char* st = ring + (size_t)s * prm.stage_bytes;
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&bars[s], nb0 + nb1);
     if (nb0)
-      bulk_g2s_plain(st, reinterpret_cast<const unsigned char*>(L.row0) + (size_t)e0 * T0::bytes,
-                     nb0, &bars[s]);
+      bulk_g2s_plain(st, L.row0 + (size_t)e0 * T0::bytes, nb0, &bars[s]);
     if (nb1)
-      bulk_g2s_plain(st + prm.stage_off1,
-                     reinterpret_cast<const unsigned char*>(L.row1) + (size_t)e0 * T1::bytes, nb1,
-                     &bars[s]);
+      bulk_g2s_plain(st + prm.stage_off1, L.row1 + (size_t)e0 * T1::bytes, nb1, &bars[s]);
   };
 
   uint32_t n_issued = 0, n_consumed = 0;
-  int cur = gwarp;
-  uint32_t rj = 0;
-  if (lane == 0) rj = reject_word(cur);
-  int cur_np = pieces_of(cur, rj);
-  int nxt = gwarp + nwarps;
-  uint32_t nxt_rj = 0;
-  if (lane == 0) nxt_rj = reject_word(nxt);
-  int nxt_np = -1;  // resolved when its first copy is due
-  uint32_t pend = 0;  // lane 0: counter value of the item after nxt
-  if (lane == 0 && nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
+  int cur = gwarp, cur_np, cur_x;
+  {
+    uint32_t rj;
+    int x;
+    if (lane == 0) prefetch(cur, rj, x);
+    cur_np = pieces_of(cur, rj);
+    cur_x = __shfl_sync(0xffffffffu, x, 0);
+  }
+  int nxt = gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
+  uint32_t nxt_rj = 0u;
+  uint32_t pend = 0u;  // lane 0: counter value of the item after nxt
+  if (lane == 0) {
+    prefetch(nxt, nxt_rj, nxt_x);
+    if (nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
+  }
   int iss_which = 0, iss_p = 0;
   int timeouts = 0;
 
@@ -587,8 +621,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   while (cur < total) {
     const int r = fast_div(cur, prm.div_nchunk);
     const int ch = cur - r * nchunk;
-    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r);
+    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, cur_x);
     const int clen = min(W, V - ch * W);
+    const bool has1 = (FLAGS & kFRow1) && L.row1 != nullptr;
     ThreadStat st0, st1;
     stat_init(st0);
     stat_init(st1);
@@ -610,7 +645,6 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       if (use_bulk) {
         if (!mbar_wait_bounded(&bars[s], ph)) ++timeouts;
       }
-      const bool has1 = (FLAGS & kFRow1) && L.row1 != nullptr;
       // Elements the bulk copy does not cover (the unaligned tail, or the whole
       // piece on the scalar path) and padding of the last vector.
       if (!use_bulk || n < kPiece) {
@@ -681,13 +715,19 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
         }
       }
       if ((FLAGS & kFStats1) && has1) {
+        // Row 1 moves to registers; the stage is refilled while its terms run.
         LaneRow<T1> R;
         lane_load(st1p, nv, R);
-        lane_stats(st1, R, lane_max(R), c);
+        const float pm1 = lane_max(R);
+        __syncwarp();
+        ++n_consumed;
+        top_up();
+        lane_stats(st1, R, pm1, c);
+      } else {
+        __syncwarp();
+        ++n_consumed;
+        top_up();
       }
-      __syncwarp();
-      ++n_consumed;
-      top_up();
     }
 
     // Per-item reduction and partial record.
@@ -695,11 +735,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     pr.G0 = pr.G1 = -INFINITY;
     pr.S0 = pr.S1 = 0.0;
     if (FLAGS & kFStats0) {
-      pr.G0 = warp_max(st0.ref);
+      pr.G0 = warp_max_redux(st0.ref);
       pr.S0 = warp_sum(rescale_pow2(st0.S, st0.ref, pr.G0));
     }
     if (FLAGS & kFStats1) {
-      pr.G1 = warp_max(st1.ref);
+      pr.G1 = warp_max_redux(st1.ref);
       pr.S1 = warp_sum(rescale_pow2(st1.S, st1.ref, pr.G1));
     }
     pr.key = kNoKey;
@@ -720,15 +760,16 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     pr.flags = flags;
     pr.pad = 0;
     if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)cur * K + lane] = list;
-    if (lane == 0) prm.part[cur] = pr;
     __syncwarp();
-    __threadfence();  // this item's partial and list before its count
     int last = 0;
     if (lane == 0) {
-      last = atomicAdd(&prm.row_counter[r], 1u) == (uint32_t)(nchunk - 1) ? 1 : 0;
-      if (last) __threadfence();
+      prm.part[cur] = pr;
+      // release: this item's partial and list before its count; acquire: the
+      // other items' records before the completing warp reads them
+      last = atom_add_acq_rel(&prm.row_counter[r], 1u) == (uint32_t)(nchunk - 1) ? 1 : 0;
     }
     last = __shfl_sync(0xffffffffu, last, 0);
+    __syncwarp();
     if (last) row_complete<T0, T1, FLAGS>(prm, r, L);
     timeouts = 0;
 
@@ -736,17 +777,13 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     cur = nxt;
     if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj);
     cur_np = nxt_np;
+    cur_x = __shfl_sync(0xffffffffu, nxt_x, 0);
     if (iss_which == 0) iss_p = 0;
     iss_which = 0;
-    if (cur < total) {
-      const int t = __shfl_sync(0xffffffffu, (int)pend, 0);
-      nxt = 2 * nwarps + t;
-    } else {
-      nxt = total;
-    }
+    nxt = cur < total ? 2 * nwarps + __shfl_sync(0xffffffffu, (int)pend, 0) : total;
     nxt_np = -1;
     if (lane == 0) {
-      nxt_rj = reject_word(nxt);
+      prefetch(nxt, nxt_rj, nxt_x);
       if (nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
     }
     top_up();
