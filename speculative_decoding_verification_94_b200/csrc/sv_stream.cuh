@@ -135,11 +135,9 @@ __device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r, int x
   return L;
 }
 
-// Add with acquire-release semantics at device scope (global memory).
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
+// Acquire-release fence at device scope.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // Warp maximum of a float through the integer reduction unit.
@@ -211,7 +209,8 @@ __device__ __forceinline__ unsigned long long row_topk_merge(const unsigned long
 // for chain rows, take the acceptance decision.  With kFTopk0 it also writes
 // the row's top-K outputs.
 template <class T0, class T1, int FLAGS>
-__device__ __noinline__ void row_complete(const StreamParams& prm, int r, const RowLoc& L) {
+__device__ __noinline__ void row_complete(const StreamParams& prm, int r, int x) {
+  const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, x);
   const int lane = threadIdx.x & 31;
   const int nchunk = prm.nchunk;
   Partial* base = prm.part + (size_t)r * nchunk;
@@ -617,6 +616,32 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     }
   };
 
+  // Deferred row counting.  sig_*: an item whose record is written but not
+  // yet counted; res_*: a count added whose result (lane 0) is not yet read.
+  int sig_r = -1, sig_x = -1, res_r = -1, res_x = -1;
+  uint32_t res_old = 0u;
+  auto resolve = [&]() {
+    if (res_r < 0) return;
+    const int last = __shfl_sync(0xffffffffu, res_old == (uint32_t)(nchunk - 1) ? 1 : 0, 0);
+    if (last) {
+      __threadfence();  // acquire: the other items' records
+      __syncwarp();
+      row_complete<T0, T1, FLAGS>(prm, res_r, res_x);
+    }
+    res_r = -1;
+  };
+  auto signal = [&]() {
+    if (sig_r < 0) return;
+    __syncwarp();
+    if (lane == 0) {
+      fence_acq_rel_gpu();  // release: the record (and list) before its count
+      res_old = atomicAdd(&prm.row_counter[sig_r], 1u);
+    }
+    res_r = sig_r;
+    res_x = sig_x;
+    sig_r = -1;
+  };
+
   top_up();
   while (cur < total) {
     const int r = fast_div(cur, prm.div_nchunk);
@@ -759,18 +784,15 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     if (__any_sync(0xffffffffu, timeouts != 0)) flags |= kPTimeout;
     pr.flags = flags;
     pr.pad = 0;
+    // Counting is deferred: the count of an item is added one item later,
+    // when its record has long been written (the release fence then costs
+    // little), and the returned count is read one item after that.
+    resolve();
+    signal();
     if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)cur * K + lane] = list;
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      prm.part[cur] = pr;
-      // release: this item's partial and list before its count; acquire: the
-      // other items' records before the completing warp reads them
-      last = atom_add_acq_rel(&prm.row_counter[r], 1u) == (uint32_t)(nchunk - 1) ? 1 : 0;
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    __syncwarp();
-    if (last) row_complete<T0, T1, FLAGS>(prm, r, L);
+    if (lane == 0) prm.part[cur] = pr;
+    sig_r = r;
+    sig_x = L.x;
     timeouts = 0;
 
     // Advance: nxt becomes current; the item after it comes from the counter.
@@ -788,6 +810,10 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     }
     top_up();
   }
+  // Count the last item and read the outstanding results.
+  resolve();
+  signal();
+  resolve();
   // Any copy still in flight (only after a timed-out wait) completes before exit.
   if (use_bulk && lane == 0)
     while (n_consumed < n_issued) {
