@@ -160,14 +160,14 @@ static int stream_chunk(int V, long long nrows) {
   return w < cap ? w : cap;
 }
 
-// Workspace: batch counter, per-request rejection words, per-row chunk
+// Workspace: batch and item counters, per-request rejection words, per-row chunk
 // counters, row records, chunk partials and (top-K) chunk lists.  Every byte
 // is zero between calls.
 static WsLayout ws_layout(int B, int nrows, int nchunk, int K) {
   WsLayout w;
   size_t o = 0;
   w.off_glob = o;
-  o += 16;
+  o += 256;  // batch counter (word 0) and the stream's item counters (words 32..63)
   w.off_reject = o;
   o = align_up(o + 4 * (size_t)B, 16);
   w.off_counter = o;
@@ -449,7 +449,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   sp.rec = w.rec;
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
-  sp.sched = w.glob + 1;
+  sp.sched = w.glob + 32;
   sp.status = device_status;
 
   FinishParams fp = {};
@@ -561,7 +561,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   sp.rec = w.rec;
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
-  sp.sched = w.glob + 1;
+  sp.sched = w.glob + 32;
   sp.status = device_status;
   cudaError_t e = dt == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
                                 : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
@@ -625,7 +625,7 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   sp.rec = w.rec;
   sp.row_counter = w.counter;
   sp.req_reject = w.reject;
-  sp.sched = w.glob + 1;
+  sp.sched = w.glob + 32;
   sp.status = device_status;
   sp.topk_logp = topk_logp;
   sp.topk_idx = topk_idx;
@@ -688,7 +688,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
     sp.rec = w.rec;
     sp.row_counter = w.counter;
     sp.req_reject = w.reject;
-  sp.sched = w.glob + 1;
+  sp.sched = w.glob + 32;
     sp.status = device_status;
     cudaError_t e = d_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFStats0>(sp, sg, s)
                                        : launch_stream<F32, F32, kFStats0>(sp, sg, s);

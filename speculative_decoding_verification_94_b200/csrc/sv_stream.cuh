@@ -32,6 +32,7 @@ constexpr int kLaneVecs = kPiece / (32 * kVec);  // 8-element vectors per lane p
 constexpr int kStages = 2;                    // ring depth per warp
 constexpr int kStreamWarps = 8;
 constexpr int kStreamThreads = kStreamWarps * 32;
+constexpr int kStripes = 32;                  // dynamic item counters (one per warp stripe)
 
 // What an item computes.
 enum StreamFlags : int {
@@ -101,7 +102,7 @@ struct StreamParams {
   int32_t* status;
   FastDiv div_nchunk;     // item -> row
   FastDiv div_B;          // chain row -> position
-  uint32_t* sched;        // [2]: dynamic item counter, exited warps (zero between calls)
+  uint32_t* sched;        // [kStripes] dynamic item counters (zero between calls)
 };
 
 // Where row r of a stream lives.
@@ -499,11 +500,14 @@ __device__ __forceinline__ void lane_stats(ThreadStat& st, const LaneRow<T>& R, 
 // The streaming kernel.
 //
 // Work distribution: warp g takes items g and g + NW first, then items
-// 2 NW + t in the order of a device-wide counter t, so the items run roughly
-// in index order (position-major for chains) and no warp waits on a slow
-// neighbour.  Lane 0 fetches the counter value of the item after next, and
-// that item's rejection word and draft token, when an item starts.  The last
-// warp to leave returns the counters to zero.
+// 2 NW + 32 t + (g mod 32) in the order of the counter t of its stripe
+// (g mod 32), so the items run roughly in index order (position-major for
+// chains) and no warp waits on a slow neighbour; 32 counters keep the atomic
+// traffic per address low.  Lane 0 fetches the counter value of the item
+// after next, and that item's rejection word and draft token, when an item
+// starts.  Every warp fetches until it draws an item past the end, so each
+// counter receives a known number of fetches; the fetch that returns the last
+// of them returns the counter to zero.
 // ---------------------------------------------------------------------------
 template <class T0, class T1, int FLAGS>
 __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_constant__ StreamParams prm) {
@@ -582,10 +586,29 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   }
   int nxt = gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
   uint32_t nxt_rj = 0u;
+  // Lane 0: the stripe counter and the number of fetches it will receive.
+  const int stripe = gwarp % kStripes;
+  uint32_t* const ctr = prm.sched + stripe;
+  uint32_t fetches = 0u;
+  {
+    const long long rest = (long long)total - 2LL * nwarps - stripe;
+    const long long valid = rest > 0 ? (rest + kStripes - 1) / kStripes : 0;
+    const int warps = nwarps / kStripes + (stripe < nwarps % kStripes ? 1 : 0);
+    fetches = (uint32_t)(valid + warps);
+  }
+  auto fetch = [&]() -> uint32_t {  // lane 0
+    const uint32_t t = atomicAdd(ctr, 1u);
+    if (t == fetches - 1u) *ctr = 0u;  // the last access of this call
+    return t;
+  };
+  auto dyn_item = [&](uint32_t t) -> int {
+    const long long d = 2LL * nwarps + (long long)t * kStripes + stripe;
+    return d < total ? (int)d : total;
+  };
   uint32_t pend = 0u;  // lane 0: counter value of the item after nxt
   if (lane == 0) {
     prefetch(nxt, nxt_rj, nxt_x);
-    if (nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
+    pend = fetch();  // every warp fetches at least once
   }
   int iss_which = 0, iss_p = 0;
   int timeouts = 0;
@@ -802,11 +825,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     cur_x = __shfl_sync(0xffffffffu, nxt_x, 0);
     if (iss_which == 0) iss_p = 0;
     iss_which = 0;
-    nxt = cur < total ? 2 * nwarps + __shfl_sync(0xffffffffu, (int)pend, 0) : total;
+    nxt = cur < total ? dyn_item(__shfl_sync(0xffffffffu, pend, 0)) : total;
     nxt_np = -1;
     if (lane == 0) {
       prefetch(nxt, nxt_rj, nxt_x);
-      if (nxt < total) pend = atomicAdd(&prm.sched[0], 1u);
+      if (nxt < total) pend = fetch();
     }
     top_up();
   }
@@ -820,15 +843,6 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       mbar_wait_bounded(&bars[n_consumed % kStages], (n_consumed / kStages) & 1u);
       ++n_consumed;
     }
-  // The last warp to leave returns the scheduling counters to zero.
-  if (lane == 0) {
-    __threadfence();
-    if (atomicAdd(&prm.sched[1], 1u) == (uint32_t)(nwarps - 1)) {
-      __threadfence();
-      prm.sched[0] = 0u;
-      prm.sched[1] = 0u;
-    }
-  }
 }
 
 }  // namespace sv
