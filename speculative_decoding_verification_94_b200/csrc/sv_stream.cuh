@@ -1,26 +1,27 @@
 // sv_stream.cuh -- the streaming pass shared by every entry point.
 //
 // Every warp is an independent worker.  Work items are chunks of W vocabulary
-// entries of one row (or of a target/draft row pair, read together); warp g
-// takes items g, g + NW, g + 2NW, ... (NW warps in the grid), so items are
-// processed roughly in index order.  Chain items are numbered position-major
-// (every request's position 0 first): an item whose request has already
-// rejected at an earlier position is skipped before any byte is loaded, so
-// once a request's fate is known its later rows are never read.
+// entries of one row (or of a target/draft row pair, read together), handed
+// out roughly in index order (static first items, then per-stripe counters;
+// see stream_kernel).  Chain items are numbered position-major (every
+// request's position 0 first): an item whose request has already rejected at
+// an earlier position is skipped before any byte is loaded, so once a
+// request's fate is known its later rows are not read.
 //
 // A warp streams its items through its own ring of kStages pieces of kPiece
 // elements; lane 0 issues bulk copies (cp.async.bulk, no multicast) up to
 // kStages pieces ahead, across item boundaries, and each piece completes on its
-// own mbarrier.  Per item the warp keeps online softmax statistics (sv_device
-// ThreadStat: exact power-of-two rescales), the element at the draft token,
-// the argmax, and a sorted warp list of the K best keys, reduces them with
-// shuffles, writes one partial record and counts the chunk into its row.  The
-// warp that completes a row combines the row's partials in chunk order (so
+// own mbarrier.  Each lane moves its share of a piece to registers and keeps
+// online softmax statistics (ThreadStat: exact power-of-two rescales), the
+// element at the draft token, the argmax, and a sorted warp list of the K best
+// keys; per item these are reduced with shuffles into one partial record.
+// Items are counted into their row one item late (deferred counting); the warp
+// whose count completes a row combines the row's partials in chunk order (so
 // the result does not depend on which warp finished last) and records the
 // row's normaliser and, for chain rows, the acceptance decision.
 //
 // No __syncthreads, no cluster barrier and no shared-memory residency: the
-// only cross-warp communication is the per-row counter and the records.
+// only cross-warp communication is the counters and the records.
 #pragma once
 
 #include "sv_device.cuh"
@@ -503,9 +504,9 @@ __device__ __forceinline__ void lane_stats(ThreadStat& st, const LaneRow<T>& R, 
 // 2 NW + 32 t + (g mod 32) in the order of the counter t of its stripe
 // (g mod 32), so the items run roughly in index order (position-major for
 // chains) and no warp waits on a slow neighbour; 32 counters keep the atomic
-// traffic per address low.  Lane 0 fetches the counter value of the item
-// after next, and that item's rejection word and draft token, when an item
-// starts.  Every warp fetches until it draws an item past the end, so each
+// traffic per address low.  A warp knows its next three items; the counter
+// value, rejection word and draft token of each are read an item before they
+// are used.  Every warp fetches until it draws an item past the end, so each
 // counter receives a known number of fetches; the fetch that returns the last
 // of them returns the counter to zero.
 // ---------------------------------------------------------------------------
@@ -605,10 +606,21 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     const long long d = 2LL * nwarps + (long long)t * kStripes + stripe;
     return d < total ? (int)d : total;
   };
-  uint32_t pend = 0u;  // lane 0: counter value of the item after nxt
+  // Three items ahead are known: cur, nxt and nxt2.  nxt's rejection word and
+  // token were read one item before they are needed; nxt2's are in flight;
+  // pend (the counter value of the item after nxt2) was fetched one item
+  // before it is read.
+  int nxt2 = total, nxt2_x = -1;  // nxt2_x: lane 0 only
+  uint32_t nxt2_rj = 0u;
+  uint32_t pend = 0u;  // lane 0
   if (lane == 0) {
     prefetch(nxt, nxt_rj, nxt_x);
     pend = fetch();  // every warp fetches at least once
+  }
+  nxt2 = dyn_item(__shfl_sync(0xffffffffu, pend, 0));
+  if (lane == 0) {
+    prefetch(nxt2, nxt2_rj, nxt2_x);
+    if (nxt2 < total) pend = fetch();
   }
   int iss_which = 0, iss_p = 0;
   int timeouts = 0;
@@ -825,11 +837,14 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     cur_x = __shfl_sync(0xffffffffu, nxt_x, 0);
     if (iss_which == 0) iss_p = 0;
     iss_which = 0;
-    nxt = cur < total ? dyn_item(__shfl_sync(0xffffffffu, pend, 0)) : total;
+    nxt = nxt2;
     nxt_np = -1;
+    nxt_rj = nxt2_rj;
+    nxt_x = nxt2_x;
+    nxt2 = nxt2 < total ? dyn_item(__shfl_sync(0xffffffffu, pend, 0)) : total;
     if (lane == 0) {
-      prefetch(nxt, nxt_rj, nxt_x);
-      if (nxt < total) pend = fetch();
+      prefetch(nxt2, nxt2_rj, nxt2_x);
+      if (nxt2 < total) pend = fetch();
     }
     top_up();
   }
