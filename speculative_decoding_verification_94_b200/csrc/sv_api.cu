@@ -217,8 +217,19 @@ static StreamGeom stream_geom(int V, long long nrows, int te, int de) {
   return g;
 }
 
+// In-stream row counting (count = -1: decide here).  It only pays when a
+// chain's positions run one after another, letting rows after a rejection be
+// skipped: every position must span at least three rounds of the resident
+// warps.  Otherwise the finisher completes the rows and the stream spends
+// nothing per item on counting.
+static int stream_count_policy(const StreamParams& p, long long resident_warps) {
+  const int forced = env_int("SV_STREAM_COUNT");
+  if (forced == 1 || forced == 2) return forced - 1;  // 1: off, 2: on
+  return (long long)p.B * p.nchunk >= 3 * resident_warps ? 1 : 0;
+}
+
 template <class T0, class T1, int FLAGS>
-static cudaError_t launch_stream(StreamParams p, const StreamGeom& g, cudaStream_t s) {
+static cudaError_t launch_stream(StreamParams& p, const StreamGeom& g, cudaStream_t s) {
   auto kernel = stream_kernel<T0, T1, FLAGS>;
   const void* kp = reinterpret_cast<const void*>(kernel);
   cudaError_t e = ensure_kernel_attrs(kp, g.smem, false);
@@ -232,6 +243,7 @@ static cudaError_t launch_stream(StreamParams p, const StreamGeom& g, cudaStream
   const long long need = (items + kStreamWarps - 1) / kStreamWarps;
   if (need < grid) grid = need;
   if (grid < 1) grid = 1;
+  if (p.count < 0) p.count = stream_count_policy(p, (long long)per_sm * sms * kStreamWarps);
   kernel<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
   return cudaGetLastError();
 }
@@ -329,7 +341,7 @@ static cudaError_t pick_plan(K kernel, const RowPlan* plans, int np, int ncluste
 }
 
 template <class TT, class DT, int DKIND>
-static cudaError_t run_chain_sample(const StreamParams& sp, const StreamGeom& sg, FinishParams fp,
+static cudaError_t run_chain_sample(StreamParams sp, const StreamGeom& sg, FinishParams fp,
                                     const RowPlan* plans, int np, bool kd, cudaStream_t s) {
   // probability drafts are not streamed: q(x) is read directly
   constexpr int base = kFStats0 | kFGather | (DKIND == kDraftLogits ? (kFRow1 | kFStats1) : 0);
@@ -340,8 +352,10 @@ static cudaError_t run_chain_sample(const StreamParams& sp, const StreamGeom& sg
   fp.L = plan.L;
   fp.use_bulk = plan.use_bulk;
   fp.lay = plan.lay;
+  static_assert(base == chain_sample_flags<DKIND, false>(), "stream and finisher flags");
   e = kd ? launch_stream<TT, DT, base | kFTopk0>(sp, sg, s) : launch_stream<TT, DT, base>(sp, sg, s);
   if (e != cudaSuccess) return e;
+  fp.sp = sp;
   return launch_clusters(fin, fp, plan, fp.B, s);
 }
 
@@ -426,6 +440,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   StreamParams sp = {};
+  sp.count = -1;  // decided at launch
   sp.rows0 = target_logits;
   sp.rows1 = greedy ? nullptr : draft;
   sp.tokens = draft_tokens;
@@ -492,7 +507,9 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
     cudaError_t e = t_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
                                        : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
     if (e != cudaSuccess) return SV_ERR_CUDA;
-    return cuda_status(launch_blocks(chain_greedy_finish, fp, (B + kWarps - 1) / kWarps, 0, s));
+    fp.sp = sp;
+    return cuda_status(t_dtype == SV_BF16 ? launch_blocks(chain_greedy_finish<BF16>, fp, B, 0, s)
+                                          : launch_blocks(chain_greedy_finish<F32>, fp, B, 0, s));
   }
 
   RowPlan plans[8];
@@ -563,6 +580,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   sp.req_reject = w.reject;
   sp.sched = w.glob + 32;
   sp.status = device_status;
+  sp.count = 0;  // no skipping in a tree: the finisher completes the rows
   cudaError_t e = dt == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
                                 : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
   if (e != cudaSuccess) return SV_ERR_CUDA;
@@ -581,7 +599,9 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   fp.rec = w.rec;
   fp.req_reject = w.reject;
   fp.status = device_status;
-  return cuda_status(launch_blocks(tree_finish, fp, B, kFixedBytes + 4 * n * 4, s));
+  fp.sp = sp;
+  return cuda_status(dt == SV_BF16 ? launch_blocks(tree_finish<BF16>, fp, B, kFixedBytes + 4 * n * 4, s)
+                                   : launch_blocks(tree_finish<F32>, fp, B, kFixedBytes + 4 * n * 4, s));
 }
 
 sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, int K,
@@ -630,6 +650,7 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   sp.topk_logp = topk_logp;
   sp.topk_idx = topk_idx;
   sp.lse = lse;
+  sp.count = 1;  // no finishing kernel: rows complete in the stream
   // one pass: the warp that completes a row merges its chunk lists and writes it
   return cuda_status(dt == SV_BF16 ? launch_stream<BF16, BF16, kFStats0 | kFTopk0>(sp, sg, s)
                                    : launch_stream<F32, F32, kFStats0 | kFTopk0>(sp, sg, s));
@@ -666,8 +687,8 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   const WsPtrs w = ws_carve(workspace, wl);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const float c = (float)(1.4426950408889634 / (double)temperature);
+  StreamParams sp = {};
   if (d_kind == SV_DRAFT_LOGITS) {
-    StreamParams sp = {};
     sp.rows0 = draft;
     sp.kind = kKindRows;
     sp.B = B * k;
@@ -676,8 +697,8 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
     sp.nrows = B * k;
     sp.W = sg.W;
     sp.nchunk = sg.nchunk;
-  sp.div_nchunk = make_fastdiv(sg.nchunk);
-  sp.div_B = make_fastdiv(sp.B);
+    sp.div_nchunk = make_fastdiv(sg.nchunk);
+    sp.div_B = make_fastdiv(sp.B);
     sp.c = c;
     sp.use_bulk = bulk_ok_row(draft, V, esize(d_dtype));
     sp.K = 1;
@@ -688,8 +709,9 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
     sp.rec = w.rec;
     sp.row_counter = w.counter;
     sp.req_reject = w.reject;
-  sp.sched = w.glob + 32;
+    sp.sched = w.glob + 32;
     sp.status = device_status;
+    sp.count = 0;  // the finisher completes the draft rows
     cudaError_t e = d_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFStats0>(sp, sg, s)
                                        : launch_stream<F32, F32, kFStats0>(sp, sg, s);
     if (e != cudaSuccess) return SV_ERR_CUDA;
@@ -718,6 +740,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   fp.req_reject = w.reject;
   fp.glob_counter = w.glob;
   fp.status = device_status;
+  fp.sp = sp;
   cudaError_t e = (d_dtype == SV_BF16) ? launch_blocks(kl_finish<BF16>, fp, B, kFixedBytes, s)
                                        : launch_blocks(kl_finish<F32>, fp, B, kFixedBytes, s);
   return cuda_status(e);

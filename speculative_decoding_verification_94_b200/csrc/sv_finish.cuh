@@ -55,7 +55,17 @@ struct FinishParams {
   uint32_t* req_reject;
   uint32_t* glob_counter;
   int32_t* status;
+  // the stream's parameters: rows it did not complete (sp.count == 0) are
+  // completed here first
+  StreamParams sp;
 };
+
+// Stream flags of the sampling chain (they fix what a row completion does).
+template <int DKIND, bool KD>
+constexpr int chain_sample_flags() {
+  return kFStats0 | kFGather | (DKIND == kDraftLogits ? (kFRow1 | kFStats1) : 0) |
+         (KD ? kFTopk0 : 0);
+}
 
 template <class TT, class DT, int DKIND>
 __device__ __forceinline__ void weights8(const unsigned char* tbuf, const unsigned char* dbuf,
@@ -126,7 +136,7 @@ __device__ __forceinline__ void zero_recs(const FinishParams& p, size_t r0, int 
 }
 
 template <class TT, class DT, int DKIND, bool KD>
-__global__ void __launch_bounds__(kThreads) chain_sample_finish(const FinishParams prm) {
+__global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
@@ -140,6 +150,16 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const FinishPara
   const ChunkGeom g = chunk_geom(rank, prm.L, V);
   const float c = prm.c;
   const bool use_bulk = prm.use_bulk != 0;
+
+  // 0. rows 0..k of the request, when the stream left them to this kernel
+  if (!prm.sp.count) {
+    const int w = threadIdx.x >> 5;
+    for (int t = rank * kWarps + w; t < P; t += C * kWarps)
+      row_complete<TT, DT, chain_sample_flags<DKIND, KD>()>(
+          prm.sp, t * B + b, t < k ? prm.tokens[(size_t)b * k + t] : -1);
+    if (threadIdx.x == 0) __threadfence();
+    cluster.sync();
+  }
 
   if (threadIdx.x < 32) {
     bool bad;
@@ -329,12 +349,20 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const FinishPara
                 prm.total, prm.glob_counter, sh);
 }
 
-// Greedy chain: one warp per request.
-__global__ void __launch_bounds__(kThreads) chain_greedy_finish(const FinishParams prm) {
-  const int lane = threadIdx.x & 31;
-  const int b = (int)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (b >= prm.B) return;
+// Greedy chain: one block per request (its warps complete the request's rows
+// when the stream left them; warp 0 takes the decision).
+template <class T>
+__global__ void __launch_bounds__(kThreads) chain_greedy_finish(const __grid_constant__ FinishParams prm) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int b = (int)blockIdx.x;
   const int k = prm.k, P = k + 1, B = prm.B;
+  if (!prm.sp.count) {
+    for (int t = w; t < P; t += kWarps)
+      row_complete<T, T, kFArgmax0>(prm.sp, t * B + b, t < k ? prm.tokens[(size_t)b * k + t] : -1);
+    __threadfence();
+    __syncthreads();
+  }
+  if (w != 0) return;
   bool bad = false;
   const int n = warp_first_rejection(prm.rec, B, k, b, &bad);
   const int tok = __ldcg(&prm.rec[(size_t)n * B + b].argmax);
@@ -353,11 +381,18 @@ __global__ void __launch_bounds__(kThreads) chain_greedy_finish(const FinishPara
 }
 
 // Greedy tree: one block per request; node rows are rows b * n + j.
-__global__ void __launch_bounds__(kThreads) tree_finish(const FinishParams prm) {
+template <class T>
+__global__ void __launch_bounds__(kThreads) tree_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
   const int n = prm.k, V = prm.V;
   const int b = (int)blockIdx.x;
+  if (!prm.sp.count) {
+    for (int t = threadIdx.x >> 5; t < n; t += kWarps)
+      row_complete<T, T, kFArgmax0>(prm.sp, b * n + t, -1);
+    __threadfence();
+    __syncthreads();
+  }
   int* garg = reinterpret_cast<int*>(smem + kFixedBytes);
   int* par = garg + n;
   int* tok = par + n;
@@ -424,12 +459,17 @@ __global__ void __launch_bounds__(kThreads) tree_finish(const FinishParams prm) 
 // rows stream first (logits) so that rec holds their normalisers; probability
 // drafts have no stream pass.
 template <class DT>
-__global__ void __launch_bounds__(kThreads) kl_finish(const FinishParams prm) {
+__global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int b = (int)blockIdx.x;
   const int k = prm.k, P = k + 1, B = prm.B, V = prm.V, K = prm.K;
+  if (!prm.draft_probs && !prm.sp.count) {
+    for (int t = w; t < k; t += kWarps) row_complete<DT, DT, kFStats0>(prm.sp, b * k + t, -1);
+    __threadfence();
+    __syncthreads();
+  }
   const double ln2 = 0.69314718055994530942;
   const double c = (double)prm.c;
   for (int i = w; i < k; i += kWarps) {

@@ -61,6 +61,7 @@ struct __align__(16) Partial {
   unsigned long long key;  // argmax key of row 0
 };
 enum : int { kPHasX = 1, kPSkipped = 2, kPTimeout = 4 };
+static_assert(sizeof(Partial) == 48, "chunk record layout");
 
 // Row record written by the warp that completes a row.
 struct __align__(16) RowRec {
@@ -104,6 +105,9 @@ struct StreamParams {
   FastDiv div_nchunk;     // item -> row
   FastDiv div_B;          // chain row -> position
   uint32_t* sched;        // [kStripes] dynamic item counters (zero between calls)
+  int count;              // 1: items are counted into rows and rows completed here
+                          //    (required for skipping); 0: partials only, rows are
+                          //    completed by the finishing kernel
 };
 
 // Where row r of a stream lives.
@@ -113,6 +117,17 @@ struct RowLoc {
   const unsigned char* row1;
   int x;               // chain: draft token of this row (-1 for the bonus row / none)
 };
+
+// A chunk record read through L2 in three 16-byte loads.
+__device__ __forceinline__ Partial load_partial(const Partial* p) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  const uint4 a = __ldcg(q), b = __ldcg(q + 1), c = __ldcg(q + 2);
+  Partial r;
+  memcpy(reinterpret_cast<unsigned char*>(&r), &a, 16);
+  memcpy(reinterpret_cast<unsigned char*>(&r) + 16, &b, 16);
+  memcpy(reinterpret_cast<unsigned char*>(&r) + 32, &c, 16);
+  return r;
+}
 
 // Row pointers of row r (the draft token is supplied separately).
 template <class T0, class T1, int FLAGS>
@@ -216,31 +231,43 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, int x)
   const int lane = threadIdx.x & 31;
   const int nchunk = prm.nchunk;
   Partial* base = prm.part + (size_t)r * nchunk;
+  // One pass: lane l folds chunks l, l + 32, ... in order into a running
+  // (reference, sum) pair; the power-of-two rescales are exact, so the sums
+  // equal those of a fold at the final reference.  Two records per lane are
+  // loaded at a time.
   float g0 = -INFINITY, g1 = -INFINITY, zx0 = 0.f, zx1 = 0.f;
+  double s0 = 0.0, s1 = 0.0;
   int flags = 0, hx = 0;
   unsigned long long key = kNoKey;
-  for (int q = lane; q < nchunk; q += 32) {
-    const Partial* pq = base + q;
-    g0 = fmaxf(g0, __ldcg(&pq->G0));
-    g1 = fmaxf(g1, __ldcg(&pq->G1));
-    const int f = __ldcg(&pq->flags);
-    flags |= f;
-    if (f & kPHasX) {
-      hx = 1;
-      zx0 = __ldcg(&pq->zx0);
-      zx1 = __ldcg(&pq->zx1);
+  auto fold = [&](const Partial& pq) {
+    if (pq.G0 > g0) {
+      s0 = rescale_pow2(s0, g0, pq.G0);
+      g0 = pq.G0;
     }
-    const unsigned long long kq = __ldcg(&pq->key);
-    key = kq > key ? kq : key;
+    s0 += rescale_pow2(pq.S0, pq.G0, g0);
+    if (pq.G1 > g1) {
+      s1 = rescale_pow2(s1, g1, pq.G1);
+      g1 = pq.G1;
+    }
+    s1 += rescale_pow2(pq.S1, pq.G1, g1);
+    flags |= pq.flags;
+    if (pq.flags & kPHasX) {
+      hx = 1;
+      zx0 = pq.zx0;
+      zx1 = pq.zx1;
+    }
+    key = pq.key > key ? pq.key : key;
+  };
+  for (int q = lane; q < nchunk; q += 64) {
+    const Partial pa = load_partial(base + q);
+    const bool two = q + 32 < nchunk;
+    const Partial pb = two ? load_partial(base + q + 32) : Partial{};
+    fold(pa);
+    if (two) fold(pb);
   }
   const float G0 = warp_max(g0), G1 = warp_max(g1);
-  double s0 = 0.0, s1 = 0.0;
-  for (int q = lane; q < nchunk; q += 32) {
-    const Partial* pq = base + q;
-    s0 += rescale_pow2(__ldcg(&pq->S0), __ldcg(&pq->G0), G0);
-    s1 += rescale_pow2(__ldcg(&pq->S1), __ldcg(&pq->G1), G1);
-  }
-  const double S0 = warp_sum(s0), S1 = warp_sum(s1);  // (every lane has read its partials)
+  const double S0 = warp_sum(rescale_pow2(s0, g0, G0)), S1 = warp_sum(rescale_pow2(s1, g1, G1));
+  // (every lane has read its records)
   for (int q = lane; q < nchunk; q += 32) base[q] = Partial{};
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) flags |= __shfl_xor_sync(0xffffffffu, flags, o);
@@ -539,7 +566,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     if (!chain || item >= total) return;
     const int r = fast_div(item, prm.div_nchunk);
     const int i = fast_div(r, prm.div_B), b = r - i * prm.B;
-    rj = load_relaxed_u32(&prm.req_reject[b]);
+    if (prm.count) rj = load_relaxed_u32(&prm.req_reject[b]);
     if (i < prm.k) x = prm.tokens[(size_t)b * prm.k + i];
   };
   // Pieces of an item (lane-uniform); 0 when skipped: an earlier position of
@@ -597,12 +624,14 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     const int warps = nwarps / kStripes + (stripe < nwarps % kStripes ? 1 : 0);
     fetches = (uint32_t)(valid + warps);
   }
-  auto fetch = [&]() -> uint32_t {  // lane 0
-    const uint32_t t = atomicAdd(ctr, 1u);
-    if (t == fetches - 1u) *ctr = 0u;  // the last access of this call
-    return t;
+  auto fetch = [&]() -> uint32_t {  // lane 0; the result is read an item later
+    return atomicAdd(ctr, 1u);
   };
-  auto dyn_item = [&](uint32_t t) -> int {
+  // The item of a fetched counter value (read by every lane from lane 0).  The
+  // lane that holds the last value of this call returns the counter to zero.
+  auto take = [&](uint32_t t0) -> int {
+    if (lane == 0 && t0 == fetches - 1u) *ctr = 0u;
+    const uint32_t t = __shfl_sync(0xffffffffu, t0, 0);
     const long long d = 2LL * nwarps + (long long)t * kStripes + stripe;
     return d < total ? (int)d : total;
   };
@@ -617,7 +646,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     prefetch(nxt, nxt_rj, nxt_x);
     pend = fetch();  // every warp fetches at least once
   }
-  nxt2 = dyn_item(__shfl_sync(0xffffffffu, pend, 0));
+  nxt2 = take(pend);
   if (lane == 0) {
     prefetch(nxt2, nxt2_rj, nxt2_x);
     if (nxt2 < total) pend = fetch();
@@ -820,10 +849,12 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     pr.flags = flags;
     pr.pad = 0;
     // Counting is deferred: the count of an item is added one item later,
-    // when its record has long been written (the release fence then costs
-    // little), and the returned count is read one item after that.
-    resolve();
-    signal();
+    // when its record has long been written, and the returned count is read
+    // one item after that.
+    if (prm.count) {
+      resolve();
+      signal();
+    }
     if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)cur * K + lane] = list;
     if (lane == 0) prm.part[cur] = pr;
     sig_r = r;
@@ -841,7 +872,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     nxt_np = -1;
     nxt_rj = nxt2_rj;
     nxt_x = nxt2_x;
-    nxt2 = nxt2 < total ? dyn_item(__shfl_sync(0xffffffffu, pend, 0)) : total;
+    nxt2 = nxt2 < total ? take(pend) : total;
     if (lane == 0) {
       prefetch(nxt2, nxt2_rj, nxt2_x);
       if (nxt2 < total) pend = fetch();
@@ -849,9 +880,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     top_up();
   }
   // Count the last item and read the outstanding results.
-  resolve();
-  signal();
-  resolve();
+  if (prm.count) {
+    resolve();
+    signal();
+    resolve();
+  }
   // Any copy still in flight (only after a timed-out wait) completes before exit.
   if (use_bulk && lane == 0)
     while (n_consumed < n_issued) {
