@@ -213,7 +213,8 @@ static StreamGeom stream_geom(int V, long long nrows, int te, int de) {
   g.nchunk = (V + g.W - 1) / g.W;
   g.stage_off1 = (int)align_up((size_t)kPiece * te, 128);
   g.stage_bytes = g.stage_off1 + (int)align_up((size_t)kPiece * de, 128);
-  g.smem = kStreamWarps * kStages * g.stage_bytes + kStreamWarps * kStages * 8;
+  g.smem = kStreamWarps * kStages * g.stage_bytes + kStreamWarps * kStages * 8 +
+           kStreamWarps * 2 * (int)sizeof(IssueDesc);
   return g;
 }
 

@@ -74,6 +74,15 @@ struct __align__(16) RowRec {
 enum RowCode : int { kRowNone = 0, kRowAccepted = 1, kRowRejected = 2, kRowSkipped = 3,
                      kRowError = 4 };
 
+// Where the bulk copies of an item come from (lane 0 of a warp, in shared
+// memory): its two rows at the chunk start and the chunk length.
+struct IssueDesc {
+  const unsigned char* src0;
+  const unsigned char* src1;  // nullptr: row 1 not streamed
+  int len;
+  int pad;
+};
+
 struct StreamParams {
   const void* rows0;      // row-0 array: target logits (chain, rows) or draft logits (KL)
   const void* rows1;      // row-1 array: draft logits / probabilities (chain sample)
@@ -544,6 +553,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   unsigned char* ring = smem + (size_t)warp * kStages * prm.stage_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kStreamWarps * kStages * prm.stage_bytes) +
                    warp * kStages;
+  IssueDesc* desc = reinterpret_cast<IssueDesc*>(smem + (size_t)kStreamWarps * kStages * prm.stage_bytes +
+                                                 (size_t)kStreamWarps * kStages * 8) +
+                    warp * 2;
   const bool use_bulk = prm.use_bulk != 0;
   const bool chain = prm.kind != kKindRows;
   const int V = prm.V, W = prm.W, nchunk = prm.nchunk;
@@ -570,8 +582,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     if (i < prm.k) x = prm.tokens[(size_t)b * prm.k + i];
   };
   // Pieces of an item (lane-uniform); 0 when skipped: an earlier position of
-  // its request rejected.
-  auto pieces_of = [&](int item, uint32_t rj) -> int {
+  // its request rejected.  Lane 0 records the item's copy sources in
+  // descriptor `slot`.
+  auto pieces_of = [&](int item, uint32_t rj, int slot) -> int {
     if (item >= total) return 0;
     const int r = fast_div(item, prm.div_nchunk);
     const int ch = item - r * nchunk;
@@ -581,27 +594,33 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       skip = __shfl_sync(0xffffffffu, rj > (uint32_t)(prm.k - i) ? 1 : 0, 0);
     }
     const int len = min(W, V - ch * W);
+    if (lane == 0 && !skip) {
+      const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, -1);
+      IssueDesc d;
+      d.src0 = L.row0 + (size_t)ch * W * T0::bytes;
+      d.src1 = ((FLAGS & kFRow1) && L.row1 != nullptr) ? L.row1 + (size_t)ch * W * T1::bytes : nullptr;
+      d.len = len;
+      d.pad = 0;
+      desc[slot] = d;
+    }
     return skip ? 0 : (len + kPiece - 1) / kPiece;
   };
 
-  // Lane 0: bulk copies of piece p of an item into ring stage s.
-  auto issue = [&](int item, int p, int s) {
-    const int r = fast_div(item, prm.div_nchunk);
-    const int ch = item - r * nchunk;
-    const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, -1);
-    const int e0 = ch * W + p * kPiece;
-    const int n = min(kPiece, min(V, ch * W + W) - e0);
+  // Lane 0: bulk copies of piece p of the item in descriptor `slot` into ring
+  // stage s.
+  auto issue = [&](int slot, int p, int s) {
+    const IssueDesc d = desc[slot];
+    const int e0 = p * kPiece;
+    const int n = min(kPiece, d.len - e0);
     const uint32_t nb0 = (uint32_t)(n * T0::bytes) & ~15u;
-    const uint32_t nb1 =
-        ((FLAGS & kFRow1) && L.row1 != nullptr) ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
+    const uint32_t nb1 = d.src1 != nullptr ? ((uint32_t)(n * T1::bytes) & ~15u) : 0u;
     unsigned char* st = ring + (size_t)s * prm.stage_bytes;
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&bars[s], nb0 + nb1);
-    if (nb0)
-      bulk_g2s_plain(st, L.row0 + (size_t)e0 * T0::bytes, nb0, &bars[s]);
-    if (nb1)
-      bulk_g2s_plain(st + prm.stage_off1, L.row1 + (size_t)e0 * T1::bytes, nb1, &bars[s]);
+    if (nb0) bulk_g2s_plain(st, d.src0 + (size_t)e0 * T0::bytes, nb0, &bars[s]);
+    if (nb1) bulk_g2s_plain(st + prm.stage_off1, d.src1 + (size_t)e0 * T1::bytes, nb1, &bars[s]);
   };
+  int slot_cur = 0;  // descriptor of cur; nxt uses the other
 
   uint32_t n_issued = 0, n_consumed = 0;
   int cur = gwarp, cur_np, cur_x;
@@ -609,7 +628,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     uint32_t rj;
     int x;
     if (lane == 0) prefetch(cur, rj, x);
-    cur_np = pieces_of(cur, rj);
+    cur_np = pieces_of(cur, rj, 0);
     cur_x = __shfl_sync(0xffffffffu, x, 0);
   }
   int nxt = gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
@@ -659,7 +678,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       int it, pp;
       if (iss_which == 0) {
         if (iss_p < cur_np) {
-          it = cur;
+          it = slot_cur;
           pp = iss_p++;
         } else {
           iss_which = 1;
@@ -667,9 +686,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
           continue;
         }
       } else {
-        if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj);
+        if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj, slot_cur ^ 1);
         if (iss_p < nxt_np) {
-          it = nxt;
+          it = slot_cur ^ 1;
           pp = iss_p++;
         } else {
           break;
@@ -863,7 +882,8 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
 
     // Advance: nxt becomes current; the item after it comes from the counter.
     cur = nxt;
-    if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj);
+    if (nxt_np < 0) nxt_np = pieces_of(nxt, nxt_rj, slot_cur ^ 1);
+    slot_cur ^= 1;
     cur_np = nxt_np;
     cur_x = __shfl_sync(0xffffffffu, nxt_x, 0);
     if (iss_which == 0) iss_p = 0;
