@@ -65,8 +65,28 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+def rank_seed(rank: int) -> int:
+    """Each replica verifies its own batch (weak scaling)."""
+    return 1000 * rank
+
+
+def reduce_max(values, dist, device):
+    """Element-wise maximum over ranks of a list of floats (timing only; no
+    data-path collective).  Every rank must call it in the same order."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_value(rows_per_rank: int, world: int, steps: int, ms_total: float) -> float:
+    """Whole-job rows/s: the rows every rank verified over the slowest rank's time."""
+    return rows_per_rank * world * steps / (ms_total * 1e-3)
+
+
 def make_workload(a, rank):
-    seed = 1000 * rank
+    seed = rank_seed(rank)
     if a.workload == "qwen_chain":
         B = a.B or 32
         k = a.k or 3
@@ -338,10 +358,7 @@ def main():
     ms_total = start.elapsed_time(end)
     ms_launch = ms_total / a.steps  # one verification call (stream + finish kernels) per step
     clk = clocks.stop(tw0, tw1)
-    if dist is not None:
-        tt = torch.tensor([ms_total, ms_launch], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, ms_launch = float(tt[0]), float(tt[1])
+    ms_total, ms_launch = reduce_max([ms_total, ms_launch], dist, dev)
     st = int(status.item())
     assert st & sv.SV_DEV_ERROR_MASK == 0, f"device status {st:#x}"
 
@@ -349,7 +366,7 @@ def main():
     full_bytes = algo_bytes
     algo_bytes = needed_bytes(kind, x, outs["accepted_len"].cpu().numpy())
     achieved = algo_bytes / (ms_launch * 1e-3) / 1e9
-    value = rows * world * a.steps / (ms_total * 1e-3)
+    value = job_value(rows, world, a.steps, ms_total)
 
     # end to end through the public call: pinned host inputs -> device, verify,
     # results -> pinned host, all inside the timed region.
@@ -386,11 +403,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ms_e2e = e0.elapsed_time(e1)
-        if dist is not None:
-            tt = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms_e2e = float(tt[0])
-        e2e = {"value": rows * world * n_e2e / (ms_e2e * 1e-3), "unit": UNIT,
+        (ms_e2e,) = reduce_max([ms_e2e], dist, dev)
+        e2e = {"value": job_value(rows, world, n_e2e, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
 
