@@ -160,6 +160,10 @@ static int stream_chunk(int V, long long nrows) {
   return w < cap ? w : cap;
 }
 
+// Record slots per row: one per piece, enough for either schedule (a record
+// per chunk of W >= kPiece elements, or one per run of pieces).
+static int record_slots(int V) { return (V + kPiece - 1) / kPiece; }
+
 // Workspace: batch and item counters, per-request rejection words, per-row chunk
 // counters, row records, chunk partials and (top-K) chunk lists.  Every byte
 // is zero between calls.
@@ -231,21 +235,33 @@ static int stream_count_policy(const StreamParams& p, long long resident_warps) 
 
 template <class T0, class T1, int FLAGS>
 static cudaError_t launch_stream(StreamParams& p, const StreamGeom& g, cudaStream_t s) {
-  auto kernel = stream_kernel<T0, T1, FLAGS>;
-  const void* kp = reinterpret_cast<const void*>(kernel);
-  cudaError_t e = ensure_kernel_attrs(kp, g.smem, false);
+  auto kd = stream_kernel<T0, T1, FLAGS>;             // dynamic items, in-stream counting
+  auto ks = stream_kernel<T0, T1, FLAGS | kFStatic>;  // static partition
+  cudaError_t e = ensure_kernel_attrs(reinterpret_cast<const void*>(kd), g.smem, false);
   if (e != cudaSuccess) return e;
+  if ((e = ensure_kernel_attrs(reinterpret_cast<const void*>(ks), g.smem, false)) != cudaSuccess)
+    return e;
   int per_sm = 0, sms = 0;
-  if ((e = blocks_per_sm(kp, kStreamThreads, g.smem, &per_sm)) != cudaSuccess) return e;
+  if ((e = blocks_per_sm(reinterpret_cast<const void*>(kd), kStreamThreads, g.smem, &per_sm)) !=
+      cudaSuccess)
+    return e;
   if ((e = sm_count(&sms)) != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  if (p.count < 0) p.count = stream_count_policy(p, (long long)per_sm * sms * kStreamWarps);
+  if (p.count == 0) {  // static partition into pieces (one record slot each)
+    p.W = kPiece;
+    p.nchunk = record_slots(p.V);
+    p.div_nchunk = make_fastdiv(p.nchunk);
+  }
   const long long items = (long long)p.nrows * p.nchunk;
   long long grid = (long long)per_sm * sms;
   const long long need = (items + kStreamWarps - 1) / kStreamWarps;
   if (need < grid) grid = need;
   if (grid < 1) grid = 1;
-  if (p.count < 0) p.count = stream_count_policy(p, (long long)per_sm * sms * kStreamWarps);
-  kernel<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
+  if (p.count == 0)
+    ks<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
+  else
+    kd<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -368,23 +384,19 @@ extern "C" {
 
 size_t sv_verify_chain_workspace_size(int B, int k, int V, int K) {
   if (B <= 0 || k < 1 || V < 1) return 256;
-  const int W = stream_chunk(V, (long long)B * (k + 1));
-  return ws_layout(B, B * (k + 1), (V + W - 1) / W, K > 0 ? K : 0).bytes;
+  return ws_layout(B, B * (k + 1), record_slots(V), K > 0 ? K : 0).bytes;
 }
 size_t sv_verify_tree_workspace_size(int B, int n, int V) {
   if (B <= 0 || n < 1 || V < 1) return 256;
-  const int W = stream_chunk(V, (long long)B * n);
-  return ws_layout(B, B * n, (V + W - 1) / W, 0).bytes;
+  return ws_layout(B, B * n, record_slots(V), 0).bytes;
 }
 size_t sv_extract_topk_workspace_size(int rows, int V, int K) {
   if (rows <= 0 || V < 1) return 256;
-  const int W = stream_chunk(V, rows);
-  return ws_layout(rows, rows, (V + W - 1) / W, K > 0 ? K : 0).bytes;
+  return ws_layout(rows, rows, record_slots(V), K > 0 ? K : 0).bytes;
 }
 size_t sv_kd_kl_loss_workspace_size(int B, int k, int V) {
   if (B <= 0 || k < 1 || V < 1) return 256;
-  const int W = stream_chunk(V, (long long)B * k);
-  return ws_layout(B, B * k, (V + W - 1) / W, 0).bytes;
+  return ws_layout(B, B * k, record_slots(V), 0).bytes;
 }
 
 static sv_status check_workspace(void* ws, size_t bytes, size_t need) {
@@ -434,7 +446,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   const int te = esize(t_dtype);
   const int de = greedy ? 0 : (d_kind == SV_DRAFT_PROBS ? 4 : esize(d_dtype));
   const StreamGeom sg = stream_geom(V, (long long)B * P, te, d_kind == SV_DRAFT_PROBS ? 0 : de);
-  const WsLayout wl = ws_layout(B, B * P, sg.nchunk, K);
+  const WsLayout wl = ws_layout(B, B * P, record_slots(V), K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);
@@ -554,7 +566,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if ((long long)B * n > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
   const StreamGeom sg = stream_geom(V, (long long)B * n, esize(dt), 0);
-  const WsLayout wl = ws_layout(B, B * n, sg.nchunk, 0);
+  const WsLayout wl = ws_layout(B, B * n, record_slots(V), 0);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);
@@ -620,7 +632,7 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if (rows > 0x7fffffff / 64) return SV_ERR_UNSUPPORTED;
   const StreamGeom sg = stream_geom(V, rows, esize(dt), 0);
-  const WsLayout wl = ws_layout(rows, rows, sg.nchunk, K);
+  const WsLayout wl = ws_layout(rows, rows, record_slots(V), K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);
@@ -682,7 +694,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if ((long long)B * k > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
   const StreamGeom sg = stream_geom(V, (long long)B * k, esize(d_dtype), 0);
-  const WsLayout wl = ws_layout(B, B * k, sg.nchunk, 0);
+  const WsLayout wl = ws_layout(B, B * k, record_slots(V), 0);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);

@@ -43,6 +43,9 @@ enum StreamFlags : int {
   kFArgmax0 = 8,   // argmax of row 0
   kFTopk0 = 16,    // top-K keys of row 0
   kFGather = 32,   // the two rows' values at the row's draft token
+  kFStatic = 64,   // static contiguous partition, no in-stream counting (the
+                   // finishing kernel completes the rows); else dynamic items
+                   // with in-stream counting and early exit
 };
 
 // How items map to rows and what the row decision is.
@@ -558,6 +561,8 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
                     warp * 2;
   const bool use_bulk = prm.use_bulk != 0;
   const bool chain = prm.kind != kKindRows;
+  constexpr bool stat = (FLAGS & kFStatic) != 0;
+  constexpr int RF = FLAGS & ~kFStatic;  // what a row completion does
   const int V = prm.V, W = prm.W, nchunk = prm.nchunk;
   const int total = prm.nrows * nchunk;
   const int nwarps = (int)gridDim.x * kStreamWarps;
@@ -578,7 +583,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     if (!chain || item >= total) return;
     const int r = fast_div(item, prm.div_nchunk);
     const int i = fast_div(r, prm.div_B), b = r - i * prm.B;
-    if (prm.count) rj = load_relaxed_u32(&prm.req_reject[b]);
+    if (!stat) rj = load_relaxed_u32(&prm.req_reject[b]);
     if (i < prm.k) x = prm.tokens[(size_t)b * prm.k + i];
   };
   // Pieces of an item (lane-uniform); 0 when skipped: an earlier position of
@@ -623,7 +628,14 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   int slot_cur = 0;  // descriptor of cur; nxt uses the other
 
   uint32_t n_issued = 0, n_consumed = 0;
-  int cur = gwarp, cur_np, cur_x;
+  // Static mode (no in-stream counting): warp g takes the contiguous items
+  // [g * total / NW, (g + 1) * total / NW) and merges consecutive items of one
+  // row into one record.  Dynamic mode: first items g and g + NW, then the
+  // stripe counters.
+  const long long lo = stat ? (long long)gwarp * total / nwarps : 0;
+  const long long hi = stat ? (long long)(gwarp + 1) * total / nwarps : 0;
+  auto stat_item = [&](long long t) -> int { return t < hi ? (int)t : total; };
+  int cur = stat ? stat_item(lo) : gwarp, cur_np, cur_x;
   {
     uint32_t rj;
     int x;
@@ -631,7 +643,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     cur_np = pieces_of(cur, rj, 0);
     cur_x = __shfl_sync(0xffffffffu, x, 0);
   }
-  int nxt = gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
+  int nxt = stat ? stat_item(lo + 1) : gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
   uint32_t nxt_rj = 0u;
   // Lane 0: the stripe counter and the number of fetches it will receive.
   const int stripe = gwarp % kStripes;
@@ -663,12 +675,12 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   uint32_t pend = 0u;  // lane 0
   if (lane == 0) {
     prefetch(nxt, nxt_rj, nxt_x);
-    pend = fetch();  // every warp fetches at least once
+    if (!stat) pend = fetch();  // every warp fetches at least once
   }
-  nxt2 = take(pend);
+  nxt2 = stat ? stat_item(lo + 2) : take(pend);
   if (lane == 0) {
     prefetch(nxt2, nxt2_rj, nxt2_x);
-    if (nxt2 < total) pend = fetch();
+    if (!stat && nxt2 < total) pend = fetch();
   }
   int iss_which = 0, iss_p = 0;
   int timeouts = 0;
@@ -709,7 +721,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     if (last) {
       __threadfence();  // acquire: the other items' records
       __syncwarp();
-      row_complete<T0, T1, FLAGS>(prm, res_r, res_x);
+      row_complete<T0, T1, RF>(prm, res_r, res_x);
     }
     res_r = -1;
   };
@@ -726,22 +738,35 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   };
 
   top_up();
+  // The statistics of a run: the items merged into one record (one item in
+  // dynamic mode).
+  ThreadStat st0, st1;
+  float best = -INFINITY;
+  int bidx = -1;
+  float zx0 = 0.f, zx1 = 0.f;
+  int hx = 0;
+  unsigned long long list = kNoKey;
+  unsigned long long thr_key = kNoKey;
+  float thr_val = -INFINITY;
+  int run_first = -1;  // the item whose record slot the run writes
   while (cur < total) {
     const int r = fast_div(cur, prm.div_nchunk);
     const int ch = cur - r * nchunk;
     const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, cur_x);
     const int clen = min(W, V - ch * W);
     const bool has1 = (FLAGS & kFRow1) && L.row1 != nullptr;
-    ThreadStat st0, st1;
-    stat_init(st0);
-    stat_init(st1);
-    float best = -INFINITY;
-    int bidx = -1;
-    float zx0 = 0.f, zx1 = 0.f;
-    int hx = 0;
-    unsigned long long list = kNoKey;
-    unsigned long long thr_key = kNoKey;
-    float thr_val = -INFINITY;
+    if (run_first < 0) {
+      run_first = cur;
+      stat_init(st0);
+      stat_init(st1);
+      best = -INFINITY;
+      bidx = -1;
+      zx0 = zx1 = 0.f;
+      hx = 0;
+      list = kNoKey;
+      thr_key = kNoKey;
+      thr_val = -INFINITY;
+    }
 
     for (int p = 0; p < cur_np; ++p) {
       const int s = (int)(n_consumed % kStages);
@@ -838,7 +863,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       }
     }
 
-    // Per-item reduction and partial record.
+    // The run ends at a row boundary, at the end of the warp's range, and
+    // after every item in dynamic mode.
+    const bool run_end = !stat || nxt >= total || ch == nchunk - 1;
+    if (run_end) {
+    // Per-run reduction and record.
     Partial pr;
     pr.G0 = pr.G1 = -INFINITY;
     pr.S0 = pr.S1 = 0.0;
@@ -870,15 +899,17 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     // Counting is deferred: the count of an item is added one item later,
     // when its record has long been written, and the returned count is read
     // one item after that.
-    if (prm.count) {
+    if (!stat) {
       resolve();
       signal();
     }
-    if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)cur * K + lane] = list;
-    if (lane == 0) prm.part[cur] = pr;
+    if ((FLAGS & kFTopk0) && lane < K) prm.cand[(size_t)run_first * K + lane] = list;
+    if (lane == 0) prm.part[run_first] = pr;
     sig_r = r;
     sig_x = L.x;
     timeouts = 0;
+    run_first = -1;
+    }
 
     // Advance: nxt becomes current; the item after it comes from the counter.
     cur = nxt;
@@ -892,15 +923,15 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     nxt_np = -1;
     nxt_rj = nxt2_rj;
     nxt_x = nxt2_x;
-    nxt2 = nxt2 < total ? take(pend) : total;
+    nxt2 = nxt2 < total ? (stat ? stat_item((long long)nxt2 + 1) : take(pend)) : total;
     if (lane == 0) {
       prefetch(nxt2, nxt2_rj, nxt2_x);
-      if (nxt2 < total) pend = fetch();
+      if (!stat && nxt2 < total) pend = fetch();
     }
     top_up();
   }
   // Count the last item and read the outstanding results.
-  if (prm.count) {
+  if (!stat) {
     resolve();
     signal();
     resolve();

@@ -367,3 +367,33 @@ def test_every_cluster_size(monkeypatch, C):
     got = sv.sv_extract_topk_kd(x.target.to(DEV), 32, 0.7)
     ref = O.topk(x.target, 32, 0.7)
     assert np.array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
+
+
+@pytest.mark.parametrize("mode", ["1", "2"])
+def test_both_stream_schedules(monkeypatch, kd256, mode):
+    """Static partition (rows completed by the finisher) and dynamic items with
+    in-stream counting and early exit give the oracle's results; the
+    workspace is all zero after every call."""
+    monkeypatch.setenv("SV_STREAM_COUNT", mode)
+    x = kd256
+    st = status_tensor()
+    kd = dict(K=32, reward=x.reward.to(DEV), wmode="group_norm", group=16)
+    got = run_chain(x, kd=kd, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & sv.SV_DEV_ERROR_MASK == 0
+    ref = O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward, x.temperature, 32,
+                      mode=O.W_GROUP_NORM, group=16)
+    assert_chain_match(got, ref, x.uniforms.numpy(), x.temperature, x.k)
+    assert_kd_match(got, ref, x.k)
+    ws = sv._WS[torch.cuda.current_device()]
+    assert int(torch.count_nonzero(ws)) == 0
+    # plain sampling and greedy chains under the same schedule
+    check_chain(inputs.make_chain(48, 3, 70001, dtype="bf16", sigma_d=1.0, temperature=0.7,
+                                  seed=7))
+    g = inputs.make_chain(48, 3, 70001, dtype="bf16", sigma_d=1.0, temperature=0.0, seed=8)
+    got = run_chain(g)
+    ref = oracle_chain(g)
+    torch.cuda.synchronize()
+    assert np.array_equal(got["accepted_len"].cpu().numpy(), ref["accepted_len"])
+    assert np.array_equal(got["out_tokens"].cpu().numpy(), ref["out_tokens"])
+    assert int(torch.count_nonzero(ws)) == 0
