@@ -32,7 +32,7 @@ int forced_cluster() {
 // Finishing plans: every power-of-two cluster size C whose chunk of
 // ceil(V / C) elements fits the shared-memory limit, C ascending.
 template <class XB>
-int feasible_plans(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* plans) {
+int feasible_plans(int V, int tb, int db, XB x_bytes, bool bulk_ok, int rows_bytes, RowPlan* plans) {
   if (V < 1 || V > kMaxV) return 0;
   const int forced = forced_cluster();
   int n = 0;
@@ -42,7 +42,8 @@ int feasible_plans(int V, int tb, int db, XB x_bytes, bool bulk_ok, RowPlan* pla
     if (L > kMaxChunk) continue;
     const int np = (L + kRound - 1) / kRound;
     RowLayout lay;
-    lay.off_t = kFixedBytes;
+    lay.off_rows = kFixedBytes;
+    lay.off_t = kFixedBytes + (int)align_up((size_t)rows_bytes, 128);
     lay.off_d = lay.off_t + (int)align_up((size_t)L * tb, 128);
     lay.off_x = lay.off_d + (int)align_up((size_t)L * db, 128);
     lay.bytes = lay.off_x + (int)align_up((size_t)x_bytes(L, np), 128);
@@ -258,6 +259,7 @@ static cudaError_t launch_stream(StreamParams& p, const StreamGeom& g, cudaStrea
   const long long need = (items + kStreamWarps - 1) / kStreamWarps;
   if (need < grid) grid = need;
   if (grid < 1) grid = 1;
+  p.nwarps_eff = (int)(grid * kStreamWarps < items ? grid * kStreamWarps : items);
   if (p.count == 0)
     ks<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
   else
@@ -279,13 +281,15 @@ static cudaError_t launch_clusters(K kernel, const Prm& prm, const RowPlan& plan
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)plan.lay.bytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)plan.C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps the stream's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, prm);
 }
 
@@ -293,8 +297,17 @@ template <class K, class Prm>
 static cudaError_t launch_blocks(K kernel, const Prm& prm, int blocks, int smem, cudaStream_t s) {
   cudaError_t e = ensure_kernel_attrs(reinterpret_cast<const void*>(kernel), smem, false);
   if (e != cudaSuccess) return e;
-  kernel<<<(unsigned)blocks, kThreads, smem, s>>>(prm);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps the stream's tail
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, prm);
 }
 
 // Clusters of plan.C CTAs of this kernel that the device holds at once.
@@ -521,8 +534,9 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
                                        : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
     if (e != cudaSuccess) return SV_ERR_CUDA;
     fp.sp = sp;
-    return cuda_status(t_dtype == SV_BF16 ? launch_blocks(chain_greedy_finish<BF16>, fp, B, 0, s)
-                                          : launch_blocks(chain_greedy_finish<F32>, fp, B, 0, s));
+    const int gsm = kFixedBytes + P * (int)sizeof(RowRec);
+    return cuda_status(t_dtype == SV_BF16 ? launch_blocks(chain_greedy_finish<BF16>, fp, B, gsm, s)
+                                          : launch_blocks(chain_greedy_finish<F32>, fp, B, gsm, s));
   }
 
   RowPlan plans[8];
@@ -532,7 +546,8 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
         const int x = npc * kThreads * 4 + kThreads * 8;
         return x < 2 * kThreads * 4 ? 2 * kThreads * 4 : x;
       },
-      bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de), plans);
+      bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de), P * (int)sizeof(RowRec),
+      plans);
   if (np == 0) return SV_ERR_UNSUPPORTED;
   cudaError_t e;
   if (d_kind == SV_DRAFT_PROBS)
@@ -613,8 +628,9 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   fp.req_reject = w.reject;
   fp.status = device_status;
   fp.sp = sp;
-  return cuda_status(dt == SV_BF16 ? launch_blocks(tree_finish<BF16>, fp, B, kFixedBytes + 4 * n * 4, s)
-                                   : launch_blocks(tree_finish<F32>, fp, B, kFixedBytes + 4 * n * 4, s));
+  const int tsm = kFixedBytes + n * (int)sizeof(RowRec) + 4 * n * 4;
+  return cuda_status(dt == SV_BF16 ? launch_blocks(tree_finish<BF16>, fp, B, tsm, s)
+                                   : launch_blocks(tree_finish<F32>, fp, B, tsm, s));
 }
 
 sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, int K,
@@ -754,8 +770,9 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   fp.glob_counter = w.glob;
   fp.status = device_status;
   fp.sp = sp;
-  cudaError_t e = (d_dtype == SV_BF16) ? launch_blocks(kl_finish<BF16>, fp, B, kFixedBytes, s)
-                                       : launch_blocks(kl_finish<F32>, fp, B, kFixedBytes, s);
+  const int ksm = kFixedBytes + k * (int)sizeof(RowRec);
+  cudaError_t e = (d_dtype == SV_BF16) ? launch_blocks(kl_finish<BF16>, fp, B, ksm, s)
+                                       : launch_blocks(kl_finish<F32>, fp, B, ksm, s);
   return cuda_status(e);
 }
 

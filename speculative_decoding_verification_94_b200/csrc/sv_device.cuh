@@ -272,6 +272,22 @@ __device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsig
   return d;
 }
 
+// Programmatic dependent launch: a kernel lets the next kernel on its stream
+// be scheduled early; the next kernel waits here until this grid has
+// completed and its memory operations are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Split cluster barrier (every thread of the cluster arrives, then waits).
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
 // 2^x on the special-function unit (ex2.approx.ftz.f32).
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -102,17 +102,46 @@ __device__ __forceinline__ float seq_sum8(const float w[8]) {
   return s;
 }
 
-// First rejection of request b from its row records (one warp, all lanes
-// return the same): n, and whether every row that decides the outcome
-// (0..n) was verified.
-__device__ __forceinline__ int warp_first_rejection(const RowRec* rec, int B, int k, int b,
-                                                    bool* bad) {
+// The request's rows in shared memory (rows[t] = row t of the request):
+// folded here from the stream's records (static schedule), or read from the
+// records the stream completed (dynamic schedule).  Warp w takes rows w, w + 8,
+// ...; every caller in a cluster does this redundantly (no barrier needed).
+// Returns nothing; rows[] is valid after the caller's __syncthreads.
+template <class T0, class T1, int FLAGS>
+__device__ __forceinline__ void load_rows(const FinishParams& prm, RowRec* rows, int nrows,
+                                          int row0, int row_stride, const int32_t* xs, int nx,
+                                          bool report) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const bool stat = !prm.sp.count;
+  for (int t = w; t < nrows; t += kWarps) {
+    const int r = row0 + t * row_stride;
+    const int x = t < nx ? xs[t] : -1;
+    RowRec rr;
+    if (stat) {
+      const RowSum s = row_combine<T0, T1, FLAGS>(prm.sp, r, x, true);
+      int err = 0;
+      rr = row_decide<FLAGS>(prm.sp, r, x, s, &err);
+      if (err && report && lane == 0) set_status(prm.status, err);
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(prm.rec + r);
+      uint4 q[3];
+      q[0] = __ldcg(src);
+      q[1] = __ldcg(src + 1);
+      q[2] = __ldcg(src + 2);
+      memcpy(&rr, q, sizeof(RowRec));
+    }
+    if (lane == 0) rows[t] = rr;
+  }
+}
+
+// First rejection n of a chain (one warp; all lanes return the same) and
+// whether every row that decides the outcome (0..n) was verified.
+__device__ __forceinline__ int first_rejection(const RowRec* rows, int k, bool* bad) {
   const int lane = threadIdx.x & 31;
   int n = k;
   for (int base = 0; base < k; base += 32) {
     const int t = base + lane;
-    const int code = t < k ? __ldcg(&rec[(size_t)t * B + b].code) : 0;
-    const unsigned m = __ballot_sync(0xffffffffu, t < k && code == kRowRejected);
+    const unsigned m = __ballot_sync(0xffffffffu, t < k && rows[t].code == kRowRejected);
     if (m) {
       n = base + __ffs(m) - 1;
       break;
@@ -121,20 +150,36 @@ __device__ __forceinline__ int warp_first_rejection(const RowRec* rec, int B, in
   bool bd = false;
   for (int base = 0; base <= n; base += 32) {
     const int t = base + lane;
-    const int code = t <= n ? __ldcg(&rec[(size_t)t * B + b].code) : kRowAccepted;
+    const int code = t <= n ? rows[t].code : kRowAccepted;
     bd |= __any_sync(0xffffffffu, code != kRowAccepted && code != kRowRejected);
   }
   *bad = bd;
   return n;
 }
 
-// Zero the row records of rows r0, r0 + stride_rows, ... (nr rows) with
-// threads t0, t0 + nt, ...
-__device__ __forceinline__ void zero_recs(const FinishParams& p, size_t r0, int stride_rows,
-                                          int nr, int t0, int nt) {
-  for (int q = t0; q < nr; q += nt) p.rec[r0 + (size_t)q * stride_rows] = RowRec{};
+// The rows' stream state back to zero: the records of the static schedule,
+// or the row records of the dynamic one.  Rows t = t0, t0 + nt, ... (warps).
+__device__ __forceinline__ void release_rows(const FinishParams& prm, int nrows, int row0,
+                                             int row_stride, int t0, int nt) {
+  const int lane = threadIdx.x & 31;
+  for (int t = t0; t < nrows; t += nt) {
+    const int r = row0 + t * row_stride;
+    if (!prm.sp.count) row_zero_records(prm.sp, r, true);
+    else if (lane == 0) prm.rec[r] = RowRec{};
+  }
 }
 
+// Chain sampling: one cluster of C CTAs per request.
+//   0. rows 0..k in every CTA (load_rows); warp 0 finds the first rejection n;
+//   1. fused KD (static schedule): the rows' top-K outputs for rows 0..n,
+//      spread over the cluster's warps; later rows' lists are cleared;
+//   2. the draw from the one row pair that needs it (residual at n < k, bonus
+//      row at n = k), staged by bulk copies, chunk masses scanned in a fixed
+//      order through distributed shared memory (the one cluster barrier);
+//   3. the rows' stream state back to zero (after the barrier: no CTA still
+//      reads it);
+//   4. the CTA that owns the drawn token writes the request's outputs (the
+//      first CTA when there is no draw: failed rows or timeouts).
 template <class TT, class DT, int DKIND, bool KD>
 __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -142,6 +187,7 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
   const int C = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
+  RowRec* rows = reinterpret_cast<RowRec*>(smem + prm.lay.off_rows);
   unsigned char* tbuf = smem + prm.lay.off_t;
   unsigned char* dbuf = smem + prm.lay.off_d;
   float* sums = reinterpret_cast<float*>(smem + prm.lay.off_x);
@@ -150,38 +196,43 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
   const ChunkGeom g = chunk_geom(rank, prm.L, V);
   const float c = prm.c;
   const bool use_bulk = prm.use_bulk != 0;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  constexpr int RF = chain_sample_flags<DKIND, KD>();
+  if (threadIdx.x == 0) sh.tok = -1;
+  pdl_wait();  // the stream's records are complete
 
-  // 0. rows 0..k of the request, when the stream left them to this kernel
-  if (!prm.sp.count) {
-    const int w = threadIdx.x >> 5;
-    for (int t = rank * kWarps + w; t < P; t += C * kWarps)
-      row_complete<TT, DT, chain_sample_flags<DKIND, KD>()>(
-          prm.sp, t * B + b, t < k ? prm.tokens[(size_t)b * k + t] : -1);
-    if (threadIdx.x == 0) __threadfence();
-    cluster.sync();
-  }
-
-  if (threadIdx.x < 32) {
+  // 0. the request's rows and its first rejection
+  load_rows<TT, DT, RF>(prm, rows, P, b, B, prm.tokens + (size_t)b * k, k, rank == 0);
+  __syncthreads();
+  if (w == 0) {
     bool bad;
-    const int n = warp_first_rejection(prm.rec, B, k, b, &bad);
-    if (threadIdx.x == 0) {
+    const int n = first_rejection(rows, k, &bad);
+    if (lane == 0) {
       sh.fin_n = bad ? -1 : n;
       sh.need = bad ? 0 : 1;
       sh.err = 0;
-      // cleared before the draw's first cluster barrier; the owning CTA writes it after
-      if (rank == 0 && !bad) prm.out_tokens[(size_t)b * P + n] = -1;
-      const RowRec* rn = &prm.rec[(size_t)n * B + b];
-      sh.Gt = __ldcg(&rn->G0);
-      sh.St = __ldcg(&rn->S0);
-      sh.Gd = __ldcg(&rn->G1);
-      sh.Sd = __ldcg(&rn->S1);
-      sh.tok = -1;
+      sh.owner = 0;
+      sh.Gt = rows[n].G0;
+      sh.St = rows[n].S0;
+      sh.Gd = rows[n].G1;
+      sh.Sd = rows[n].S1;
     }
   }
   __syncthreads();
   const int n = sh.fin_n;
 
-  // 1. the draw, from row pair n (residual) or the bonus row k (target only).
+  // 1. fused KD outputs of rows 0..n (static schedule; the dynamic schedule
+  //    wrote them in the stream)
+  if (KD && !prm.sp.count) {
+    for (int t = rank * kWarps + w; t < P; t += C * kWarps) {
+      const RowRec& rr = rows[t];
+      row_outputs<TT, DT, RF>(prm.sp, t * B + b, t < k ? prm.tokens[(size_t)b * k + t] : -1,
+                              rr.L0, rr.L1, 0, n >= 0 && t <= n, true);
+    }
+  }
+
+  // 2. the draw, from row pair n (residual) or the bonus row k (target only)
+  bool arrived = false;
   if (sh.need) {
     const bool pair = n < k;
     const void* trow = row_ptr<TT>(prm.target, (size_t)b * P + n, V);
@@ -201,9 +252,9 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         const int e = p * kRound + (int)threadIdx.x * kVec;
         float s = 0.f;
         if (e < g.nvec * kVec) {
-          float w[8];
-          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, w);
-          s = seq_sum8(w);
+          float wv[8];
+          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, wv);
+          s = seq_sum8(wv);
         }
         sums[p * kThreads + threadIdx.x] = s;
       }
@@ -213,11 +264,10 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         for (int p = 0; p < g.npieces; ++p) Rc += sh.ptot[p];
         sh.R = Rc;
       }
-      cluster.sync();  // chunk masses visible
-      if (threadIdx.x < 32) {
+      cluster.sync();  // chunk masses visible; every CTA has read the rows' records
+      if (w == 0) {
         // chunk q owns [incl(q-1), incl(q)) of the cumulative mass; the scan
         // runs in the same order in every CTA.
-        const int lane = threadIdx.x;
         const double Rq = lane < C ? cluster.map_shared_rank(&sh, lane)->R : 0.0;
         const double incl = warp_scan_incl(Rq);
         const double R = __shfl_sync(0xffffffffu, incl, 31);
@@ -232,14 +282,17 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
           sh.redo = (R == 0.0 && mode == kModeResidual && !tmo) ? 1 : 0;
           sh.owner = (R > 0.0 && !tmo && myO <= tt && tt < hi) ? 1 : 0;
           if (tmo && rank == 0) set_status(prm.status, SV_DEV_TIMEOUT);
-          sh.err = tmo ? 1 : 0;
+          sh.err = (tmo || !(R > 0.0)) ? 1 : 0;
         }
       }
       __syncthreads();
+      cluster_arrive_release();  // done with the other CTAs' shared memory
+      arrived = true;
       if (!sh.redo) break;
       if (rank == 0 && threadIdx.x == 0) set_status(prm.status, SV_DEV_RESIDUAL_ZERO);
       mode = kModeP;
-      cluster.sync();  // nobody still reads sh.R of the first attempt
+      cluster_wait_acquire();  // nobody still reads sh.R of the first attempt
+      arrived = false;
     }
     if (sh.owner) {
       if (threadIdx.x == 0) {
@@ -284,15 +337,15 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         if (fb) ts = sh.last_pos;
         if ((int)threadIdx.x == ts) {
           const int e = pp * kRound + ts * kVec;
-          float w[8];
-          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, w);
+          float wv[8];
+          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, wv);
           const double b0 = sh.base + (ts > 0 ? incl_arr[ts - 1] : 0.0);
           float a = 0.f;
           int pick = -1, lastq = -1;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            a = __fadd_rn(a, w[q]);
-            if (w[q] > 0.f) lastq = q;
+            a = __fadd_rn(a, wv[q]);
+            if (wv[q] > 0.f) lastq = q;
             if (!fb && pick < 0 && b0 + (double)a > sh.tt) pick = q;
           }
           if (pick < 0) pick = lastq;
@@ -300,16 +353,35 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         }
         __syncthreads();
       }
-      if (threadIdx.x == 0) prm.out_tokens[(size_t)b * P + n] = sh.tok;
     }
+  } else {
+    cluster.sync();  // every CTA has read the rows' records
   }
 
-  // 2. fused KD: the stream wrote rows 0..n; later rows are not verified and
-  // are defined as empty.
-  if (KD) {
-    // rows after the emitted position: not verified, defined as empty
-    if (rank == 0) {
-      const int first_undef = n < 0 ? 0 : n + 1;
+  // 3. the rows' stream state back to zero
+  release_rows(prm, P, b, B, rank * kWarps + w, C * kWarps);
+
+  // 4. outputs, by the owner of the drawn token (or the first CTA without a draw)
+  const bool writer = sh.need ? (sh.owner != 0 || (sh.err && rank == 0)) : rank == 0;
+  if (writer) {
+    if (threadIdx.x == 0) {
+      int nn = n;
+      if (nn >= 0 && (!sh.need || sh.err)) nn = -1;
+      if (nn >= 0 && (sh.tok < 0 || sh.tok >= V)) nn = -1;
+      sh.fin_n = nn;
+      prm.accepted_len[b] = nn;
+      prm.req_reject[b] = 0u;
+    }
+    __syncthreads();
+    const int nf = sh.fin_n;
+    for (int t = threadIdx.x; t < P; t += kThreads) {
+      int v = -1;
+      if (nf >= 0) v = t < nf ? prm.tokens[(size_t)b * k + t] : (t == nf ? sh.tok : -1);
+      prm.out_tokens[(size_t)b * P + t] = v;
+    }
+    if (KD) {
+      // rows after the emitted position are not verified: defined as empty
+      const int first_undef = nf < 0 ? 0 : nf + 1;
       for (int t = first_undef * prm.K + (int)threadIdx.x; t < P * prm.K; t += kThreads) {
         prm.topk_logp[(size_t)b * P * prm.K + t] = NAN;
         prm.topk_idx[(size_t)b * P * prm.K + t] = -1;
@@ -318,66 +390,42 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         prm.lse[(size_t)b * P + t] = NAN;
       for (int t = first_undef + (int)threadIdx.x; t < k; t += kThreads)
         prm.kl[(size_t)b * k + t] = NAN;
+      __syncthreads();
+      kd_finalize(b, nf, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
+                  prm.total, prm.glob_counter, sh);
     }
   }
-  if (threadIdx.x == 0) __threadfence();
-  cluster.sync();  // draw, KD rows and every read of the records are done
-
-  // 3. outputs (rank 0) and workspace hygiene (every CTA).
-  zero_recs(prm, (size_t)b, B, P, rank * kThreads + (int)threadIdx.x, C * kThreads);
-  if (rank != 0) return;
-  if (threadIdx.x == 0) {
-    int nn = n;
-    if (nn >= 0 && sh.need && sh.err) nn = -1;
-    if (nn >= 0) {
-      const int tk = __ldcg(&prm.out_tokens[(size_t)b * P + nn]);
-      if (tk < 0 || tk >= V) nn = -1;
-    }
-    sh.fin_n = nn;
-    prm.accepted_len[b] = nn;
-    prm.req_reject[b] = 0u;
-  }
-  __syncthreads();
-  const int nf = sh.fin_n;
-  for (int t = threadIdx.x; t < P; t += kThreads) {
-    if (nf >= 0 && t == nf) continue;  // the drawn token, written by the owning CTA
-    const int v = (nf >= 0 && t < nf) ? prm.tokens[(size_t)b * k + t] : -1;
-    prm.out_tokens[(size_t)b * P + t] = v;
-  }
-  if (KD)
-    kd_finalize(b, nf, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
-                prm.total, prm.glob_counter, sh);
+  if (arrived) cluster_wait_acquire();  // keep this CTA's shared memory until all have read it
 }
 
-// Greedy chain: one block per request (its warps complete the request's rows
-// when the stream left them; warp 0 takes the decision).
+// Greedy chain: one block per request.
 template <class T>
 __global__ void __launch_bounds__(kThreads) chain_greedy_finish(const __grid_constant__ FinishParams prm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  RowRec* rows = reinterpret_cast<RowRec*>(smem + kFixedBytes);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int b = (int)blockIdx.x;
   const int k = prm.k, P = k + 1, B = prm.B;
-  if (!prm.sp.count) {
-    for (int t = w; t < P; t += kWarps)
-      row_complete<T, T, kFArgmax0>(prm.sp, t * B + b, t < k ? prm.tokens[(size_t)b * k + t] : -1);
-    __threadfence();
-    __syncthreads();
+  pdl_wait();
+  load_rows<T, T, kFArgmax0>(prm, rows, P, b, B, prm.tokens + (size_t)b * k, k, true);
+  __syncthreads();
+  if (w == 0) {
+    bool bad = false;
+    const int n = first_rejection(rows, k, &bad);
+    const int tok = rows[n].argmax;
+    if (tok < 0 || tok >= prm.V) bad = true;
+    for (int t = lane; t < P; t += 32) {
+      int v = -1;
+      if (!bad) v = (t < n) ? prm.tokens[(size_t)b * k + t] : (t == n ? tok : -1);
+      prm.out_tokens[(size_t)b * P + t] = v;
+    }
+    if (lane == 0) {
+      prm.accepted_len[b] = bad ? -1 : n;
+      prm.req_reject[b] = 0u;
+    }
   }
-  if (w != 0) return;
-  bool bad = false;
-  const int n = warp_first_rejection(prm.rec, B, k, b, &bad);
-  const int tok = __ldcg(&prm.rec[(size_t)n * B + b].argmax);
-  if (tok < 0 || tok >= prm.V) bad = true;
-  for (int t = lane; t < P; t += 32) {
-    int v = -1;
-    if (!bad) v = (t < n) ? prm.tokens[(size_t)b * k + t] : (t == n ? tok : -1);
-    prm.out_tokens[(size_t)b * P + t] = v;
-  }
-  __syncwarp();
-  zero_recs(prm, (size_t)b, B, P, lane, 32);
-  if (lane == 0) {
-    prm.accepted_len[b] = bad ? -1 : n;
-    prm.req_reject[b] = 0u;
-  }
+  __syncthreads();  // (every warp has read the rows' state)
+  release_rows(prm, P, b, B, w, kWarps);
 }
 
 // Greedy tree: one block per request; node rows are rows b * n + j.
@@ -387,21 +435,18 @@ __global__ void __launch_bounds__(kThreads) tree_finish(const __grid_constant__ 
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
   const int n = prm.k, V = prm.V;
   const int b = (int)blockIdx.x;
-  if (!prm.sp.count) {
-    for (int t = threadIdx.x >> 5; t < n; t += kWarps)
-      row_complete<T, T, kFArgmax0>(prm.sp, b * n + t, -1);
-    __threadfence();
-    __syncthreads();
-  }
-  int* garg = reinterpret_cast<int*>(smem + kFixedBytes);
+  RowRec* rows = reinterpret_cast<RowRec*>(smem + kFixedBytes);
+  int* garg = reinterpret_cast<int*>(smem + kFixedBytes + (size_t)n * sizeof(RowRec));
   int* par = garg + n;
   int* tok = par + n;
   int* dep = tok + n;
+  pdl_wait();
+  load_rows<T, T, kFArgmax0>(prm, rows, n, b * n, 1, nullptr, 0, true);
+  __syncthreads();
   int err_any = 0;
   for (int t = threadIdx.x; t < n; t += kThreads) {
-    const RowRec* r = &prm.rec[(size_t)b * n + t];
-    const int code = __ldcg(&r->code);
-    garg[t] = code == kRowAccepted ? __ldcg(&r->argmax) : -1;
+    const int code = rows[t].code;
+    garg[t] = code == kRowAccepted ? rows[t].argmax : -1;
     err_any |= (code != kRowAccepted);
     par[t] = prm.parents[(size_t)b * n + t];
     tok[t] = prm.tokens[(size_t)b * n + t];
@@ -452,26 +497,25 @@ __global__ void __launch_bounds__(kThreads) tree_finish(const __grid_constant__ 
       ot[Lb] = garg[best];
     }
   }
-  zero_recs(prm, (size_t)b * n, 1, n, threadIdx.x, kThreads);
+  release_rows(prm, n, b * n, 1, threadIdx.x >> 5, kWarps);
 }
 
 // KD loss: one block per request, one warp per draft row (b, i < k).  Draft
-// rows stream first (logits) so that rec holds their normalisers; probability
-// drafts have no stream pass.
+// logit rows are folded from the stream's records first; probability drafts
+// have no stream pass.
 template <class DT>
 __global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
+  RowRec* rows = reinterpret_cast<RowRec*>(smem + kFixedBytes);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int b = (int)blockIdx.x;
   const int k = prm.k, P = k + 1, B = prm.B, V = prm.V, K = prm.K;
-  if (!prm.draft_probs && !prm.sp.count) {
-    for (int t = w; t < k; t += kWarps) row_complete<DT, DT, kFStats0>(prm.sp, b * k + t, -1);
-    __threadfence();
-    __syncthreads();
-  }
   const double ln2 = 0.69314718055994530942;
   const double c = (double)prm.c;
+  pdl_wait();
+  if (!prm.draft_probs) load_rows<DT, DT, kFStats0>(prm, rows, k, b * k, 1, nullptr, 0, true);
+  __syncthreads();
   for (int i = w; i < k; i += kWarps) {
     const size_t trow = (size_t)b * P + i;
     const size_t drow = (size_t)b * k + i;
@@ -485,9 +529,8 @@ __global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ Fi
     double L1 = 0.0;
     int err = 0;
     if (!prm.draft_probs) {
-      const int code = __ldcg(&prm.rec[drow].code);
-      L1 = __ldcg(&prm.rec[drow].L0);
-      if (code != kRowAccepted) err = 1;
+      L1 = rows[i].L0;
+      if (rows[i].code != kRowAccepted) err = 1;
     }
     double m = lp;
 #pragma unroll
@@ -522,7 +565,7 @@ __global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ Fi
     sh.fin_n = n;
   }
   __syncthreads();
-  if (!prm.draft_probs) zero_recs(prm, (size_t)b * k, 1, k, threadIdx.x, kThreads);
+  if (!prm.draft_probs) release_rows(prm, k, b * k, 1, w, kWarps);
   kd_finalize(b, sh.fin_n, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
               prm.total, prm.glob_counter, sh);
 }

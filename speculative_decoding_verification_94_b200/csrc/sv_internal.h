@@ -12,6 +12,7 @@ namespace sv {
 // Shared-memory layout of a finishing kernel: fixed block, then the staged
 // chunk(s) of one row pair, then a scratch region.
 struct RowLayout {
+  int off_rows;  // per-row records of the request (RowRec each)
   int off_t;   // target chunk
   int off_d;   // draft chunk
   int off_x;   // scratch (per-piece weight sums, scan values, KD merge buffers)

@@ -117,6 +117,7 @@ struct StreamParams {
   FastDiv div_nchunk;     // item -> row
   FastDiv div_B;          // chain row -> position
   uint32_t* sched;        // [kStripes] dynamic item counters (zero between calls)
+  int nwarps_eff;         // static partition: warps with a range (<= the grid's warps)
   int count;              // 1: items are counted into rows and rows completed here
                           //    (required for skipping); 0: partials only, rows are
                           //    completed by the finishing kernel
@@ -193,60 +194,107 @@ __device__ __forceinline__ uint32_t load_relaxed_u32(const uint32_t* p) {
   return *reinterpret_cast<const volatile uint32_t*>(p);
 }
 
-// Top K keys of row r from the stream's per-chunk lists (each sorted, best
-// first), best first in lanes 0..K-1.  The chunk heads are merged first; a
-// chunk whose head is not above the K-th best key so far holds nothing that
-// can enter, so only the few chunks with a larger head are read in full.
-__device__ __forceinline__ unsigned long long row_topk_merge(const unsigned long long* lists,
-                                                             int nchunk, int K) {
+// The record slots of row r: one per chunk (dynamic schedule), or, for the
+// static partition, one per run: the row start unless a warp range starts
+// there, and every warp range start inside the row.  Warp w's range starts at
+// floor(w * total / NWs) (total = rows * slots per row, NWs = prm.nwarps_eff).
+struct SlotMap {
+  long long a;      // first slot of the row
+  long long total;  // slots of the stream
+  int nw;           // warps of the static partition (0: one slot per chunk)
+  int wA;           // first warp whose range starts inside the row
+  int head;         // 1: the row start is a slot of its own
+  int nseg;         // slots of the row
+};
+
+__device__ __forceinline__ SlotMap slot_map(const StreamParams& p, int r, bool stat) {
+  SlotMap m;
+  m.a = (long long)r * p.nchunk;
+  m.total = (long long)p.nrows * p.nchunk;
+  if (!stat) {
+    m.nw = 0;
+    m.wA = 0;
+    m.head = 1;
+    m.nseg = p.nchunk;
+    return m;
+  }
+  const long long nw = p.nwarps_eff;
+  const long long e = m.a + p.nchunk;
+  const long long wA = (m.a * nw + m.total - 1) / m.total;  // ceil
+  const long long wB = (e * nw + m.total - 1) / m.total;
+  m.nw = (int)nw;
+  m.wA = (int)wA;
+  m.head = (wA >= wB || (wA * m.total) / nw != m.a) ? 1 : 0;
+  m.nseg = m.head + (int)(wB - wA);
+  return m;
+}
+
+__device__ __forceinline__ long long slot_at(const SlotMap& m, int q) {
+  if (m.nw == 0) return m.a + q;
+  if (m.head && q == 0) return m.a;
+  return ((long long)(m.wA + q - m.head) * m.total) / m.nw;
+}
+
+// Top K keys of a row from its slots' lists (each sorted, best first), best
+// first in lanes 0..K-1.  The heads are merged first; a list whose head is not
+// above the K-th best key so far holds nothing that can enter, so only the few
+// lists with a larger head are read in full.
+__device__ __forceinline__ unsigned long long row_topk_merge(const unsigned long long* cand,
+                                                             const SlotMap& m, int K) {
   const int lane = threadIdx.x & 31;
   unsigned long long list = kNoKey;
-  for (int q0 = 0; q0 < nchunk; q0 += 32) {
+  for (int q0 = 0; q0 < m.nseg; q0 += 32) {
     const int q = q0 + lane;
-    const unsigned long long h = q < nchunk ? __ldcg(&lists[(size_t)q * K]) : kNoKey;
+    const unsigned long long h = q < m.nseg ? __ldcg(&cand[slot_at(m, q) * K]) : kNoKey;
     list = warp_merge_desc(list, warp_sort_desc(h));
   }
   unsigned long long thr = __shfl_sync(0xffffffffu, list, K - 1);
-  for (int q0 = 0; q0 < nchunk; q0 += 32) {
+  for (int q0 = 0; q0 < m.nseg; q0 += 32) {
     const int q = q0 + lane;
-    const unsigned long long h = q < nchunk ? __ldcg(&lists[(size_t)q * K]) : kNoKey;
-    unsigned m = __ballot_sync(0xffffffffu, h > thr);
-    while (m) {
-      // up to four chunks at a time: their keys 1..K-1 (the heads are merged)
+    const long long sq = q < m.nseg ? slot_at(m, q) : 0;
+    const unsigned long long h = q < m.nseg ? __ldcg(&cand[sq * K]) : kNoKey;
+    unsigned msk = __ballot_sync(0xffffffffu, h > thr);
+    while (msk) {
+      // up to four lists at a time: their keys 1..K-1 (the heads are merged)
       unsigned long long x[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         x[t] = kNoKey;
-        if (m) {
-          const int src = __ffs(m) - 1;
-          m &= m - 1;
-          if (lane + 1 < K) x[t] = __ldcg(&lists[(size_t)(q0 + src) * K + lane + 1]);
+        if (msk) {
+          const int src = __ffs(msk) - 1;
+          msk &= msk - 1;
+          const long long ss = __shfl_sync(0xffffffffu, sq, src);
+          if (lane + 1 < K) x[t] = __ldcg(&cand[ss * K + lane + 1]);
         }
       }
 #pragma unroll
       for (int t = 0; t < 4; ++t) list = warp_merge_desc(list, x[t]);
       thr = __shfl_sync(0xffffffffu, list, K - 1);
-      m &= __ballot_sync(0xffffffffu, h > thr);
+      msk &= __ballot_sync(0xffffffffu, h > thr);
     }
   }
   return list;
 }
 
-// The warp that counted a row's last chunk: combine the row's partials in
-// chunk order (lane l takes chunks l, l+32, ...; butterflies across lanes),
-// return the row's partials (and chunk lists) to zero, record the row and,
-// for chain rows, take the acceptance decision.  With kFTopk0 it also writes
-// the row's top-K outputs.
+// A row's statistics folded from its records (every lane holds the same).
+struct RowSum {
+  float G0, G1;
+  double S0, S1;
+  double L0, L1;  // log2 of the partition functions: G + log2(S)
+  float zx0, zx1;
+  int flags;
+  int hx;
+  unsigned long long key;
+};
+
+// Fold row r's records (warp-collective, read-only).  Lane l folds slots l,
+// l + 32, ... in order into a running (reference, sum) pair; the power-of-two
+// rescales are exact, so the sums equal those of a fold at the final
+// reference.  Two records per lane are loaded at a time.
 template <class T0, class T1, int FLAGS>
-__device__ __noinline__ void row_complete(const StreamParams& prm, int r, int x) {
-  const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, x);
+__device__ __noinline__ RowSum row_combine(const StreamParams& prm, int r, int x, bool stat) {
   const int lane = threadIdx.x & 31;
-  const int nchunk = prm.nchunk;
-  Partial* base = prm.part + (size_t)r * nchunk;
-  // One pass: lane l folds chunks l, l + 32, ... in order into a running
-  // (reference, sum) pair; the power-of-two rescales are exact, so the sums
-  // equal those of a fold at the final reference.  Two records per lane are
-  // loaded at a time.
+  const SlotMap m = slot_map(prm, r, stat);
   float g0 = -INFINITY, g1 = -INFINITY, zx0 = 0.f, zx1 = 0.f;
   double s0 = 0.0, s1 = 0.0;
   int flags = 0, hx = 0;
@@ -270,124 +318,166 @@ __device__ __noinline__ void row_complete(const StreamParams& prm, int r, int x)
     }
     key = pq.key > key ? pq.key : key;
   };
-  for (int q = lane; q < nchunk; q += 64) {
-    const Partial pa = load_partial(base + q);
-    const bool two = q + 32 < nchunk;
-    const Partial pb = two ? load_partial(base + q + 32) : Partial{};
+  for (int q = lane; q < m.nseg; q += 64) {
+    const Partial pa = load_partial(prm.part + slot_at(m, q));
+    const bool two = q + 32 < m.nseg;
+    const Partial pb = two ? load_partial(prm.part + slot_at(m, q + 32)) : Partial{};
     fold(pa);
     if (two) fold(pb);
   }
-  const float G0 = warp_max(g0), G1 = warp_max(g1);
-  const double S0 = warp_sum(rescale_pow2(s0, g0, G0)), S1 = warp_sum(rescale_pow2(s1, g1, G1));
-  // (every lane has read its records)
-  for (int q = lane; q < nchunk; q += 32) base[q] = Partial{};
+  RowSum s;
+  s.G0 = warp_max(g0);
+  s.G1 = warp_max(g1);
+  s.S0 = warp_sum(rescale_pow2(s0, g0, s.G0));
+  s.S1 = warp_sum(rescale_pow2(s1, g1, s.G1));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) flags |= __shfl_xor_sync(0xffffffffu, flags, o);
-  key = warp_max_u64(key);
+  s.flags = flags;
+  s.key = warp_max_u64(key);
   const unsigned hm = __ballot_sync(0xffffffffu, hx != 0);
+  s.hx = hm != 0u;
+  s.zx0 = s.zx1 = 0.f;
   if (hm) {
     const int src = __ffs(hm) - 1;
-    zx0 = __shfl_sync(0xffffffffu, zx0, src);
-    zx1 = __shfl_sync(0xffffffffu, zx1, src);
+    s.zx0 = __shfl_sync(0xffffffffu, zx0, src);
+    s.zx1 = __shfl_sync(0xffffffffu, zx1, src);
     // a draft row that is not streamed (probabilities): q(x) read directly
-    if (!(FLAGS & kFRow1) && L.row1 != nullptr)
-      zx1 = load1<T1>(reinterpret_cast<const unsigned char*>(L.row1), L.x);
-  }
-  const double L0 = (double)G0 + log2(S0);
-  const double L1 = (double)G1 + log2(S1);
-  int err = 0;
-  if (flags & kPTimeout) err |= SV_DEV_TIMEOUT;
-  if ((FLAGS & kFStats0) && G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
-  if ((FLAGS & kFStats1) && L.row1 != nullptr && G1 == -INFINITY) err |= SV_DEV_NO_FINITE;
-  const bool skipped = prm.kind != kKindRows && (flags & kPSkipped);
-
-  if (FLAGS & kFTopk0) {
-    const int K = prm.K;
-    unsigned long long* lists = prm.cand + (size_t)r * nchunk * K;
-    const unsigned long long kk = row_topk_merge(lists, nchunk, K);
-    __syncwarp();
-    for (int t = lane; t < nchunk * K; t += 32) lists[t] = 0ull;
-    if (!skipped) {
-      const double ln2 = 0.69314718055994530942;
-      const bool rows = prm.kind == kKindRows;
-      const size_t orow = rows ? (size_t)r : (size_t)L.b * (prm.k + 1) + L.i;
-      // a failed row of a plain top-K call reads as NaN; chain rows are
-      // judged by the caller of the chain (accepted_len -1)
-      const bool nan_out = rows && err != 0;
-      double lp = -INFINITY;
-      int j = -1;
-      if (lane < K) {
-        j = key_index(kk);
-        lp = ((double)key_value(kk) * (double)prm.c - L0) * ln2;
-        prm.topk_logp[orow * K + lane] = nan_out ? NAN : (float)lp;
-        prm.topk_idx[orow * K + lane] = j;
-      }
-      if (lane == 0) prm.lse[orow] = nan_out ? NAN : (float)(L0 * ln2);
-      if (!rows && L.row1 != nullptr) {
-        // KL(p~ || q) over the renormalised top-K of the target row
-        double m = lp;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
-        double s = (lane < K) ? exp(lp - m) : 0.0;
-        s = warp_sum(s);
-        const double lse_k = m + log(s);
-        double term = 0.0;
-        if (lane < K && j >= 0 && j < prm.V) {
-          const float zd = load1<T1>(reinterpret_cast<const unsigned char*>(L.row1), j);
-          const double log_pt = lp - lse_k;
-          const double pt = exp(log_pt);
-          const double log_q = (FLAGS & kFStats1) ? ((double)zd * (double)prm.c - L1) * ln2
-                                                  : log((double)zd);
-          term = (pt == 0.0) ? 0.0 : pt * (log_pt - log_q);
-        }
-        term = warp_sum(term);
-        if (lane == 0) prm.kl[(size_t)L.b * prm.k + L.i] = (float)term;
-      }
+    if (!(FLAGS & kFRow1) && prm.rows1 != nullptr && prm.kind != kKindRows) {
+      const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, x);
+      if (L.row1 != nullptr) s.zx1 = load1<T1>(L.row1, x);
     }
   }
-  if (lane != 0) return;
-  if (prm.kind == kKindRows && (FLAGS & kFTopk0)) {
-    // a plain top-K call has no second pass: no record
-    if (err) set_status(prm.status, err);
-    prm.row_counter[r] = 0u;
-    return;
-  }
+  s.L0 = (double)s.G0 + log2(s.S0);
+  s.L1 = (double)s.G1 + log2(s.S1);
+  return s;
+}
+
+// A completed row's record: code (RowCode) and error bits (lane-uniform, no
+// side effects).  Chain sampling takes the ratio test u * q(x) < p(x) in
+// float64 from the row's log-partitions; greedy chains compare the draft
+// token with the argmax.
+template <int FLAGS>
+__device__ __forceinline__ RowRec row_decide(const StreamParams& prm, int r, int x,
+                                             const RowSum& s, int* err_out) {
   RowRec rec;
-  rec.G0 = G0;
-  rec.G1 = G1;
-  rec.S0 = S0;
-  rec.S1 = S1;
-  rec.L0 = L0;
-  rec.L1 = L1;
-  rec.argmax = key_index(key);
-  int code = kRowAccepted;
+  rec.G0 = s.G0;
+  rec.G1 = s.G1;
+  rec.S0 = s.S0;
+  rec.S1 = s.S1;
+  rec.L0 = s.L0;
+  rec.L1 = s.L1;
+  rec.argmax = key_index(s.key);
+  int err = 0, code = kRowAccepted;
+  if (s.flags & kPTimeout) err |= SV_DEV_TIMEOUT;
+  if ((FLAGS & kFStats0) && s.G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
   if (prm.kind != kKindRows) {
-    const int i = L.i, b = L.b, k = prm.k;
-    if (skipped) {
+    const int i = fast_div(r, prm.div_B), b = r - i * prm.B, k = prm.k;
+    if ((FLAGS & kFStats1) && i < k && s.G1 == -INFINITY) err |= SV_DEV_NO_FINITE;
+    if (s.flags & kPSkipped) {
       err = 0;
       code = kRowSkipped;
     } else if (prm.kind == kKindChainSample) {
-      if (i < k && !hm) err |= SV_DEV_BAD_TOKEN;
+      if (i < k && !s.hx) err |= SV_DEV_BAD_TOKEN;
       if (!err && i < k) {
         const double c = (double)prm.c;
-        const double px = exp2((double)zx0 * c - L0);
-        const double qx = (FLAGS & kFStats1) ? exp2((double)zx1 * c - L1) : (double)zx1;
+        const double px = exp2((double)s.zx0 * c - s.L0);
+        const double qx = (FLAGS & kFStats1) ? exp2((double)s.zx1 * c - s.L1) : (double)s.zx1;
         const double u = (double)prm.u[(size_t)b * (k + 1) + i];
         code = (u * qx < px) ? kRowAccepted : kRowRejected;
       }
     } else {  // greedy: accept iff the draft token is the argmax
-      if (i < k && (L.x < 0 || L.x >= prm.V)) err |= SV_DEV_BAD_TOKEN;
-      if (!err && i < k) code = (L.x == rec.argmax) ? kRowAccepted : kRowRejected;
+      if (i < k && (x < 0 || x >= prm.V)) err |= SV_DEV_BAD_TOKEN;
+      if (!err && i < k) code = (x == rec.argmax) ? kRowAccepted : kRowRejected;
     }
-    if (code == kRowRejected && !err) atomicMax(&prm.req_reject[b], (uint32_t)(k - i));
   }
-  if (err) {
-    set_status(prm.status, err);
-    code = kRowError;
-  }
+  if (err) code = kRowError;
   rec.code = code;
-  prm.rec[r] = rec;
-  prm.row_counter[r] = 0u;
+  *err_out = err;
+  return rec;
+}
+
+// Top-K outputs of a completed row (kFTopk0; warp-collective): merge the
+// row's lists and return them to zero; with `outputs`, write the row's top-K
+// log-probabilities, indices and lse (and, for a chain row with a draft row,
+// KL(p~ || q)).  L0/L1: the row's log2-partitions.  A failed row of a plain
+// top-K call reads as NaN.
+template <class T0, class T1, int FLAGS>
+__device__ __noinline__ void row_outputs(const StreamParams& prm, int r, int x, double L0,
+                                         double L1, int err, bool outputs, bool stat) {
+  const int lane = threadIdx.x & 31;
+  const SlotMap m = slot_map(prm, r, stat);
+  const int K = prm.K;
+  const unsigned long long kk = row_topk_merge(prm.cand, m, K);
+  __syncwarp();
+  for (int q = 0; q < m.nseg; ++q) {
+    const long long sq = slot_at(m, q);
+    if (lane < K) prm.cand[sq * K + lane] = 0ull;
+  }
+  if (!outputs) return;
+  const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, x);
+  const double ln2 = 0.69314718055994530942;
+  const bool rows = prm.kind == kKindRows;
+  const size_t orow = rows ? (size_t)r : (size_t)L.b * (prm.k + 1) + L.i;
+  const bool nan_out = rows && err != 0;
+  double lp = -INFINITY;
+  int j = -1;
+  if (lane < K) {
+    j = key_index(kk);
+    lp = ((double)key_value(kk) * (double)prm.c - L0) * ln2;
+    prm.topk_logp[orow * K + lane] = nan_out ? NAN : (float)lp;
+    prm.topk_idx[orow * K + lane] = j;
+  }
+  if (lane == 0) prm.lse[orow] = nan_out ? NAN : (float)(L0 * ln2);
+  if (!rows && L.row1 != nullptr) {
+    // KL(p~ || q) over the renormalised top-K of the target row
+    double mx = lp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    double se = (lane < K) ? exp(lp - mx) : 0.0;
+    se = warp_sum(se);
+    const double lse_k = mx + log(se);
+    double term = 0.0;
+    if (lane < K && j >= 0 && j < prm.V) {
+      const float zd = load1<T1>(L.row1, j);
+      const double log_pt = lp - lse_k;
+      const double pt = exp(log_pt);
+      const double log_q =
+          (FLAGS & kFStats1) ? ((double)zd * (double)prm.c - L1) * ln2 : log((double)zd);
+      term = (pt == 0.0) ? 0.0 : pt * (log_pt - log_q);
+    }
+    term = warp_sum(term);
+    if (lane == 0) prm.kl[(size_t)L.b * prm.k + L.i] = (float)term;
+  }
+}
+
+// Return row r's records to zero (warp-collective).
+__device__ __forceinline__ void row_zero_records(const StreamParams& prm, int r, bool stat) {
+  const int lane = threadIdx.x & 31;
+  const SlotMap m = slot_map(prm, r, stat);
+  for (int q = lane; q < m.nseg; q += 32) prm.part[slot_at(m, q)] = Partial{};
+}
+
+// In-stream completion (dynamic schedule): the warp whose count completed row
+// r decides it, publishes its record (and a rejection to the request's
+// rejection word, so that later positions are skipped) and commits it.
+template <class T0, class T1, int FLAGS>
+__device__ __noinline__ void row_complete(const StreamParams& prm, int r, int x) {
+  const int lane = threadIdx.x & 31;
+  const RowSum s = row_combine<T0, T1, FLAGS>(prm, r, x, false);
+  int err = 0;
+  const RowRec rec = row_decide<FLAGS>(prm, r, x, s, &err);
+  if (lane == 0) {
+    if (rec.code == kRowRejected) {
+      const int i = fast_div(r, prm.div_B), b = r - i * prm.B;
+      atomicMax(&prm.req_reject[b], (uint32_t)(prm.k - i));
+    }
+    if (err) set_status(prm.status, err);
+    // a plain top-K call has no second pass: no record
+    if (!(prm.kind == kKindRows && (FLAGS & kFTopk0))) prm.rec[r] = rec;
+    prm.row_counter[r] = 0u;
+  }
+  if (FLAGS & kFTopk0) row_outputs<T0, T1, FLAGS>(prm, r, x, s.L0, s.L1, err, rec.code != kRowSkipped, false);
+  row_zero_records(prm, r, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -570,6 +660,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   const float c = prm.c;
   const int K = prm.K;
   const unsigned kmask = K >= 32 ? 0xffffffffu : ((1u << K) - 1u);
+  pdl_launch_dependents();  // the finisher may be scheduled as resources free up
   if (lane == 0 && use_bulk) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
@@ -632,8 +723,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   // [g * total / NW, (g + 1) * total / NW) and merges consecutive items of one
   // row into one record.  Dynamic mode: first items g and g + NW, then the
   // stripe counters.
-  const long long lo = stat ? (long long)gwarp * total / nwarps : 0;
-  const long long hi = stat ? (long long)(gwarp + 1) * total / nwarps : 0;
+  const int nws = prm.nwarps_eff;
+  const long long lo = (stat && gwarp < nws) ? (long long)gwarp * total / nws : 0;
+  const long long hi = (stat && gwarp < nws) ? (long long)(gwarp + 1) * total / nws : 0;
   auto stat_item = [&](long long t) -> int { return t < hi ? (int)t : total; };
   int cur = stat ? stat_item(lo) : gwarp, cur_np, cur_x;
   {
