@@ -26,17 +26,17 @@ int env_int(const char* name) {
 
 int forced_cluster() {
   const int c = env_int("SV_CLUSTER_CTAS");
-  return (c == 1 || c == 2 || c == 4 || c == 8 || c == 16) ? c : 0;
+  return (c >= 1 && c <= kMaxCluster) ? c : 0;
 }
 
-// Finishing plans: every power-of-two cluster size C whose chunk of
+// Finishing plans: every cluster size C (1..16) whose chunk of
 // ceil(V / C) elements fits the shared-memory limit, C ascending.
 template <class XB>
 int feasible_plans(int V, int tb, int db, XB x_bytes, bool bulk_ok, int rows_bytes, RowPlan* plans) {
   if (V < 1 || V > kMaxV) return 0;
   const int forced = forced_cluster();
   int n = 0;
-  for (int C = 1; C <= kMaxCluster; C *= 2) {
+  for (int C = 1; C <= kMaxCluster; ++C) {
     if (forced && C != forced) continue;
     const int L = (int)align_up((size_t)((V + C - 1) / C), kVec);
     if (L > kMaxChunk) continue;
@@ -539,7 +539,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
                                           : launch_blocks(chain_greedy_finish<F32>, fp, B, gsm, s));
   }
 
-  RowPlan plans[8];
+  RowPlan plans[kMaxCluster];
   const int np = feasible_plans(
       V, te, de,
       [](int, int npc) {

@@ -198,6 +198,15 @@ __device__ __forceinline__ uint32_t load_relaxed_u32(const uint32_t* p) {
 // static partition, one per run: the row start unless a warp range starts
 // there, and every warp range start inside the row.  Warp w's range starts at
 // floor(w * total / NWs) (total = rows * slots per row, NWs = prm.nwarps_eff).
+// floor(num / den) for 0 <= num < 2^53, 0 < den: a float64 estimate, then an
+// exact integer correction (avoids a 64-bit integer division).
+__device__ __forceinline__ long long floor_div(long long num, long long den) {
+  long long q = (long long)((double)num / (double)den);
+  if (q * den > num) --q;
+  else if ((q + 1) * den <= num) ++q;
+  return q;
+}
+
 struct SlotMap {
   long long a;      // first slot of the row
   long long total;  // slots of the stream
@@ -220,11 +229,11 @@ __device__ __forceinline__ SlotMap slot_map(const StreamParams& p, int r, bool s
   }
   const long long nw = p.nwarps_eff;
   const long long e = m.a + p.nchunk;
-  const long long wA = (m.a * nw + m.total - 1) / m.total;  // ceil
-  const long long wB = (e * nw + m.total - 1) / m.total;
+  const long long wA = floor_div(m.a * nw + m.total - 1, m.total);  // ceil
+  const long long wB = floor_div(e * nw + m.total - 1, m.total);
   m.nw = (int)nw;
   m.wA = (int)wA;
-  m.head = (wA >= wB || (wA * m.total) / nw != m.a) ? 1 : 0;
+  m.head = (wA >= wB || floor_div(wA * m.total, nw) != m.a) ? 1 : 0;
   m.nseg = m.head + (int)(wB - wA);
   return m;
 }
@@ -232,7 +241,7 @@ __device__ __forceinline__ SlotMap slot_map(const StreamParams& p, int r, bool s
 __device__ __forceinline__ long long slot_at(const SlotMap& m, int q) {
   if (m.nw == 0) return m.a + q;
   if (m.head && q == 0) return m.a;
-  return ((long long)(m.wA + q - m.head) * m.total) / m.nw;
+  return floor_div((long long)(m.wA + q - m.head) * m.total, m.nw);
 }
 
 // Top K keys of a row from its slots' lists (each sorted, best first), best
@@ -661,6 +670,25 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   const int K = prm.K;
   const unsigned kmask = K >= 32 ? 0xffffffffu : ((1u << K) - 1u);
   pdl_launch_dependents();  // the finisher may be scheduled as resources free up
+  // Static schedule: this warp's pieces [lo, hi); an item is a run of them
+  // within one row (the record slot is the run's first piece).
+  const int nws = prm.nwarps_eff;
+  const long long lo = (stat && gwarp < nws) ? (long long)gwarp * total / nws : 0;
+  const long long hi = (stat && gwarp < nws) ? (long long)(gwarp + 1) * total / nws : 0;
+  auto run_end = [&](int item) -> long long {  // static: one past the run's last piece
+    const long long re = (long long)(fast_div(item, prm.div_nchunk) + 1) * nchunk;
+    return re < hi ? re : hi;
+  };
+  auto next_run = [&](int item) -> int {  // static: the run after the one starting at item
+    if (item >= total) return total;
+    const long long e = run_end(item);
+    return e < hi ? (int)e : total;
+  };
+  // Elements of an item whose first piece is piece ch of its row.
+  auto item_len = [&](int item, int ch) -> int {
+    if (!stat) return min(W, V - ch * W);
+    return (int)min((run_end(item) - item) * (long long)kPiece, (long long)(V - ch * kPiece));
+  };
   if (lane == 0 && use_bulk) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
@@ -689,7 +717,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       const int i = fast_div(r, prm.div_B);
       skip = __shfl_sync(0xffffffffu, rj > (uint32_t)(prm.k - i) ? 1 : 0, 0);
     }
-    const int len = min(W, V - ch * W);
+    const int len = item_len(item, ch);
     if (lane == 0 && !skip) {
       const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, -1);
       IssueDesc d;
@@ -723,11 +751,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   // [g * total / NW, (g + 1) * total / NW) and merges consecutive items of one
   // row into one record.  Dynamic mode: first items g and g + NW, then the
   // stripe counters.
-  const int nws = prm.nwarps_eff;
-  const long long lo = (stat && gwarp < nws) ? (long long)gwarp * total / nws : 0;
-  const long long hi = (stat && gwarp < nws) ? (long long)(gwarp + 1) * total / nws : 0;
-  auto stat_item = [&](long long t) -> int { return t < hi ? (int)t : total; };
-  int cur = stat ? stat_item(lo) : gwarp, cur_np, cur_x;
+  int cur = stat ? (lo < hi ? (int)lo : total) : gwarp, cur_np, cur_x;
   {
     uint32_t rj;
     int x;
@@ -735,7 +759,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     cur_np = pieces_of(cur, rj, 0);
     cur_x = __shfl_sync(0xffffffffu, x, 0);
   }
-  int nxt = stat ? stat_item(lo + 1) : gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
+  int nxt = stat ? next_run(cur) : gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
   uint32_t nxt_rj = 0u;
   // Lane 0: the stripe counter and the number of fetches it will receive.
   const int stripe = gwarp % kStripes;
@@ -769,7 +793,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     prefetch(nxt, nxt_rj, nxt_x);
     if (!stat) pend = fetch();  // every warp fetches at least once
   }
-  nxt2 = stat ? stat_item(lo + 2) : take(pend);
+  nxt2 = stat ? next_run(nxt) : take(pend);
   if (lane == 0) {
     prefetch(nxt2, nxt2_rj, nxt2_x);
     if (!stat && nxt2 < total) pend = fetch();
@@ -845,7 +869,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     const int r = fast_div(cur, prm.div_nchunk);
     const int ch = cur - r * nchunk;
     const RowLoc L = locate_row<T0, T1, FLAGS>(prm, r, cur_x);
-    const int clen = min(W, V - ch * W);
+    const int clen = item_len(cur, ch);
     const bool has1 = (FLAGS & kFRow1) && L.row1 != nullptr;
     if (run_first < 0) {
       run_first = cur;
@@ -957,8 +981,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
 
     // The run ends at a row boundary, at the end of the warp's range, and
     // after every item in dynamic mode.
-    const bool run_end = !stat || nxt >= total || ch == nchunk - 1;
-    if (run_end) {
+    {
     // Per-run reduction and record.
     Partial pr;
     pr.G0 = pr.G1 = -INFINITY;
@@ -1015,7 +1038,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     nxt_np = -1;
     nxt_rj = nxt2_rj;
     nxt_x = nxt2_x;
-    nxt2 = nxt2 < total ? (stat ? stat_item((long long)nxt2 + 1) : take(pend)) : total;
+    nxt2 = nxt2 < total ? (stat ? next_run(nxt2) : take(pend)) : total;
     if (lane == 0) {
       prefetch(nxt2, nxt2_rj, nxt2_x);
       if (!stat && nxt2 < total) pend = fetch();

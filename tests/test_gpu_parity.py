@@ -358,7 +358,7 @@ def test_deterministic_and_workspace_reuse(kd256):
         assert bitwise_equal(a[key], c[key]), key
 
 
-@pytest.mark.parametrize("C", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("C", [1, 2, 3, 4, 8, 12, 16])
 def test_every_cluster_size(monkeypatch, C):
     """The row plan's cluster size must not change any result."""
     monkeypatch.setenv("SV_CLUSTER_CTAS", str(C))
