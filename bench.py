@@ -33,9 +33,10 @@ from speculative_decoding_verification_94_b200 import inputs  # noqa: E402
 METRIC = "verified rows/s"
 UNIT = "rows/s"
 L2_BYTES = 126 * 1024 * 1024
-# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the chain
-# kernel, from profiles/ (None until a capture of the current kernel exists).
-NCU_TRAFFIC = {}
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per call (stream kernel +
+# finisher, one full capture of each on this workload); absent for a workload
+# without a capture of the current kernels.
+NCU_TRAFFIC = {"qwen_chain_verify": (68.114176 + 0.710912 + 18.583552) * 1e6}
 # kernels one verification call launches: the streaming pass and the finisher
 LAUNCHES_PER_CALL = 2
 
