@@ -165,6 +165,38 @@ SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, co
                           void* stream);
 
 /*
+ * sv_verify_chain_noalloc -- sv_verify_chain without a caller-supplied
+ * workspace.  The pages have no counterpart: this is a convenience of this
+ * library for callers that cannot allocate device memory around a call, such
+ * as host code running under another framework's allocator, or a plugin
+ * interface that hands over only input and output pointers, so that they
+ * cannot own a workspace buffer.
+ *
+ *   Arguments, results and errors are those of sv_verify_chain.
+ *   The scratch is a fixed array of SV_NOALLOC_MAX_BYTES per device inside
+ *   libsv.  The first call on a device (with that device current) performs a
+ *   one-time setup that looks up the array's device address; make that first
+ *   call before any stream capture.
+ *   A call whose sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0)
+ *   exceeds SV_NOALLOC_MAX_BYTES returns SV_ERR_WORKSPACE and launches
+ *   nothing.  At V = 151936 that allows about B*(k+1) <= 570 target rows
+ *   without KD and about 90 with K = 32.
+ *   The array starts zero-filled and every completed call returns it to zero,
+ *   so nothing needs clearing.  All calls on a device share the one array:
+ *   calls that can run at the same time (on different streams, or from host
+ *   threads without mutual ordering) race on it and must be ordered by the
+ *   caller.
+ */
+#define SV_NOALLOC_MAX_BYTES (4u << 20)
+SV_API sv_status sv_verify_chain_noalloc(const void* target_logits, sv_dtype t_dtype,
+                                         const void* draft, sv_dtype d_dtype,
+                                         sv_draft_kind d_kind, const int32_t* draft_tokens,
+                                         const float* uniforms, int B, int k, int V,
+                                         float temperature, int32_t* accepted_len,
+                                         int32_t* out_tokens, const sv_kd_args* kd,
+                                         int32_t* device_status, void* stream);
+
+/*
  * sv_verify_tree_greedy -- greedy (T = 0) verification of B candidate trees
  * (reading notes section 3: EAGLE trees of depth s, top-t branching, n nodes).
  *

@@ -564,6 +564,43 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   return cuda_status(e);
 }
 
+// Scratch of sv_verify_chain_noalloc: one fixed, zero-initialised array per
+// device (every completed call returns it to zero), and its device address,
+// looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_ws[SV_NOALLOC_MAX_BYTES];
+static void* g_noalloc_ptr[64];
+
+static sv_status noalloc_workspace(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SV_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return SV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || p == nullptr)
+      return SV_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SV_OK;
+}
+
+sv_status sv_verify_chain_noalloc(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                                  sv_dtype d_dtype, sv_draft_kind d_kind,
+                                  const int32_t* draft_tokens, const float* uniforms, int B, int k,
+                                  int V, float temperature, int32_t* accepted_len,
+                                  int32_t* out_tokens, const sv_kd_args* kd,
+                                  int32_t* device_status, void* stream) {
+  const size_t need = sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0);
+  if (need > (size_t)SV_NOALLOC_MAX_BYTES) return SV_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const sv_status st = noalloc_workspace(&ws);
+  if (st != SV_OK) return st;
+  return sv_verify_chain(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens, uniforms, B,
+                         k, V, temperature, accepted_len, out_tokens, kd, ws,
+                         (size_t)SV_NOALLOC_MAX_BYTES, device_status, stream);
+}
+
 sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* node_tokens,
                                 const int32_t* parents, int B, int n, int V, int max_depth,
                                 int32_t* accepted_len, int32_t* out_tokens,

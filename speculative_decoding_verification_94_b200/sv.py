@@ -26,7 +26,7 @@ SV_DEV_BAD_TOKEN, SV_DEV_NO_FINITE, SV_DEV_TIMEOUT, SV_DEV_BAD_TREE = 0x1, 0x2, 
 SV_DEV_BAD_INDEX, SV_DEV_ERROR_MASK = 0x10, 0xFF
 SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
-EXPORTS = ("sv_verify_chain", "sv_verify_tree_greedy", "sv_extract_topk_kd", "sv_kd_kl_loss",
+EXPORTS = ("sv_verify_chain", "sv_verify_chain_noalloc", "sv_verify_tree_greedy", "sv_extract_topk_kd", "sv_kd_kl_loss",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
            "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size",
            "sv_device_status_check", "sv_status_string", "sv_version")
@@ -66,6 +66,9 @@ def lib() -> ctypes.CDLL:
             vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
             L.sv_verify_chain.argtypes = [vp, ci, vp, ci, ci, vp, vp, ci, ci, ci, cf, vp, vp,
                                           ctypes.POINTER(sv_kd_args), vp, sz, vp, vp]
+            L.sv_verify_chain_noalloc.argtypes = [vp, ci, vp, ci, ci, vp, vp, ci, ci, ci, cf, vp,
+                                                  vp, ctypes.POINTER(sv_kd_args), vp, vp]
+            L.sv_verify_chain_noalloc.restype = ci
             L.sv_verify_tree_greedy.argtypes = [vp, ci, vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, sz,
                                                 vp, vp]
             L.sv_extract_topk_kd.argtypes = [vp, ci, ci, ci, ci, cf, vp, vp, vp, vp, sz, vp, vp]
@@ -208,6 +211,52 @@ def sv_verify_chain(target: torch.Tensor, draft: torch.Tensor | None, draft_toke
         B, k, V, T, _p(o["accepted_len"]), _p(o["out_tokens"]), kd_ptr, _p(w), w.numel(),
         _p(device_status), _stream(dev, stream))
     _check(rc, "sv_verify_chain")
+    return o
+
+
+def sv_verify_chain_noalloc(target: torch.Tensor, draft: torch.Tensor | None,
+                            draft_tokens: torch.Tensor, uniforms: torch.Tensor | None,
+                            temperature: float, *, draft_kind: str = "logits",
+                            kd: dict | None = None, out: dict | None = None,
+                            device_status: torch.Tensor | None = None, stream=None) -> dict:
+    """sv_verify_chain with the library's fixed per-device scratch instead of a
+    workspace (see sv.h for its size limit and ordering rule).  Outputs are
+    allocated here unless given in `out`; the C call itself allocates nothing."""
+    _dev(target, "target")
+    B, P, V = target.shape
+    k = P - 1
+    dev = target.device
+    _dev(draft_tokens, "draft_tokens", torch.int32)
+    dk = SV_DRAFT_PROBS if draft_kind == "probs" else SV_DRAFT_LOGITS
+    if draft is not None:
+        _dev(draft, "draft")
+    if uniforms is not None:
+        _dev(uniforms, "uniforms", torch.float32)
+    o = dict(out or {})
+    o.setdefault("accepted_len", torch.empty(B, dtype=torch.int32, device=dev))
+    o.setdefault("out_tokens", torch.empty(B, P, dtype=torch.int32, device=dev))
+    kd_ptr = None
+    if kd is not None:
+        K = int(kd.get("K", 32))
+        o.setdefault("topk_logp", torch.empty(B, P, K, dtype=torch.float32, device=dev))
+        o.setdefault("topk_idx", torch.empty(B, P, K, dtype=torch.int32, device=dev))
+        o.setdefault("lse", torch.empty(B, P, dtype=torch.float32, device=dev))
+        o.setdefault("kl", torch.empty(B, k, dtype=torch.float32, device=dev))
+        o.setdefault("loss", torch.empty(B, dtype=torch.float32, device=dev))
+        o.setdefault("total", torch.empty(1, dtype=torch.float32, device=dev))
+        reward = _dev(kd["reward"], "reward", torch.float32)
+        wmode = SV_W_GROUP_NORM if kd.get("wmode", "raw") == "group_norm" else SV_W_RAW
+        kd_ptr = ctypes.byref(sv_kd_args(K, o["topk_logp"].data_ptr(), o["topk_idx"].data_ptr(),
+                                         o["lse"].data_ptr(), o["kl"].data_ptr(),
+                                         reward.data_ptr(), wmode, int(kd.get("group", 1)),
+                                         float(kd.get("clip", 0.0)), o["loss"].data_ptr(),
+                                         o["total"].data_ptr()))
+    rc = lib().sv_verify_chain_noalloc(
+        _p(target), _dtype_code(target), _p(draft),
+        _dtype_code(draft) if draft is not None else SV_F32, dk, _p(draft_tokens), _p(uniforms),
+        B, k, V, float(temperature), _p(o["accepted_len"]), _p(o["out_tokens"]), kd_ptr,
+        _p(device_status), _stream(dev, stream))
+    _check(rc, "sv_verify_chain_noalloc")
     return o
 
 
