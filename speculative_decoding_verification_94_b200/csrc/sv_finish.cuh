@@ -181,7 +181,7 @@ __device__ __forceinline__ void release_rows(const FinishParams& prm, int nrows,
 //   4. the CTA that owns the drawn token writes the request's outputs (the
 //      first CTA when there is no draw: failed rows or timeouts).
 template <class TT, class DT, int DKIND, bool KD>
-__global__ void __launch_bounds__(kThreads, 4) chain_sample_finish(const __grid_constant__ FinishParams prm) {
+__global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
@@ -199,13 +199,6 @@ __global__ void __launch_bounds__(kThreads, 4) chain_sample_finish(const __grid_
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   constexpr int RF = chain_sample_flags<DKIND, KD>();
   if (threadIdx.x == 0) sh.tok = -1;
-  // Row pair 0 (the most frequent place of the first rejection) is staged
-  // before the stream has finished: the logits are inputs, not its results.
-  const bool spec = use_bulk;
-  if (spec)
-    stage_chunks<TT, DT, true>(sh, tbuf, dbuf, row_ptr<TT>(prm.target, (size_t)b * P, V),
-                               row_ptr<DT>(prm.draft, (size_t)b * k, V), g, true,
-                               DKIND == kDraftProbs);
   pdl_wait();  // the stream's records are complete
 
   // 0. the request's rows and its first rejection
@@ -244,24 +237,11 @@ __global__ void __launch_bounds__(kThreads, 4) chain_sample_finish(const __grid_
     const bool pair = n < k;
     const void* trow = row_ptr<TT>(prm.target, (size_t)b * P + n, V);
     const void* drow = pair ? row_ptr<DT>(prm.draft, (size_t)b * k + n, V) : nullptr;
-    uint32_t phase = 0;
-    if (!spec) {
-      if (pair)
-        stage_chunks<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, use_bulk, DKIND == kDraftProbs);
-      else
-        stage_chunks<TT, DT, false>(sh, tbuf, dbuf, trow, drow, g, use_bulk, false);
-    } else if (n != 0) {
-      // the speculative copies land first, then the buffers take row pair n
-      if (threadIdx.x == 0) {
-        for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, true, 0);
-        if (pair)
-          issue_item_copies<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, policy_evict_first());
-        else
-          issue_item_copies<TT, DT, false>(sh, tbuf, dbuf, trow, drow, g, policy_evict_first());
-      }
-      phase = 1;
-    }
-    for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, use_bulk, phase);
+    if (pair)
+      stage_chunks<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, use_bulk, DKIND == kDraftProbs);
+    else
+      stage_chunks<TT, DT, false>(sh, tbuf, dbuf, trow, drow, g, use_bulk, false);
+    for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, use_bulk);
     __syncthreads();
     int mode = pair ? kModeResidual : kModeP;
     const float Gt = sh.Gt, Gd = sh.Gd;
@@ -375,8 +355,6 @@ __global__ void __launch_bounds__(kThreads, 4) chain_sample_finish(const __grid_
       }
     }
   } else {
-    if (spec && threadIdx.x == 0)  // no draw: the speculative copies land before exit
-      for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, true, 0);
     cluster.sync();  // every CTA has read the rows' records
   }
 
