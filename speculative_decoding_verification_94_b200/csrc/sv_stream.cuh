@@ -863,7 +863,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   int hx = 0;
   unsigned long long list = kNoKey;
   unsigned long long thr_key = kNoKey;
+  unsigned long long thr_floor = kNoKey;  // lower bound of the run's K-th best key
   float thr_val = -INFINITY;
+  bool seed = false;
   int run_first = -1;  // the item whose record slot the run writes
   while (cur < total) {
     const int r = fast_div(cur, prm.div_nchunk);
@@ -881,7 +883,9 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       hx = 0;
       list = kNoKey;
       thr_key = kNoKey;
+      thr_floor = kNoKey;
       thr_val = -INFINITY;
+      seed = true;
     }
 
     for (int p = 0; p < cur_np; ++p) {
@@ -938,6 +942,16 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
           }
         }
         if (FLAGS & kFTopk0) {
+          if (seed) {
+            // The smallest lane maximum of the run's first piece: every lane
+            // holds an element at least that large, so the run's K best (K <=
+            // 32) are too; nothing below it needs to enter the list.
+            const float t = order_float(__reduce_min_sync(0xffffffffu, float_order(pm)));
+            thr_floor = (unsigned long long)float_order(t) << 32;
+            thr_key = thr_floor > thr_key ? thr_floor : thr_key;
+            thr_val = key_value(thr_key);
+            seed = false;
+          }
 #pragma unroll
           for (int v = 0; v < kLaneVecs; ++v) {
             const int vi = v * 32 + lane;
@@ -954,7 +968,8 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
                   const unsigned long long key = topk_key(xs[q], e0 + sbase + q);
                   if (key > thr_key) {
                     warp_list_insert(list, key, kmask);
-                    thr_key = __shfl_sync(0xffffffffu, list, K - 1);
+                    const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
+                    thr_key = kth > thr_floor ? kth : thr_floor;
                   }
                 }
               }
