@@ -668,7 +668,6 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   const int gwarp = (int)blockIdx.x * kStreamWarps + warp;
   const float c = prm.c;
   const int K = prm.K;
-  const unsigned kmask = K >= 32 ? 0xffffffffu : ((1u << K) - 1u);
   pdl_launch_dependents();  // the finisher may be scheduled as resources free up
   // Static schedule: this warp's pieces [lo, hi); an item is a run of them
   // within one row (the record slot is the run's first piece).
@@ -952,29 +951,35 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
             thr_val = key_value(thr_key);
             seed = false;
           }
+          // Candidates are found lane-parallel in registers: each round, every
+          // lane offers its best key above the threshold that it has not yet
+          // offered; the 32 offers are sorted and merged into the list.
+          unsigned pmask = 0;  // this lane's vectors that can hold a candidate
 #pragma unroll
-          for (int v = 0; v < kLaneVecs; ++v) {
-            const int vi = v * 32 + lane;
-            unsigned m = __ballot_sync(0xffffffffu, vi < nv && vec_max(R, v) >= thr_val);
-            while (m) {
-              const int src = __ffs(m) - 1;
-              m &= m - 1;
-              const int sbase = (v * 32 + src) * kVec;
+          for (int v = 0; v < kLaneVecs; ++v)
+            if (v * 32 + lane < nv && vec_max(R, v) >= thr_val) pmask |= 1u << v;
+          unsigned long long last = ~0ull;
+          while (__any_sync(0xffffffffu, pmask != 0)) {
+            unsigned long long cand = kNoKey;
+            for (unsigned mm = pmask; mm; mm &= mm - 1) {
+              const int vi = (__ffs(mm) - 1) * 32 + lane;
               float xs[8];
-              load8<T0>(st, sbase, xs);  // every lane reads the source lane's vector
+              load8<T0>(st, vi * kVec, xs);  // (the stage is still this piece's)
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                if (sbase + q < n) {
-                  const unsigned long long key = topk_key(xs[q], e0 + sbase + q);
-                  if (key > thr_key) {
-                    warp_list_insert(list, key, kmask);
-                    const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
-                    thr_key = kth > thr_floor ? kth : thr_floor;
-                  }
+              for (int t = 0; t < 8; ++t) {
+                if (vi * kVec + t < n) {
+                  const unsigned long long key = topk_key(xs[t], e0 + vi * kVec + t);
+                  if (key > thr_key && key < last && key > cand) cand = key;
                 }
               }
             }
+            if (cand == kNoKey) pmask = 0;
+            if (!__any_sync(0xffffffffu, cand != kNoKey)) break;
+            list = warp_merge_desc(list, warp_sort_desc(cand));
+            const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
+            thr_key = kth > thr_floor ? kth : thr_floor;
             thr_val = thr_key == kNoKey ? -INFINITY : key_value(thr_key);
+            if (cand != kNoKey) last = cand;
           }
         }
       }
