@@ -974,8 +974,17 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
               }
             }
             if (cand == kNoKey) pmask = 0;
-            if (!__any_sync(0xffffffffu, cand != kNoKey)) break;
-            list = warp_merge_desc(list, warp_sort_desc(cand));
+            unsigned cm = __ballot_sync(0xffffffffu, cand != kNoKey);
+            if (!cm) break;
+            if (__popc(cm) <= 4) {  // few offers: insert them one by one
+              while (cm) {
+                const int src = __ffs(cm) - 1;
+                cm &= cm - 1;
+                warp_list_insert(list, __shfl_sync(0xffffffffu, cand, src), 0xffffffffu);
+              }
+            } else {
+              list = warp_merge_desc(list, warp_sort_desc(cand));
+            }
             const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
             thr_key = kth > thr_floor ? kth : thr_floor;
             thr_val = thr_key == kNoKey ? -INFINITY : key_value(thr_key);
