@@ -954,13 +954,20 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
           // Candidates are found lane-parallel in registers: each round, every
           // lane offers its best key above the threshold that it has not yet
           // offered; the 32 offers are sorted and merged into the list.
-          unsigned pmask = 0;  // this lane's vectors that can hold a candidate
+          // This lane's vectors that can hold a candidate.  The list holds
+          // only earlier pieces' keys here, so a value equal to the list's
+          // K-th cannot enter (larger index); the floor admits equal values.
+          unsigned pmask = 0;
+          const bool strict = thr_key != thr_floor;
 #pragma unroll
-          for (int v = 0; v < kLaneVecs; ++v)
-            if (v * 32 + lane < nv && vec_max(R, v) >= thr_val) pmask |= 1u << v;
+          for (int v = 0; v < kLaneVecs; ++v) {
+            const float vm = vec_max(R, v);
+            if (v * 32 + lane < nv && (vm > thr_val || (!strict && vm == thr_val))) pmask |= 1u << v;
+          }
           unsigned long long last = ~0ull;
           while (__any_sync(0xffffffffu, pmask != 0)) {
             unsigned long long cand = kNoKey;
+            int more = 0;  // keys above the threshold besides the offer
             for (unsigned mm = pmask; mm; mm &= mm - 1) {
               const int vi = (__ffs(mm) - 1) * 32 + lane;
               float xs[8];
@@ -969,11 +976,14 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
               for (int t = 0; t < 8; ++t) {
                 if (vi * kVec + t < n) {
                   const unsigned long long key = topk_key(xs[t], e0 + vi * kVec + t);
-                  if (key > thr_key && key < last && key > cand) cand = key;
+                  if (key > thr_key && key < last) {
+                    more += cand != kNoKey;
+                    if (key > cand) cand = key;
+                  }
                 }
               }
             }
-            if (cand == kNoKey) pmask = 0;
+            if (cand == kNoKey || more == 0) pmask = 0;  // nothing left after this offer
             unsigned cm = __ballot_sync(0xffffffffu, cand != kNoKey);
             if (!cm) break;
             if (__popc(cm) <= 4) {  // few offers: insert them one by one
