@@ -179,7 +179,7 @@ SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, co
  *   call before any stream capture.
  *   A call whose sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0)
  *   exceeds SV_NOALLOC_MAX_BYTES returns SV_ERR_WORKSPACE and launches
- *   nothing.  At V = 151936 that allows about B*(k+1) <= 290 target rows
+ *   nothing.  At V = 151936 that allows about B*(k+1) <= 570 target rows
  *   without KD and about 90 with K = 32.
  *   The array starts zero-filled and every completed call returns it to zero,
  *   so nothing needs clearing.  All calls on a device share the one array:

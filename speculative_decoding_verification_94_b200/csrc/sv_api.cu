@@ -161,13 +161,9 @@ static int stream_chunk(int V, long long nrows) {
   return w < cap ? w : cap;
 }
 
-// Static-schedule slot unit: half a piece, so that warp ranges balance to a
-// half piece; a whole piece when top-K lists are kept (one list per slot).
-static int slot_unit(int K) { return K > 0 ? kPiece : kPiece / 2; }
-
-// Record slots per row: one per slot unit, enough for either schedule (a
-// record per chunk of W >= kPiece elements, or one per run of slots).
-static int record_slots(int V, int K) { return (V + slot_unit(K) - 1) / slot_unit(K); }
+// Record slots per row: one per piece, enough for either schedule (a record
+// per chunk of W >= kPiece elements, or one per run of pieces).
+static int record_slots(int V) { return (V + kPiece - 1) / kPiece; }
 
 // Workspace: batch and item counters, per-request rejection words, per-row chunk
 // counters, row records, chunk partials and (top-K) chunk lists.  Every byte
@@ -253,10 +249,9 @@ static cudaError_t launch_stream(StreamParams& p, const StreamGeom& g, cudaStrea
   if ((e = sm_count(&sms)) != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   if (p.count < 0) p.count = stream_count_policy(p, (long long)per_sm * sms * kStreamWarps);
-  if (p.count == 0) {  // static partition into slots (one record slot each)
-    const int K = (FLAGS & kFTopk0) ? p.K : 0;
-    p.W = slot_unit(K);
-    p.nchunk = record_slots(p.V, K);
+  if (p.count == 0) {  // static partition into pieces (one record slot each)
+    p.W = kPiece;
+    p.nchunk = record_slots(p.V);
     p.div_nchunk = make_fastdiv(p.nchunk);
   }
   const long long items = (long long)p.nrows * p.nchunk;
@@ -402,19 +397,19 @@ extern "C" {
 
 size_t sv_verify_chain_workspace_size(int B, int k, int V, int K) {
   if (B <= 0 || k < 1 || V < 1) return 256;
-  return ws_layout(B, B * (k + 1), record_slots(V, K > 0 ? K : 0), K > 0 ? K : 0).bytes;
+  return ws_layout(B, B * (k + 1), record_slots(V), K > 0 ? K : 0).bytes;
 }
 size_t sv_verify_tree_workspace_size(int B, int n, int V) {
   if (B <= 0 || n < 1 || V < 1) return 256;
-  return ws_layout(B, B * n, record_slots(V, 0), 0).bytes;
+  return ws_layout(B, B * n, record_slots(V), 0).bytes;
 }
 size_t sv_extract_topk_workspace_size(int rows, int V, int K) {
   if (rows <= 0 || V < 1) return 256;
-  return ws_layout(rows, rows, record_slots(V, K > 0 ? K : 0), K > 0 ? K : 0).bytes;
+  return ws_layout(rows, rows, record_slots(V), K > 0 ? K : 0).bytes;
 }
 size_t sv_kd_kl_loss_workspace_size(int B, int k, int V) {
   if (B <= 0 || k < 1 || V < 1) return 256;
-  return ws_layout(B, B * k, record_slots(V, 0), 0).bytes;
+  return ws_layout(B, B * k, record_slots(V), 0).bytes;
 }
 
 static sv_status check_workspace(void* ws, size_t bytes, size_t need) {
@@ -464,7 +459,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   const int te = esize(t_dtype);
   const int de = greedy ? 0 : (d_kind == SV_DRAFT_PROBS ? 4 : esize(d_dtype));
   const StreamGeom sg = stream_geom(V, (long long)B * P, te, d_kind == SV_DRAFT_PROBS ? 0 : de);
-  const WsLayout wl = ws_layout(B, B * P, record_slots(V, K), K);
+  const WsLayout wl = ws_layout(B, B * P, record_slots(V), K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);
@@ -623,7 +618,7 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if ((long long)B * n > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
   const StreamGeom sg = stream_geom(V, (long long)B * n, esize(dt), 0);
-  const WsLayout wl = ws_layout(B, B * n, record_slots(V, 0), 0);
+  const WsLayout wl = ws_layout(B, B * n, record_slots(V), 0);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);
@@ -690,7 +685,7 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if (rows > 0x7fffffff / 64) return SV_ERR_UNSUPPORTED;
   const StreamGeom sg = stream_geom(V, rows, esize(dt), 0);
-  const WsLayout wl = ws_layout(rows, rows, record_slots(V, K), K);
+  const WsLayout wl = ws_layout(rows, rows, record_slots(V), K);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);
@@ -752,7 +747,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
   if ((long long)B * k > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
   const StreamGeom sg = stream_geom(V, (long long)B * k, esize(d_dtype), 0);
-  const WsLayout wl = ws_layout(B, B * k, record_slots(V, 0), 0);
+  const WsLayout wl = ws_layout(B, B * k, record_slots(V), 0);
   sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
   if (st != SV_OK) return st;
   const WsPtrs w = ws_carve(workspace, wl);

@@ -686,7 +686,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   // Elements of an item whose first piece is piece ch of its row.
   auto item_len = [&](int item, int ch) -> int {
     if (!stat) return min(W, V - ch * W);
-    return (int)min((run_end(item) - item) * (long long)W, (long long)(V - ch * W));
+    return (int)min((run_end(item) - item) * (long long)kPiece, (long long)(V - ch * kPiece));
   };
   if (lane == 0 && use_bulk) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
