@@ -36,7 +36,7 @@ L2_BYTES = 126 * 1024 * 1024
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per call (stream kernel +
 # finisher, one full capture of each on this workload); absent for a workload
 # without a capture of the current kernels.
-NCU_TRAFFIC = {"qwen_chain_verify": (68.114176 + 0.710912 + 18.583552) * 1e6}
+NCU_TRAFFIC = {"qwen_chain_verify": (68.115200 + 0.634624 + 18.584064) * 1e6}
 # kernels one verification call launches: the streaming pass and the finisher
 LAUNCHES_PER_CALL = 2
 
@@ -420,7 +420,7 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f32", "data": "synthetic",
                 "config": dict(cfg, l2=f"{ncopy} rotating input copies "
-                                       f"({ncopy * algo_bytes / 2**20:.0f} MiB > 2x L2)",
+                                       f"({ncopy * full_bytes / 2**20:.0f} MiB > 2x L2)",
                                parallelism=f"dp{world}" if world > 1 else "single"),
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                              "unit": "GB/s", "frac": achieved / peak,
