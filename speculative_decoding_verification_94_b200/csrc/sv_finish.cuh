@@ -248,21 +248,15 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
     const float invSt = (float)(1.0 / sh.St);
     const float invSd = (DKIND == kDraftLogits && pair) ? (float)(1.0 / sh.Sd) : 1.f;
     for (int attempt = 0; attempt < 2; ++attempt) {
-      // two pieces per iteration: independent exp2 chains for the scheduler
-      for (int p = 0; p < g.npieces; p += 2) {
-        float s2[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int e = (p + h) * kRound + (int)threadIdx.x * kVec;
-          s2[h] = 0.f;
-          if (p + h < g.npieces && e < g.nvec * kVec) {
-            float wv[8];
-            weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, wv);
-            s2[h] = seq_sum8(wv);
-          }
+      for (int p = 0; p < g.npieces; ++p) {
+        const int e = p * kRound + (int)threadIdx.x * kVec;
+        float s = 0.f;
+        if (e < g.nvec * kVec) {
+          float wv[8];
+          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, wv);
+          s = seq_sum8(wv);
         }
-        sums[p * kThreads + threadIdx.x] = s2[0];
-        if (p + 1 < g.npieces) sums[(p + 1) * kThreads + threadIdx.x] = s2[1];
+        sums[p * kThreads + threadIdx.x] = s;
       }
       piece_totals(sums, g.npieces, sh);
       if (threadIdx.x == 0) {

@@ -119,13 +119,9 @@ __device__ __forceinline__ void drain_pieces(RowShared& sh, const ChunkGeom& g, 
 // order (warp butterflies, then warps in index order).  Collective.
 __device__ __forceinline__ void piece_totals(const float* sums, int npieces, RowShared& sh) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int p = 0; p < npieces; p += 2) {  // two independent reductions at a time
-    const double v0 = warp_sum((double)sums[p * kThreads + threadIdx.x]);
-    const double v1 = p + 1 < npieces ? warp_sum((double)sums[(p + 1) * kThreads + threadIdx.x]) : 0.0;
-    if (lane == 0) {
-      sh.wsum[w][p] = v0;
-      if (p + 1 < npieces) sh.wsum[w][p + 1] = v1;
-    }
+  for (int p = 0; p < npieces; ++p) {
+    const double v = warp_sum((double)sums[p * kThreads + threadIdx.x]);
+    if (lane == 0) sh.wsum[w][p] = v;
   }
   __syncthreads();
   if ((int)threadIdx.x < npieces) {
