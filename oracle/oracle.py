@@ -71,9 +71,12 @@ def _lib(plant: int = 0) -> ctypes.CDLL:
         L.oracle_kl.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, ci, cd, f64p, f64p, ci]
         L.oracle_reward_loss.argtypes = [f64p, i32p, f64p, ci, ci, ci, ci, cd, f64p, f64p, f64p]
         L.oracle_softmax.argtypes = [vp, ci, ci, ci, cd, f64p, f64p]
+        L.oracle_kd_grad.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, cd, i32p, f64p, ci, ci,
+                                     cd, f64p, ci]
         L.oracle_max_threads.argtypes = []
         for name in ("oracle_verify_chain", "oracle_tree_greedy", "oracle_topk", "oracle_kl",
-                     "oracle_reward_loss", "oracle_softmax", "oracle_max_threads"):
+                     "oracle_reward_loss", "oracle_softmax", "oracle_kd_grad",
+                     "oracle_max_threads"):
             getattr(L, name).restype = ci
         _LIBS[plant] = L
     return _LIBS[plant]
@@ -231,6 +234,26 @@ def reward_loss(kl_values, accepted_len, reward, *, mode: int = W_RAW, group: in
                                    _ptr(total, ctypes.c_double))
     _check(rc, "reward_loss")
     return dict(w=w, loss=loss, total=float(total[0]))
+
+
+def kd_grad(topk_logp, topk_idx, draft, accepted_len, reward, temperature: float, *,
+            mode: int = W_RAW, group: int = 1, clip: float = 0.0, threads: int = 0):
+    """d loss / d draft logits [B, k, V] (float64) of the reward-weighted KD loss."""
+    lp = _np(topk_logp, np.float64)
+    ix = _np(topk_idx, np.int32)
+    B, P, K = lp.shape
+    k = P - 1
+    d, ddt = _raw(draft)
+    V = d.shape[-1]
+    acc = _np(accepted_len, np.int32)
+    r = _np(reward, np.float64)
+    g = np.zeros((B, k, V), np.float64)
+    rc = _lib().oracle_kd_grad(_ptr(lp, ctypes.c_double), _ptr(ix, ctypes.c_int32), B, k, K,
+                               d.ctypes.data, ddt, V, float(np.float32(temperature)),
+                               _ptr(acc, ctypes.c_int32), _ptr(r, ctypes.c_double), mode, group,
+                               float(clip), _ptr(g, ctypes.c_double), threads)
+    _check(rc, "kd_grad")
+    return g
 
 
 def softmax(logits, temperature: float) -> dict:

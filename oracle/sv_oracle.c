@@ -541,6 +541,74 @@ int oracle_reward_loss(const double* kl, const int32_t* accepted_len, const doub
   return OR_OK;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Gradient of the reward-weighted KD loss with respect to the draft logits   */
+/* ([RWKD]; reading notes section 4, Algorithm 1 step 3: the drafter's        */
+/* gradient flows into the current q_theta only, never into the stored       */
+/* log q).  From d log q_j / d z_l = (delta_jl - q_l) / T and sum_j p~_j = 1:  */
+/*   d loss_b / d z_d[b, i, l] = w_b [i < n_b] (q_il - p~_il [l in K]) / T.    */
+/* Logit drafts only; w_b as in oracle_reward_loss.  grad [B, k, V].          */
+/* ------------------------------------------------------------------------ */
+int oracle_kd_grad(const double* topk_logp, const int32_t* topk_idx, int B, int k, int K,
+                   const void* draft, int d_dtype, int V, double T,
+                   const int32_t* accepted_len, const double* reward, int mode, int group,
+                   double clip, double* grad, int nthreads) {
+  if (B < 0 || k < 1 || K < 1 || K > V || !(T > 0.0) || !topk_logp || !topk_idx || !draft ||
+      !accepted_len || !reward || !grad)
+    return OR_BAD_ARG;
+  if (mode == OR_W_GROUP_NORM && (group < 1 || B % group != 0)) return OR_BAD_ARG;
+  set_threads(nthreads);
+  const int P = k + 1;
+  int err = OR_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int row = 0; row < B * k; ++row) {
+    int b = row / k, i = row % k;
+    double* g = grad + (size_t)row * V;
+    for (int j = 0; j < V; ++j) g[j] = 0.0;
+    double wb = reward[b];
+    if (mode == OR_W_GROUP_NORM) {
+      int g0 = (b / group) * group;
+      double gs = 0.0;
+      for (int t = g0; t < g0 + group; ++t) gs += reward[t];
+      wb = gs == 0.0 ? 0.0 : reward[b] / gs;
+    }
+    if (clip > 0.0) wb = wb > clip ? clip : (wb < -clip ? -clip : wb);
+    int n = accepted_len[b];
+    if (n < 0 || n > k) {
+#pragma omp atomic write
+      err = OR_BAD_ARG;
+      continue;
+    }
+    if (i >= n || wb == 0.0) continue;
+    size_t drow = (size_t)row * (size_t)V;
+    double lse_d = softmax_row(draft, d_dtype, drow, V, T, NULL);
+    if (isnan(lse_d)) {
+#pragma omp atomic write
+      err = OR_NO_FINITE;
+      continue;
+    }
+    for (int j = 0; j < V; ++j) g[j] = wb * exp(load_value(draft, d_dtype, drow + (size_t)j) / T - lse_d) / T;
+    const double* lp = topk_logp + ((size_t)b * P + i) * K;
+    const int32_t* ix = topk_idx + ((size_t)b * P + i) * K;
+    double mk = -INFINITY;
+    for (int t = 0; t < K; ++t)
+      if (lp[t] > mk) mk = lp[t];
+    double sk = 0.0;
+    for (int t = 0; t < K; ++t) sk += exp(lp[t] - mk);
+    double lse_k = mk + log(sk);
+    for (int t = 0; t < K; ++t) {
+      int j = ix[t];
+      if (j < 0 || j >= V) {
+#pragma omp atomic write
+        err = OR_BAD_TOKEN;
+        continue;
+      }
+      g[j] -= wb * exp(lp[t] - lse_k) / T;
+    }
+  }
+  return err;
+}
+
 /* Temperature softmax of `rows` rows (exposed so that the tests can compare
  * the oracle's normalisation against an independent library routine). */
 int oracle_softmax(const void* logits, int dtype, int rows, int V, double T, double* p,

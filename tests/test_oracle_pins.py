@@ -359,3 +359,54 @@ def test_oracle_is_thread_count_invariant(oracle):
     b = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 0.7, threads=8)
     for key in ("accepted_len", "out_tokens", "p_x", "cdf_margin"):
         assert np.array_equal(a[key], b[key], equal_nan=True)
+
+
+# --------------------------------------------------------------------------
+# KD gradient into the draft logits (reading notes section 4, Algorithm 1
+# step 3: gradient only into the current q_theta; section 5: reward weights).
+# --------------------------------------------------------------------------
+def _kd_case(seed, B=4, k=2, V=12, K=4, T=0.8):
+    rng = np.random.default_rng(seed)
+    # logits on a 1/1024 grid: z +- 1/1024 is exact in float32
+    draft = np.round(rng.normal(0, 1.5, (B, k, V)) * 1024) / 1024
+    lp = np.sort(rng.normal(-2, 1, (B, k + 1, K)), axis=-1)[..., ::-1].copy()
+    ix = np.stack([rng.permutation(V)[:K] for _ in range(B * (k + 1))]).reshape(B, k + 1, K)
+    acc = np.array([k, 1, 0, 2][:B], np.int32)
+    reward = np.array([0.85, 0.3, 0.6, 0.0][:B])
+    return draft.astype(np.float32), lp, ix.astype(np.int32), acc, reward, T
+
+
+def _kd_loss(oracle, draft, lp, ix, acc, reward, T, mode, group):
+    kl = oracle.kl(lp, ix, torch.from_numpy(draft), T)["kl"]
+    return oracle.reward_loss(kl, acc, reward, mode=mode, group=group)["total"]
+
+
+@pytest.mark.parametrize("mode,group", [(0, 1), (1, 2)])
+def test_kd_gradient_matches_central_differences(oracle, mode, group):
+    draft, lp, ix, acc, reward, T = _kd_case(3)
+    g = oracle.kd_grad(lp, ix, torch.from_numpy(draft), acc, reward, T, mode=mode, group=group)
+    h = 1.0 / 1024
+    num = np.zeros_like(g)
+    for b in range(draft.shape[0]):
+        for i in range(draft.shape[1]):
+            for j in range(draft.shape[2]):
+                zp, zm = draft.copy(), draft.copy()
+                zp[b, i, j] += h
+                zm[b, i, j] -= h
+                num[b, i, j] = (_kd_loss(oracle, zp, lp, ix, acc, reward, T, mode, group) -
+                                _kd_loss(oracle, zm, lp, ix, acc, reward, T, mode, group)) / (2 * h)
+    scale = np.abs(g).max()
+    assert scale > 0
+    assert np.abs(num - g).max() <= 2e-5 * scale, np.abs(num - g).max() / scale
+
+
+def test_kd_gradient_rows_sum_to_zero_and_vanish_where_unused(oracle):
+    draft, lp, ix, acc, reward, T = _kd_case(4)
+    g = oracle.kd_grad(lp, ix, torch.from_numpy(draft), acc, reward, T)
+    for b in range(draft.shape[0]):
+        for i in range(draft.shape[1]):
+            if i >= acc[b] or reward[b] == 0.0:
+                assert not g[b, i].any()
+            else:
+                assert abs(g[b, i].sum()) < 1e-12 * max(1.0, np.abs(g[b, i]).max())
+                assert g[b, i].max() > 0 > g[b, i].min()
