@@ -254,6 +254,29 @@ SV_API sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, 
                         float* total, void* workspace, size_t workspace_bytes,
                         int32_t* device_status, void* stream);
 
+/*
+ * sv_kd_grad -- gradient of the reward-weighted KD loss with respect to the
+ * draft logits, the drafter update of the reading notes, section 4 (Algorithm
+ * 1 step 3: the gradient flows into the current q_theta only) with the reward
+ * weights of section 5.  With q = softmax(draft[b, i] / T) and p~ as in
+ * sv_kd_kl_loss:
+ *   grad[b, i, j] = w_b * (q_j - p~_j [j in topk_idx[b, i, :]]) / T  for i < accepted_len[b],
+ *   grad[b, i, j] = 0                                                 otherwise,
+ * which is d loss[b] / d draft[b, i, j] for the loss of sv_kd_kl_loss.
+ *   topk_logp, topk_idx [B, k+1, K]; draft [B, k, V] logits (d_dtype);
+ *   accepted_len [B]; reward [B]; grad [B, k, V] fp32 out.  T > 0.
+ *   A row whose statistics fail (no finite logit) or whose top-K indices are
+ *   out of range is set to NaN, with the matching SV_DEV_* bit.
+ *   workspace: sv_kd_grad_workspace_size(B, k, V) bytes.
+ */
+SV_API size_t sv_kd_grad_workspace_size(int B, int k, int V);
+SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
+                            const void* draft, sv_dtype d_dtype, int V, float temperature,
+                            const int32_t* accepted_len, const float* reward,
+                            sv_weight_mode wmode, int group, float clip, float* grad,
+                            void* workspace, size_t workspace_bytes, int32_t* device_status,
+                            void* stream);
+
 /* Map a device status word (read back by the caller) to a host status:
  * SV_OK, SV_ERR_TIMEOUT if SV_DEV_TIMEOUT is set, else SV_ERR_DEVICE_CHECK
  * if any other error bit is set.  Informational bits are ignored. */

@@ -813,6 +813,87 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   return cuda_status(e);
 }
 
+size_t sv_kd_grad_workspace_size(int B, int k, int V) { return sv_kd_kl_loss_workspace_size(B, k, V); }
+
+sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
+                     const void* draft, sv_dtype d_dtype, int V, float temperature,
+                     const int32_t* accepted_len, const float* reward, sv_weight_mode wmode,
+                     int group, float clip, float* grad, void* workspace, size_t workspace_bytes,
+                     int32_t* device_status, void* stream) {
+  if (B < 0 || k < 1 || k > 255 || K < 1 || K > kMaxK || V < 1 || K > V) return SV_ERR_INVALID_ARG;
+  if (!scale_ok(temperature) || !dtype_ok(d_dtype)) return SV_ERR_INVALID_ARG;
+  if (wmode != SV_W_RAW && wmode != SV_W_GROUP_NORM) return SV_ERR_INVALID_ARG;
+  if (wmode == SV_W_GROUP_NORM && (group < 1 || (B > 0 && B % group != 0)))
+    return SV_ERR_INVALID_ARG;
+  if (!isfinite(clip)) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
+  if (!topk_logp || !topk_idx || !draft || !accepted_len || !reward || !grad)
+    return SV_ERR_INVALID_ARG;
+  if (!aligned(topk_logp, 4) || !aligned(topk_idx, 4) || !aligned(draft, esize(d_dtype)) ||
+      !aligned(accepted_len, 4) || !aligned(reward, 4) || !aligned(grad, 4))
+    return SV_ERR_INVALID_ARG;
+  if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
+  if ((long long)B * k > 0x7fffffffLL / 64 || (long long)B * k * V > (1LL << 40))
+    return SV_ERR_UNSUPPORTED;
+  const StreamGeom sg = stream_geom(V, (long long)B * k, esize(d_dtype), 0);
+  const WsLayout wl = ws_layout(B, B * k, record_slots(V), 0);
+  sv_status st = check_workspace(workspace, workspace_bytes, wl.bytes);
+  if (st != SV_OK) return st;
+  const WsPtrs w = ws_carve(workspace, wl);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const float c = (float)(1.4426950408889634 / (double)temperature);
+  StreamParams sp = {};
+  sp.rows0 = draft;
+  sp.kind = kKindRows;
+  sp.B = B * k;
+  sp.k = 1;
+  sp.V = V;
+  sp.nrows = B * k;
+  sp.W = sg.W;
+  sp.nchunk = sg.nchunk;
+  sp.div_nchunk = make_fastdiv(sg.nchunk);
+  sp.div_B = make_fastdiv(sp.B);
+  sp.c = c;
+  sp.use_bulk = bulk_ok_row(draft, V, esize(d_dtype));
+  sp.K = 1;
+  sp.stage_bytes = sg.stage_bytes;
+  sp.stage_off1 = sg.stage_off1;
+  sp.part = w.part;
+  sp.cand = w.cand;
+  sp.rec = w.rec;
+  sp.row_counter = w.counter;
+  sp.req_reject = w.reject;
+  sp.sched = w.glob + 32;
+  sp.status = device_status;
+  sp.count = 0;  // the gradient kernel folds the rows
+  cudaError_t e = d_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFStats0>(sp, sg, s)
+                                     : launch_stream<F32, F32, kFStats0>(sp, sg, s);
+  if (e != cudaSuccess) return SV_ERR_CUDA;
+  FinishParams fp = {};
+  fp.draft = draft;
+  fp.B = B;
+  fp.k = k;
+  fp.K = K;
+  fp.V = V;
+  fp.c = c;
+  fp.temperature = temperature;
+  fp.in_topk_logp = topk_logp;
+  fp.in_topk_idx = topk_idx;
+  fp.in_accepted_len = accepted_len;
+  fp.reward = reward;
+  fp.wmode = wmode;
+  fp.group = group < 1 ? 1 : group;
+  fp.clip = clip;
+  fp.grad = grad;
+  fp.part = w.part;
+  fp.rec = w.rec;
+  fp.status = device_status;
+  fp.sp = sp;
+  e = (d_dtype == SV_BF16) ? launch_blocks(kd_grad_kernel<BF16>, fp, B * k, kFixedBytes, s)
+                           : launch_blocks(kd_grad_kernel<F32>, fp, B * k, kFixedBytes, s);
+  return cuda_status(e);
+}
+
 sv_status sv_device_status_check(int32_t w) {
   if (w & SV_DEV_TIMEOUT) return SV_ERR_TIMEOUT;
   if (w & SV_DEV_ERROR_MASK) return SV_ERR_DEVICE_CHECK;

@@ -48,6 +48,9 @@ struct FinishParams {
   const int32_t* in_topk_idx;
   const int32_t* in_accepted_len;
   int draft_probs;
+  // KD gradient (sv_kd_grad)
+  float* grad;
+  float temperature;
   // stream scratch
   Partial* part;
   unsigned long long* cand;
@@ -568,6 +571,87 @@ __global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ Fi
   if (!prm.draft_probs) release_rows(prm, k, b * k, 1, w, kWarps);
   kd_finalize(b, sh.fin_n, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
               prm.total, prm.glob_counter, sh);
+}
+
+// Gradient of the reward-weighted KD loss with respect to the draft logits:
+// one block per draft row (b, i).  grad = w_b (q - p~ [j in K]) / T for
+// i < n_b (zero otherwise), q = softmax(z / T) from the row's folded
+// statistics: q_j = 2^((z_j c - G) - log2 S), the exact integer reference G
+// taken first so that the float argument stays small.
+template <class DT>
+__global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant__ FinishParams prm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  RowShared& sh = *reinterpret_cast<RowShared*>(smem);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = (int)blockIdx.x;
+  const int k = prm.k, P = k + 1, V = prm.V, K = prm.K;
+  const int b = row / k, i = row - b * k;
+  float* g = prm.grad + (size_t)row * V;
+  pdl_wait();
+  if (w == 0) {
+    const int n = prm.in_accepted_len[b];
+    const double wb = reward_weight(prm.reward, b, prm.wmode, prm.group, prm.clip);
+    int active = (n >= 0 && n <= k && i < n && wb != 0.0) ? 1 : 0;
+    if (n < 0 || n > k) {
+      if (lane == 0 && i == 0) set_status(prm.status, SV_DEV_BAD_INDEX);
+    }
+    // the row's statistics (every draft row was streamed)
+    const RowSum st = row_combine<DT, DT, kFStats0>(prm.sp, row, -1, true);
+    row_zero_records(prm.sp, row, true);
+    int bad = st.G0 == -INFINITY || (st.flags & kPTimeout);
+    if (active && bad && lane == 0)
+      set_status(prm.status, (st.flags & kPTimeout) ? SV_DEV_TIMEOUT : SV_DEV_NO_FINITE);
+    // p~ over the kept entries of target row (b, i)
+    double lp = -INFINITY;
+    int j = -1;
+    if (lane < K) {
+      lp = (double)prm.in_topk_logp[((size_t)b * P + i) * K + lane];
+      j = prm.in_topk_idx[((size_t)b * P + i) * K + lane];
+    }
+    const int badj = __any_sync(0xffffffffu, lane < K && (j < 0 || j >= V));
+    if (active && badj && lane == 0) set_status(prm.status, SV_DEV_BAD_INDEX);
+    double m = lp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    double se = (lane < K) ? exp(lp - m) : 0.0;
+    se = warp_sum(se);
+    const double pt = (lane < K) ? exp(lp - (m + log(se))) : 0.0;
+    if (lane == 0) {
+      sh.need = active ? (bad || badj ? 2 : 1) : 0;  // 0: zeros, 1: gradient, 2: NaN
+      sh.Gt = st.G0;
+      sh.St = log2(st.S0);  // log2 S, the fractional part of the log2-partition
+      sh.R = wb / (double)prm.temperature;
+    }
+    if (lane < 32) {  // the kept entries' p~, for the fix-up below
+      sh.topk[lane] = (lane < K) ? ((unsigned long long)(uint32_t)j << 32) |
+                                       (unsigned long long)__float_as_uint((float)pt)
+                                 : 0ull;
+    }
+  }
+  __syncthreads();
+  const int mode = sh.need;
+  const float c = prm.c, G = sh.Gt, l2s = (float)sh.St, scale = (float)sh.R;
+  const typename DT::storage* z = reinterpret_cast<const typename DT::storage*>(
+      row_ptr<DT>(prm.draft, (size_t)row, V));
+  for (int e = threadIdx.x; e < V; e += kThreads) {
+    float v = 0.f;
+    if (mode == 1) {
+      const float zf = load1<DT>(reinterpret_cast<const unsigned char*>(z), e);
+      v = scale * ex2(fmaf(zf, c, -G) - l2s);
+    } else if (mode == 2) {
+      v = NAN;
+    }
+    g[e] = v;
+  }
+  __syncthreads();  // the kept entries are rewritten after the plain writes
+  if (mode == 1 && w == 0 && lane < K) {
+    const unsigned long long t = sh.topk[lane];
+    const int j = (int)(t >> 32);
+    const float pt = __uint_as_float((uint32_t)(t & 0xffffffffu));
+    const float zf = load1<DT>(reinterpret_cast<const unsigned char*>(z), j);
+    const float q = ex2(fmaf(zf, c, -G) - l2s);
+    g[j] = scale * (q - pt);
+  }
 }
 
 }  // namespace sv

@@ -26,7 +26,8 @@ SV_DEV_BAD_TOKEN, SV_DEV_NO_FINITE, SV_DEV_TIMEOUT, SV_DEV_BAD_TREE = 0x1, 0x2, 
 SV_DEV_BAD_INDEX, SV_DEV_ERROR_MASK = 0x10, 0xFF
 SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
-EXPORTS = ("sv_verify_chain", "sv_verify_chain_noalloc", "sv_verify_tree_greedy", "sv_extract_topk_kd", "sv_kd_kl_loss",
+EXPORTS = ("sv_verify_chain", "sv_verify_chain_noalloc", "sv_verify_tree_greedy", "sv_kd_grad",
+           "sv_kd_grad_workspace_size", "sv_extract_topk_kd", "sv_kd_kl_loss",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
            "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size",
            "sv_device_status_check", "sv_status_string", "sv_version")
@@ -74,8 +75,12 @@ def lib() -> ctypes.CDLL:
             L.sv_extract_topk_kd.argtypes = [vp, ci, ci, ci, ci, cf, vp, vp, vp, vp, sz, vp, vp]
             L.sv_kd_kl_loss.argtypes = [vp, vp, ci, ci, ci, vp, ci, ci, ci, cf, vp, vp, ci, ci, cf,
                                         vp, vp, vp, vp, sz, vp, vp]
+            L.sv_kd_grad.argtypes = [vp, vp, ci, ci, ci, vp, ci, ci, cf, vp, vp, ci, ci, cf, vp,
+                                     vp, sz, vp, vp]
+            L.sv_kd_grad_workspace_size.argtypes = [ci, ci, ci]
+            L.sv_kd_grad_workspace_size.restype = sz
             for f in ("sv_verify_chain", "sv_verify_tree_greedy", "sv_extract_topk_kd",
-                      "sv_kd_kl_loss", "sv_device_status_check"):
+                      "sv_kd_kl_loss", "sv_kd_grad", "sv_device_status_check"):
                 getattr(L, f).restype = ci
             L.sv_device_status_check.argtypes = [ctypes.c_int32]
             L.sv_verify_chain_workspace_size.argtypes = [ci, ci, ci, ci]
@@ -344,3 +349,30 @@ def sv_device_status_check(word: int) -> int:
 
 def sv_version() -> int:
     return int(lib().sv_version())
+
+
+def sv_kd_grad(topk_logp: torch.Tensor, topk_idx: torch.Tensor, draft: torch.Tensor,
+               accepted_len: torch.Tensor, reward: torch.Tensor, temperature: float, *,
+               wmode: str = "raw", group: int = 1, clip: float = 0.0,
+               out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+               device_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """d loss / d draft logits [B, k, V] fp32 of the reward-weighted KD loss (see sv.h)."""
+    _dev(topk_logp, "topk_logp", torch.float32)
+    _dev(topk_idx, "topk_idx", torch.int32)
+    _dev(draft, "draft")
+    _dev(accepted_len, "accepted_len", torch.int32)
+    _dev(reward, "reward", torch.float32)
+    B, P, K = topk_logp.shape
+    k = P - 1
+    V = draft.shape[-1]
+    dev = draft.device
+    g = out if out is not None else torch.empty(B, k, V, dtype=torch.float32, device=dev)
+    nbytes = int(lib().sv_kd_grad_workspace_size(B, k, V))
+    w = ws if ws is not None else workspace(dev, B, nbytes)
+    wm = SV_W_GROUP_NORM if wmode == "group_norm" else SV_W_RAW
+    rc = lib().sv_kd_grad(_p(topk_logp), _p(topk_idx), B, k, K, _p(draft), _dtype_code(draft), V,
+                          float(temperature), _p(accepted_len), _p(reward), wm, int(group),
+                          float(clip), _p(g), _p(w), w.numel(), _p(device_status),
+                          _stream(dev, stream))
+    _check(rc, "sv_kd_grad")
+    return g

@@ -397,3 +397,54 @@ def test_both_stream_schedules(monkeypatch, kd256, mode):
     assert np.array_equal(got["accepted_len"].cpu().numpy(), ref["accepted_len"])
     assert np.array_equal(got["out_tokens"].cpu().numpy(), ref["out_tokens"])
     assert int(torch.count_nonzero(ws)) == 0
+
+
+def _grad_check(x, acc, reward, ref_top, mode, group, T):
+    """sv_kd_grad against the oracle on the same top-K buffers and lengths."""
+    lp = torch.from_numpy(ref_top["topk_logp"].astype(np.float32))
+    ix = torch.from_numpy(ref_top["topk_idx"].astype(np.int32))
+    st = status_tensor()
+    got = sv.sv_kd_grad(lp.to(DEV), ix.to(DEV), x.draft.to(DEV),
+                        torch.from_numpy(acc).to(DEV), x.reward.to(DEV), T,
+                        wmode="group_norm" if mode == O.W_GROUP_NORM else "raw", group=group,
+                        device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & sv.SV_DEV_ERROR_MASK == 0
+    ref = O.kd_grad(lp.numpy().astype(np.float64), ix.numpy(), x.draft, acc,
+                    x.reward.numpy().astype(np.float64), T, mode=mode, group=group)
+    g = got.cpu().numpy().astype(np.float64)
+    # tolerance: 1e-5 of the magnitude the rounding acts on, |w|/T (q_j + p~_j)
+    w = O.reward_loss(np.zeros((x.B, x.k)), acc, x.reward.numpy().astype(np.float64),
+                      mode=mode, group=group)["w"]
+    q = O.softmax(x.draft, T)["p"].reshape(x.B, x.k, -1)
+    mag = q.copy()
+    B, P, K = lp.shape
+    pt = np.exp(lp.numpy() - np.log(np.exp(lp.numpy().astype(np.float64)).sum(-1, keepdims=True)))
+    for b in range(B):
+        for i in range(x.k):
+            mag[b, i, ix[b, i].numpy()] += pt[b, i]
+    mag *= (np.abs(w) / T)[:, None, None]
+    err = np.abs(g - ref)
+    assert (err <= 1e-5 * mag + 1e-30).all(), float((err / np.maximum(mag, 1e-300)).max())
+    active = np.arange(x.k)[None, :] < acc[:, None]
+    assert not g[~active].any()
+    return got
+
+
+def test_kd_grad_small_and_ragged():
+    x = inputs.make_chain(6, 3, 1001, dtype="f32", model="gauss", sigma_t=2.0, sigma_d=0.5,
+                          temperature=1.0, seed=21)
+    ref = O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward, 1.0, 8)
+    acc = ref["accepted_len"].astype(np.int32)
+    acc[0] = 3  # at least one request with every draft kept
+    _grad_check(x, acc, x.reward, ref, O.W_RAW, 1, 1.0)
+
+
+def test_kd_grad_full_vocabulary(kd256):
+    x = inputs.ChainInputs(kd256.target[:32].contiguous(), kd256.draft[:32].contiguous(),
+                           kd256.draft_tokens[:32].contiguous(), kd256.uniforms[:32].contiguous(),
+                           kd256.reward[:32].contiguous(), kd256.temperature)
+    ref = O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward, x.temperature, 32,
+                      mode=O.W_GROUP_NORM, group=16)
+    acc = ref["accepted_len"].astype(np.int32)
+    _grad_check(x, acc, x.reward, ref, O.W_GROUP_NORM, 16, x.temperature)
