@@ -31,6 +31,11 @@ sys.path.insert(0, ROOT)
 from speculative_decoding_verification_94_b200 import inputs  # noqa: E402
 
 METRIC = "verified rows/s"
+GRAD_METRIC = "kd-gradient draft rows/s"
+
+
+def metric_of(kind):
+    return GRAD_METRIC if kind == "grad" else METRIC
 UNIT = "rows/s"
 L2_BYTES = 126 * 1024 * 1024
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per call (stream kernel +
@@ -48,7 +53,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="qwen_chain",
-                    choices=["qwen_chain", "kd", "tree", "tiny", "sweep"])
+                    choices=["qwen_chain", "kd", "kd_grad", "tree", "tiny", "sweep"])
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--sigma", type=float, default=1.0)
@@ -106,6 +111,13 @@ def make_workload(a, rank):
         x = inputs.kd_chain(B=B, k=k, seed=seed)
         return "kd", x, dict(workload="fused_verify_kd", B=B, k=k, V=x.V, input_dtype="bf16",
                              temperature=1.0, K=32, weighting="group_norm", group=16)
+    if a.workload == "kd_grad":
+        B = a.B or 256
+        k = a.k or 3
+        x = inputs.kd_chain(B=B, k=k, seed=seed)
+        return "grad", x, dict(workload="kd_gradient", B=B, k=k, V=x.V, input_dtype="bf16",
+                               temperature=1.0, K=32, weighting="group_norm", group=16,
+                               output="fp32 [B, k, V]")
     if a.workload == "tiny":
         x = inputs.tiny_chain(seed=seed)
         return "chain", x, dict(workload="tiny_chain_verify", B=4, k=3, V=1024,
@@ -125,6 +137,13 @@ def needed_bytes(kind, x, accepted_len):
     Rows after the first rejection are not part of the computation."""
     if kind == "tree":
         return rows_and_bytes(kind, x)[1]
+    if kind == "grad":
+        # the draft rows whose gradient is not zero are read once; every row of
+        # the fp32 gradient is written; plus the top-K buffers and small inputs
+        B, k, V = x.draft.shape
+        n = np.asarray(accepted_len, np.int64)
+        return int(np.sum(n) * V * x.draft.element_size() + B * k * V * 4 +
+                   B * (k + 1) * 32 * 8 + B * 8)
     B, P, V = x.target.shape
     k = P - 1
     te, de = x.target.element_size(), x.draft.element_size()
@@ -143,6 +162,9 @@ def rows_and_bytes(kind, x):
         B, n, V = x.logits.shape
         es = x.logits.element_size()
         return B * n, B * n * V * es + B * n * 8 + B * 4 + 2 * B * (x.max_depth + 1) * 4
+    if kind == "grad":  # draft rows per step; every draft row read twice, gradient written
+        B, k, V = x.draft.shape
+        return B * k, B * k * V * (2 * x.draft.element_size() + 4) + B * (k + 1) * 32 * 8 + B * 8
     B, P, V = x.target.shape
     k = P - 1
     te, de = x.target.element_size(), x.draft.element_size()
@@ -210,6 +232,13 @@ def oracle_step_fn(kind, x, threads=0):
         return lambda: O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward,
                                    x.temperature, 32, mode=O.W_GROUP_NORM, group=16,
                                    threads=threads)
+    if kind == "grad":
+        ref = O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward, x.temperature,
+                          32, mode=O.W_GROUP_NORM, group=16, threads=threads)
+        lp, ix, acc = ref["topk_logp"], ref["topk_idx"], ref["accepted_len"]
+        r = x.reward.numpy().astype(np.float64)
+        return lambda: O.kd_grad(lp, ix, x.draft, acc, r, x.temperature, mode=O.W_GROUP_NORM,
+                                 group=16, threads=threads)
     return lambda: O.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, x.temperature,
                                   threads=threads)
 
@@ -245,7 +274,8 @@ def run_reference(a):
         fn()
     dt = time.perf_counter() - t0
     value = rows * a.steps / dt
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+    line = {"impl": "reference", "metric": metric_of(kind), "value": value, "unit": UNIT,
+            "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * dt / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": cfg,
@@ -297,6 +327,23 @@ def main():
             s = d or sets[i % ncopy]
             sv.sv_verify_tree_greedy(s["logits"], s["tok"], s["par"], x.max_depth, out=outs,
                                      device_status=status)
+    elif kind == "grad":
+        B, k, V = x.draft.shape
+        sets = [dict(d=x.draft.to(dev)) for _ in range(ncopy)]
+        # the top-K buffers and accepted lengths come from one fused verification
+        pre = sv.sv_verify_chain(x.target.to(dev), sets[0]["d"], x.draft_tokens.to(dev),
+                                 x.uniforms.to(dev), x.temperature,
+                                 kd=dict(K=32, reward=x.reward.to(dev), wmode="group_norm",
+                                         group=16))
+        gin = dict(lp=pre["topk_logp"], ix=pre["topk_idx"], r=x.reward.to(dev))
+        outs = dict(grad=torch.empty(B, k, V, device=dev), accepted_len=pre["accepted_len"])
+        torch.cuda.synchronize(dev)
+
+        def step(i, d=None):
+            s = d or sets[i % ncopy]
+            sv.sv_kd_grad(gin["lp"], gin["ix"], s["d"], outs["accepted_len"], gin["r"],
+                          x.temperature, wmode="group_norm", group=16, out=outs["grad"],
+                          device_status=status)
     else:
         sets = [dict(t=x.target.to(dev), d=x.draft.to(dev), tok=x.draft_tokens.to(dev),
                      u=x.uniforms.to(dev), r=x.reward.to(dev)) for _ in range(ncopy)]
@@ -376,13 +423,16 @@ def main():
         if kind == "tree":
             host = dict(logits=x.logits.pin_memory(), tok=x.node_tokens.pin_memory(),
                         par=x.parents.pin_memory())
+        elif kind == "grad":
+            host = dict(d=x.draft.pin_memory())
         else:
             host = dict(t=x.target.pin_memory(), d=x.draft.pin_memory(),
                         tok=x.draft_tokens.pin_memory(), u=x.uniforms.pin_memory(),
                         r=x.reward.pin_memory())
         dsts = sets[0]
         res_h = {k2: torch.empty(v.shape, dtype=v.dtype).pin_memory()
-                 for k2, v in outs.items() if k2 in ("accepted_len", "out_tokens", "total")}
+                 for k2, v in outs.items()
+                 if k2 in (("grad",) if kind == "grad" else ("accepted_len", "out_tokens", "total"))}
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = sum(v.numel() * v.element_size() for v in res_h.values())
         n_e2e = max(3, min(a.steps, 50))
@@ -415,7 +465,7 @@ def main():
 
     if rank == 0:
         traffic = NCU_TRAFFIC.get(cfg["workload"])
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        line = {"metric": metric_of(kind), "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_total / a.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f32", "data": "synthetic",
@@ -428,9 +478,9 @@ def main():
                              "algorithmic_bytes_per_launch": algo_bytes,
                              "full_read_bytes_per_launch": full_bytes,
                              "call_us": ms_launch * 1e3,
-                             "kernel": ("sv_verify_tree_greedy" if kind == "tree"
-                                        else "sv_verify_chain") +
-                             " call: stream_kernel + finishing kernel, timed together"},
+                             "kernel": {"tree": "sv_verify_tree_greedy",
+                                        "grad": "sv_kd_grad"}.get(kind, "sv_verify_chain") +
+                             " call: stream_kernel + second kernel, timed together"},
                 "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / 8000.0,
                 "e2e": e2e, "gpu_launches": LAUNCHES_PER_CALL * a.steps, "clocks": clk,
                 "cpu_baseline": cpu}
