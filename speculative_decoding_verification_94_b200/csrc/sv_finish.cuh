@@ -633,13 +633,31 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
   const float c = prm.c, G = sh.Gt, l2s = (float)sh.St, scale = (float)sh.R;
   const typename DT::storage* z = reinterpret_cast<const typename DT::storage*>(
       row_ptr<DT>(prm.draft, (size_t)row, V));
-  for (int e = threadIdx.x; e < V; e += kThreads) {
-    float v = 0.f;
+  // 8 elements per thread and step: one 16- or 32-byte load, two 16-byte
+  // streaming stores (when the row and the gradient row are 16-byte aligned)
+  const bool vec = (reinterpret_cast<uintptr_t>(z) % 16 == 0) &&
+                   (reinterpret_cast<uintptr_t>(g) % 16 == 0);
+  const int nvec = vec ? V / kVec : 0;
+  const float fill = mode == 2 ? NAN : 0.f;
+#pragma unroll 4
+  for (int t = threadIdx.x; t < nvec; t += kThreads) {
+    float v[8];
+    if (mode == 1) {
+      load8<DT>(reinterpret_cast<const unsigned char*>(z), t * kVec, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = scale * ex2(fmaf(v[q], c, -G) - l2s);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = fill;
+    }
+    __stcs(reinterpret_cast<float4*>(g + (size_t)t * kVec), make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(reinterpret_cast<float4*>(g + (size_t)t * kVec + 4), make_float4(v[4], v[5], v[6], v[7]));
+  }
+  for (int e = nvec * kVec + threadIdx.x; e < V; e += kThreads) {
+    float v = fill;
     if (mode == 1) {
       const float zf = load1<DT>(reinterpret_cast<const unsigned char*>(z), e);
       v = scale * ex2(fmaf(zf, c, -G) - l2s);
-    } else if (mode == 2) {
-      v = NAN;
     }
     g[e] = v;
   }
