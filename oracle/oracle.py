@@ -69,10 +69,11 @@ def _lib(plant: int = 0) -> ctypes.CDLL:
         L.oracle_tree_greedy.argtypes = [vp, ci, i32p, i32p, ci, ci, ci, ci, i32p, i32p, i32p, ci]
         L.oracle_topk.argtypes = [vp, ci, ci, ci, ci, cd, f64p, i32p, f64p, ci]
         L.oracle_kl.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, ci, cd, f64p, f64p, ci]
-        L.oracle_reward_loss.argtypes = [f64p, i32p, f64p, ci, ci, ci, ci, cd, f64p, f64p, f64p]
+        L.oracle_reward_loss.argtypes = [f64p, i32p, f64p, ci, ci, ci, ci, cd, ci, f64p, f64p,
+                                         f64p]
         L.oracle_softmax.argtypes = [vp, ci, ci, ci, cd, f64p, f64p]
         L.oracle_kd_grad.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, cd, i32p, f64p, ci, ci,
-                                     cd, f64p, ci]
+                                     cd, ci, f64p, ci]
         L.oracle_max_threads.argtypes = []
         for name in ("oracle_verify_chain", "oracle_tree_greedy", "oracle_topk", "oracle_kl",
                      "oracle_reward_loss", "oracle_softmax", "oracle_kd_grad",
@@ -219,7 +220,7 @@ def kl(topk_logp, topk_idx, draft, temperature: float, *, draft_kind: int = DRAF
 
 
 def reward_loss(kl_values, accepted_len, reward, *, mode: int = W_RAW, group: int = 1,
-                clip: float = 0.0) -> dict:
+                clip: float = 0.0, positions: int = 0) -> dict:
     """Reward-weighted KD loss per request and its sum."""
     klv = _np(kl_values, np.float64)
     B, k = klv.shape
@@ -230,14 +231,16 @@ def reward_loss(kl_values, accepted_len, reward, *, mode: int = W_RAW, group: in
     total = np.zeros(1, np.float64)
     rc = _lib().oracle_reward_loss(_ptr(klv, ctypes.c_double), _ptr(acc, ctypes.c_int32),
                                    _ptr(r, ctypes.c_double), B, k, mode, group, float(clip),
-                                   _ptr(w, ctypes.c_double), _ptr(loss, ctypes.c_double),
+                                   int(positions), _ptr(w, ctypes.c_double),
+                                   _ptr(loss, ctypes.c_double),
                                    _ptr(total, ctypes.c_double))
     _check(rc, "reward_loss")
     return dict(w=w, loss=loss, total=float(total[0]))
 
 
 def kd_grad(topk_logp, topk_idx, draft, accepted_len, reward, temperature: float, *,
-            mode: int = W_RAW, group: int = 1, clip: float = 0.0, threads: int = 0):
+            mode: int = W_RAW, group: int = 1, clip: float = 0.0, positions: int = 0,
+            threads: int = 0):
     """d loss / d draft logits [B, k, V] (float64) of the reward-weighted KD loss."""
     lp = _np(topk_logp, np.float64)
     ix = _np(topk_idx, np.int32)
@@ -251,7 +254,7 @@ def kd_grad(topk_logp, topk_idx, draft, accepted_len, reward, temperature: float
     rc = _lib().oracle_kd_grad(_ptr(lp, ctypes.c_double), _ptr(ix, ctypes.c_int32), B, k, K,
                                d.ctypes.data, ddt, V, float(np.float32(temperature)),
                                _ptr(acc, ctypes.c_int32), _ptr(r, ctypes.c_double), mode, group,
-                               float(clip), _ptr(g, ctypes.c_double), threads)
+                               float(clip), int(positions), _ptr(g, ctypes.c_double), threads)
     _check(rc, "kd_grad")
     return g
 
@@ -270,12 +273,13 @@ def softmax(logits, temperature: float) -> dict:
 
 def verify_kd(target, draft, draft_tokens, uniforms, reward, temperature: float, K: int, *,
               mode: int = W_RAW, group: int = 1, clip: float = 0.0,
-              draft_kind: int = DRAFT_LOGITS, threads: int = 0) -> dict:
+              draft_kind: int = DRAFT_LOGITS, positions: int = 0, threads: int = 0) -> dict:
     """Chain verification followed by the KD quantities, each step as above."""
     v = verify_chain(target, draft, draft_tokens, uniforms, temperature,
                      draft_kind=draft_kind, threads=threads)
     tk = topk(target, K, temperature, threads=threads)
     d = kl(tk["topk_logp"], tk["topk_idx"], draft, temperature, draft_kind=draft_kind,
            threads=threads)
-    rl = reward_loss(d["kl"], v["accepted_len"], reward, mode=mode, group=group, clip=clip)
+    rl = reward_loss(d["kl"], v["accepted_len"], reward, mode=mode, group=group, clip=clip,
+                     positions=positions)
     return {**v, **tk, **d, **rl}

@@ -41,7 +41,8 @@
  *  - argmax and top-K ties go to the lowest vocabulary index;
  *  - top-K log-probs are full-vocabulary log-softmax values; the KD target
  *    p~ renormalises them over the K kept entries;
- *  - the KD loss sums the accepted draft positions i < n_acc.
+ *  - the KD loss sums the accepted draft positions i < n_acc (optionally the
+ *    first rejected position as well).
  */
 #include <math.h>
 #include <stdint.h>
@@ -510,12 +511,15 @@ int oracle_kl(const double* topk_logp, const int32_t* topk_idx, int B, int k, in
 /*                                                                            */
 /* w_b = r_b (RAW) or r_b / sum_{b' in group(b)} r_b' (GROUP_NORM, groups of  */
 /* `group` consecutive requests; a zero group sum gives w = 0); clip > 0      */
-/* clamps w to [-clip, clip].  loss_b = w_b * sum_{i < accepted_len[b]}       */
-/* kl[b, i] (0 when w_b == 0: a zero-weight sample contributes nothing);      */
-/* total = sum_b loss_b.                                                      */
+/* clamps w to [-clip, clip].  loss_b = w_b * sum_{i < m_b} kl[b, i] (0 when  */
+/* w_b == 0: a zero-weight sample contributes nothing); total = sum_b loss_b. */
+/* m_b = accepted_len[b] (positions = 0: the accepted drafts), or, with       */
+/* positions = 1, one more when a draft was rejected (n < k): the first       */
+/* rejected position too, as drafters that learn from their rejected          */
+/* proposals do ("Draft-OPD" page).                                           */
 /* ------------------------------------------------------------------------ */
 int oracle_reward_loss(const double* kl, const int32_t* accepted_len, const double* reward,
-                       int B, int k, int mode, int group, double clip, double* w,
+                       int B, int k, int mode, int group, double clip, int positions, double* w,
                        double* loss, double* total) {
   if (B < 0 || k < 1 || !kl || !accepted_len || !reward || !loss || !total) return OR_BAD_ARG;
   if (mode == OR_W_GROUP_NORM && (group < 1 || B % group != 0)) return OR_BAD_ARG;
@@ -532,8 +536,9 @@ int oracle_reward_loss(const double* kl, const int32_t* accepted_len, const doub
     if (w) w[b] = wb;
     int n = accepted_len[b];
     if (n < 0 || n > k) return OR_BAD_ARG;
+    int m = (positions && n < k) ? n + 1 : n;
     double s = 0.0;
-    for (int i = 0; i < n; ++i) s += kl[(size_t)b * k + i];
+    for (int i = 0; i < m; ++i) s += kl[(size_t)b * k + i];
     loss[b] = wb == 0.0 ? 0.0 : wb * s;
     sum += loss[b];
   }
@@ -547,12 +552,12 @@ int oracle_reward_loss(const double* kl, const int32_t* accepted_len, const doub
 /* gradient flows into the current q_theta only, never into the stored       */
 /* log q).  From d log q_j / d z_l = (delta_jl - q_l) / T and sum_j p~_j = 1:  */
 /*   d loss_b / d z_d[b, i, l] = w_b [i < n_b] (q_il - p~_il [l in K]) / T.    */
-/* Logit drafts only; w_b as in oracle_reward_loss.  grad [B, k, V].          */
+/* Logit drafts only; w_b and the positions i < m_b as in oracle_reward_loss. */
 /* ------------------------------------------------------------------------ */
 int oracle_kd_grad(const double* topk_logp, const int32_t* topk_idx, int B, int k, int K,
                    const void* draft, int d_dtype, int V, double T,
                    const int32_t* accepted_len, const double* reward, int mode, int group,
-                   double clip, double* grad, int nthreads) {
+                   double clip, int positions, double* grad, int nthreads) {
   if (B < 0 || k < 1 || K < 1 || K > V || !(T > 0.0) || !topk_logp || !topk_idx || !draft ||
       !accepted_len || !reward || !grad)
     return OR_BAD_ARG;
@@ -579,7 +584,8 @@ int oracle_kd_grad(const double* topk_logp, const int32_t* topk_idx, int B, int 
       err = OR_BAD_ARG;
       continue;
     }
-    if (i >= n || wb == 0.0) continue;
+    int m = (positions && n < k) ? n + 1 : n;
+    if (i >= m || wb == 0.0) continue;
     size_t drow = (size_t)row * (size_t)V;
     double lse_d = softmax_row(draft, d_dtype, drow, V, T, NULL);
     if (isnan(lse_d)) {

@@ -376,15 +376,17 @@ def _kd_case(seed, B=4, k=2, V=12, K=4, T=0.8):
     return draft.astype(np.float32), lp, ix.astype(np.int32), acc, reward, T
 
 
-def _kd_loss(oracle, draft, lp, ix, acc, reward, T, mode, group):
+def _kd_loss(oracle, draft, lp, ix, acc, reward, T, mode, group, positions=0):
     kl = oracle.kl(lp, ix, torch.from_numpy(draft), T)["kl"]
-    return oracle.reward_loss(kl, acc, reward, mode=mode, group=group)["total"]
+    return oracle.reward_loss(kl, acc, reward, mode=mode, group=group,
+                              positions=positions)["total"]
 
 
-@pytest.mark.parametrize("mode,group", [(0, 1), (1, 2)])
-def test_kd_gradient_matches_central_differences(oracle, mode, group):
+@pytest.mark.parametrize("mode,group,positions", [(0, 1, 0), (1, 2, 0), (0, 1, 1)])
+def test_kd_gradient_matches_central_differences(oracle, mode, group, positions):
     draft, lp, ix, acc, reward, T = _kd_case(3)
-    g = oracle.kd_grad(lp, ix, torch.from_numpy(draft), acc, reward, T, mode=mode, group=group)
+    g = oracle.kd_grad(lp, ix, torch.from_numpy(draft), acc, reward, T, mode=mode, group=group,
+                       positions=positions)
     h = 1.0 / 1024
     num = np.zeros_like(g)
     for b in range(draft.shape[0]):
@@ -393,8 +395,10 @@ def test_kd_gradient_matches_central_differences(oracle, mode, group):
                 zp, zm = draft.copy(), draft.copy()
                 zp[b, i, j] += h
                 zm[b, i, j] -= h
-                num[b, i, j] = (_kd_loss(oracle, zp, lp, ix, acc, reward, T, mode, group) -
-                                _kd_loss(oracle, zm, lp, ix, acc, reward, T, mode, group)) / (2 * h)
+                num[b, i, j] = (_kd_loss(oracle, zp, lp, ix, acc, reward, T, mode, group,
+                                         positions) -
+                                _kd_loss(oracle, zm, lp, ix, acc, reward, T, mode, group,
+                                         positions)) / (2 * h)
     scale = np.abs(g).max()
     assert scale > 0
     assert np.abs(num - g).max() <= 2e-5 * scale, np.abs(num - g).max() / scale
@@ -410,3 +414,22 @@ def test_kd_gradient_rows_sum_to_zero_and_vanish_where_unused(oracle):
             else:
                 assert abs(g[b, i].sum()) < 1e-12 * max(1.0, np.abs(g[b, i]).max())
                 assert g[b, i].max() > 0 > g[b, i].min()
+
+
+def test_kd_mask_with_the_first_rejected_position(oracle):
+    """positions=1 (the Draft-OPD variant) adds position n when a draft was
+    rejected (n < k) and changes nothing when every draft was accepted."""
+    rng = np.random.default_rng(5)
+    B, k = 6, 3
+    kl = rng.uniform(0, 1, (B, k))
+    acc = np.array([0, 1, 2, 3, 1, 3], np.int32)
+    rw = rng.uniform(0.1, 1, B)
+    r0 = oracle.reward_loss(kl, acc, rw)
+    r1 = oracle.reward_loss(kl, acc, rw, positions=1)
+    for b in range(B):
+        n = acc[b]
+        extra = rw[b] * kl[b, n] if n < k else 0.0
+        assert r1["loss"][b] == pytest.approx(r0["loss"][b] + extra, rel=1e-14, abs=1e-15)
+    bumped = np.minimum(acc + 1, k).astype(np.int32)
+    r2 = oracle.reward_loss(kl, bumped, rw)
+    assert np.allclose(r1["loss"], r2["loss"], rtol=1e-14, atol=0)
