@@ -101,8 +101,11 @@ typedef struct sv_kd_args {
   sv_weight_mode wmode;       /* reward weighting */
   int group;                  /* GROUP_NORM group size (B % group == 0); ignored for RAW */
   float clip;                 /* > 0: clamp w to [-clip, clip]; <= 0: no clipping */
-  float* loss;                /* [B]         out: w_b * sum_{i < accepted_len[b]} kl[b, i] (0 if w_b == 0) */
+  float* loss;                /* [B]         out: w_b * sum_{i < m_b} kl[b, i] (0 if w_b == 0) */
   float* total;               /* [1]         out: sum_b loss[b], fixed summation order */
+  int positions;              /* the KD positions: 0: m_b = accepted_len[b] (the accepted drafts);
+                                 1: also the first rejected position, m_b = n + 1 when n < k (as
+                                 drafters that learn from rejected proposals do, "Draft-OPD" page) */
 } sv_kd_args;
 
 /* Bytes of zero-filled workspace needed by each call (K = 0: no fused KD).
@@ -243,15 +246,16 @@ SV_API sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, i
  *   renormalised kept target mass), log q_j = log softmax(draft[b, i] / T)_j
  *   (or log of the given probability) at j = topk_idx[b, i, :],
  *   kl[b, i] = sum_j p~_j (log p~_j - log q_j) (+inf when q_j = 0 < p~_j).
- *   loss[b] = w_b * sum_{i < accepted_len[b]} kl[b, i] (0 when w_b == 0),
+ *   loss[b] = w_b * sum_{i < m_b} kl[b, i] (0 when w_b == 0), m_b as in
+ *   sv_kd_args.positions (accepted_len[b], or one more at a rejection),
  *   total[0] = sum_b loss[b]; w_b as in sv_weight_mode, optionally clipped.
  *   accepted_len [B] int32 in [0, k]; reward [B] fp32; T > 0.
  */
 SV_API sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
                         const void* draft, sv_dtype d_dtype, sv_draft_kind d_kind, int V,
                         float temperature, const int32_t* accepted_len, const float* reward,
-                        sv_weight_mode wmode, int group, float clip, float* kl, float* loss,
-                        float* total, void* workspace, size_t workspace_bytes,
+                        sv_weight_mode wmode, int group, float clip, int positions, float* kl,
+                        float* loss, float* total, void* workspace, size_t workspace_bytes,
                         int32_t* device_status, void* stream);
 
 /*
@@ -260,9 +264,10 @@ SV_API sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, 
  * 1 step 3: the gradient flows into the current q_theta only) with the reward
  * weights of section 5.  With q = softmax(draft[b, i] / T) and p~ as in
  * sv_kd_kl_loss:
- *   grad[b, i, j] = w_b * (q_j - p~_j [j in topk_idx[b, i, :]]) / T  for i < accepted_len[b],
+ *   grad[b, i, j] = w_b * (q_j - p~_j [j in topk_idx[b, i, :]]) / T  for i < m_b,
  *   grad[b, i, j] = 0                                                 otherwise,
- * which is d loss[b] / d draft[b, i, j] for the loss of sv_kd_kl_loss.
+ * which is d loss[b] / d draft[b, i, j] for the loss of sv_kd_kl_loss with
+ * the same `positions` (m_b as in sv_kd_args).
  *   topk_logp, topk_idx [B, k+1, K]; draft [B, k, V] logits (d_dtype);
  *   accepted_len [B]; reward [B]; grad [B, k, V] fp32 out.  T > 0.
  *   A row whose statistics fail (no finite logit) or whose top-K indices are
@@ -273,7 +278,7 @@ SV_API size_t sv_kd_grad_workspace_size(int B, int k, int V);
 SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
                             const void* draft, sv_dtype d_dtype, int V, float temperature,
                             const int32_t* accepted_len, const float* reward,
-                            sv_weight_mode wmode, int group, float clip, float* grad,
+                            sv_weight_mode wmode, int group, float clip, int positions, float* grad,
                             void* workspace, size_t workspace_bytes, int32_t* device_status,
                             void* stream);
 

@@ -523,6 +523,7 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
     fp.clip = kd->clip;
     fp.loss = kd->loss;
     fp.total = kd->total;
+    fp.positions = kd->positions ? 1 : 0;
     sp.topk_logp = kd->topk_logp;
     sp.topk_idx = kd->topk_idx;
     sp.lse = kd->lse;
@@ -725,8 +726,8 @@ sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, i
 sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
                         const void* draft, sv_dtype d_dtype, sv_draft_kind d_kind, int V,
                         float temperature, const int32_t* accepted_len, const float* reward,
-                        sv_weight_mode wmode, int group, float clip, float* kl, float* loss,
-                        float* total, void* workspace, size_t workspace_bytes,
+                        sv_weight_mode wmode, int group, float clip, int positions, float* kl,
+                        float* loss, float* total, void* workspace, size_t workspace_bytes,
                         int32_t* device_status, void* stream) {
   if (B < 0 || k < 1 || k > 255 || K < 1 || K > kMaxK || V < 1 || K > V) return SV_ERR_INVALID_ARG;
   if (!scale_ok(temperature)) return SV_ERR_INVALID_ARG;
@@ -798,6 +799,7 @@ sv_status sv_kd_kl_loss(const float* topk_logp, const int32_t* topk_idx, int B, 
   fp.wmode = wmode;
   fp.group = group < 1 ? 1 : group;
   fp.clip = clip;
+  fp.positions = positions ? 1 : 0;
   fp.kl = kl;
   fp.loss = loss;
   fp.total = total;
@@ -818,8 +820,8 @@ size_t sv_kd_grad_workspace_size(int B, int k, int V) { return sv_kd_kl_loss_wor
 sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int B, int k, int K,
                      const void* draft, sv_dtype d_dtype, int V, float temperature,
                      const int32_t* accepted_len, const float* reward, sv_weight_mode wmode,
-                     int group, float clip, float* grad, void* workspace, size_t workspace_bytes,
-                     int32_t* device_status, void* stream) {
+                     int group, float clip, int positions, float* grad, void* workspace,
+                     size_t workspace_bytes, int32_t* device_status, void* stream) {
   if (B < 0 || k < 1 || k > 255 || K < 1 || K > kMaxK || V < 1 || K > V) return SV_ERR_INVALID_ARG;
   if (!scale_ok(temperature) || !dtype_ok(d_dtype)) return SV_ERR_INVALID_ARG;
   if (wmode != SV_W_RAW && wmode != SV_W_GROUP_NORM) return SV_ERR_INVALID_ARG;
@@ -884,6 +886,7 @@ sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int B, int
   fp.wmode = wmode;
   fp.group = group < 1 ? 1 : group;
   fp.clip = clip;
+  fp.positions = positions ? 1 : 0;
   fp.grad = grad;
   fp.part = w.part;
   fp.rec = w.rec;

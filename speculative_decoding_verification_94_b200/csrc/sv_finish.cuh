@@ -48,6 +48,7 @@ struct FinishParams {
   const int32_t* in_topk_idx;
   const int32_t* in_accepted_len;
   int draft_probs;
+  int positions;  // KD positions (sv_kd_args.positions)
   // KD gradient (sv_kd_grad)
   float* grad;
   float temperature;
@@ -394,8 +395,8 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
       for (int t = first_undef + (int)threadIdx.x; t < k; t += kThreads)
         prm.kl[(size_t)b * k + t] = NAN;
       __syncthreads();
-      kd_finalize(b, nf, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
-                  prm.total, prm.glob_counter, sh);
+      kd_finalize(b, nf, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
+                  prm.positions, prm.loss, prm.total, prm.glob_counter, sh);
     }
   }
   if (arrived) cluster_wait_acquire();  // keep this CTA's shared memory until all have read it
@@ -569,8 +570,8 @@ __global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ Fi
   }
   __syncthreads();
   if (!prm.draft_probs) release_rows(prm, k, b * k, 1, w, kWarps);
-  kd_finalize(b, sh.fin_n, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip, prm.loss,
-              prm.total, prm.glob_counter, sh);
+  kd_finalize(b, sh.fin_n, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
+              prm.positions, prm.loss, prm.total, prm.glob_counter, sh);
 }
 
 // Gradient of the reward-weighted KD loss with respect to the draft logits:
@@ -591,7 +592,8 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
   if (w == 0) {
     const int n = prm.in_accepted_len[b];
     const double wb = reward_weight(prm.reward, b, prm.wmode, prm.group, prm.clip);
-    int active = (n >= 0 && n <= k && i < n && wb != 0.0) ? 1 : 0;
+    const int npos = (prm.positions && n >= 0 && n < k) ? n + 1 : n;  // KD positions
+    int active = (n >= 0 && n <= k && i < npos && wb != 0.0) ? 1 : 0;
     if (n < 0 || n > k) {
       if (lane == 0 && i == 0) set_status(prm.status, SV_DEV_BAD_INDEX);
     }

@@ -44,7 +44,8 @@ class sv_kd_args(ctypes.Structure):
                 ("topk_idx", ctypes.c_void_p), ("lse", ctypes.c_void_p),
                 ("kl", ctypes.c_void_p), ("reward", ctypes.c_void_p),
                 ("wmode", ctypes.c_int), ("group", ctypes.c_int), ("clip", ctypes.c_float),
-                ("loss", ctypes.c_void_p), ("total", ctypes.c_void_p)]
+                ("loss", ctypes.c_void_p), ("total", ctypes.c_void_p),
+                ("positions", ctypes.c_int)]
 
 
 _lib = None
@@ -74,9 +75,9 @@ def lib() -> ctypes.CDLL:
                                                 vp, vp]
             L.sv_extract_topk_kd.argtypes = [vp, ci, ci, ci, ci, cf, vp, vp, vp, vp, sz, vp, vp]
             L.sv_kd_kl_loss.argtypes = [vp, vp, ci, ci, ci, vp, ci, ci, ci, cf, vp, vp, ci, ci, cf,
-                                        vp, vp, vp, vp, sz, vp, vp]
-            L.sv_kd_grad.argtypes = [vp, vp, ci, ci, ci, vp, ci, ci, cf, vp, vp, ci, ci, cf, vp,
-                                     vp, sz, vp, vp]
+                                        ci, vp, vp, vp, vp, sz, vp, vp]
+            L.sv_kd_grad.argtypes = [vp, vp, ci, ci, ci, vp, ci, ci, cf, vp, vp, ci, ci, cf, ci,
+                                     vp, vp, sz, vp, vp]
             L.sv_kd_grad_workspace_size.argtypes = [ci, ci, ci]
             L.sv_kd_grad_workspace_size.restype = sz
             for f in ("sv_verify_chain", "sv_verify_tree_greedy", "sv_extract_topk_kd",
@@ -207,7 +208,7 @@ def sv_verify_chain(target: torch.Tensor, draft: torch.Tensor | None, draft_toke
                                          o["lse"].data_ptr(), o["kl"].data_ptr(),
                                          reward.data_ptr(), wmode, int(kd.get("group", 1)),
                                          float(kd.get("clip", 0.0)), o["loss"].data_ptr(),
-                                         o["total"].data_ptr()))
+                                         o["total"].data_ptr(), int(kd.get("positions", 0))))
     nbytes = sv_verify_chain_workspace_size(B, k, V, int(kd.get("K", 32)) if kd else 0)
     w = ws if ws is not None else workspace(dev, B, nbytes)
     rc = lib().sv_verify_chain(
@@ -315,8 +316,9 @@ def sv_extract_topk_kd(logits: torch.Tensor, K: int, temperature: float, *,
 def sv_kd_kl_loss(topk_logp: torch.Tensor, topk_idx: torch.Tensor, draft: torch.Tensor,
                   temperature: float, accepted_len: torch.Tensor, reward: torch.Tensor, *,
                   draft_kind: str = "logits", wmode: str = "raw", group: int = 1,
-                  clip: float = 0.0, out: dict | None = None, ws: torch.Tensor | None = None,
-                  device_status: torch.Tensor | None = None, stream=None) -> dict:
+                  clip: float = 0.0, positions: int = 0, out: dict | None = None,
+                  ws: torch.Tensor | None = None, device_status: torch.Tensor | None = None,
+                  stream=None) -> dict:
     """Reward-weighted KD loss from top-K buffers [B, k+1, K] and draft [B, k, V]."""
     _dev(topk_logp, "topk_logp", torch.float32)
     _dev(topk_idx, "topk_idx", torch.int32)
@@ -337,7 +339,8 @@ def sv_kd_kl_loss(topk_logp: torch.Tensor, topk_idx: torch.Tensor, draft: torch.
     wm = SV_W_GROUP_NORM if wmode == "group_norm" else SV_W_RAW
     rc = lib().sv_kd_kl_loss(_p(topk_logp), _p(topk_idx), B, k, K, _p(draft), _dtype_code(draft),
                              dk, V, float(temperature), _p(accepted_len), _p(reward), wm,
-                             int(group), float(clip), _p(o["kl"]), _p(o["loss"]), _p(o["total"]),
+                             int(group), float(clip), int(positions), _p(o["kl"]), _p(o["loss"]),
+                             _p(o["total"]),
                              _p(w), w.numel(), _p(device_status), _stream(dev, stream))
     _check(rc, "sv_kd_kl_loss")
     return o
@@ -353,7 +356,7 @@ def sv_version() -> int:
 
 def sv_kd_grad(topk_logp: torch.Tensor, topk_idx: torch.Tensor, draft: torch.Tensor,
                accepted_len: torch.Tensor, reward: torch.Tensor, temperature: float, *,
-               wmode: str = "raw", group: int = 1, clip: float = 0.0,
+               wmode: str = "raw", group: int = 1, clip: float = 0.0, positions: int = 0,
                out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
                device_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """d loss / d draft logits [B, k, V] fp32 of the reward-weighted KD loss (see sv.h)."""
@@ -372,7 +375,7 @@ def sv_kd_grad(topk_logp: torch.Tensor, topk_idx: torch.Tensor, draft: torch.Ten
     wm = SV_W_GROUP_NORM if wmode == "group_norm" else SV_W_RAW
     rc = lib().sv_kd_grad(_p(topk_logp), _p(topk_idx), B, k, K, _p(draft), _dtype_code(draft), V,
                           float(temperature), _p(accepted_len), _p(reward), wm, int(group),
-                          float(clip), _p(g), _p(w), w.numel(), _p(device_status),
+                          float(clip), int(positions), _p(g), _p(w), w.numel(), _p(device_status),
                           _stream(dev, stream))
     _check(rc, "sv_kd_grad")
     return g

@@ -141,8 +141,8 @@ def test_other_entry_points_validate(lib):
                                   None) == sv.SV_ERR_WORKSPACE
     # KL loss: probs must be fp32, group must divide B
     assert lib.sv_kd_kl_loss(f, f, 4, 3, 32, f, sv.SV_BF16, sv.SV_DRAFT_PROBS, 1000, 1.0, f, f,
-                             0, 1, 0.0, f, f, f, f, 1 << 20, None, None) == E
+                             0, 1, 0.0, 0, f, f, f, f, 1 << 20, None, None) == E
     assert lib.sv_kd_kl_loss(f, f, 4, 3, 32, f, sv.SV_BF16, sv.SV_DRAFT_LOGITS, 1000, 1.0, f, f,
-                             1, 3, 0.0, f, f, f, f, 1 << 20, None, None) == E
+                             1, 3, 0.0, 0, f, f, f, f, 1 << 20, None, None) == E
     assert lib.sv_kd_kl_loss(f, f, 4, 3, 32, f, sv.SV_BF16, sv.SV_DRAFT_LOGITS, 1000, 1.0, f, f,
-                             0, 1, 0.0, f, f, f, None, 1 << 20, None, None) == sv.SV_ERR_WORKSPACE
+                             0, 1, 0.0, 0, f, f, f, None, 1 << 20, None, None) == sv.SV_ERR_WORKSPACE

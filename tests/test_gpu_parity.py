@@ -448,3 +448,47 @@ def test_kd_grad_full_vocabulary(kd256):
                       mode=O.W_GROUP_NORM, group=16)
     acc = ref["accepted_len"].astype(np.int32)
     _grad_check(x, acc, x.reward, ref, O.W_GROUP_NORM, 16, x.temperature)
+
+
+def test_kd_first_rejected_position(kd256):
+    """positions=1 (the Draft-OPD variant): the loss and the gradient also
+    cover the first rejected position."""
+    x = inputs.ChainInputs(kd256.target[:32].contiguous(), kd256.draft[:32].contiguous(),
+                           kd256.draft_tokens[:32].contiguous(), kd256.uniforms[:32].contiguous(),
+                           kd256.reward[:32].contiguous(), kd256.temperature)
+    st = status_tensor()
+    kd = dict(K=32, reward=x.reward.to(DEV), wmode="group_norm", group=16, positions=1)
+    got = run_chain(x, kd=kd, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & sv.SV_DEV_ERROR_MASK == 0
+    ref = O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward, x.temperature, 32,
+                      mode=O.W_GROUP_NORM, group=16, positions=1)
+    assert_chain_match(got, ref, x.uniforms.numpy(), x.temperature, x.k)
+    acc = got["accepted_len"].cpu().numpy()
+    assert (acc < x.k).any()
+    rl = O.reward_loss(ref["kl"], acc, x.reward.numpy().astype(np.float64), mode=O.W_GROUP_NORM,
+                       group=16, positions=1)
+    m = np.where(acc < x.k, acc + 1, acc)
+    mag = np.array([abs(rl["w"][b]) * ref["scale"][b, :m[b]].sum() for b in range(x.B)])
+    assert_close(got["loss"].cpu().numpy(), rl["loss"], mag, "loss")
+    assert_close(got["total"].cpu().numpy(), [rl["total"]], [mag.sum()], "total")
+    # the standalone loss and the gradient with the same positions
+    lp = torch.from_numpy(ref["topk_logp"].astype(np.float32))
+    ix = torch.from_numpy(ref["topk_idx"].astype(np.int32))
+    accd = torch.from_numpy(acc.astype(np.int32)).to(DEV)
+    kl = sv.sv_kd_kl_loss(lp.to(DEV), ix.to(DEV), x.draft.to(DEV), x.temperature, accd,
+                          x.reward.to(DEV), wmode="group_norm", group=16, positions=1)
+    torch.cuda.synchronize()
+    assert_close(kl["loss"].cpu().numpy(), rl["loss"], mag, "standalone loss")
+    g = sv.sv_kd_grad(lp.to(DEV), ix.to(DEV), x.draft.to(DEV), accd, x.reward.to(DEV),
+                      x.temperature, wmode="group_norm", group=16, positions=1)
+    gref = O.kd_grad(lp.numpy().astype(np.float64), ix.numpy(), x.draft, acc.astype(np.int32),
+                     x.reward.numpy().astype(np.float64), x.temperature, mode=O.W_GROUP_NORM,
+                     group=16, positions=1)
+    torch.cuda.synchronize()
+    gg = g.cpu().numpy().astype(np.float64)
+    row_active = np.arange(x.k)[None, :] < m[:, None]
+    assert np.array_equal(np.abs(gg).sum(-1) > 0, np.abs(gref).sum(-1) > 0)
+    assert (row_active >= (np.abs(gref).sum(-1) > 0)).all()
+    scale = np.abs(gref).max(axis=-1, keepdims=True) + 1e-30
+    assert (np.abs(gg - gref) <= 1e-4 * scale).all()
