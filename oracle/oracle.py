@@ -65,11 +65,12 @@ def _lib(plant: int = 0) -> ctypes.CDLL:
                                 ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double))
         ci, cd = ctypes.c_int, ctypes.c_double
         L.oracle_verify_chain.argtypes = [vp, ci, vp, ci, ci, i32p, f32p, ci, ci, ci, cd, i32p, i32p,
-                                          f64p, f64p, f64p, i32p, i32p, ci]
+                                          i32p, i32p, f64p, f64p, f64p, i32p, i32p, ci]
         L.oracle_tree_greedy.argtypes = [vp, ci, i32p, i32p, ci, ci, ci, ci, i32p, i32p, i32p, ci]
         L.oracle_topk.argtypes = [vp, ci, ci, ci, ci, cd, f64p, i32p, f64p, ci]
         L.oracle_kl.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, ci, cd, f64p, f64p, ci]
-        L.oracle_reward_loss.argtypes = [f64p, i32p, f64p, ci, ci, ci, ci, cd, ci, f64p, f64p,
+        L.oracle_reward_loss.argtypes = [f64p, i32p, f64p, ci, ci, ci, ci, cd, ci, i32p, i32p,
+                                         f64p, f64p,
                                          f64p]
         L.oracle_softmax.argtypes = [vp, ci, ci, ci, cd, f64p, f64p]
         L.oracle_kd_grad.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, cd, i32p, f64p, ci, ci,
@@ -122,6 +123,17 @@ def _ptr(a, ctype):
     return a.ctypes.data_as(ctypes.POINTER(ctype))
 
 
+def _opt_i32(x, n: int):
+    """An optional int32 [n] argument (None passes NULL); the pointer keeps the
+    converted array alive for the call."""
+    if x is None:
+        return None
+    a = _np(x, np.int32).reshape(-1)
+    if a.size != n:
+        raise ValueError(f"expected {n} entries, got {a.size}")
+    return _ptr(a, ctypes.c_int32)
+
+
 def _check(rc: int, what: str):
     if rc != 0:
         raise OracleError(f"{what}: {_ERRORS.get(rc, rc)}")
@@ -129,7 +141,7 @@ def _check(rc: int, what: str):
 
 def verify_chain(target, draft, draft_tokens, uniforms, temperature: float, *,
                  draft_kind: int = DRAFT_LOGITS, threads: int = 0, plant: int = 0,
-                 allow_errors: bool = False) -> dict:
+                 allow_errors: bool = False, draft_len=None, active=None) -> dict:
     """Chain verification of B requests with k draft tokens each.
 
     target [B, k+1, V] and draft [B, k, V] (fp32 or bf16; draft may be fp32
@@ -157,6 +169,7 @@ def verify_chain(target, draft, draft_tokens, uniforms, temperature: float, *,
     rc = _lib(plant).oracle_verify_chain(
         t.ctypes.data, tdt, None if d is None else d.ctypes.data, ddt, draft_kind,
         _ptr(x, ctypes.c_int32), _ptr(u, ctypes.c_float), B, k, V, T,
+        _opt_i32(draft_len, B), _opt_i32(active, B),
         _ptr(acc, ctypes.c_int32), _ptr(out, ctypes.c_int32), _ptr(px, ctypes.c_double),
         _ptr(qx, ctypes.c_double), _ptr(margin, ctypes.c_double), _ptr(srow, ctypes.c_int32),
         _ptr(fb, ctypes.c_int32), threads)
@@ -220,7 +233,7 @@ def kl(topk_logp, topk_idx, draft, temperature: float, *, draft_kind: int = DRAF
 
 
 def reward_loss(kl_values, accepted_len, reward, *, mode: int = W_RAW, group: int = 1,
-                clip: float = 0.0, positions: int = 0) -> dict:
+                clip: float = 0.0, positions: int = 0, draft_len=None, active=None) -> dict:
     """Reward-weighted KD loss per request and its sum."""
     klv = _np(kl_values, np.float64)
     B, k = klv.shape
@@ -231,7 +244,8 @@ def reward_loss(kl_values, accepted_len, reward, *, mode: int = W_RAW, group: in
     total = np.zeros(1, np.float64)
     rc = _lib().oracle_reward_loss(_ptr(klv, ctypes.c_double), _ptr(acc, ctypes.c_int32),
                                    _ptr(r, ctypes.c_double), B, k, mode, group, float(clip),
-                                   int(positions), _ptr(w, ctypes.c_double),
+                                   int(positions), _opt_i32(draft_len, B),
+                                   _opt_i32(active, B), _ptr(w, ctypes.c_double),
                                    _ptr(loss, ctypes.c_double),
                                    _ptr(total, ctypes.c_double))
     _check(rc, "reward_loss")
@@ -273,13 +287,14 @@ def softmax(logits, temperature: float) -> dict:
 
 def verify_kd(target, draft, draft_tokens, uniforms, reward, temperature: float, K: int, *,
               mode: int = W_RAW, group: int = 1, clip: float = 0.0,
-              draft_kind: int = DRAFT_LOGITS, positions: int = 0, threads: int = 0) -> dict:
+              draft_kind: int = DRAFT_LOGITS, positions: int = 0, threads: int = 0,
+              draft_len=None, active=None) -> dict:
     """Chain verification followed by the KD quantities, each step as above."""
     v = verify_chain(target, draft, draft_tokens, uniforms, temperature,
-                     draft_kind=draft_kind, threads=threads)
+                     draft_kind=draft_kind, threads=threads, draft_len=draft_len, active=active)
     tk = topk(target, K, temperature, threads=threads)
     d = kl(tk["topk_logp"], tk["topk_idx"], draft, temperature, draft_kind=draft_kind,
            threads=threads)
     rl = reward_loss(d["kl"], v["accepted_len"], reward, mode=mode, group=group, clip=clip,
-                     positions=positions)
+                     positions=positions, draft_len=draft_len, active=active)
     return {**v, **tk, **d, **rl}

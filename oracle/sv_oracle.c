@@ -169,17 +169,30 @@ static int inverse_cdf(const double* w, int V, double u, double* margin) {
 /* sampled), fallback [B] (1 when the residual mass was zero).                */
 /* T == 0 selects greedy verification.                                        */
 /* ------------------------------------------------------------------------ */
+/* draft_len [B] (may be NULL: k for every request): request b drafted
+ * k_b <= k tokens; it uses target rows 0..k_b, draft rows 0..k_b-1, the
+ * uniforms 0..k_b-1 for the tests and uniform k_b for the draw.  active [B]
+ * (may be NULL: all active): an inactive request verifies nothing,
+ * accepted_len = 0 and every out_token -1 (no token is emitted).          */
 int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int d_dtype,
                         int d_kind, const int32_t* draft_tokens, const float* u, int B,
-                        int k, int V, double T, int32_t* accepted_len, int32_t* out_tokens,
-                        double* p_x, double* q_x, double* cdf_margin, int32_t* sample_row,
-                        int32_t* fallback, int nthreads) {
+                        int k, int V, double T, const int32_t* draft_len, const int32_t* active,
+                        int32_t* accepted_len, int32_t* out_tokens, double* p_x, double* q_x,
+                        double* cdf_margin, int32_t* sample_row, int32_t* fallback,
+                        int nthreads) {
   if (B < 0 || k < 1 || V < 1 || !(T >= 0.0) || !target || !draft_tokens || !accepted_len ||
       !out_tokens)
     return OR_BAD_ARG;
   if (T > 0.0 && (!draft || !u)) return OR_BAD_ARG;
-  for (size_t i = 0; i < (size_t)B * (size_t)k; ++i)
-    if (draft_tokens[i] < 0 || draft_tokens[i] >= V) return OR_BAD_TOKEN;
+  for (int b = 0; b < B; ++b) {
+    const int kb = draft_len ? draft_len[b] : k;
+    if (kb < 0 || kb > k) return OR_BAD_ARG;
+    if (active && !active[b]) continue;
+    for (int i = 0; i < kb; ++i) {
+      const int32_t t = draft_tokens[(size_t)b * k + i];
+      if (t < 0 || t >= V) return OR_BAD_TOKEN;
+    }
+  }
   set_threads(nthreads);
   const int P = k + 1;
   int err = OR_OK;
@@ -203,12 +216,18 @@ int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int 
         for (int i = 0; i < k; ++i) p_x[(size_t)b * k + i] = q_x[(size_t)b * k + i] = NAN;
       if (cdf_margin) cdf_margin[b] = INFINITY;
       if (fallback) fallback[b] = 0;
+      if (active && !active[b]) {  /* nothing verified, nothing emitted */
+        accepted_len[b] = 0;
+        if (sample_row) sample_row[b] = -1;
+        continue;
+      }
+      const int kb = draft_len ? draft_len[b] : k;
 
       if (T == 0.0) {
         /* Greedy: accept x_i iff it equals the target argmax at row i; emit
          * the target argmax at the first mismatch, or at row k. */
-        int n = k, emit = -1;
-        for (int i = 0; i < k; ++i) {
+        int n = kb, emit = -1;
+        for (int i = 0; i < kb; ++i) {
           int g = argmax_row(target, t_dtype, ((size_t)b * P + i) * (size_t)V, V);
           if (x[i] != g) {
             n = i;
@@ -216,7 +235,7 @@ int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int 
             break;
           }
         }
-        if (n == k) emit = argmax_row(target, t_dtype, ((size_t)b * P + k) * (size_t)V, V);
+        if (n == kb) emit = argmax_row(target, t_dtype, ((size_t)b * P + kb) * (size_t)V, V);
         for (int i = 0; i < n; ++i) out[i] = x[i];
         out[n] = emit;
         accepted_len[b] = n;
@@ -224,8 +243,8 @@ int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int 
         continue;
       }
 
-      int n = k, emit = -1, bad = 0;
-      for (int i = 0; i < k; ++i) {
+      int n = kb, emit = -1, bad = 0;
+      for (int i = 0; i < kb; ++i) {
         size_t trow = ((size_t)b * P + i) * (size_t)V;
         size_t drow = ((size_t)b * k + i) * (size_t)V;
         if (isnan(softmax_row(target, t_dtype, trow, V, T, p))) {
@@ -263,10 +282,10 @@ int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int 
           r[j] = d > 0.0 ? d : 0.0;
         }
         double mg;
-        emit = inverse_cdf(r, V, (double)u[(size_t)b * P + k], &mg);
+        emit = inverse_cdf(r, V, (double)u[(size_t)b * P + kb], &mg);
         if (emit < 0) {
           /* Zero residual mass: sample the target row itself. */
-          emit = inverse_cdf(p, V, (double)u[(size_t)b * P + k], &mg);
+          emit = inverse_cdf(p, V, (double)u[(size_t)b * P + kb], &mg);
           if (fallback) fallback[b] = 1;
         }
         if (cdf_margin) cdf_margin[b] = mg;
@@ -278,9 +297,13 @@ int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int 
         err = OR_NO_FINITE;
         continue;
       }
-      if (n == k) {
-        /* Every draft accepted: one bonus token from the target row k. */
+      if (n == kb) {
+        /* Every draft accepted: one bonus token from the target row k_b. */
+#if OR_PLANT == 3
         size_t trow = ((size_t)b * P + k) * (size_t)V;
+#else
+        size_t trow = ((size_t)b * P + kb) * (size_t)V;
+#endif
         if (isnan(softmax_row(target, t_dtype, trow, V, T, p))) {
           accepted_len[b] = -1;
 #pragma omp atomic write
@@ -288,7 +311,7 @@ int oracle_verify_chain(const void* target, int t_dtype, const void* draft, int 
           continue;
         }
         double mg;
-        emit = inverse_cdf(p, V, (double)u[(size_t)b * P + k], &mg);
+        emit = inverse_cdf(p, V, (double)u[(size_t)b * P + kb], &mg);
         if (cdf_margin) cdf_margin[b] = mg;
       }
       for (int i = 0; i < n; ++i) out[i] = x[i];
@@ -517,9 +540,13 @@ int oracle_kl(const double* topk_logp, const int32_t* topk_idx, int B, int k, in
 /* positions = 1, one more when a draft was rejected (n < k): the first       */
 /* rejected position too, as drafters that learn from their rejected          */
 /* proposals do ("Draft-OPD" page).                                           */
+/* Ragged batches: draft_len [B] (may be NULL: k) moves the "rejected" test   */
+/* to n < k_b; a request with active[b] == 0 (active may be NULL) has         */
+/* loss_b = 0.                                                                */
 /* ------------------------------------------------------------------------ */
 int oracle_reward_loss(const double* kl, const int32_t* accepted_len, const double* reward,
-                       int B, int k, int mode, int group, double clip, int positions, double* w,
+                       int B, int k, int mode, int group, double clip, int positions,
+                       const int32_t* draft_len, const int32_t* active, double* w,
                        double* loss, double* total) {
   if (B < 0 || k < 1 || !kl || !accepted_len || !reward || !loss || !total) return OR_BAD_ARG;
   if (mode == OR_W_GROUP_NORM && (group < 1 || B % group != 0)) return OR_BAD_ARG;
@@ -534,12 +561,13 @@ int oracle_reward_loss(const double* kl, const int32_t* accepted_len, const doub
     }
     if (clip > 0.0) wb = wb > clip ? clip : (wb < -clip ? -clip : wb);
     if (w) w[b] = wb;
+    const int kb = draft_len ? draft_len[b] : k;
     int n = accepted_len[b];
-    if (n < 0 || n > k) return OR_BAD_ARG;
-    int m = (positions && n < k) ? n + 1 : n;
+    if (kb < 0 || kb > k || n < 0 || n > kb) return OR_BAD_ARG;
+    int m = (positions && n < kb) ? n + 1 : n;
     double s = 0.0;
     for (int i = 0; i < m; ++i) s += kl[(size_t)b * k + i];
-    loss[b] = wb == 0.0 ? 0.0 : wb * s;
+    loss[b] = (wb == 0.0 || (active && !active[b])) ? 0.0 : wb * s;
     sum += loss[b];
   }
   *total = sum;

@@ -433,3 +433,138 @@ def test_kd_mask_with_the_first_rejected_position(oracle):
     bumped = np.minimum(acc + 1, k).astype(np.int32)
     r2 = oracle.reward_loss(kl, bumped, rw)
     assert np.allclose(r1["loss"], r2["loss"], rtol=1e-14, atol=0)
+
+
+# --------------------------------------------------------------------------
+# Ragged batches: request b drafted k_b <= k tokens; inactive requests emit
+# nothing.
+# --------------------------------------------------------------------------
+def _ragged_mc(oracle, plant=0):
+    rng = np.random.default_rng(31)
+    k, V, B = 3, 8, 200_000
+    zt = rng.normal(0, 1.5, (k + 1, V)).astype(np.float32)
+    d = rng.dirichlet(np.full(V, 0.7), size=k).astype(np.float32)
+    x = inputs.make_chain_fixed(B, zt, d, draft_kind="probs", temperature=1.0, seed=9)
+    klen = rng.integers(0, k + 1, B).astype(np.int32)
+    act = (rng.random(B) < 0.9).astype(np.int32)
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 1.0,
+                            draft_kind=oracle.DRAFT_PROBS, draft_len=klen, active=act,
+                            plant=plant)
+    p = torch.softmax(torch.from_numpy(zt).double(), -1).numpy()
+    return r, p, d.astype(np.float64), klen, act
+
+
+def _ragged_pvalues(r, p, klen, act):
+    k, V = p.shape[0] - 1, p.shape[1]
+    acc, out = r["accepted_len"], r["out_tokens"]
+    pv = []
+    for i in range(k + 1):
+        reached = (act == 1) & (klen >= i) & (acc >= i)
+        counts = np.bincount(out[reached, i], minlength=V)
+        pv.append(scipy.stats.chisquare(counts, p[i] * reached.sum()).pvalue)
+    return pv
+
+
+def test_ragged_planted_bonus_row_is_caught(oracle):
+    """A bonus drawn from row k instead of row k_b (plant 3) fails the
+    ragged losslessness pin."""
+    oracle.build(plant=3)
+    r, p, q, klen, act = _ragged_mc(oracle, plant=3)
+    assert min(_ragged_pvalues(r, p, klen, act)) < 1e-6
+
+
+def test_ragged_chain_is_lossless(oracle):
+    """With per-request draft lengths k_b the emitted token at every position
+    i <= k_b is still distributed as the target row i, and position i < k_b
+    accepts at the rate sum_x min(p_i, q_i) (Leviathan et al.); inactive
+    requests emit nothing.  A bonus drawn from the wrong row (k instead of
+    k_b) fails the chi-square test at position k_b."""
+    r, p, q, klen, act = _ragged_mc(oracle)
+    k, V = 3, 8
+    acc, out = r["accepted_len"], r["out_tokens"]
+    off = act == 0
+    assert (acc[off] == 0).all() and (out[off] == -1).all()
+    on = act == 1
+    assert (acc[on] <= klen[on]).all()
+    for b in np.flatnonzero(on)[:2000]:
+        n = acc[b]
+        assert (out[b, n + 1:] == -1).all() and out[b, n] >= 0
+    for i, pval in enumerate(_ragged_pvalues(r, p, klen, act)):
+        assert pval > 1e-3, (i, pval)
+    for i in range(k):
+        tested = on & (klen > i) & (acc >= i)
+        if tested.any():
+            a = (acc[tested] > i).mean()
+            alpha = np.minimum(p[i], q[i]).sum()
+            sd = math.sqrt(alpha * (1 - alpha) / tested.sum())
+            assert abs(a - alpha) < 4 * sd, (i, a, alpha)
+
+
+def test_ragged_chain_equals_the_shorter_chain(oracle):
+    """Request b of a ragged batch gives exactly the result of a chain of
+    k_b drafts on the same rows, with the uniforms u_0..u_{k_b} (the draw
+    takes u_{k_b}); k_b = 0 is an inverse-CDF draw from the target row 0."""
+    T = 0.8
+    x = inputs.make_chain(12, 4, 500, dtype="bf16", temperature=T, seed=21)
+    klen = np.array([4, 3, 2, 1, 0, 4, 2, 0, 1, 3, 3, 4], np.int32)
+    r = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, T, draft_len=klen)
+    for b in range(12):
+        kb = int(klen[b])
+        if kb == 0:
+            z = x.target[b, 0].double().numpy() / float(np.float32(T))
+            pz = np.exp(z - scipy.special.logsumexp(z))
+            u0 = float(x.uniforms[b, 0])
+            want = int(np.searchsorted(np.cumsum(pz), u0 * pz.sum(), side="right"))
+            assert r["accepted_len"][b] == 0 and r["out_tokens"][b, 0] == want
+            assert (r["out_tokens"][b, 1:] == -1).all()
+            continue
+        s = oracle.verify_chain(x.target[b:b + 1, :kb + 1].contiguous(),
+                                x.draft[b:b + 1, :kb].contiguous(),
+                                x.draft_tokens[b:b + 1, :kb].contiguous(),
+                                x.uniforms[b:b + 1, :kb + 1].contiguous(), T)
+        assert r["accepted_len"][b] == s["accepted_len"][0]
+        assert list(r["out_tokens"][b, :kb + 1]) == list(s["out_tokens"][0])
+        assert (r["out_tokens"][b, kb + 1:] == -1).all()
+
+
+def test_ragged_greedy_chain_bruteforce(oracle):
+    rng = np.random.default_rng(8)
+    B, k, V = 200, 4, 30
+    z = _quantised_rows(rng, (B, k + 1, V))
+    first_max = z.argmax(-1)
+    x = np.where(rng.random((B, k)) < 0.8, first_max[:, :k], rng.integers(0, V, (B, k)))
+    klen = rng.integers(0, k + 1, B).astype(np.int32)
+    act = (rng.random(B) < 0.85).astype(np.int32)
+    x[np.arange(k)[None, :] >= klen[:, None]] = -7  # never read: outside the drafts
+    x[act == 0] = -7
+    r = oracle.verify_chain(torch.from_numpy(z), None, torch.from_numpy(x.astype(np.int32)),
+                            None, 0.0, draft_len=klen, active=act)
+    for b in range(B):
+        if not act[b]:
+            assert r["accepted_len"][b] == 0 and (r["out_tokens"][b] == -1).all()
+            continue
+        n = 0
+        while n < klen[b] and x[b, n] == first_max[b, n]:
+            n += 1
+        assert r["accepted_len"][b] == n
+        assert list(r["out_tokens"][b, :n]) == list(x[b, :n])
+        assert r["out_tokens"][b, n] == first_max[b, n]
+        assert (r["out_tokens"][b, n + 1:] == -1).all()
+
+
+def test_ragged_kd_mask_and_inactive_requests(oracle):
+    """With draft lengths the first-rejected-position rule tests n < k_b, and
+    an inactive request contributes nothing to the loss."""
+    rng = np.random.default_rng(6)
+    B, k = 6, 4
+    kl = rng.uniform(0, 1, (B, k))
+    klen = np.array([4, 2, 2, 0, 3, 1], np.int32)
+    acc = np.array([1, 2, 1, 0, 3, 1], np.int32)
+    act = np.array([1, 1, 1, 1, 1, 0], np.int32)
+    rw = rng.uniform(0.1, 1, B)
+    r = oracle.reward_loss(kl, acc, rw, positions=1, draft_len=klen, active=act)
+    want = [rw[0] * kl[0, :2].sum(), rw[1] * kl[1, :2].sum(), rw[2] * kl[2, :2].sum(), 0.0,
+            rw[4] * kl[4, :3].sum(), 0.0]
+    assert np.allclose(r["loss"], want, rtol=1e-14, atol=0)
+    with pytest.raises(oracle.OracleError):
+        oracle.reward_loss(kl, np.array([3, 0, 0, 0, 0, 0], np.int32), rw, draft_len=klen * 0 + 2)
