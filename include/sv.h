@@ -86,6 +86,7 @@ typedef enum sv_weight_mode { SV_W_RAW = 0, SV_W_GROUP_NORM = 1 } sv_weight_mode
 #define SV_DEV_TIMEOUT 0x4        /* a bounded wait for a bulk copy gave up */
 #define SV_DEV_BAD_TREE 0x8       /* parents[] is not a tree in BFS order, or depth > max_depth */
 #define SV_DEV_BAD_INDEX 0x10     /* a top-K index outside [0, V) given to sv_kd_kl_loss */
+#define SV_DEV_BAD_LEN 0x20       /* a draft_len outside [0, k] given to sv_verify_chain_ragged */
 #define SV_DEV_ERROR_MASK 0xff
 #define SV_DEV_RESIDUAL_ZERO 0x100 /* info: a rejection met zero residual mass; the target row was sampled */
 #define SV_DEV_TOPK_SLOW 0x200     /* info: massive ties sent a top-K through the slow exact path */
@@ -166,6 +167,41 @@ SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, co
                           int32_t* accepted_len, int32_t* out_tokens, const sv_kd_args* kd,
                           void* workspace, size_t workspace_bytes, int32_t* device_status,
                           void* stream);
+
+/*
+ * sv_verify_chain_ragged -- sv_verify_chain for a batch whose requests
+ * drafted different numbers of tokens, some of which may be idle.
+ *
+ * Operation: that of sv_verify_chain with k replaced per request by
+ *   k_b = draft_len[b] (0 <= k_b <= k; k itself is the padded length).  The
+ *   pages verify each request's own draft chain; a batch that mixes chain
+ *   lengths, or that holds finished requests, is padded to one k here, and
+ *   the padding is never read.  Request b tests drafts 0..k_b-1 with
+ *   uniforms[b, 0..k_b-1], draws the resample or the bonus token with
+ *   uniforms[b, k_b], and takes the bonus from target row k_b.  k_b = 0
+ *   draws one token from target row 0.  A request with active[b] == 0 is
+ *   idle: none of its rows is read, accepted_len = 0 and every out_token is
+ *   -1; with kd, its rows are empty and its loss is 0.
+ *
+ * Arguments: those of sv_verify_chain, plus
+ *   draft_len  [B] int32 device, or NULL (k for every request).  A value
+ *              outside [0, k] fails that request (accepted_len -1, outputs
+ *              -1 / NaN) and sets SV_DEV_BAD_LEN.
+ *   active     [B] int32 device, or NULL (every request active).
+ *   Row and draft-token entries past k_b (and all entries of an idle request)
+ *   are not read and need not be valid.  With kd and positions = 1, the first
+ *   rejected position is added when n < k_b.
+ *   Layouts, workspace size and errors are those of sv_verify_chain.
+ */
+SV_API sv_status sv_verify_chain_ragged(const void* target_logits, sv_dtype t_dtype,
+                                        const void* draft, sv_dtype d_dtype,
+                                        sv_draft_kind d_kind, const int32_t* draft_tokens,
+                                        const float* uniforms, const int32_t* draft_len,
+                                        const int32_t* active, int B, int k, int V,
+                                        float temperature, int32_t* accepted_len,
+                                        int32_t* out_tokens, const sv_kd_args* kd,
+                                        void* workspace, size_t workspace_bytes,
+                                        int32_t* device_status, void* stream);
 
 /*
  * sv_verify_chain_noalloc -- sv_verify_chain without a caller-supplied

@@ -383,7 +383,11 @@ static cudaError_t run_chain_sample(StreamParams sp, const StreamGeom& sg, Finis
   fp.use_bulk = plan.use_bulk;
   fp.lay = plan.lay;
   static_assert(base == chain_sample_flags<DKIND, false>(), "stream and finisher flags");
-  e = kd ? launch_stream<TT, DT, base | kFTopk0>(sp, sg, s) : launch_stream<TT, DT, base>(sp, sg, s);
+  const bool rg = sp.klen != nullptr || sp.active != nullptr;
+  e = kd ? (rg ? launch_stream<TT, DT, base | kFTopk0 | kFRagged>(sp, sg, s)
+               : launch_stream<TT, DT, base | kFTopk0>(sp, sg, s))
+         : (rg ? launch_stream<TT, DT, base | kFRagged>(sp, sg, s)
+               : launch_stream<TT, DT, base>(sp, sg, s));
   if (e != cudaSuccess) return e;
   fp.sp = sp;
   return launch_clusters(fin, fp, plan, fp.B, s);
@@ -417,13 +421,19 @@ static sv_status check_workspace(void* ws, size_t bytes, size_t need) {
   return SV_OK;
 }
 
-sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
-                          sv_dtype d_dtype, sv_draft_kind d_kind, const int32_t* draft_tokens,
-                          const float* uniforms, int B, int k, int V, float temperature,
-                          int32_t* accepted_len, int32_t* out_tokens, const sv_kd_args* kd,
-                          void* workspace, size_t workspace_bytes, int32_t* device_status,
-                          void* stream) {
+}  // extern "C"
+
+// Chain verification, padded (draft_len == active == nullptr) or ragged.
+static sv_status verify_chain_impl(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                                   sv_dtype d_dtype, sv_draft_kind d_kind,
+                                   const int32_t* draft_tokens, const float* uniforms,
+                                   const int32_t* draft_len, const int32_t* active, int B, int k,
+                                   int V, float temperature, int32_t* accepted_len,
+                                   int32_t* out_tokens, const sv_kd_args* kd, void* workspace,
+                                   size_t workspace_bytes, int32_t* device_status, void* stream) {
   if (B < 0 || k < 1 || k > 255 || V < 1) return SV_ERR_INVALID_ARG;
+  if ((draft_len && !aligned(draft_len, 4)) || (active && !aligned(active, 4)))
+    return SV_ERR_INVALID_ARG;
   if (!(temperature >= 0.f) || !isfinite(temperature)) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(t_dtype)) return SV_ERR_INVALID_ARG;
   if (kd && (kd->K < 1 || kd->K > kMaxK || kd->K > V)) return SV_ERR_INVALID_ARG;
@@ -492,6 +502,8 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   sp.req_reject = w.reject;
   sp.sched = w.glob + 32;
   sp.status = device_status;
+  sp.klen = draft_len;
+  sp.active = active;
 
   FinishParams fp = {};
   fp.target = target_logits;
@@ -531,8 +543,13 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
   }
 
   if (greedy) {
-    cudaError_t e = t_dtype == SV_BF16 ? launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s)
-                                       : launch_stream<F32, F32, kFArgmax0>(sp, sg, s);
+    const bool rg = draft_len != nullptr || active != nullptr;
+    cudaError_t e =
+        t_dtype == SV_BF16
+            ? (rg ? launch_stream<BF16, BF16, kFArgmax0 | kFRagged>(sp, sg, s)
+                  : launch_stream<BF16, BF16, kFArgmax0>(sp, sg, s))
+            : (rg ? launch_stream<F32, F32, kFArgmax0 | kFRagged>(sp, sg, s)
+                  : launch_stream<F32, F32, kFArgmax0>(sp, sg, s));
     if (e != cudaSuccess) return SV_ERR_CUDA;
     fp.sp = sp;
     const int gsm = kFixedBytes + P * (int)sizeof(RowRec);
@@ -563,6 +580,31 @@ sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const voi
             ? run_chain_sample<F32, BF16, kDraftLogits>(sp, sg, fp, plans, np, kd, s)
             : run_chain_sample<F32, F32, kDraftLogits>(sp, sg, fp, plans, np, kd, s);
   return cuda_status(e);
+}
+
+extern "C" {
+
+sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                          sv_dtype d_dtype, sv_draft_kind d_kind, const int32_t* draft_tokens,
+                          const float* uniforms, int B, int k, int V, float temperature,
+                          int32_t* accepted_len, int32_t* out_tokens, const sv_kd_args* kd,
+                          void* workspace, size_t workspace_bytes, int32_t* device_status,
+                          void* stream) {
+  return verify_chain_impl(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens, uniforms,
+                           nullptr, nullptr, B, k, V, temperature, accepted_len, out_tokens, kd,
+                           workspace, workspace_bytes, device_status, stream);
+}
+
+sv_status sv_verify_chain_ragged(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                                 sv_dtype d_dtype, sv_draft_kind d_kind,
+                                 const int32_t* draft_tokens, const float* uniforms,
+                                 const int32_t* draft_len, const int32_t* active, int B, int k,
+                                 int V, float temperature, int32_t* accepted_len,
+                                 int32_t* out_tokens, const sv_kd_args* kd, void* workspace,
+                                 size_t workspace_bytes, int32_t* device_status, void* stream) {
+  return verify_chain_impl(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens, uniforms,
+                           draft_len, active, B, k, V, temperature, accepted_len, out_tokens, kd,
+                           workspace, workspace_bytes, device_status, stream);
 }
 
 // Scratch of sv_verify_chain_noalloc: one fixed, zero-initialised array per

@@ -205,40 +205,47 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
   if (threadIdx.x == 0) sh.tok = -1;
   pdl_wait();  // the stream's records are complete
 
-  // 0. the request's rows and its first rejection
-  load_rows<TT, DT, RF>(prm, rows, P, b, B, prm.tokens + (size_t)b * k, k, rank == 0);
+  // 0. the request's rows 0..k_b and its first rejection (k_b < 0: an
+  //    inactive request or an invalid draft count: no row)
+  const int kb = req_kb(prm.sp, b);
+  const int nld = kb < 0 ? 0 : kb + 1;
+  load_rows<TT, DT, RF>(prm, rows, nld, b, B, prm.tokens + (size_t)b * k, nld - 1, rank == 0);
   __syncthreads();
   if (w == 0) {
-    bool bad;
-    const int n = first_rejection(rows, k, &bad);
+    bool bad = true;
+    const int n = kb < 0 ? 0 : first_rejection(rows, kb, &bad);
     if (lane == 0) {
       sh.fin_n = bad ? -1 : n;
       sh.need = bad ? 0 : 1;
       sh.err = 0;
       sh.owner = 0;
-      sh.Gt = rows[n].G0;
-      sh.St = rows[n].S0;
-      sh.Gd = rows[n].G1;
-      sh.Sd = rows[n].S1;
+      if (!bad) {
+        sh.Gt = rows[n].G0;
+        sh.St = rows[n].S0;
+        sh.Gd = rows[n].G1;
+        sh.Sd = rows[n].S1;
+      }
+      if (kb == -2 && rank == 0) set_status(prm.status, SV_DEV_BAD_LEN);
     }
   }
   __syncthreads();
   const int n = sh.fin_n;
 
   // 1. fused KD outputs of rows 0..n (static schedule; the dynamic schedule
-  //    wrote them in the stream)
+  //    wrote them in the stream); the other rows' lists are cleared
   if (KD && !prm.sp.count) {
     for (int t = rank * kWarps + w; t < P; t += C * kWarps) {
-      const RowRec& rr = rows[t];
-      row_outputs<TT, DT, RF>(prm.sp, t * B + b, t < k ? prm.tokens[(size_t)b * k + t] : -1,
-                              rr.L0, rr.L1, 0, n >= 0 && t <= n, true);
+      const bool ld = t < nld;
+      row_outputs<TT, DT, RF>(prm.sp, t * B + b, t < kb ? prm.tokens[(size_t)b * k + t] : -1,
+                              ld ? rows[t].L0 : 0.0, ld ? rows[t].L1 : 0.0, 0,
+                              n >= 0 && t <= n, true);
     }
   }
 
-  // 2. the draw, from row pair n (residual) or the bonus row k (target only)
+  // 2. the draw, from row pair n (residual) or the bonus row k_b (target only)
   bool arrived = false;
   if (sh.need) {
-    const bool pair = n < k;
+    const bool pair = n < kb;
     const void* trow = row_ptr<TT>(prm.target, (size_t)b * P + n, V);
     const void* drow = pair ? row_ptr<DT>(prm.draft, (size_t)b * k + n, V) : nullptr;
     if (pair)
@@ -280,7 +287,7 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         const int tmo = warp_sum_int(lane < C ? cluster.map_shared_rank(&sh, lane)->timeouts : 0);
         if (lane == 0) {
           const double myO = rank > 0 ? lo : 0.0;
-          const double tt = (double)prm.u[(size_t)b * P + k] * R;
+          const double tt = (double)prm.u[(size_t)b * P + kb] * R;
           sh.tt = tt;
           sh.base = myO;
           sh.redo = (R == 0.0 && mode == kModeResidual && !tmo) ? 1 : 0;
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
       if (nn >= 0 && (!sh.need || sh.err)) nn = -1;
       if (nn >= 0 && (sh.tok < 0 || sh.tok >= V)) nn = -1;
       sh.fin_n = nn;
-      prm.accepted_len[b] = nn;
+      prm.accepted_len[b] = kb == -1 ? 0 : nn;  // an inactive request accepts nothing
       prm.req_reject[b] = 0u;
     }
     __syncthreads();
@@ -392,10 +399,12 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
       }
       for (int t = first_undef + (int)threadIdx.x; t < P; t += kThreads)
         prm.lse[(size_t)b * P + t] = NAN;
-      for (int t = first_undef + (int)threadIdx.x; t < k; t += kThreads)
+      // draft rows past the request's own drafts (k_b <= k) have no KL either
+      const int kl_undef = min(first_undef, kb < 0 ? 0 : kb);
+      for (int t = kl_undef + (int)threadIdx.x; t < k; t += kThreads)
         prm.kl[(size_t)b * k + t] = NAN;
       __syncthreads();
-      kd_finalize(b, nf, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
+      kd_finalize(b, nf, B, k, kb, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
                   prm.positions, prm.loss, prm.total, prm.glob_counter, sh);
     }
   }
@@ -411,20 +420,23 @@ __global__ void __launch_bounds__(kThreads) chain_greedy_finish(const __grid_con
   const int b = (int)blockIdx.x;
   const int k = prm.k, P = k + 1, B = prm.B;
   pdl_wait();
-  load_rows<T, T, kFArgmax0>(prm, rows, P, b, B, prm.tokens + (size_t)b * k, k, true);
+  const int kb = req_kb(prm.sp, b);  // rows 0..k_b (none when k_b < 0)
+  const int nld = kb < 0 ? 0 : kb + 1;
+  load_rows<T, T, kFArgmax0>(prm, rows, nld, b, B, prm.tokens + (size_t)b * k, nld - 1, true);
   __syncthreads();
   if (w == 0) {
-    bool bad = false;
-    const int n = first_rejection(rows, k, &bad);
-    const int tok = rows[n].argmax;
+    bool bad = true;
+    const int n = kb < 0 ? 0 : first_rejection(rows, kb, &bad);
+    const int tok = kb < 0 ? -1 : rows[n].argmax;
     if (tok < 0 || tok >= prm.V) bad = true;
+    if (kb == -2 && lane == 0) set_status(prm.status, SV_DEV_BAD_LEN);
     for (int t = lane; t < P; t += 32) {
       int v = -1;
       if (!bad) v = (t < n) ? prm.tokens[(size_t)b * k + t] : (t == n ? tok : -1);
       prm.out_tokens[(size_t)b * P + t] = v;
     }
     if (lane == 0) {
-      prm.accepted_len[b] = bad ? -1 : n;
+      prm.accepted_len[b] = kb == -1 ? 0 : (bad ? -1 : n);
       prm.req_reject[b] = 0u;
     }
   }
@@ -570,7 +582,7 @@ __global__ void __launch_bounds__(kThreads) kl_finish(const __grid_constant__ Fi
   }
   __syncthreads();
   if (!prm.draft_probs) release_rows(prm, k, b * k, 1, w, kWarps);
-  kd_finalize(b, sh.fin_n, B, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
+  kd_finalize(b, sh.fin_n, B, k, k, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
               prm.positions, prm.loss, prm.total, prm.glob_counter, sh);
 }
 

@@ -164,13 +164,14 @@ __device__ __forceinline__ bool arrive_last(uint32_t* counter, uint32_t total, R
 
 // Loss of request b, then (if it is the last request) the total.  Called by
 // the whole block that finalized request b.  kl rows are read through L2.
-__device__ inline void kd_finalize(int b, int n, int B, int k, const float* kl, const float* reward,
+__device__ inline void kd_finalize(int b, int n, int B, int k, int kb, const float* kl,
+                            const float* reward,
                             int wmode, int group, float clip, int positions, float* loss,
                             float* total, uint32_t* glob_counter, RowShared& sh) {
   if (threadIdx.x == 0) {
     // the KD positions: the accepted drafts, and with `positions` the first
-    // rejected one as well
-    const int m = (positions && n >= 0 && n < k) ? n + 1 : n;
+    // rejected one as well (kb: the request's draft count)
+    const int m = (positions && n >= 0 && n < kb) ? n + 1 : n;
     double s = 0.0;
     for (int i = 0; i < m; ++i) s += (double)__ldcg(&kl[(size_t)b * k + i]);
     const double w = (n < 0) ? 0.0 : reward_weight(reward, b, wmode, group, clip);

@@ -46,6 +46,9 @@ enum StreamFlags : int {
   kFStatic = 64,   // static contiguous partition, no in-stream counting (the
                    // finishing kernel completes the rows); else dynamic items
                    // with in-stream counting and early exit
+  kFRagged = 128,  // chain requests with their own draft counts or an active
+                   // mask: rows a request does not use are skipped, and row
+                   // k_b streams its target row only
 };
 
 // How items map to rows and what the row decision is.
@@ -121,7 +124,23 @@ struct StreamParams {
   int count;              // 1: items are counted into rows and rows completed here
                           //    (required for skipping); 0: partials only, rows are
                           //    completed by the finishing kernel
+  // Ragged chains (both may be null): request b drafted klen[b] <= k tokens
+  // (rows 0..klen[b] are used, row klen[b] being its bonus row); a request
+  // with active[b] == 0 uses no row.
+  const int32_t* klen;
+  const int32_t* active;
 };
+
+// Draft count k_b of chain request b: k, or klen[b]; -1 for an inactive
+// request, -2 when klen[b] lies outside [0, k].  Rows i > k_b of the request
+// are not read.  (The streaming loop asks only in its kFRagged variants.)
+__device__ __forceinline__ int req_kb(const StreamParams& p, int b) {
+  if (p.klen == nullptr && p.active == nullptr) return p.k;
+  if (p.active != nullptr && __ldg(&p.active[b]) == 0) return -1;
+  if (p.klen == nullptr) return p.k;
+  const int kb = __ldg(&p.klen[b]);
+  return (kb < 0 || kb > p.k) ? -2 : kb;
+}
 
 // Where row r of a stream lives.
 struct RowLoc {
@@ -159,7 +178,7 @@ __device__ __forceinline__ RowLoc locate_row(const StreamParams& p, int r, int x
   const int P = p.k + 1;
   L.row0 = reinterpret_cast<const unsigned char*>(p.rows0) + ((size_t)L.b * P + L.i) * p.V * T0::bytes;
   L.row1 = nullptr;
-  if (p.rows1 != nullptr && L.i < p.k)
+  if (p.rows1 != nullptr && L.i < ((FLAGS & kFRagged) ? req_kb(p, L.b) : p.k))
     L.row1 = reinterpret_cast<const unsigned char*>(p.rows1) +
              ((size_t)L.b * p.k + L.i) * p.V * T1::bytes;
   return L;
@@ -380,7 +399,7 @@ __device__ __forceinline__ RowRec row_decide(const StreamParams& prm, int r, int
   if (s.flags & kPTimeout) err |= SV_DEV_TIMEOUT;
   if ((FLAGS & kFStats0) && s.G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
   if (prm.kind != kKindRows) {
-    const int i = fast_div(r, prm.div_B), b = r - i * prm.B, k = prm.k;
+    const int i = fast_div(r, prm.div_B), b = r - i * prm.B, k = req_kb(prm, b);
     if ((FLAGS & kFStats1) && i < k && s.G1 == -INFINITY) err |= SV_DEV_NO_FINITE;
     if (s.flags & kPSkipped) {
       err = 0;
@@ -391,7 +410,7 @@ __device__ __forceinline__ RowRec row_decide(const StreamParams& prm, int r, int
         const double c = (double)prm.c;
         const double px = exp2((double)s.zx0 * c - s.L0);
         const double qx = (FLAGS & kFStats1) ? exp2((double)s.zx1 * c - s.L1) : (double)s.zx1;
-        const double u = (double)prm.u[(size_t)b * (k + 1) + i];
+        const double u = (double)prm.u[(size_t)b * (prm.k + 1) + i];
         code = (u * qx < px) ? kRowAccepted : kRowRejected;
       }
     } else {  // greedy: accept iff the draft token is the argmax
@@ -437,7 +456,7 @@ __device__ __noinline__ void row_outputs(const StreamParams& prm, int r, int x, 
     prm.topk_idx[orow * K + lane] = j;
   }
   if (lane == 0) prm.lse[orow] = nan_out ? NAN : (float)(L0 * ln2);
-  if (!rows && L.row1 != nullptr) {
+  if (!rows && L.row1 != nullptr && L.i < req_kb(prm, L.b)) {
     // KL(p~ || q) over the renormalised top-K of the target row
     double mx = lp;
 #pragma unroll
@@ -702,10 +721,16 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
     const int r = fast_div(item, prm.div_nchunk);
     const int i = fast_div(r, prm.div_B), b = r - i * prm.B;
     if (!stat) rj = load_relaxed_u32(&prm.req_reject[b]);
-    if (i < prm.k) x = prm.tokens[(size_t)b * prm.k + i];
+    if (FLAGS & kFRagged) {
+      const int kb = req_kb(prm, b);
+      if (i > kb) rj = 0xffffffffu;  // a row its request does not use
+      if (i < kb) x = prm.tokens[(size_t)b * prm.k + i];
+    } else if (i < prm.k) {
+      x = prm.tokens[(size_t)b * prm.k + i];
+    }
   };
   // Pieces of an item (lane-uniform); 0 when skipped: an earlier position of
-  // its request rejected.  Lane 0 records the item's copy sources in
+  // its request rejected, or the request does not use the row.  Lane 0 records the item's copy sources in
   // descriptor `slot`.
   auto pieces_of = [&](int item, uint32_t rj, int slot) -> int {
     if (item >= total) return 0;

@@ -23,10 +23,10 @@ SV_F32, SV_BF16 = 0, 1
 SV_DRAFT_LOGITS, SV_DRAFT_PROBS = 0, 1
 SV_W_RAW, SV_W_GROUP_NORM = 0, 1
 SV_DEV_BAD_TOKEN, SV_DEV_NO_FINITE, SV_DEV_TIMEOUT, SV_DEV_BAD_TREE = 0x1, 0x2, 0x4, 0x8
-SV_DEV_BAD_INDEX, SV_DEV_ERROR_MASK = 0x10, 0xFF
+SV_DEV_BAD_INDEX, SV_DEV_BAD_LEN, SV_DEV_ERROR_MASK = 0x10, 0x20, 0xFF
 SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
-EXPORTS = ("sv_verify_chain", "sv_verify_chain_noalloc", "sv_verify_tree_greedy", "sv_kd_grad",
+EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc", "sv_verify_tree_greedy", "sv_kd_grad",
            "sv_kd_grad_workspace_size", "sv_extract_topk_kd", "sv_kd_kl_loss",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
            "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size",
@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
             vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
             L.sv_verify_chain.argtypes = [vp, ci, vp, ci, ci, vp, vp, ci, ci, ci, cf, vp, vp,
                                           ctypes.POINTER(sv_kd_args), vp, sz, vp, vp]
+            L.sv_verify_chain_ragged.argtypes = [vp, ci, vp, ci, ci, vp, vp, vp, vp, ci, ci, ci,
+                                                 cf, vp, vp, ctypes.POINTER(sv_kd_args), vp, sz,
+                                                 vp, vp]
+            L.sv_verify_chain_ragged.restype = ci
             L.sv_verify_chain_noalloc.argtypes = [vp, ci, vp, ci, ci, vp, vp, ci, ci, ci, cf, vp,
                                                   vp, ctypes.POINTER(sv_kd_args), vp, vp]
             L.sv_verify_chain_noalloc.restype = ci
@@ -176,9 +180,37 @@ def sv_verify_chain(target: torch.Tensor, draft: torch.Tensor | None, draft_toke
     target [B, k+1, V], draft [B, k, V] (logits, or fp32 probabilities with
     draft_kind="probs"), draft_tokens [B, k] int32, uniforms [B, k+1] fp32.
     kd: None or dict(K=32, reward=[B] fp32, wmode="raw"|"group_norm",
-    group=16, clip=0.0) for the fused top-K / KL / loss outputs.
+    group=16, clip=0.0, positions=0) for the fused top-K / KL / loss outputs.
     Returns the output tensors (allocated unless given in `out`).
     """
+    return _verify_chain(target, draft, draft_tokens, uniforms, temperature, None, None,
+                         draft_kind, kd, out, ws, device_status, stream)
+
+
+def sv_verify_chain_ragged(target: torch.Tensor, draft: torch.Tensor | None,
+                           draft_tokens: torch.Tensor, uniforms: torch.Tensor | None,
+                           temperature: float, *, draft_len: torch.Tensor | None = None,
+                           active: torch.Tensor | None = None, draft_kind: str = "logits",
+                           kd: dict | None = None, out: dict | None = None,
+                           ws: torch.Tensor | None = None,
+                           device_status: torch.Tensor | None = None, stream=None) -> dict:
+    """sv_verify_chain for requests with their own draft counts (see sv.h).
+
+    draft_len [B] int32 (k_b <= k; None: k) and active [B] int32 (0: an idle
+    request; None: all active), both on the device; the rest as in
+    sv_verify_chain, padded to k."""
+    B = target.shape[0]
+    for name, t in (("draft_len", draft_len), ("active", active)):
+        if t is not None:
+            _dev(t, name, torch.int32)
+            if t.numel() != B:
+                raise ValueError(f"{name} must have {B} entries")
+    return _verify_chain(target, draft, draft_tokens, uniforms, temperature, draft_len, active,
+                         draft_kind, kd, out, ws, device_status, stream)
+
+
+def _verify_chain(target, draft, draft_tokens, uniforms, temperature, draft_len, active,
+                  draft_kind, kd, out, ws, device_status, stream) -> dict:
     _dev(target, "target")
     B, P, V = target.shape
     k = P - 1
@@ -211,12 +243,17 @@ def sv_verify_chain(target: torch.Tensor, draft: torch.Tensor | None, draft_toke
                                          o["total"].data_ptr(), int(kd.get("positions", 0))))
     nbytes = sv_verify_chain_workspace_size(B, k, V, int(kd.get("K", 32)) if kd else 0)
     w = ws if ws is not None else workspace(dev, B, nbytes)
-    rc = lib().sv_verify_chain(
-        _p(target), _dtype_code(target), _p(draft),
-        _dtype_code(draft) if draft is not None else SV_F32, dk, _p(draft_tokens), _p(uniforms),
-        B, k, V, T, _p(o["accepted_len"]), _p(o["out_tokens"]), kd_ptr, _p(w), w.numel(),
-        _p(device_status), _stream(dev, stream))
-    _check(rc, "sv_verify_chain")
+    head = (_p(target), _dtype_code(target), _p(draft),
+            _dtype_code(draft) if draft is not None else SV_F32, dk, _p(draft_tokens),
+            _p(uniforms))
+    tail = (B, k, V, T, _p(o["accepted_len"]), _p(o["out_tokens"]), kd_ptr, _p(w), w.numel(),
+            _p(device_status), _stream(dev, stream))
+    if draft_len is None and active is None:
+        rc = lib().sv_verify_chain(*head, *tail)
+        _check(rc, "sv_verify_chain")
+    else:
+        rc = lib().sv_verify_chain_ragged(*head, _p(draft_len), _p(active), *tail)
+        _check(rc, "sv_verify_chain_ragged")
     return o
 
 
@@ -256,7 +293,7 @@ def sv_verify_chain_noalloc(target: torch.Tensor, draft: torch.Tensor | None,
                                          o["lse"].data_ptr(), o["kl"].data_ptr(),
                                          reward.data_ptr(), wmode, int(kd.get("group", 1)),
                                          float(kd.get("clip", 0.0)), o["loss"].data_ptr(),
-                                         o["total"].data_ptr()))
+                                         o["total"].data_ptr(), int(kd.get("positions", 0))))
     rc = lib().sv_verify_chain_noalloc(
         _p(target), _dtype_code(target), _p(draft),
         _dtype_code(draft) if draft is not None else SV_F32, dk, _p(draft_tokens), _p(uniforms),
