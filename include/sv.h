@@ -324,6 +324,35 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
 SV_API sv_status sv_device_status_check(int32_t device_status_word);
 
 /* Static description of a status code. */
+/*
+ * sv_sched_select -- the runtime half of the adaptive speculative decoding
+ * scheduler (reading notes, section 3 "G1 解法: Adaptive Speculative Decoding
+ * Server": an offline solver profiles throughput over configurations x batch
+ * sizes; at each decoding step the scheduler looks up the best configuration
+ * for the current active batch and falls back to plain target decoding when
+ * the predicted speedup is below 1).  Host code: no device memory, no stream.
+ *
+ * Arguments (all host memory, caller-owned):
+ *   throughput  [n_cfg, n_batch] fp32: profiled throughput (tokens/s or any
+ *               unit where higher is better) of configuration c at batch
+ *               size batches[j]; finite, >= 0, and > 0 in row `nonspec`.
+ *   batches     [n_batch] int32, strictly ascending, >= 1.
+ *   nonspec     the row of plain (non-speculative) target decoding.
+ *   active_batch >= 1: the current number of active requests.
+ *   config      out: the configuration to run.
+ *   predicted_speedup  out (may be NULL): the best speculative configuration's
+ *               predicted throughput over plain decoding's at active_batch
+ *               (the value compared with 1; 0 when n_cfg == 1).
+ * Lookup model: each row is interpolated linearly in the batch size between
+ * the two profiled sizes around active_batch, and held constant outside the
+ * profiled range.  The best speculative row is the largest interpolated
+ * throughput (lowest index on ties); it is chosen unless its speedup is
+ * below 1.  Invalid arguments return SV_ERR_INVALID_ARG.
+ */
+SV_API sv_status sv_sched_select(const float* throughput, const int32_t* batches, int n_cfg,
+                                 int n_batch, int nonspec, int active_batch, int32_t* config,
+                                 float* predicted_speedup);
+
 SV_API const char* sv_status_string(sv_status s);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

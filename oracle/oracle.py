@@ -298,3 +298,41 @@ def verify_kd(target, draft, draft_tokens, uniforms, reward, temperature: float,
     rl = reward_loss(d["kl"], v["accepted_len"], reward, mode=mode, group=group, clip=clip,
                      positions=positions, draft_len=draft_len, active=active)
     return {**v, **tk, **d, **rl}
+
+
+def sched_select(throughput, batches, nonspec: int, active_batch: int):
+    """Adaptive scheduler lookup ("ReSpec ... (reading notes)", section 3 "G1
+    解法: Adaptive Speculative Decoding Server": the solver's profiled
+    throughput per configuration and batch size; the scheduler picks the best
+    configuration for the active batch and falls back to plain decoding when
+    the predicted speedup is below 1).  Reading: each configuration's
+    throughput is interpolated linearly between the profiled batch sizes
+    around the active batch (held at the end values outside them); the best
+    speculative configuration is the largest (lowest index on ties).
+    Returns (config, best speculative speedup), in float64 from the float32
+    table."""
+    thr = [[float(np.float32(v)) for v in row] for row in np.asarray(throughput)]
+    bs = [int(b) for b in batches]
+    n_cfg = len(thr)
+
+    def interp(row):
+        if active_batch <= bs[0]:
+            return row[0]
+        if active_batch >= bs[-1]:
+            return row[-1]
+        for j in range(len(bs) - 1):
+            if bs[j] <= active_batch < bs[j + 1]:
+                t = (active_batch - bs[j]) / (bs[j + 1] - bs[j])
+                return row[j] + t * (row[j + 1] - row[j])
+        raise AssertionError("unreachable")
+
+    base = interp(thr[nonspec])
+    best, best_thr = -1, 0.0
+    for c in range(n_cfg):
+        if c == nonspec:
+            continue
+        v = interp(thr[c])
+        if best < 0 or v > best_thr:
+            best, best_thr = c, v
+    speedup = 0.0 if best < 0 else best_thr / base
+    return (nonspec if best < 0 or speedup < 1.0 else best), speedup

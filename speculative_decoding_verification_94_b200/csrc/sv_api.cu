@@ -945,6 +945,48 @@ sv_status sv_device_status_check(int32_t w) {
   return SV_OK;
 }
 
+sv_status sv_sched_select(const float* throughput, const int32_t* batches, int n_cfg,
+                          int n_batch, int nonspec, int active_batch, int32_t* config,
+                          float* predicted_speedup) {
+  if (!throughput || !batches || !config || n_cfg < 1 || n_batch < 1 || nonspec < 0 ||
+      nonspec >= n_cfg || active_batch < 1)
+    return SV_ERR_INVALID_ARG;
+  for (int j = 0; j < n_batch; ++j)
+    if (batches[j] < 1 || (j > 0 && batches[j] <= batches[j - 1])) return SV_ERR_INVALID_ARG;
+  for (long long i = 0; i < (long long)n_cfg * n_batch; ++i)
+    if (!(throughput[i] >= 0.f) || !isfinite(throughput[i])) return SV_ERR_INVALID_ARG;
+  // the two profiled sizes around the active batch and the weight of the upper one
+  int j0 = 0, j1 = 0;
+  double t = 0.0;
+  if (active_batch >= batches[n_batch - 1]) {
+    j0 = j1 = n_batch - 1;
+  } else if (active_batch > batches[0]) {
+    while (batches[j1] <= active_batch) ++j1;
+    j0 = j1 - 1;
+    t = (double)(active_batch - batches[j0]) / (double)(batches[j1] - batches[j0]);
+  }
+  auto at = [&](int c) {
+    const double a = throughput[(size_t)c * n_batch + j0], b = throughput[(size_t)c * n_batch + j1];
+    return a + t * (b - a);
+  };
+  const double base = at(nonspec);
+  if (!(base > 0.0)) return SV_ERR_INVALID_ARG;
+  int best = -1;
+  double best_thr = 0.0;
+  for (int c = 0; c < n_cfg; ++c) {
+    if (c == nonspec) continue;
+    const double v = at(c);
+    if (best < 0 || v > best_thr) {
+      best = c;
+      best_thr = v;
+    }
+  }
+  const double speedup = best < 0 ? 0.0 : best_thr / base;
+  *config = (best < 0 || speedup < 1.0) ? nonspec : best;
+  if (predicted_speedup) *predicted_speedup = (float)speedup;
+  return SV_OK;
+}
+
 const char* sv_status_string(sv_status s) {
   switch (s) {
     case SV_OK: return "ok";

@@ -26,8 +26,9 @@ SV_DEV_BAD_TOKEN, SV_DEV_NO_FINITE, SV_DEV_TIMEOUT, SV_DEV_BAD_TREE = 0x1, 0x2, 
 SV_DEV_BAD_INDEX, SV_DEV_BAD_LEN, SV_DEV_ERROR_MASK = 0x10, 0x20, 0xFF
 SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
-EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc", "sv_verify_tree_greedy", "sv_kd_grad",
-           "sv_kd_grad_workspace_size", "sv_extract_topk_kd", "sv_kd_kl_loss",
+EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc",
+           "sv_verify_tree_greedy", "sv_kd_grad", "sv_kd_grad_workspace_size",
+           "sv_extract_topk_kd", "sv_kd_kl_loss", "sv_sched_select",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
            "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size",
            "sv_device_status_check", "sv_status_string", "sv_version")
@@ -95,6 +96,8 @@ def lib() -> ctypes.CDLL:
             for f in ("sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
                       "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size"):
                 getattr(L, f).restype = sz
+            L.sv_sched_select.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp]
+            L.sv_sched_select.restype = ci
             L.sv_status_string.argtypes = [ci]
             L.sv_status_string.restype = ctypes.c_char_p
             L.sv_version.argtypes = []
@@ -160,6 +163,25 @@ def sv_verify_chain_workspace_size(B: int, k: int, V: int, K: int = 0) -> int:
 
 def sv_verify_tree_workspace_size(B: int, n: int, V: int) -> int:
     return int(lib().sv_verify_tree_workspace_size(B, n, V))
+
+
+def sv_sched_select(throughput, batches, nonspec: int, active_batch: int) -> tuple[int, float]:
+    """Adaptive scheduler lookup (see sv.h): the configuration to run at
+    `active_batch` from a profiled throughput table [n_cfg, n_batch] over
+    ascending batch sizes, and the best speculative configuration's predicted
+    speedup.  Host arrays; nothing touches the GPU."""
+    import numpy as np
+    thr = np.ascontiguousarray(throughput, dtype=np.float32)
+    bs = np.ascontiguousarray(batches, dtype=np.int32)
+    if thr.ndim != 2 or bs.ndim != 1 or thr.shape[1] != bs.shape[0]:
+        raise ValueError("throughput must be [n_cfg, n_batch] and batches [n_batch]")
+    cfg = ctypes.c_int32(-1)
+    sp = ctypes.c_float(0.0)
+    rc = lib().sv_sched_select(thr.ctypes.data, bs.ctypes.data, thr.shape[0], thr.shape[1],
+                               int(nonspec), int(active_batch), ctypes.addressof(cfg),
+                               ctypes.addressof(sp))
+    _check(rc, "sv_sched_select")
+    return int(cfg.value), float(sp.value)
 
 
 def sv_extract_topk_workspace_size(rows: int, V: int, K: int) -> int:
