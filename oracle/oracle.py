@@ -66,6 +66,8 @@ def _lib(plant: int = 0) -> ctypes.CDLL:
         ci, cd = ctypes.c_int, ctypes.c_double
         L.oracle_verify_chain.argtypes = [vp, ci, vp, ci, ci, i32p, f32p, ci, ci, ci, cd, i32p, i32p,
                                           i32p, i32p, f64p, f64p, f64p, i32p, i32p, ci]
+        L.oracle_tree_sample.argtypes = [vp, ci, vp, ci, ci, i32p, i32p, f32p, ci, ci, ci, cd, ci,
+                                         i32p, i32p, i32p, f64p, f64p, i32p, i32p, ci]
         L.oracle_tree_greedy.argtypes = [vp, ci, i32p, i32p, ci, ci, ci, ci, i32p, i32p, i32p, ci]
         L.oracle_topk.argtypes = [vp, ci, ci, ci, ci, cd, f64p, i32p, f64p, ci]
         L.oracle_kl.argtypes = [f64p, i32p, ci, ci, ci, vp, ci, ci, ci, cd, f64p, f64p, ci]
@@ -177,6 +179,36 @@ def verify_chain(target, draft, draft_tokens, uniforms, temperature: float, *,
         _check(rc, "verify_chain")
     return dict(accepted_len=acc, out_tokens=out, p_x=px, q_x=qx, cdf_margin=margin,
                 sample_row=srow, fallback=fb, status=rc)
+
+
+def tree_sample(target, draft, node_tokens, parents, uniforms, temperature: float,
+                max_depth: int, *, draft_kind: int = DRAFT_LOGITS, threads: int = 0,
+                plant: int = 0) -> dict:
+    """Sampling verification of B candidate trees of n nodes by multi-step
+    speculative sampling: target and draft [B, n, V], uniforms [B, n]."""
+    t, tdt = _raw(target)
+    d, ddt = _raw(draft)
+    B, n, V = t.shape
+    tok = _np(node_tokens, np.int32).reshape(B, n)
+    par = _np(parents, np.int32).reshape(B, n)
+    u = _np(uniforms, np.float32).reshape(B, n)
+    W = max_depth + 1
+    acc = np.zeros(B, np.int32)
+    out = np.zeros((B, W), np.int32)
+    nodes = np.zeros((B, W), np.int32)
+    tm = np.zeros(B, np.float64)
+    cm = np.zeros(B, np.float64)
+    fb = np.zeros(B, np.int32)
+    nt = np.zeros(B, np.int32)
+    rc = _lib(plant).oracle_tree_sample(
+        t.ctypes.data, tdt, d.ctypes.data, ddt, draft_kind, _ptr(tok, ctypes.c_int32),
+        _ptr(par, ctypes.c_int32), _ptr(u, ctypes.c_float), B, n, V,
+        float(np.float32(temperature)), max_depth, _ptr(acc, ctypes.c_int32),
+        _ptr(out, ctypes.c_int32), _ptr(nodes, ctypes.c_int32), _ptr(tm, ctypes.c_double),
+        _ptr(cm, ctypes.c_double), _ptr(fb, ctypes.c_int32), _ptr(nt, ctypes.c_int32), threads)
+    _check(rc, "tree_sample")
+    return dict(accepted_len=acc, out_tokens=out, accepted_nodes=nodes, test_margin=tm,
+                cdf_margin=cm, fallback=fb, n_tests=nt)
 
 
 def tree_greedy(logits, node_tokens, parents, max_depth: int, *, threads: int = 0) -> dict:

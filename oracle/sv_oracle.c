@@ -22,6 +22,13 @@
  *         the target's (Leviathan et al. 2023).  The equation body itself was
  *         lost from the page; min(1, p(x)/q(x)) is the named textbook rule.
  *  [TREE] same notes, section 3 "G1 解法": EAGLE candidate trees (s, t, n).
+ *  [MSS]  the pages name the trees but no rule for verifying them by
+ *         sampling; the rule restated here is the multi-step speculative
+ *         sampling of SpecInfer (Miao et al., "SpecInfer: Accelerating Large
+ *         Language Model Serving with Tree-based Speculative Inference and
+ *         Verification"), the recursive rejection sampling EAGLE adopts: it
+ *         keeps the target's distribution when every node's children are
+ *         drawn independently from that node's draft distribution.
  *  [TOPK] same notes, section 4 "G2 解法", worked example: keep the top-K=32
  *         target log-probs of the V=151936 row; KD target KL(softmax(log p) || q).
  *  [RWKD] ReSpec blog, section "奖励加权的适应机制": L_KD = w(r) * sum_t
@@ -401,6 +408,154 @@ int oracle_tree_greedy(const void* logits, int dtype, const int32_t* node_tokens
     free(g);
     free(depth);
     free(acc);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sampling tree verification ([TREE] for the trees; [MSS] for the rule).     */
+/*                                                                            */
+/* target [B, n, V]: the target distribution after each node; draft [B, n, V] */
+/* (logits or probabilities): the draft distribution the node's children     */
+/* were drawn from; node_tokens, parents as in oracle_tree_greedy; u [B, n]:  */
+/* column j >= 1 tests node j, column 0 drives the one final draw.            */
+/* Multi-step speculative sampling walks from the root.  At node v, r = p_v;  */
+/* its children are tried in ascending index order: child c with token x is   */
+/* accepted iff u_c * q_v(x) < r(x) (probability min(1, r(x)/q_v(x))), and    */
+/* the walk moves to c; otherwise r becomes max(0, r - q_v) / sum max(0,      */
+/* r - q_v) and the next child is tried.  When no child is accepted (or v is  */
+/* a leaf) one token is drawn from r by inverse CDF with u_0.  A zero         */
+/* residual mass (probability zero when the children are drawn from q_v)      */
+/* ends the tests at v and draws from p_v.  Outputs as oracle_tree_greedy;    */
+/* diagnostics (may be NULL): test_margin [B] = min over the tests of         */
+/* |u_c - r(x)/q_v(x)| (q_v(x) > 0; +inf without such a test), cdf_margin     */
+/* [B], fallback [B], n_tests [B].                                            */
+/* ------------------------------------------------------------------------ */
+int oracle_tree_sample(const void* target, int t_dtype, const void* draft, int d_dtype,
+                       int d_kind, const int32_t* node_tokens, const int32_t* parents,
+                       const float* u, int B, int n, int V, double T, int max_depth,
+                       int32_t* accepted_len, int32_t* out_tokens, int32_t* accepted_nodes,
+                       double* test_margin, double* cdf_margin, int32_t* fallback,
+                       int32_t* n_tests, int nthreads) {
+  if (B < 0 || n < 1 || V < 1 || max_depth < 0 || !(T > 0.0) || !target || !draft ||
+      !node_tokens || !parents || !u || !accepted_len || !out_tokens || !accepted_nodes)
+    return OR_BAD_ARG;
+  for (int b = 0; b < B; ++b) {
+    const int32_t* par = parents + (size_t)b * n;
+    if (par[0] != -1) return OR_BAD_TREE;
+    int* depth = (int*)malloc(sizeof(int) * (size_t)n);
+    if (!depth) return OR_NOMEM;
+    depth[0] = 0;
+    int ok = 1;
+    for (int j = 1; j < n && ok; ++j) {
+      if (par[j] < 0 || par[j] >= j) ok = 0;
+      else {
+        depth[j] = depth[par[j]] + 1;
+        if (depth[j] > max_depth) ok = 0;
+      }
+      if (node_tokens[(size_t)b * n + j] < 0 || node_tokens[(size_t)b * n + j] >= V) ok = 0;
+    }
+    free(depth);
+    if (!ok) return OR_BAD_TREE;
+  }
+  set_threads(nthreads);
+  const int W = max_depth + 1;
+  int err = OR_OK;
+#pragma omp parallel
+  {
+    double* p = (double*)malloc(sizeof(double) * (size_t)V);
+    double* q = (double*)malloc(sizeof(double) * (size_t)V);
+    double* r = (double*)malloc(sizeof(double) * (size_t)V);
+    if (!p || !q || !r) {
+#pragma omp atomic write
+      err = OR_NOMEM;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+      if (!p || !q || !r) continue;
+      const int32_t* par = parents + (size_t)b * n;
+      const int32_t* tok = node_tokens + (size_t)b * n;
+      const float* ub = u + (size_t)b * n;
+      int32_t* on = accepted_nodes + (size_t)b * W;
+      int32_t* ot = out_tokens + (size_t)b * W;
+      for (int d = 0; d < W; ++d) on[d] = ot[d] = -1;
+      double tm = INFINITY, mg = INFINITY;
+      int fb = 0, tests = 0, depth = 0, v = 0, emit = -1, bad = 0;
+      on[0] = 0;
+      for (;;) {
+        const size_t row = ((size_t)b * n + v) * (size_t)V;
+        if (isnan(softmax_row(target, t_dtype, row, V, T, p))) {
+          bad = 1;
+          break;
+        }
+        if (d_kind == OR_DRAFT_LOGITS) {
+          if (isnan(softmax_row(draft, d_dtype, row, V, T, q))) {
+            bad = 1;
+            break;
+          }
+        } else {
+          for (int j = 0; j < V; ++j) q[j] = load_value(draft, d_dtype, row + (size_t)j);
+        }
+        memcpy(r, p, sizeof(double) * (size_t)V);
+        int next = -1;
+        for (int c = v + 1; c < n; ++c) {
+          if (par[c] != v) continue;
+          const int x = tok[c];
+          const double uc = (double)ub[c];
+          ++tests;
+#if OR_PLANT == 4
+          const double rx = p[x]; /* planted mistake: siblings tested against p, not the residual */
+#else
+          const double rx = r[x];
+#endif
+          if (q[x] > 0.0) {
+            const double gap = fabs(uc - rx / q[x]);
+            if (gap < tm) tm = gap;
+          }
+          if (uc * q[x] < rx) { /* accept with probability min(1, r(x) / q(x)) */
+            next = c;
+            break;
+          }
+          double s = 0.0;
+          for (int j = 0; j < V; ++j) {
+            const double d = r[j] - q[j];
+            r[j] = d > 0.0 ? d : 0.0;
+            s += r[j];
+          }
+          if (!(s > 0.0)) { /* zero residual mass: draw from the target row */
+            memcpy(r, p, sizeof(double) * (size_t)V);
+            fb = 1;
+            break;
+          }
+          for (int j = 0; j < V; ++j) r[j] /= s;
+        }
+        if (next >= 0) {
+          ++depth;
+          on[depth] = next;
+          ot[depth - 1] = tok[next];
+          v = next;
+          continue;
+        }
+        emit = inverse_cdf(r, V, (double)ub[0], &mg);
+        break;
+      }
+      if (bad || emit < 0) {
+        for (int d = 0; d < W; ++d) on[d] = ot[d] = -1;
+        accepted_len[b] = -1;
+#pragma omp atomic write
+        err = OR_NO_FINITE;
+      } else {
+        ot[depth] = emit;
+        accepted_len[b] = depth;
+      }
+      if (test_margin) test_margin[b] = tm;
+      if (cdf_margin) cdf_margin[b] = mg;
+      if (fallback) fallback[b] = fb;
+      if (n_tests) n_tests[b] = tests;
+    }
+    free(p);
+    free(q);
+    free(r);
   }
   return err;
 }

@@ -568,3 +568,137 @@ def test_ragged_kd_mask_and_inactive_requests(oracle):
     assert np.allclose(r["loss"], want, rtol=1e-14, atol=0)
     with pytest.raises(oracle.OracleError):
         oracle.reward_loss(kl, np.array([3, 0, 0, 0, 0, 0], np.int32), rw, draft_len=klen * 0 + 2)
+
+
+# --------------------------------------------------------------------------
+# Sampling tree verification (multi-step speculative sampling, SpecInfer).
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("draft_kind", ["logits", "probs"])
+def test_tree_sample_single_path_equals_chain(oracle, draft_kind):
+    """A tree that is one path of k children is chain verification: the same
+    ratio tests, the residual at the first rejection, the bonus at the leaf
+    (node j+1 tests with the chain's u_j, the final draw takes u_k)."""
+    B, k, V, T = 60, 4, 300, 0.8
+    x = inputs.make_chain(B, k, V, dtype="bf16", temperature=T, sigma_d=0.6, seed=17)
+    draft = x.draft
+    kind = oracle.DRAFT_LOGITS
+    if draft_kind == "probs":
+        draft = torch.softmax(x.draft.float() / float(np.float32(T)), -1)
+        kind = oracle.DRAFT_PROBS
+    chain = oracle.verify_chain(x.target, draft, x.draft_tokens, x.uniforms, T, draft_kind=kind)
+    n = k + 1
+    par = np.tile(np.arange(-1, k, dtype=np.int32), (B, 1))
+    tok = np.zeros((B, n), np.int32)
+    tok[:, 1:] = x.draft_tokens.numpy()
+    leaf = draft[:, k - 1:k]  # the leaf's draft row is never used for a test
+    tdraft = torch.cat([draft, leaf], dim=1).contiguous()
+    u = np.zeros((B, n), np.float32)
+    u[:, 1:] = x.uniforms.numpy()[:, :k]
+    u[:, 0] = x.uniforms.numpy()[:, k]
+    tr = oracle.tree_sample(x.target, tdraft, tok, par, u, T, k, draft_kind=kind)
+    assert np.array_equal(tr["accepted_len"], chain["accepted_len"])
+    assert np.array_equal(tr["out_tokens"], chain["out_tokens"])
+    for b in range(B):
+        a = tr["accepted_len"][b]
+        assert list(tr["accepted_nodes"][b, :a + 1]) == list(range(a + 1))
+    assert len(set(chain["accepted_len"].tolist())) > 2
+
+
+def _tree_mc(oracle, plant=0, B=200_000, V=5, m1=3, m2=2, seed=23):
+    """Depth-2 trees whose rows depend only on the path's tokens: the root's
+    m1 children and each depth-1 node's m2 children are drawn independently
+    from the draft row of their parent's context."""
+    rng = np.random.default_rng(seed)
+    p0 = rng.dirichlet(np.full(V, 0.8))
+    p1 = rng.dirichlet(np.full(V, 0.8), size=V)
+    p2 = rng.dirichlet(np.full(V, 0.8), size=(V, V))
+    q0 = rng.dirichlet(np.full(V, 0.8))
+    q1 = rng.dirichlet(np.full(V, 0.8), size=V)
+    n = 1 + m1 + m1 * m2
+    par = np.full((B, n), -1, np.int32)
+    par[:, 1:1 + m1] = 0
+    for i in range(m1):
+        par[:, 1 + m1 + i * m2:1 + m1 + (i + 1) * m2] = 1 + i
+    tok = np.zeros((B, n), np.int32)
+    tok[:, 1:1 + m1] = rng.choice(V, size=(B, m1), p=q0)
+    cum1 = np.cumsum(q1, axis=1)
+    for i in range(m1):
+        t1 = tok[:, 1 + i]
+        draws = (rng.random((B, m2))[:, :, None] > cum1[t1][:, None, :]).sum(-1)
+        tok[:, 1 + m1 + i * m2:1 + m1 + (i + 1) * m2] = np.minimum(draws, V - 1)
+    logp = np.zeros((B, n, V), np.float32)
+    qd = np.zeros((B, n, V), np.float32)
+    logp[:, 0] = np.log(p0)
+    qd[:, 0] = q0
+    for i in range(m1):
+        t1 = tok[:, 1 + i]
+        logp[:, 1 + i] = np.log(p1[t1])
+        qd[:, 1 + i] = q1[t1]
+        for j in range(m2):
+            c = 1 + m1 + i * m2 + j
+            logp[:, c] = np.log(p2[t1, tok[:, c]])
+            qd[:, c] = q0  # a leaf's draft row is never used for a test
+    u = inputs.uniforms24(np.random.default_rng(seed + 1), (B, n))
+    r = oracle.tree_sample(torch.from_numpy(logp), torch.from_numpy(qd), tok, par, u, 1.0, 2,
+                           draft_kind=oracle.DRAFT_PROBS, plant=plant)
+    # the target rows as stored (fp32 log-probabilities, renormalised at T = 1)
+    def sm(z):
+        z = z.astype(np.float64)
+        e = np.exp(z - z.max(-1, keepdims=True))
+        return e / e.sum(-1, keepdims=True)
+    return r, sm(np.log(p0).astype(np.float32)), sm(np.log(p1).astype(np.float32)), \
+        sm(np.log(p2).astype(np.float32)), q0.astype(np.float32).astype(np.float64)
+
+
+def _tree_pvalues(r, P0, P1, P2, min_count=400):
+    acc, out = r["accepted_len"], r["out_tokens"]
+    V = P0.shape[0]
+    pv = [scipy.stats.chisquare(np.bincount(out[:, 0], minlength=V), P0 * len(acc)).pvalue]
+    for t in range(V):
+        sel = (acc >= 1) & (out[:, 0] == t)
+        if sel.sum() >= min_count:
+            pv.append(scipy.stats.chisquare(np.bincount(out[sel, 1], minlength=V),
+                                            P1[t] * sel.sum()).pvalue)
+        for t2 in range(V):
+            sel2 = sel & (acc >= 2) & (out[:, 1] == t2)
+            if sel2.sum() >= min_count:
+                pv.append(scipy.stats.chisquare(np.bincount(out[sel2, 2], minlength=V),
+                                                P2[t, t2] * sel2.sum()).pvalue)
+    return pv
+
+
+def test_tree_sample_is_lossless(oracle):
+    """Every emitted token follows the target row of its context (SpecInfer's
+    theorem for multi-step speculative sampling), at all three positions; the
+    root rejects all m children with probability prod_i (1 - sum_x min(q, r_i)),
+    r_0 = p and r_{i+1} the normalised max(0, r_i - q)."""
+    r, P0, P1, P2, q0 = _tree_mc(oracle)
+    pv = _tree_pvalues(r, P0, P1, P2)
+    assert len(pv) > 10
+    assert min(pv) > 1e-4, pv
+    rr, none = P0.copy(), 1.0
+    for _ in range(3):
+        none *= 1.0 - np.minimum(q0, rr).sum()
+        rr = np.maximum(rr - q0, 0.0)
+        rr /= rr.sum()
+    got = (r["accepted_len"] == 0).mean()
+    sd = math.sqrt(none * (1 - none) / len(r["accepted_len"]))
+    assert abs(got - none) < 4 * sd, (got, none)
+    assert (r["fallback"] == 0).all()
+
+
+def test_tree_sample_planted_sibling_mistake_is_caught(oracle):
+    """Testing every sibling against p instead of the running residual (plant
+    4) over-accepts drafted tokens and must fail the losslessness pin."""
+    oracle.build(plant=4)
+    r, P0, P1, P2, _ = _tree_mc(oracle, plant=4)
+    assert min(_tree_pvalues(r, P0, P1, P2)) < 1e-6
+
+
+def test_tree_sample_rejects_malformed_trees(oracle):
+    z = torch.zeros(1, 3, 4)
+    tok = np.array([[0, 1, 2]], np.int32)
+    u = np.full((1, 3), 0.5, np.float32)
+    for par, depth in (([[-1, 0, 2]], 2), ([[0, 0, 1]], 2), ([[-1, 0, 1]], 1)):
+        with pytest.raises(oracle.OracleError):
+            oracle.tree_sample(z, z, tok, np.array(par, np.int32), u, 1.0, depth)
