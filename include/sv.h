@@ -260,6 +260,53 @@ SV_API sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const in
                                 int32_t* device_status, void* stream);
 
 /*
+ * sv_verify_tree_sample -- sampling (T > 0) verification of B candidate
+ * trees.  The reading notes (section 3) name the EAGLE trees but no sampling
+ * rule; the rule is the multi-step speculative sampling of SpecInfer (Miao et
+ * al., "SpecInfer: Accelerating Large Language Model Serving with Tree-based
+ * Speculative Inference and Verification"), the recursive rejection sampling
+ * EAGLE adopts.
+ *
+ * Operation: from the root, at node v (p_v = softmax(target[b, v, :] / T),
+ *   q_v = softmax(draft[b, v, :] / T) or the given probabilities), r = p_v;
+ *   the children of v are tried in ascending node order: child c with token
+ *   x is accepted iff uniforms[b, c] * q_v(x) < r(x) (probability
+ *   min(1, r(x)/q_v(x))), and the walk moves to c; otherwise r becomes
+ *   max(0, r - q_v) normalised and the next child is tried.  A node with no
+ *   accepted child (or none at all) draws one token from r by inverse CDF in
+ *   ascending vocabulary order with uniforms[b, 0].  A zero residual mass
+ *   (probability zero when children are drawn from q_v) draws from p_v and
+ *   sets SV_DEV_RESIDUAL_ZERO.  The emitted tokens follow the target's
+ *   distribution when the children of every node are drawn independently
+ *   from its draft row.
+ *
+ * Arguments
+ *   target_logits [B, n, V] (t_dtype): row j is the target distribution after
+ *                 node j.
+ *   draft         [B, n, V]: row j is the draft distribution node j's children
+ *                 were drawn from: logits (d_dtype), or fp32 probabilities.
+ *                 Rows of leaves are read only when the walk reaches them.
+ *   node_tokens, parents, max_depth as in sv_verify_tree_greedy.
+ *   uniforms      [B, n] fp32 in [0, 1): column j >= 1 tests node j, column 0
+ *                 drives the final draw.
+ *   T > 0.  1 <= n <= 1024, 0 <= max_depth < n, 1 <= V <= 524288.
+ *   accepted_len, accepted_nodes, out_tokens as in sv_verify_tree_greedy
+ *   (the token after the path is the drawn one).  Invalid trees or tokens set
+ *   SV_DEV_BAD_TREE / SV_DEV_BAD_TOKEN, a row without a finite value
+ *   SV_DEV_NO_FINITE; the request then has accepted_len -1 and -1 outputs.
+ *   No workspace: each request's rows are read by one thread-block cluster,
+ *   and only the rows of the nodes the walk visits.
+ */
+SV_API sv_status sv_verify_tree_sample(const void* target_logits, sv_dtype t_dtype,
+                                       const void* draft, sv_dtype d_dtype,
+                                       sv_draft_kind d_kind, const int32_t* node_tokens,
+                                       const int32_t* parents, const float* uniforms, int B,
+                                       int n, int V, int max_depth, float temperature,
+                                       int32_t* accepted_len, int32_t* out_tokens,
+                                       int32_t* accepted_nodes, int32_t* device_status,
+                                       void* stream);
+
+/*
  * sv_extract_topk_kd -- the distillation buffer of the reading notes,
  * section 4: for each of `rows` rows of V logits, the K largest logits
  * (value desc, index asc) as full-vocabulary log-probs at temperature T.

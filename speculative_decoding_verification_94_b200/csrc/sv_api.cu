@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "sv_finish.cuh"
+#include "sv_tree_sample.cuh"
 
 namespace sv {
 
@@ -711,6 +712,87 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   const int tsm = kFixedBytes + n * (int)sizeof(RowRec) + 4 * n * 4;
   return cuda_status(dt == SV_BF16 ? launch_blocks(tree_finish<BF16>, fp, B, tsm, s)
                                    : launch_blocks(tree_finish<F32>, fp, B, tsm, s));
+}
+
+}  // extern "C"
+
+template <class TT, class DT, int DKIND>
+static cudaError_t run_tree_sample(FinishParams fp, int te, int de, bool bulk_ok, cudaStream_t s) {
+  RowPlan plans[kMaxCluster];
+  const int rows_bytes = (int)sizeof(TreeShared) + 4 * fp.k * (int)sizeof(int);
+  const int np = feasible_plans(
+      fp.V, te, de,
+      [](int, int npc) {
+        const int x = npc * kThreads * 4 + kThreads * 8;
+        return x < 2 * kThreads * 4 ? 2 * kThreads * 4 : x;
+      },
+      bulk_ok, rows_bytes, plans);
+  if (np == 0) return cudaErrorInvalidConfiguration;
+  auto kern = tree_sample_kernel<TT, DT, DKIND>;
+  RowPlan plan;
+  cudaError_t e = pick_plan(kern, plans, np, fp.B, &plan);
+  if (e != cudaSuccess) return e;
+  fp.L = plan.L;
+  fp.use_bulk = plan.use_bulk;
+  fp.lay = plan.lay;
+  return launch_clusters(kern, fp, plan, fp.B, s);
+}
+
+extern "C" {
+
+sv_status sv_verify_tree_sample(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                                sv_dtype d_dtype, sv_draft_kind d_kind, const int32_t* node_tokens,
+                                const int32_t* parents, const float* uniforms, int B, int n, int V,
+                                int max_depth, float temperature, int32_t* accepted_len,
+                                int32_t* out_tokens, int32_t* accepted_nodes,
+                                int32_t* device_status, void* stream) {
+  if (B < 0 || n < 1 || n > 1024 || V < 1 || max_depth < 0 || max_depth >= n)
+    return SV_ERR_INVALID_ARG;
+  if (!dtype_ok(t_dtype) || !dtype_ok(d_dtype)) return SV_ERR_INVALID_ARG;
+  if (d_kind != SV_DRAFT_LOGITS && d_kind != SV_DRAFT_PROBS) return SV_ERR_INVALID_ARG;
+  if (d_kind == SV_DRAFT_PROBS && d_dtype != SV_F32) return SV_ERR_INVALID_ARG;
+  if (!scale_ok(temperature)) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
+  if (!target_logits || !draft || !node_tokens || !parents || !uniforms || !accepted_len ||
+      !out_tokens || !accepted_nodes)
+    return SV_ERR_INVALID_ARG;
+  const int te = esize(t_dtype), de = esize(d_dtype);
+  if (!aligned(target_logits, te) || !aligned(draft, de) || !aligned(node_tokens, 4) ||
+      !aligned(parents, 4) || !aligned(uniforms, 4) || !aligned(accepted_len, 4) ||
+      !aligned(out_tokens, 4) || !aligned(accepted_nodes, 4))
+    return SV_ERR_INVALID_ARG;
+  if (device_status && !aligned(device_status, 4)) return SV_ERR_INVALID_ARG;
+  if (V > kMaxV) return SV_ERR_UNSUPPORTED;
+  if ((long long)B * kMaxCluster > 0x7fffffffLL) return SV_ERR_UNSUPPORTED;
+  FinishParams fp = {};
+  fp.target = target_logits;
+  fp.draft = draft;
+  fp.tokens = node_tokens;
+  fp.parents = parents;
+  fp.u = uniforms;
+  fp.B = B;
+  fp.k = n;
+  fp.V = V;
+  fp.max_depth = max_depth;
+  fp.c = (float)(1.4426950408889634 / (double)temperature);
+  fp.accepted_len = accepted_len;
+  fp.out_tokens = out_tokens;
+  fp.accepted_nodes = accepted_nodes;
+  fp.status = device_status;
+  const bool bulk = bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d_kind == SV_DRAFT_PROBS)
+    e = t_dtype == SV_BF16 ? run_tree_sample<BF16, F32, kDraftProbs>(fp, te, de, bulk, s)
+                           : run_tree_sample<F32, F32, kDraftProbs>(fp, te, de, bulk, s);
+  else if (t_dtype == SV_BF16)
+    e = d_dtype == SV_BF16 ? run_tree_sample<BF16, BF16, kDraftLogits>(fp, te, de, bulk, s)
+                           : run_tree_sample<BF16, F32, kDraftLogits>(fp, te, de, bulk, s);
+  else
+    e = d_dtype == SV_BF16 ? run_tree_sample<F32, BF16, kDraftLogits>(fp, te, de, bulk, s)
+                           : run_tree_sample<F32, F32, kDraftLogits>(fp, te, de, bulk, s);
+  if (e == cudaErrorInvalidConfiguration) return SV_ERR_UNSUPPORTED;
+  return cuda_status(e);
 }
 
 sv_status sv_extract_topk_kd(const void* logits, sv_dtype dt, int rows, int V, int K,

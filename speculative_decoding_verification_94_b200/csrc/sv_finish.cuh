@@ -11,6 +11,8 @@
 // the reward-weighted losses.  Every finisher returns the row records it read
 // to zero (the stream zeroes the partials), so the workspace stays zero
 // between calls.
+#pragma once
+
 #include "sv_rowops.cuh"
 #include "sv_stream.cuh"
 

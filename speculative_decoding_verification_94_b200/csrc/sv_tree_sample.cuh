@@ -1,0 +1,408 @@
+// sv_tree_sample.cuh -- sampling verification of candidate trees.
+//
+// The rule is the multi-step speculative sampling of SpecInfer (Miao et al.,
+// "SpecInfer: Accelerating Large Language Model Serving with Tree-based
+// Speculative Inference and Verification"), the recursive rejection sampling
+// that EAGLE adopts; the ReSpec reading notes (section 3, "G1 解法") name the
+// EAGLE trees (depth s, top-t branching, n nodes) it runs on.  From the root,
+// at node v with target row p_v and draft row q_v, r = p_v and the children of
+// v are tried in ascending index order: child c with token x is accepted iff
+// u_c * q_v(x) < r(x); on a rejection r becomes max(0, r - q_v) normalised.
+// The walk moves to the first accepted child; a node whose children are all
+// rejected (or a leaf) draws one token from r.
+//
+// Residual form used here: after i rejections r is proportional to
+// max(0, p - sigma_i q) with sigma_0 = 0 and sigma_{i+1} = sigma_i + M_i, where
+// M_i = sum_j max(0, p_j - sigma_i q_j) (M_0 = 1).  So the test of the next
+// child is u * q(x) * M_i < max(0, p(x) - sigma_i q(x)), and only a rejection
+// costs a pass over the row pair.
+//
+// One cluster of C CTAs per request.  Each visited node's row pair is staged
+// into the cluster's shared memory (CTA q holds vocabulary chunk q), the
+// rows' log-partitions and every residual mass are combined across the
+// cluster in rank order through distributed shared memory, so every CTA takes
+// the same decisions; the CTA that owns the drawn token writes the outputs.
+// Nothing is read for nodes off the accepted path.
+#pragma once
+
+#include "sv_finish.cuh"
+
+namespace sv {
+
+// Per-CTA values of one cluster combine.  Two slots, used alternately: a CTA
+// writes slot s again only after every CTA has passed the barrier that ended
+// the previous read of s.
+struct TreePart {
+  float Gt, Gd;
+  double St, Sd;
+  double R;  // chunk mass of the current weights
+  int timeouts;
+  int pad;
+};
+
+struct TreeShared {
+  TreePart part[2];
+  double Lt, Ld;     // log2-partitions of the staged rows
+  double M, lo, hi;  // residual mass of the cluster, this CTA's share [lo, hi)
+  double tt;         // the draw's target in [0, M)
+  int nkids, err, owner, tok, piece, first_thread, last_pos, pad;
+};
+
+template <class TT, class DT, int DKIND>
+__device__ __forceinline__ void tree_weights8(const unsigned char* tbuf, const unsigned char* dbuf,
+                                              int e, float c, float Gt, float invSt, float Gd,
+                                              float invSd, float sg, float w[8]) {
+  float zt[8];
+  load8<TT>(tbuf, e, zt);
+  float q[8];
+  if (DKIND == kDraftLogits) {
+    float zd[8];
+    load8<DT>(dbuf, e, zd);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) q[t] = __fmul_rn(ex2(fmaf(zd[t], c, -Gd)), invSd);
+  } else {
+    load8<F32>(dbuf, e, q);
+  }
+  // p - sigma q with one rounding: exactly p at sigma = 0, and exactly 0 where
+  // p == q at sigma = 1
+#pragma unroll
+  for (int t = 0; t < 8; ++t)
+    w[t] = fmaxf(__fmaf_rn(-sg, q[t], __fmul_rn(ex2(fmaf(zt[t], c, -Gt)), invSt)), 0.f);
+}
+
+// Sampling tree verification: one cluster of C CTAs per request.
+template <class TT, class DT, int DKIND>
+__global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_constant__ FinishParams prm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  RowShared& sh = *reinterpret_cast<RowShared*>(smem);
+  TreeShared& ts = *reinterpret_cast<TreeShared*>(smem + prm.lay.off_rows);
+  const int n = prm.k, V = prm.V, W = prm.max_depth + 1;
+  int* par = reinterpret_cast<int*>(&ts + 1);
+  int* tok = par + n;
+  int* kids = tok + n;
+  int* pth = kids + n;
+  unsigned char* tbuf = smem + prm.lay.off_t;
+  unsigned char* dbuf = smem + prm.lay.off_d;
+  const int b = (int)(blockIdx.x / (unsigned)C);
+  const ChunkGeom g = chunk_geom(rank, prm.L, V);
+  float* sums = reinterpret_cast<float*>(smem + prm.lay.off_x);
+  double* incl_arr = reinterpret_cast<double*>(sums + g.npieces * kThreads);
+  const float c = prm.c;
+  const bool use_bulk = prm.use_bulk != 0;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  pdl_wait();
+
+  // 0. the tree, checked the same way in every CTA
+  int bad_tree = 0, bad_tok = 0;
+  for (int t = threadIdx.x; t < n; t += kThreads) {
+    const int pj = prm.parents[(size_t)b * n + t];
+    const int x = prm.tokens[(size_t)b * n + t];
+    par[t] = pj;
+    tok[t] = x;
+    if (t == 0 ? pj != -1 : (pj < 0 || pj >= t)) bad_tree = 1;
+    if (t > 0 && (x < 0 || x >= V)) bad_tok = 1;
+  }
+  bad_tree = __syncthreads_or(bad_tree);
+  if (!bad_tree) {
+    // depth of every node <= max_depth (parents precede children, so every
+    // walk up ends at the root; it stops early once too deep)
+    for (int t = threadIdx.x; t < n; t += kThreads) {
+      int j = t, d = 0;
+      while (j > 0 && d <= prm.max_depth) {
+        j = par[j];
+        ++d;
+      }
+      if (d > prm.max_depth) bad_tree = 1;
+    }
+  }
+  bad_tree = __syncthreads_or(bad_tree);
+  bad_tok = __syncthreads_or(bad_tok);
+  if (bad_tree || bad_tok) {
+    if (rank == 0) {
+      if (threadIdx.x == 0) {
+        set_status(prm.status, bad_tree ? SV_DEV_BAD_TREE : SV_DEV_BAD_TOKEN);
+        prm.accepted_len[b] = -1;
+      }
+      for (int d = threadIdx.x; d < W; d += kThreads) {
+        prm.out_tokens[(size_t)b * W + d] = -1;
+        prm.accepted_nodes[(size_t)b * W + d] = -1;
+      }
+    }
+    return;  // no CTA has touched another's shared memory
+  }
+  if (threadIdx.x == 0) {
+    init_piece_barriers(sh, g, use_bulk);
+    pth[0] = 0;
+  }
+  __syncthreads();
+
+  int red = 0;  // cluster combines so far (selects the slot)
+  // Chunk masses of the weights max(0, p - sg q) into sums[] and ts.part,
+  // then the cluster total M and this CTA's share [lo, hi).  Collective over
+  // the cluster.
+  auto residual_pass = [&](float sg, float Gt, float invSt, float Gd, float invSd) {
+    for (int p = 0; p < g.npieces; ++p) {
+      const int e = p * kRound + (int)threadIdx.x * kVec;
+      float s = 0.f;
+      if (e < g.nvec * kVec) {
+        float wv[8];
+        tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c, Gt, invSt, Gd, invSd, sg, wv);
+        s = seq_sum8(wv);
+      }
+      sums[p * kThreads + threadIdx.x] = s;
+    }
+    piece_totals(sums, g.npieces, sh);
+    const int slot = red & 1;
+    ++red;
+    if (threadIdx.x == 0) {
+      double Rc = 0.0;
+      for (int p = 0; p < g.npieces; ++p) Rc += sh.ptot[p];
+      ts.part[slot].R = Rc;
+    }
+    cluster.sync();
+    if (w == 0) {
+      const double Rq = lane < C ? cluster.map_shared_rank(&ts.part[slot], lane)->R : 0.0;
+      const double incl = warp_scan_incl(Rq);
+      const double tot = __shfl_sync(0xffffffffu, incl, 31);
+      const double lo = __shfl_sync(0xffffffffu, incl, rank > 0 ? rank - 1 : 0);
+      const double hi = __shfl_sync(0xffffffffu, incl, rank);
+      if (lane == 0) {
+        ts.M = tot;
+        ts.lo = rank > 0 ? lo : 0.0;
+        ts.hi = hi;
+      }
+    }
+    __syncthreads();
+  };
+
+  int v = 0, depth = 0, visit = 0, err = 0;
+  bool drawn = false;
+  for (;;) {
+    // a. stage the row pair of node v
+    const size_t row = (size_t)b * n + v;
+    const void* trow = row_ptr<TT>(prm.target, row, V);
+    const void* drow = row_ptr<DT>(prm.draft, row, V);
+    if (threadIdx.x == 0) {
+      sh.timeouts = 0;
+      if (use_bulk) {
+        fence_proxy_async_smem();  // earlier reads of the buffers precede the copies
+        issue_item_copies<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, policy_evict_first());
+      }
+    }
+    scalar_fill<TT>(tbuf, trow, g, use_bulk, false);
+    scalar_fill<DT>(dbuf, drow, g, use_bulk, DKIND == kDraftProbs);
+    __syncthreads();
+    for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, use_bulk, (uint32_t)(visit & 1));
+    __syncthreads();
+
+    // b. the rows' statistics, combined over the cluster
+    ThreadStat a, d;
+    stat_init(a);
+    stat_init(d);
+    for (int p = 0; p < g.npieces; ++p) {
+      const int e = p * kRound + (int)threadIdx.x * kVec;
+      if (e < g.nvec * kVec) {
+        float z[8];
+        const float mt = load8_max<TT>(tbuf, e, z);
+        stat_update(a, z, mt, c);
+        if (DKIND == kDraftLogits) {
+          const float md = load8_max<DT>(dbuf, e, z);
+          stat_update(d, z, md, c);
+        }
+      }
+    }
+    CtaStat ca, cd;
+    stat_block2(a, d, sh.redf2, sh.redd2, &ca, &cd);
+    {
+      const int slot = red & 1;
+      ++red;
+      if (threadIdx.x == 0) {
+        ts.part[slot].Gt = ca.G;
+        ts.part[slot].St = ca.S;
+        ts.part[slot].Gd = cd.G;
+        ts.part[slot].Sd = cd.S;
+        ts.part[slot].timeouts = sh.timeouts;
+      }
+      cluster.sync();
+      if (w == 0) {
+        const TreePart* q = cluster.map_shared_rank(&ts.part[slot], lane < C ? lane : 0);
+        float Gt, Gd;
+        double St, Sd;
+        warp_stat_combine(lane < C ? q->Gt : -INFINITY, lane < C ? q->St : 0.0, &Gt, &St);
+        warp_stat_combine(lane < C ? q->Gd : -INFINITY, lane < C ? q->Sd : 0.0, &Gd, &Sd);
+        const int tmo = warp_sum_int(lane < C ? q->timeouts : 0);
+        if (lane == 0) {
+          sh.Gt = Gt;
+          sh.St = St;
+          sh.Gd = Gd;
+          sh.Sd = Sd;
+          ts.Lt = (double)Gt + log2(St);
+          ts.Ld = (double)Gd + log2(Sd);
+          ts.err = tmo ? SV_DEV_TIMEOUT
+                       : ((Gt == -INFINITY || (DKIND == kDraftLogits && Gd == -INFINITY))
+                              ? SV_DEV_NO_FINITE
+                              : 0);
+        }
+      } else if (w == 1) {
+        // the children of v in ascending order
+        int m = 0;
+        for (int base = v + 1; base < n; base += 32) {
+          const int j = base + lane;
+          const bool is = j < n && par[j] == v;
+          const unsigned bal = __ballot_sync(0xffffffffu, is);
+          if (is) kids[m + __popc(bal & ((1u << lane) - 1u))] = j;
+          m += __popc(bal);
+        }
+        if (lane == 0) ts.nkids = m;
+      }
+      __syncthreads();
+    }
+    if (ts.err) {
+      err = ts.err;
+      break;
+    }
+
+    // c. the children's tests against the running residual
+    const float Gt = sh.Gt, Gd = sh.Gd;
+    const float invSt = (float)(1.0 / sh.St);
+    const float invSd = DKIND == kDraftLogits ? (float)(1.0 / sh.Sd) : 1.f;
+    const double Lt = ts.Lt, Ld = ts.Ld, cd64 = (double)c;
+    double sigma = 0.0, M = 1.0;
+    bool have = false, fallback = false;
+    int next = -1;
+    for (int i = 0; i < ts.nkids; ++i) {
+      const int node = kids[i];
+      const int x = tok[node];
+      const double px = exp2((double)load1<TT>(reinterpret_cast<const unsigned char*>(trow), x) * cd64 - Lt);
+      const double qx =
+          DKIND == kDraftLogits
+              ? exp2((double)load1<DT>(reinterpret_cast<const unsigned char*>(drow), x) * cd64 - Ld)
+              : (double)load1<F32>(reinterpret_cast<const unsigned char*>(drow), x);
+      const double rx = fmax(px - sigma * qx, 0.0);
+      const double uc = (double)prm.u[(size_t)b * n + node];
+      if (uc * qx * M < rx) {  // accepted with probability min(1, r(x) / q(x))
+        next = node;
+        break;
+      }
+      sigma += M;
+      residual_pass((float)sigma, Gt, invSt, Gd, invSd);
+      M = ts.M;
+      have = true;
+      if (!(M > 0.0)) {  // zero residual mass: draw from the target row
+        fallback = true;
+        break;
+      }
+    }
+    if (next >= 0) {
+      ++depth;
+      if (threadIdx.x == 0) pth[depth] = next;
+      v = next;
+      ++visit;
+      continue;  // (depth <= max_depth: checked above)
+    }
+
+    // d. the draw from max(0, p - sigma q) (p itself at sigma = 0)
+    if (fallback) {
+      if (rank == 0 && threadIdx.x == 0) set_status(prm.status, SV_DEV_RESIDUAL_ZERO);
+      sigma = 0.0;
+      have = false;
+    }
+    if (!have) residual_pass((float)sigma, Gt, invSt, Gd, invSd);
+    if (threadIdx.x == 0) {
+      ts.tt = (double)prm.u[(size_t)b * n] * ts.M;
+      ts.owner = (ts.M > 0.0 && ts.lo <= ts.tt && ts.tt < ts.hi) ? 1 : 0;
+      ts.tok = -1;
+      if (!(ts.M > 0.0)) ts.err = SV_DEV_NO_FINITE;
+    }
+    __syncthreads();
+    err = ts.err;
+    if (ts.owner) {
+      if (threadIdx.x == 0) {
+        double base = ts.lo;
+        int pp = -1;
+        for (int p = 0; p < g.npieces; ++p) {
+          if (base + sh.ptot[p] > ts.tt) {
+            pp = p;
+            break;
+          }
+          base += sh.ptot[p];
+        }
+        if (pp < 0) {  // rounding pushed the target past this chunk: last piece with mass
+          double b2 = ts.lo;
+          base = ts.lo;
+          for (int p = 0; p < g.npieces; ++p) {
+            if (sh.ptot[p] > 0.0) {
+              pp = p;
+              base = b2;
+            }
+            b2 += sh.ptot[p];
+          }
+        }
+        ts.piece = pp;
+        ts.lo = base;
+        ts.first_thread = kThreads;
+        ts.last_pos = -1;
+      }
+      __syncthreads();
+      const int pp = ts.piece;
+      if (pp >= 0) {
+        const float s = sums[pp * kThreads + threadIdx.x];
+        double tot;
+        const double incl = block_scan_incl((double)s, sh.redd, &tot);
+        incl_arr[threadIdx.x] = incl;
+        if (ts.lo + incl > ts.tt) atomicMin(&ts.first_thread, (int)threadIdx.x);
+        if (s > 0.f) atomicMax(&ts.last_pos, (int)threadIdx.x);
+        __syncthreads();
+        int tsel = ts.first_thread;
+        const bool fb = (tsel == kThreads);
+        if (fb) tsel = ts.last_pos;
+        if ((int)threadIdx.x == tsel) {
+          const int e = pp * kRound + tsel * kVec;
+          float wv[8];
+          tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c, Gt, invSt, Gd, invSd, (float)sigma, wv);
+          const double b0 = ts.lo + (tsel > 0 ? incl_arr[tsel - 1] : 0.0);
+          float acc = 0.f;
+          int pick = -1, lastq = -1;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            acc = __fadd_rn(acc, wv[q]);
+            if (wv[q] > 0.f) lastq = q;
+            if (!fb && pick < 0 && b0 + (double)acc > ts.tt) pick = q;
+          }
+          if (pick < 0) pick = lastq;
+          ts.tok = pick < 0 ? -1 : g.j0 + e + pick;
+        }
+        __syncthreads();
+      }
+      drawn = true;
+    }
+    break;
+  }
+
+  // 4. outputs, by the owner of the drawn token (the first CTA on an error)
+  const bool writer = err ? rank == 0 : drawn;
+  if (writer) {
+    const int tk = err ? -1 : ts.tok;
+    const bool ok = !err && tk >= 0 && tk < V;
+    if (threadIdx.x == 0) {
+      if (err) set_status(prm.status, err);
+      prm.accepted_len[b] = ok ? depth : -1;
+    }
+    for (int d = threadIdx.x; d < W; d += kThreads) {
+      int on = -1, ot = -1;
+      if (ok && d <= depth) {
+        on = pth[d];
+        ot = d < depth ? tok[pth[d + 1]] : tk;
+      }
+      prm.accepted_nodes[(size_t)b * W + d] = on;
+      prm.out_tokens[(size_t)b * W + d] = ot;
+    }
+  }
+  drain_pieces(sh, g, use_bulk, (uint32_t)(visit & 1));
+  cluster.sync();  // no CTA leaves while another may still read its shared memory
+}
+
+}  // namespace sv

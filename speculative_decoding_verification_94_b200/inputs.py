@@ -161,6 +161,86 @@ class TreeInputs:
     meta: dict = field(default_factory=dict)
 
 
+def _tree_shape(brng: np.random.Generator, par: np.ndarray, depth_counts, branching: int):
+    """Fill par (BFS order: depth d holds depth_counts[d-1] nodes, each with a
+    parent drawn among the previous depth's nodes that have fewer than
+    ``branching`` children); return {parent: [children ascending]}."""
+    prev = [0]
+    nxt = 1
+    for cnt in depth_counts:
+        kids = {p: 0 for p in prev}
+        level = []
+        for _ in range(cnt):
+            choices = [p for p in prev if kids[p] < branching]
+            p = int(choices[brng.integers(len(choices))])
+            kids[p] += 1
+            par[nxt] = p
+            level.append(nxt)
+            nxt += 1
+        prev = level
+    children: dict[int, list[int]] = {}
+    for j in range(1, len(par)):
+        children.setdefault(int(par[j]), []).append(j)
+    return children
+
+
+@dataclass
+class TreeSampleInputs:
+    target: torch.Tensor       # [B, n, V] logits
+    draft: torch.Tensor        # [B, n, V] logits (or fp32 probabilities)
+    node_tokens: torch.Tensor  # [B, n] int32 (root token unused)
+    parents: torch.Tensor      # [B, n] int32, parents[:, 0] = -1
+    uniforms: torch.Tensor     # [B, n] fp32: column j >= 1 tests node j, column 0 the draw
+    temperature: float
+    max_depth: int
+    draft_kind: str = "logits"
+    meta: dict = field(default_factory=dict)
+
+
+def make_tree_sample(B: int = 8, V: int = V_QWEN, *, depth_counts=(8, 8, 8, 4, 3),
+                     branching: int = 8, dtype: str = "bf16", model: str = "zipf",
+                     sigma_t: float = 3.0, sigma_d: float = 1.0, zipf_s: float = 1.1,
+                     temperature: float = 0.7, seed: int = 0) -> TreeSampleInputs:
+    """Candidate trees (shapes as make_tree) for sampling verification: target
+    rows as make_chain's, draft logit rows z_t + sigma_d * N(0, 1), and the
+    children of every node drawn independently (with replacement) from the
+    stored draft row of their parent at temperature T, by Gumbel-max."""
+    n = 1 + sum(depth_counts)
+    T = float(np.float32(temperature))
+    tgt = np.empty((B, n, V), np.float32)
+    dft = np.empty((B, n, V), np.float32)
+    tok = np.zeros((B, n), np.int32)
+    par = np.full((B, n), -1, np.int32)
+    brng = _batch_rng(seed)
+    for b in range(B):
+        children = _tree_shape(brng, par[b], depth_counts, branching)
+        for j in range(n):
+            rng = _row_rng(seed, b * n + j)
+            noise_t = rng.standard_normal(V, dtype=np.float32)
+            noise_d = rng.standard_normal(V, dtype=np.float32)
+            if model == "zipf":
+                perm = rng.permutation(V)
+                prior = (-zipf_s * np.log1p(perm.astype(np.float64))).astype(np.float32)
+                zt = np.float32(sigma_t) * noise_t + prior
+            elif model == "gauss":
+                zt = np.float32(sigma_t) * noise_t
+            else:
+                raise ValueError(model)
+            tgt[b, j] = zt
+            dft[b, j] = zt + np.float32(sigma_d) * noise_d
+            kids = children.get(j, [])
+            if not kids:
+                continue
+            score = _cast(dft[b, j], dtype).double().numpy() / T
+            for c in kids:
+                g = -np.log(-np.log(rng.random(V) * (1 - 2.0**-53) + 2.0**-54))
+                tok[b, c] = int(np.argmax(score + g))
+    u = uniforms24(_batch_rng(seed + 7919), (B, n))
+    return TreeSampleInputs(_cast(tgt, dtype), _cast(dft, dtype), torch.from_numpy(tok),
+                            torch.from_numpy(par), torch.from_numpy(u), T, len(depth_counts),
+                            meta=dict(B=B, n=n, V=V, seed=seed))
+
+
 def make_tree(B: int = 8, V: int = V_QWEN, *, depth_counts=(8, 8, 8, 4, 3), branching: int = 8,
               plant_prob: float = 0.6, plant_value: float = 40.0, dtype: str = "bf16",
               sigma_t: float = 3.0, zipf_s: float = 1.1, seed: int = 0) -> TreeInputs:
@@ -181,22 +261,7 @@ def make_tree(B: int = 8, V: int = V_QWEN, *, depth_counts=(8, 8, 8, 4, 3), bran
             noise = rng.standard_normal(V, dtype=np.float32)
             perm = rng.permutation(V)
             z[b, j] = sigma_t * noise + (-zipf_s * np.log1p(perm.astype(np.float64))).astype(np.float32)
-        prev = [0]
-        nxt = 1
-        for cnt in depth_counts:
-            kids = {p: 0 for p in prev}
-            level = []
-            for _ in range(cnt):
-                choices = [p for p in prev if kids[p] < branching]
-                p = int(choices[brng.integers(len(choices))])
-                kids[p] += 1
-                par[b, nxt] = p
-                level.append(nxt)
-                nxt += 1
-            prev = level
-        children: dict[int, list[int]] = {}
-        for j in range(1, n):
-            children.setdefault(int(par[b, j]), []).append(j)
+        children = _tree_shape(brng, par[b], depth_counts, branching)
         for p, ch in children.items():
             toks = brng.choice(V, size=len(ch), replace=False)
             for j, t in zip(ch, toks):

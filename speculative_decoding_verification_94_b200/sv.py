@@ -28,7 +28,7 @@ SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
 EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc",
            "sv_verify_tree_greedy", "sv_kd_grad", "sv_kd_grad_workspace_size",
-           "sv_extract_topk_kd", "sv_kd_kl_loss", "sv_sched_select",
+           "sv_verify_tree_sample", "sv_extract_topk_kd", "sv_kd_kl_loss", "sv_sched_select",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
            "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size",
            "sv_device_status_check", "sv_status_string", "sv_version")
@@ -96,6 +96,9 @@ def lib() -> ctypes.CDLL:
             for f in ("sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
                       "sv_extract_topk_workspace_size", "sv_kd_kl_loss_workspace_size"):
                 getattr(L, f).restype = sz
+            L.sv_verify_tree_sample.argtypes = [vp, ci, vp, ci, ci, vp, vp, vp, ci, ci, ci, ci,
+                                                cf, vp, vp, vp, vp, vp]
+            L.sv_verify_tree_sample.restype = ci
             L.sv_sched_select.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp]
             L.sv_sched_select.restype = ci
             L.sv_status_string.argtypes = [ci]
@@ -347,6 +350,36 @@ def sv_verify_tree_greedy(logits: torch.Tensor, node_tokens: torch.Tensor,
                                      _p(o["out_tokens"]), _p(o["accepted_nodes"]), _p(w),
                                      w.numel(), _p(device_status), _stream(dev, stream))
     _check(rc, "sv_verify_tree_greedy")
+    return o
+
+
+def sv_verify_tree_sample(target: torch.Tensor, draft: torch.Tensor, node_tokens: torch.Tensor,
+                          parents: torch.Tensor, uniforms: torch.Tensor, temperature: float,
+                          max_depth: int, *, draft_kind: str = "logits", out: dict | None = None,
+                          device_status: torch.Tensor | None = None, stream=None) -> dict:
+    """Sampling verification of B candidate trees (see sv.h): target and draft
+    [B, n, V] (draft logits, or fp32 probabilities with draft_kind="probs"),
+    node_tokens and parents [B, n] int32, uniforms [B, n] fp32."""
+    _dev(target, "target")
+    _dev(draft, "draft")
+    B, n, V = target.shape
+    dev = target.device
+    _dev(node_tokens, "node_tokens", torch.int32)
+    _dev(parents, "parents", torch.int32)
+    _dev(uniforms, "uniforms", torch.float32)
+    W = max_depth + 1
+    o = dict(out or {})
+    o.setdefault("accepted_len", torch.empty(B, dtype=torch.int32, device=dev))
+    o.setdefault("out_tokens", torch.empty(B, W, dtype=torch.int32, device=dev))
+    o.setdefault("accepted_nodes", torch.empty(B, W, dtype=torch.int32, device=dev))
+    dk = SV_DRAFT_PROBS if draft_kind == "probs" else SV_DRAFT_LOGITS
+    rc = lib().sv_verify_tree_sample(_p(target), _dtype_code(target), _p(draft),
+                                     _dtype_code(draft), dk, _p(node_tokens), _p(parents),
+                                     _p(uniforms), B, n, V, max_depth, float(temperature),
+                                     _p(o["accepted_len"]), _p(o["out_tokens"]),
+                                     _p(o["accepted_nodes"]), _p(device_status),
+                                     _stream(dev, stream))
+    _check(rc, "sv_verify_tree_sample")
     return o
 
 
