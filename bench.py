@@ -53,7 +53,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="qwen_chain",
-                    choices=["qwen_chain", "kd", "kd_grad", "tree", "tiny", "sweep"])
+                    choices=["qwen_chain", "kd", "kd_grad", "tree", "tree_sample", "tiny",
+                             "sweep"])
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--sigma", type=float, default=1.0)
@@ -127,6 +128,12 @@ def make_workload(a, rank):
         return "tree", t, dict(workload="greedy_tree_verify", B=t.logits.shape[0],
                                n=t.logits.shape[1], V=t.logits.shape[2], depth=t.max_depth,
                                branching=8, input_dtype="bf16", temperature=0.0)
+    if a.workload == "tree_sample":
+        t = inputs.make_tree_sample(B=a.B or 8, seed=seed)
+        B, n, V = t.target.shape
+        return "tree_sample", t, dict(workload="sampling_tree_verify", B=B, n=n, V=V,
+                                      depth=t.max_depth, branching=8, input_dtype="bf16",
+                                      temperature=0.7, draft_sigma=1.0)
     raise ValueError(a.workload)
 
 
@@ -137,6 +144,12 @@ def needed_bytes(kind, x, accepted_len):
     Rows after the first rejection are not part of the computation."""
     if kind == "tree":
         return rows_and_bytes(kind, x)[1]
+    if kind == "tree_sample":
+        # the target/draft row pairs of the visited nodes (root .. last accepted)
+        B, n, V = x.target.shape
+        visits = int(np.sum(np.asarray(accepted_len, np.int64) + 1))
+        return (visits * V * (x.target.element_size() + x.draft.element_size()) + B * n * 12 +
+                B * 4 + 2 * B * (x.max_depth + 1) * 4)
     if kind == "grad":
         # the draft rows whose gradient is not zero are read once; every row of
         # the fp32 gradient is written; plus the top-K buffers and small inputs
@@ -162,6 +175,10 @@ def rows_and_bytes(kind, x):
         B, n, V = x.logits.shape
         es = x.logits.element_size()
         return B * n, B * n * V * es + B * n * 8 + B * 4 + 2 * B * (x.max_depth + 1) * 4
+    if kind == "tree_sample":
+        B, n, V = x.target.shape
+        return B * n, (B * n * V * (x.target.element_size() + x.draft.element_size()) +
+                       B * n * 12 + B * 4 + 2 * B * (x.max_depth + 1) * 4)
     if kind == "grad":  # draft rows per step; every draft row read twice, gradient written
         B, k, V = x.draft.shape
         return B * k, B * k * V * (2 * x.draft.element_size() + 4) + B * (k + 1) * 32 * 8 + B * 8
@@ -228,6 +245,9 @@ def oracle_step_fn(kind, x, threads=0):
     if kind == "tree":
         return lambda: O.tree_greedy(x.logits, x.node_tokens, x.parents, x.max_depth,
                                      threads=threads)
+    if kind == "tree_sample":
+        return lambda: O.tree_sample(x.target, x.draft, x.node_tokens, x.parents, x.uniforms,
+                                     x.temperature, x.max_depth, threads=threads)
     if kind == "kd":
         return lambda: O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward,
                                    x.temperature, 32, mode=O.W_GROUP_NORM, group=16,
@@ -327,6 +347,19 @@ def main():
             s = d or sets[i % ncopy]
             sv.sv_verify_tree_greedy(s["logits"], s["tok"], s["par"], x.max_depth, out=outs,
                                      device_status=status)
+    elif kind == "tree_sample":
+        sets = [dict(t=x.target.to(dev), d=x.draft.to(dev), tok=x.node_tokens.to(dev),
+                     par=x.parents.to(dev), u=x.uniforms.to(dev)) for _ in range(ncopy)]
+        B = x.target.shape[0]
+        outs = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=dev),
+                    out_tokens=torch.empty(B, x.max_depth + 1, dtype=torch.int32, device=dev),
+                    accepted_nodes=torch.empty(B, x.max_depth + 1, dtype=torch.int32,
+                                               device=dev))
+
+        def step(i, d=None):
+            s = d or sets[i % ncopy]
+            sv.sv_verify_tree_sample(s["t"], s["d"], s["tok"], s["par"], s["u"], x.temperature,
+                                     x.max_depth, out=outs, device_status=status)
     elif kind == "grad":
         B, k, V = x.draft.shape
         sets = [dict(d=x.draft.to(dev)) for _ in range(ncopy)]
@@ -423,6 +456,10 @@ def main():
         if kind == "tree":
             host = dict(logits=x.logits.pin_memory(), tok=x.node_tokens.pin_memory(),
                         par=x.parents.pin_memory())
+        elif kind == "tree_sample":
+            host = dict(t=x.target.pin_memory(), d=x.draft.pin_memory(),
+                        tok=x.node_tokens.pin_memory(), par=x.parents.pin_memory(),
+                        u=x.uniforms.pin_memory())
         elif kind == "grad":
             host = dict(d=x.draft.pin_memory())
         else:
@@ -478,11 +515,15 @@ def main():
                              "algorithmic_bytes_per_launch": algo_bytes,
                              "full_read_bytes_per_launch": full_bytes,
                              "call_us": ms_launch * 1e3,
-                             "kernel": {"tree": "sv_verify_tree_greedy",
-                                        "grad": "sv_kd_grad"}.get(kind, "sv_verify_chain") +
-                             " call: stream_kernel + second kernel, timed together"},
+                             "kernel": ("sv_verify_tree_sample call: tree_sample_kernel, one "
+                                        "launch" if kind == "tree_sample" else
+                                        {"tree": "sv_verify_tree_greedy",
+                                         "grad": "sv_kd_grad"}.get(kind, "sv_verify_chain") +
+                                        " call: stream_kernel + second kernel, timed together")},
                 "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / 8000.0,
-                "e2e": e2e, "gpu_launches": LAUNCHES_PER_CALL * a.steps, "clocks": clk,
+                "e2e": e2e,
+                "gpu_launches": (1 if kind == "tree_sample" else LAUNCHES_PER_CALL) * a.steps,
+                "clocks": clk,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -719,7 +719,8 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
 template <class TT, class DT, int DKIND>
 static cudaError_t run_tree_sample(FinishParams fp, int te, int de, bool bulk_ok, cudaStream_t s) {
   RowPlan plans[kMaxCluster];
-  const int rows_bytes = (int)sizeof(TreeShared) + 4 * fp.k * (int)sizeof(int);
+  // per node: 4 int, 2 float, 2 double, 1 float
+  const int rows_bytes = (int)sizeof(TreeShared) + 44 * fp.k;
   const int np = feasible_plans(
       fp.V, te, de,
       [](int, int npc) {

@@ -84,6 +84,11 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
   int* tok = par + n;
   int* kids = tok + n;
   int* pth = kids + n;
+  float* kzt = reinterpret_cast<float*>(pth + n);  // the children's target logits
+  float* kzd = kzt + n;                            // ... and draft logits (or probabilities)
+  double* kpx = reinterpret_cast<double*>(kzd + n);  // p(x) and q(x) of each child
+  double* kqx = kpx + n;
+  float* ku = reinterpret_cast<float*>(kqx + n);     // each child's uniform
   unsigned char* tbuf = smem + prm.lay.off_t;
   unsigned char* dbuf = smem + prm.lay.off_d;
   const int b = (int)(blockIdx.x / (unsigned)C);
@@ -94,6 +99,15 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
   const bool use_bulk = prm.use_bulk != 0;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   pdl_wait();
+  // the root's row pair is needed by every valid tree: its copies start first
+  const void* root_t = row_ptr<TT>(prm.target, (size_t)b * n, V);
+  const void* root_d = row_ptr<DT>(prm.draft, (size_t)b * n, V);
+  if (threadIdx.x == 0) {
+    init_piece_barriers(sh, g, use_bulk);
+    sh.timeouts = 0;
+    if (use_bulk)
+      issue_item_copies<TT, DT, true>(sh, tbuf, dbuf, root_t, root_d, g, policy_evict_first());
+  }
 
   // 0. the tree, checked the same way in every CTA
   int bad_tree = 0, bad_tok = 0;
@@ -131,12 +145,13 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
         prm.accepted_nodes[(size_t)b * W + d] = -1;
       }
     }
-    return;  // no CTA has touched another's shared memory
+    // no CTA has touched another's shared memory; the root's copies land
+    // before this CTA's shared memory is released
+    if (use_bulk && threadIdx.x == 0)
+      for (int p = 0; p < g.npieces; ++p) mbar_wait_bounded(&sh.bars[p], 0u);
+    return;
   }
-  if (threadIdx.x == 0) {
-    init_piece_barriers(sh, g, use_bulk);
-    pth[0] = 0;
-  }
+  if (threadIdx.x == 0) pth[0] = 0;
   __syncthreads();
 
   int red = 0;  // cluster combines so far (selects the slot)
@@ -144,7 +159,9 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
   // then the cluster total M and this CTA's share [lo, hi).  Collective over
   // the cluster.
   auto residual_pass = [&](float sg, float Gt, float invSt, float Gd, float invSd) {
-    for (int p = 0; p < g.npieces; ++p) {
+#pragma unroll 4
+    for (int p = 0; p < kMaxPieces; ++p) {
+      if (p >= g.npieces) break;
       const int e = p * kRound + (int)threadIdx.x * kVec;
       float s = 0.f;
       if (e < g.nvec * kVec) {
@@ -181,36 +198,82 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
   int v = 0, depth = 0, visit = 0, err = 0;
   bool drawn = false;
   for (;;) {
-    // a. stage the row pair of node v
+    // a. stage the row pair of node v (after every warp has left the previous
+    //    node's tests, which read kids[] and ts.nkids)
+    __syncthreads();
     const size_t row = (size_t)b * n + v;
     const void* trow = row_ptr<TT>(prm.target, row, V);
     const void* drow = row_ptr<DT>(prm.draft, row, V);
-    if (threadIdx.x == 0) {
+    if (visit > 0 && threadIdx.x == 0) {  // (the root's copies were issued at the start)
       sh.timeouts = 0;
       if (use_bulk) {
         fence_proxy_async_smem();  // earlier reads of the buffers precede the copies
         issue_item_copies<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, policy_evict_first());
       }
     }
+    if (w == 1) {
+      // the children of v in ascending order
+      int m = 0;
+      for (int base = v + 1; base < n; base += 32) {
+        const int j = base + lane;
+        const bool is = j < n && par[j] == v;
+        const unsigned bal = __ballot_sync(0xffffffffu, is);
+        if (is) kids[m + __popc(bal & ((1u << lane) - 1u))] = j;
+        m += __popc(bal);
+      }
+      if (lane == 0) ts.nkids = m;
+    }
     scalar_fill<TT>(tbuf, trow, g, use_bulk, false);
     scalar_fill<DT>(dbuf, drow, g, use_bulk, DKIND == kDraftProbs);
     __syncthreads();
+    // the two values each child's test reads, fetched while the copies land
+    for (int i = threadIdx.x; i < ts.nkids; i += kThreads) {
+      const int x = tok[kids[i]];
+      kzt[i] = load1<TT>(reinterpret_cast<const unsigned char*>(trow), x);
+      kzd[i] = load1<DT>(reinterpret_cast<const unsigned char*>(drow), x);
+      ku[i] = prm.u[(size_t)b * n + kids[i]];
+    }
     for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, use_bulk, (uint32_t)(visit & 1));
     __syncthreads();
 
     // b. the rows' statistics, combined over the cluster
+    // (two passes over the staged chunk: the maxima, then the exp2 terms
+    //  against one reference, so that the iterations are independent)
     ThreadStat a, d;
     stat_init(a);
     stat_init(d);
-    for (int p = 0; p < g.npieces; ++p) {
-      const int e = p * kRound + (int)threadIdx.x * kVec;
-      if (e < g.nvec * kVec) {
-        float z[8];
-        const float mt = load8_max<TT>(tbuf, e, z);
-        stat_update(a, z, mt, c);
-        if (DKIND == kDraftLogits) {
-          const float md = load8_max<DT>(dbuf, e, z);
-          stat_update(d, z, md, c);
+    {
+      float mt = -INFINITY, md = -INFINITY;
+#pragma unroll 4
+      for (int p = 0; p < kMaxPieces; ++p) {
+        if (p >= g.npieces) break;
+        const int e = p * kRound + (int)threadIdx.x * kVec;
+        if (e < g.nvec * kVec) {
+          mt = fmaxf(mt, max8<TT>(tbuf, e));
+          if (DKIND == kDraftLogits) md = fmaxf(md, max8<DT>(dbuf, e));
+        }
+      }
+      stat_cover(a, mt, c);
+      if (DKIND == kDraftLogits) stat_cover(d, md, c);
+      const bool fa = a.ref != -INFINITY, fd = DKIND == kDraftLogits && d.ref != -INFINITY;
+#pragma unroll 4
+      for (int p = 0; p < kMaxPieces; ++p) {
+        if (p >= g.npieces) break;
+        const int e = p * kRound + (int)threadIdx.x * kVec;
+        if (e < g.nvec * kVec) {
+          float z[8], t[8];
+          if (fa) {
+            load8<TT>(tbuf, e, z);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = ex2(fmaf(z[k], c, -a.ref));
+            a.S += (double)(((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7])));
+          }
+          if (fd) {
+            load8<DT>(dbuf, e, z);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = ex2(fmaf(z[k], c, -d.ref));
+            d.S += (double)(((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7])));
+          }
         }
       }
     }
@@ -246,17 +309,6 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
                               ? SV_DEV_NO_FINITE
                               : 0);
         }
-      } else if (w == 1) {
-        // the children of v in ascending order
-        int m = 0;
-        for (int base = v + 1; base < n; base += 32) {
-          const int j = base + lane;
-          const bool is = j < n && par[j] == v;
-          const unsigned bal = __ballot_sync(0xffffffffu, is);
-          if (is) kids[m + __popc(bal & ((1u << lane) - 1u))] = j;
-          m += __popc(bal);
-        }
-        if (lane == 0) ts.nkids = m;
       }
       __syncthreads();
     }
@@ -265,24 +317,27 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
       break;
     }
 
-    // c. the children's tests against the running residual
+    // c. the children's tests against the running residual (p(x) and q(x) of
+    //    every child first, in parallel)
     const float Gt = sh.Gt, Gd = sh.Gd;
     const float invSt = (float)(1.0 / sh.St);
     const float invSd = DKIND == kDraftLogits ? (float)(1.0 / sh.Sd) : 1.f;
-    const double Lt = ts.Lt, Ld = ts.Ld, cd64 = (double)c;
+    {
+      const double Lt = ts.Lt, Ld = ts.Ld, cd64 = (double)c;
+      for (int i = threadIdx.x; i < ts.nkids; i += kThreads) {
+        kpx[i] = exp2((double)kzt[i] * cd64 - Lt);
+        kqx[i] = DKIND == kDraftLogits ? exp2((double)kzd[i] * cd64 - Ld) : (double)kzd[i];
+      }
+      __syncthreads();
+    }
     double sigma = 0.0, M = 1.0;
     bool have = false, fallback = false;
     int next = -1;
     for (int i = 0; i < ts.nkids; ++i) {
       const int node = kids[i];
-      const int x = tok[node];
-      const double px = exp2((double)load1<TT>(reinterpret_cast<const unsigned char*>(trow), x) * cd64 - Lt);
-      const double qx =
-          DKIND == kDraftLogits
-              ? exp2((double)load1<DT>(reinterpret_cast<const unsigned char*>(drow), x) * cd64 - Ld)
-              : (double)load1<F32>(reinterpret_cast<const unsigned char*>(drow), x);
+      const double px = kpx[i], qx = kqx[i];
       const double rx = fmax(px - sigma * qx, 0.0);
-      const double uc = (double)prm.u[(size_t)b * n + node];
+      const double uc = (double)ku[i];
       if (uc * qx * M < rx) {  // accepted with probability min(1, r(x) / q(x))
         next = node;
         break;
