@@ -38,10 +38,12 @@ def metric_of(kind):
     return GRAD_METRIC if kind == "grad" else METRIC
 UNIT = "rows/s"
 L2_BYTES = 126 * 1024 * 1024
-# ncu dram__bytes_read.sum + dram__bytes_write.sum per call (stream kernel +
-# finisher, one full capture of each on this workload); absent for a workload
-# without a capture of the current kernels.
-NCU_TRAFFIC = {"qwen_chain_verify": (68.115200 + 0.634624 + 18.584064) * 1e6}
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
+# kernel, from one full capture of the current build on this workload (the
+# chain's stream kernel; the sampling tree's single kernel); absent for a
+# workload without such a capture.
+NCU_TRAFFIC = {"qwen_chain_verify": (68.114176 + 0.436992) * 1e6,
+               "sampling_tree_verify": 10.566912e6}
 # kernels one verification call launches: the streaming pass and the finisher
 LAUNCHES_PER_CALL = 2
 
