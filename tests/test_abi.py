@@ -146,3 +146,35 @@ def test_other_entry_points_validate(lib):
                              1, 3, 0.0, 0, f, f, f, f, 1 << 20, None, None) == E
     assert lib.sv_kd_kl_loss(f, f, 4, 3, 32, f, sv.SV_BF16, sv.SV_DRAFT_LOGITS, 1000, 1.0, f, f,
                              0, 1, 0.0, 0, f, f, f, None, 1 << 20, None, None) == sv.SV_ERR_WORKSPACE
+
+
+@no_gpu
+def test_ragged_chain_and_sampling_tree_validate(lib):
+    E = sv.SV_ERR_INVALID_ARG
+    f = FAKE
+
+    def ragged(dl, act, ws=f):
+        return lib.sv_verify_chain_ragged(f, sv.SV_BF16, f, sv.SV_BF16, sv.SV_DRAFT_LOGITS, f, f,
+                                          dl, act, 4, 3, 1024, 1.0, f, f, None, ws, 1 << 20,
+                                          None, None)
+    assert ragged(ctypes.c_void_p(0x10002), None) == E  # misaligned draft_len
+    assert ragged(None, ctypes.c_void_p(0x10001)) == E  # misaligned active
+    assert ragged(f, f, ws=None) == sv.SV_ERR_WORKSPACE  # arrays fine, fails on the workspace
+
+    def tree(**kw):
+        a = dict(t=f, tdt=sv.SV_BF16, d=f, ddt=sv.SV_BF16, dk=sv.SV_DRAFT_LOGITS, tok=f, par=f,
+                 u=f, B=4, n=32, V=1024, depth=5, T=0.7, acc=f, out=f, nodes=f)
+        a.update(kw)
+        return lib.sv_verify_tree_sample(a["t"], a["tdt"], a["d"], a["ddt"], a["dk"], a["tok"],
+                                         a["par"], a["u"], a["B"], a["n"], a["V"], a["depth"],
+                                         a["T"], a["acc"], a["out"], a["nodes"], None, None)
+    assert tree(T=0.0) == E                      # sampling needs T > 0
+    assert tree(n=0) == E
+    assert tree(n=2000) == E
+    assert tree(depth=32) == E                   # max_depth >= n
+    assert tree(dk=sv.SV_DRAFT_PROBS) == E       # probabilities must be fp32
+    assert tree(u=None) == E
+    assert tree(par=None) == E
+    assert tree(d=ctypes.c_void_p(0x10001)) == E  # misaligned bf16 row
+    assert tree(V=600000) == sv.SV_ERR_UNSUPPORTED
+    assert tree(B=0) == sv.SV_OK                 # nothing to do, nothing enqueued
