@@ -1,0 +1,51 @@
+"""The benchmark's byte counts (the numerators of its roofline figures),
+checked on CPU against sums written out from the tensors themselves: the
+stored bytes of every logit, and the bytes verification needs given the
+accepted lengths (rows after a request's first rejection, or off a tree's
+accepted path, are not needed)."""
+import numpy as np
+import torch
+
+import bench
+from speculative_decoding_verification_94_b200 import inputs
+
+
+def _nbytes(*ts):
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+def test_chain_stored_and_needed_bytes():
+    x = inputs.make_chain(3, 3, 257, dtype="bf16", seed=1)
+    rows, full = bench.rows_and_bytes("chain", x)
+    assert rows == 3 * 4
+    io = _nbytes(x.draft_tokens, x.uniforms) + 3 * 4 + 3 * 4 * 4  # accepted_len, out_tokens
+    assert full == _nbytes(x.target, x.draft) + io
+    acc = np.array([0, 2, 3], np.int32)
+    # request 0: pair 0; request 1: pairs 0..2; request 2: pairs 0..2 and the bonus row 3
+    pair = 257 * 2 * 2
+    want = (1 + 3 + 3) * pair + 257 * 2 + io
+    assert bench.needed_bytes("chain", x, acc) == want
+
+
+def test_sampling_tree_bytes_count_visited_nodes():
+    t = inputs.make_tree_sample(B=2, V=300, depth_counts=(2, 2), branching=2, seed=2)
+    B, n, V = t.target.shape
+    rows, full = bench.rows_and_bytes("tree_sample", t)
+    assert rows == B * n
+    small = _nbytes(t.node_tokens, t.parents, t.uniforms) + B * 4 + 2 * B * (t.max_depth + 1) * 4
+    assert full == _nbytes(t.target, t.draft) + small
+    acc = np.array([2, 0], np.int32)  # visits: root..depth 2 (3 nodes), root only (1 node)
+    assert bench.needed_bytes("tree_sample", t, acc) == 4 * V * (2 + 2) + small
+
+
+def test_greedy_tree_reads_every_node():
+    t = inputs.make_tree(B=2, V=300, depth_counts=(2, 2), branching=2, seed=3)
+    rows, full = bench.rows_and_bytes("tree", t)
+    assert rows == 2 * t.logits.shape[1]
+    assert bench.needed_bytes("tree", t, np.zeros(2, np.int32)) == full
+    assert full >= _nbytes(t.logits)
+
+
+def test_job_value_is_whole_job_rows_per_second():
+    # 2 ranks x 10 steps x 128 rows in 5 ms of the slowest rank
+    assert bench.job_value(128, 2, 10, 5.0) == 128 * 2 * 10 / 5e-3
