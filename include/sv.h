@@ -63,7 +63,7 @@ extern "C" {
 typedef enum sv_status {
   SV_OK = 0,
   SV_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, size or mode out of range */
-  SV_ERR_UNSUPPORTED = 2,  /* valid but beyond this build (e.g. V too large for one row plan) */
+  SV_ERR_UNSUPPORTED = 2,  /* valid but beyond the library's limits (e.g. V too large for one row plan) */
   SV_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, attribute, device query) */
   SV_ERR_DEVICE_CHECK = 4, /* returned by sv_device_status_check() for SV_DEV_* error bits */
   SV_ERR_TIMEOUT = 5,      /* returned by sv_device_status_check() for SV_DEV_TIMEOUT */
