@@ -359,6 +359,21 @@ def test_oracle_is_thread_count_invariant(oracle):
     b = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 0.7, threads=8)
     for key in ("accepted_len", "out_tokens", "p_x", "cdf_margin"):
         assert np.array_equal(a[key], b[key], equal_nan=True)
+    klen = np.arange(24, dtype=np.int32) % 4
+    act = (np.arange(24) % 5 != 0).astype(np.int32)
+    a = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 0.7, threads=1,
+                            draft_len=klen, active=act)
+    b = oracle.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, 0.7, threads=8,
+                            draft_len=klen, active=act)
+    for key in ("accepted_len", "out_tokens", "cdf_margin"):
+        assert np.array_equal(a[key], b[key], equal_nan=True)
+    t = inputs.make_tree_sample(B=24, V=500, depth_counts=(3, 3, 2), branching=3, seed=13)
+    a = oracle.tree_sample(t.target, t.draft, t.node_tokens, t.parents, t.uniforms,
+                           t.temperature, t.max_depth, threads=1)
+    b = oracle.tree_sample(t.target, t.draft, t.node_tokens, t.parents, t.uniforms,
+                           t.temperature, t.max_depth, threads=8)
+    for key in ("accepted_len", "out_tokens", "accepted_nodes", "test_margin", "cdf_margin"):
+        assert np.array_equal(a[key], b[key])
 
 
 # --------------------------------------------------------------------------
