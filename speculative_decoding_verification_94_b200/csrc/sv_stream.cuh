@@ -1,12 +1,17 @@
 // sv_stream.cuh -- the streaming pass shared by every entry point.
 //
-// Every warp is an independent worker.  Work items are chunks of W vocabulary
-// entries of one row (or of a target/draft row pair, read together), handed
-// out roughly in index order (static first items, then per-stripe counters;
-// see stream_kernel).  Chain items are numbered position-major (every
-// request's position 0 first): an item whose request has already rejected at
-// an earlier position is skipped before any byte is loaded, so once a
-// request's fate is known its later rows are not read.
+// Every warp is an independent worker.  Two schedules (chosen per call):
+//  - static (kFStatic): warp g takes a contiguous range of 1024-element pieces
+//    of the row-major piece space and writes one record per run of pieces
+//    within a row; the finishing kernel folds each row's records;
+//  - dynamic: work items are chunks of W vocabulary entries of one row (or of
+//    a target/draft row pair, read together), handed out roughly in index
+//    order (first items, then per-stripe counters; see stream_kernel), and
+//    the stream itself completes the rows.
+// Chain items are numbered position-major (every request's position 0
+// first): an item whose request has already rejected at an earlier position
+// (dynamic schedule), or whose row the request does not use (ragged batches,
+// either schedule), is skipped before any byte is loaded.
 //
 // A warp streams its items through its own ring of kStages pieces of kPiece
 // elements; lane 0 issues bulk copies (cp.async.bulk, no multicast) up to
@@ -15,10 +20,11 @@
 // online softmax statistics (ThreadStat: exact power-of-two rescales), the
 // element at the draft token, the argmax, and a sorted warp list of the K best
 // keys; per item these are reduced with shuffles into one partial record.
-// Items are counted into their row one item late (deferred counting); the warp
-// whose count completes a row combines the row's partials in chunk order (so
-// the result does not depend on which warp finished last) and records the
-// row's normaliser and, for chain rows, the acceptance decision.
+// Dynamic schedule: items are counted into their row one item late (deferred
+// counting); the warp whose count completes a row combines the row's partials
+// in chunk order (so the result does not depend on which warp finished last)
+// and records the row's normaliser and, for chain rows, the acceptance
+// decision.
 //
 // No __syncthreads, no cluster barrier and no shared-memory residency: the
 // only cross-warp communication is the counters and the records.
