@@ -1,16 +1,18 @@
 // sv_finish.cuh -- the finishing pass of every entry point (after the stream).
 //
-// Chain sampling: one C-CTA cluster per request reads the request's row
-// records, finds the first rejection n (or n = k), and draws the emitted token
-// from the one row pair that needs it: residual max(0, p_n - q_n) or, for
-// n = k, the bonus row p_k, by inverse CDF in ascending vocabulary order.  The
-// row pair is staged in shared memory (bulk copies), the CTA chunk masses are
-// combined in a fixed order through distributed shared memory and the owning
-// CTA locates the draw.  Fused KD rows were written by the stream; the
-// finisher marks the rows after the emitted position as undefined and forms
-// the reward-weighted losses.  Every finisher returns the row records it read
-// to zero (the stream zeroes the partials), so the workspace stays zero
-// between calls.
+// Chain sampling: one C-CTA cluster per request folds (static schedule) or
+// reads (dynamic schedule) the request's row records, finds the first
+// rejection n (or n = k_b, the request's draft count), and draws the emitted
+// token from the one row pair that needs it: residual max(0, p_n - q_n) or,
+// for n = k_b, the bonus row p_{k_b}, by inverse CDF in ascending vocabulary
+// order.  The row pair is staged in shared memory (bulk copies), the CTA
+// chunk masses are combined in a fixed order through distributed shared
+// memory and the owning CTA locates the draw.  Fused KD rows are written here
+// (static schedule) or were written by the stream (dynamic); the finisher
+// marks the rows after the emitted position as undefined and forms the
+// reward-weighted losses.  Every finisher returns the stream state it read
+// (the static schedule's records, or the dynamic schedule's row records) to
+// zero, so the workspace stays zero between calls.
 #pragma once
 
 #include "sv_rowops.cuh"
