@@ -55,8 +55,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="qwen_chain",
-                    choices=["qwen_chain", "kd", "kd_grad", "tree", "tree_sample", "tiny",
-                             "sweep"])
+                    choices=["qwen_chain", "kd", "kd_grad", "tree", "tree_sample", "ragged",
+                             "tiny", "sweep"])
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--sigma", type=float, default=1.0)
@@ -130,6 +130,14 @@ def make_workload(a, rank):
         return "tree", t, dict(workload="greedy_tree_verify", B=t.logits.shape[0],
                                n=t.logits.shape[1], V=t.logits.shape[2], depth=t.max_depth,
                                branching=8, input_dtype="bf16", temperature=0.0)
+    if a.workload == "ragged":
+        B = a.B or 32
+        k = a.k or 3
+        x = inputs.qwen_chain(B=B, k=k, sigma_d=1.0, seed=seed)
+        x.meta["draft_len"], x.meta["active"] = inputs.ragged_lengths(B, k, seed=seed)
+        return "ragged", x, dict(workload="ragged_chain_verify", B=B, k=k, V=x.V,
+                                 input_dtype="bf16", temperature=0.7, draft_sigma=1.0,
+                                 draft_len="uniform on 0..k", idle_fraction=0.15)
     if a.workload == "tree_sample":
         t = inputs.make_tree_sample(B=a.B or 8, seed=seed)
         B, n, V = t.target.shape
@@ -152,6 +160,18 @@ def needed_bytes(kind, x, accepted_len):
         visits = int(np.sum(np.asarray(accepted_len, np.int64) + 1))
         return (visits * V * (x.target.element_size() + x.draft.element_size()) + B * n * 12 +
                 B * 4 + 2 * B * (x.max_depth + 1) * 4)
+    if kind == "ragged":
+        # per active request: pairs 0..min(n, k_b - 1) and the bonus row k_b
+        # when n = k_b; idle requests read nothing
+        B, P, V = x.target.shape
+        te, de = x.target.element_size(), x.draft.element_size()
+        kb = x.meta["draft_len"].numpy().astype(np.int64)
+        on = x.meta["active"].numpy() != 0
+        n = np.asarray(accepted_len, np.int64)
+        pairs = np.where(on, np.minimum(n, kb - 1) + 1, 0)
+        bonus = on & (n == kb)
+        return (int(np.sum(pairs)) * V * (te + de) + int(np.sum(bonus)) * V * te +
+                _ragged_io(x))
     if kind == "grad":
         # the draft rows whose gradient is not zero are read once; every row of
         # the fp32 gradient is written; plus the top-K buffers and small inputs
@@ -171,8 +191,20 @@ def needed_bytes(kind, x, accepted_len):
     return by
 
 
+def _ragged_io(x):
+    B, P = x.target.shape[:2]
+    return (B * (P - 1) * 4 + B * P * 4 + 2 * B * 4) + B * 4 + B * P * 4
+
+
 def rows_and_bytes(kind, x):
     """Verified rows per step and the bytes of reading every logit once + I/O."""
+    if kind == "ragged":  # the rows the active requests use
+        V = x.target.shape[2]
+        te, de = x.target.element_size(), x.draft.element_size()
+        kb = x.meta["draft_len"].numpy().astype(np.int64)
+        on = x.meta["active"].numpy() != 0
+        rows = int(np.sum((kb + 1)[on]))
+        return rows, (rows * V * te + int(np.sum(kb[on])) * V * de) + _ragged_io(x)
     if kind == "tree":
         B, n, V = x.logits.shape
         es = x.logits.element_size()
@@ -250,6 +282,10 @@ def oracle_step_fn(kind, x, threads=0):
     if kind == "tree_sample":
         return lambda: O.tree_sample(x.target, x.draft, x.node_tokens, x.parents, x.uniforms,
                                      x.temperature, x.max_depth, threads=threads)
+    if kind == "ragged":
+        return lambda: O.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms,
+                                      x.temperature, threads=threads,
+                                      draft_len=x.meta["draft_len"], active=x.meta["active"])
     if kind == "kd":
         return lambda: O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward,
                                    x.temperature, 32, mode=O.W_GROUP_NORM, group=16,
@@ -362,6 +398,19 @@ def main():
             s = d or sets[i % ncopy]
             sv.sv_verify_tree_sample(s["t"], s["d"], s["tok"], s["par"], s["u"], x.temperature,
                                      x.max_depth, out=outs, device_status=status)
+    elif kind == "ragged":
+        sets = [dict(t=x.target.to(dev), d=x.draft.to(dev), tok=x.draft_tokens.to(dev),
+                     u=x.uniforms.to(dev), kl=x.meta["draft_len"].to(dev),
+                     act=x.meta["active"].to(dev)) for _ in range(ncopy)]
+        B, P = x.target.shape[0], x.target.shape[1]
+        outs = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=dev),
+                    out_tokens=torch.empty(B, P, dtype=torch.int32, device=dev))
+
+        def step(i, d=None):
+            s = d or sets[i % ncopy]
+            sv.sv_verify_chain_ragged(s["t"], s["d"], s["tok"], s["u"], x.temperature,
+                                      draft_len=s["kl"], active=s["act"], out=outs,
+                                      device_status=status)
     elif kind == "grad":
         B, k, V = x.draft.shape
         sets = [dict(d=x.draft.to(dev)) for _ in range(ncopy)]
@@ -462,6 +511,10 @@ def main():
             host = dict(t=x.target.pin_memory(), d=x.draft.pin_memory(),
                         tok=x.node_tokens.pin_memory(), par=x.parents.pin_memory(),
                         u=x.uniforms.pin_memory())
+        elif kind == "ragged":
+            host = dict(t=x.target.pin_memory(), d=x.draft.pin_memory(),
+                        tok=x.draft_tokens.pin_memory(), u=x.uniforms.pin_memory(),
+                        kl=x.meta["draft_len"].pin_memory(), act=x.meta["active"].pin_memory())
         elif kind == "grad":
             host = dict(d=x.draft.pin_memory())
         else:
@@ -519,8 +572,9 @@ def main():
                              "call_us": ms_launch * 1e3,
                              "kernel": ("sv_verify_tree_sample call: tree_sample_kernel, one "
                                         "launch" if kind == "tree_sample" else
-                                        {"tree": "sv_verify_tree_greedy",
-                                         "grad": "sv_kd_grad"}.get(kind, "sv_verify_chain") +
+                                        {"tree": "sv_verify_tree_greedy", "grad": "sv_kd_grad",
+                                         "ragged": "sv_verify_chain_ragged"}.get(
+                                             kind, "sv_verify_chain") +
                                         " call: stream_kernel + second kernel, timed together")},
                 "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / 8000.0,
                 "e2e": e2e,

@@ -273,6 +273,20 @@ def make_tree(B: int = 8, V: int = V_QWEN, *, depth_counts=(8, 8, 8, 4, 3), bran
                       len(depth_counts), meta=dict(B=B, n=n, V=V, seed=seed))
 
 
+def ragged_lengths(B: int, k: int, seed: int = 0, idle_frac: float = 0.15):
+    """Per-request draft counts k_b uniform on 0..k and an active mask (a
+    request is idle with probability idle_frac); the first min(B, k+1)
+    requests are active with k_b = 0, 1, .., k so that every length occurs.
+    Returns int32 tensors (draft_len, active)."""
+    rng = _batch_rng(seed + 104729)
+    klen = rng.integers(0, k + 1, B).astype(np.int32)
+    act = (rng.random(B) >= idle_frac).astype(np.int32)
+    m = min(B, k + 1)
+    klen[:m] = np.arange(m, dtype=np.int32)
+    act[:m] = 1
+    return torch.from_numpy(klen), torch.from_numpy(act)
+
+
 # The workloads, by what they are.
 def tiny_chain(seed: int = 0) -> ChainInputs:
     """B=4, k=3, V=1024 fp32, z_t ~ N(0, 2^2), z_d = z_t + N(0, 0.5^2), T=1."""

@@ -49,3 +49,24 @@ def test_greedy_tree_reads_every_node():
 def test_job_value_is_whole_job_rows_per_second():
     # 2 ranks x 10 steps x 128 rows in 5 ms of the slowest rank
     assert bench.job_value(128, 2, 10, 5.0) == 128 * 2 * 10 / 5e-3
+
+
+def test_ragged_bytes_count_only_used_rows():
+    x = inputs.make_chain(4, 3, 300, dtype="bf16", seed=4)
+    x.meta["draft_len"] = torch.tensor([0, 3, 2, 1], dtype=torch.int32)
+    x.meta["active"] = torch.tensor([1, 1, 0, 1], dtype=torch.int32)
+    rows, full = bench.rows_and_bytes("ragged", x)
+    assert rows == 1 + 4 + 2  # idle request 2 uses no row
+    io = _nbytes(x.draft_tokens, x.uniforms) + 2 * 4 * 4 + 4 * 4 + 4 * 4 * 4
+    row = 300 * 2
+    assert full == (7 * row + (0 + 3 + 1) * row) + io
+    acc = np.array([0, 1, 0, 1], np.int32)
+    # request 0: bonus row 0; request 1: pairs 0..1; request 3: pair 0 and bonus row 1
+    assert bench.needed_bytes("ragged", x, acc) == (0 + 2 + 1) * 2 * row + 2 * row + io
+
+
+def test_ragged_lengths_cover_every_length():
+    kl, act = inputs.ragged_lengths(32, 3, seed=0)
+    assert kl.dtype == torch.int32 and act.dtype == torch.int32
+    assert set(kl.tolist()) == {0, 1, 2, 3} and (act[:4] == 1).all()
+    assert ((kl >= 0) & (kl <= 3)).all() and 0 < int(act.sum()) <= 32
