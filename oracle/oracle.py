@@ -7,7 +7,8 @@ imports this module; the CUDA library and this oracle share no code.
 Each function takes host arrays (torch CPU tensors or numpy arrays), widens
 nothing itself (the C code widens bf16/fp32 to float64 exactly) and returns
 numpy arrays.  See the header of ``sv_oracle.c`` for the definitions followed
-and the pages they come from.
+and the pages they come from.  One function is plain Python: ``sched_select``,
+the adaptive scheduler's table lookup (no float64 arithmetic to speak of).
 """
 from __future__ import annotations
 
