@@ -39,13 +39,19 @@ def metric_of(kind):
 UNIT = "rows/s"
 L2_BYTES = 126 * 1024 * 1024
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
-# kernel, from one full capture of the current build on this workload (the
-# chain's stream kernel; the sampling tree's single kernel); absent for a
-# workload without such a capture.
-NCU_TRAFFIC = {"qwen_chain_verify": (68.114176 + 0.436992) * 1e6,
-               "sampling_tree_verify": 10.566912e6}
-# kernels one verification call launches: the streaming pass and the finisher
-LAUNCHES_PER_CALL = 2
+# kernel, from one capture of the current build on this workload, with the
+# profiles/ summary that holds it; absent for a workload whose kernel changed
+# since its last capture.
+NCU_TRAFFIC: dict = {}
+# kernels one call launches: chains of k <= 30 run as one persistent kernel;
+# the greedy tree and the KD gradient as a streaming pass plus a second kernel
+LAUNCHES = {"chain": 1, "kd": 1, "ragged": 1, "tree_sample": 1, "tree": 2, "grad": 2}
+KERNEL_NAME = {"chain": "chain_kernel (sv_verify_chain: one persistent launch per call)",
+               "kd": "chain_kernel with fused top-K / KL (sv_verify_chain: one launch per call)",
+               "ragged": "chain_kernel (sv_verify_chain_ragged: one launch per call)",
+               "tree_sample": "tree_sample_kernel (sv_verify_tree_sample: one launch per call)",
+               "tree": "sv_verify_tree_greedy call: stream_kernel + tree_finish, timed together",
+               "grad": "sv_kd_grad call: stream_kernel + kd_grad_kernel, timed together"}
 
 
 def parse():
@@ -56,7 +62,9 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="qwen_chain",
                     choices=["qwen_chain", "kd", "kd_grad", "tree", "tree_sample", "ragged",
-                             "tiny", "sweep"])
+                             "tiny", "sweep", "sched_table"])
+    ap.add_argument("--table-out", default=None,
+                    help="sched_table: write the measured verify-cost table (JSON) here")
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--sigma", type=float, default=1.0)
@@ -345,10 +353,106 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+SCHED_KS = (1, 3, 5, 7)
+SCHED_BATCHES = (1, 2, 4, 8, 16, 32)
+
+
+def graph_time_us(step, steps, dev):
+    """Mean device time of one call: `steps` calls captured in a CUDA graph,
+    replayed once untimed and once between CUDA events."""
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            step(i)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s = torch.cuda.current_stream(dev)
+    e0.record(s)
+    g.replay()
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    return 1e3 * e0.elapsed_time(e1) / steps
+
+
+def run_sched_table(a):
+    """The measured verify-cost table of the adaptive scheduler's lookup: the
+    device time of one verification call for k in SCHED_KS drafts and for
+    plain decoding (one token sampled from the target row: the ragged call
+    with every draft count 0), at active batches SCHED_BATCHES, V=151936
+    bf16, T=0.7, draft noise sigma (default 1.0).  Throughput of a
+    configuration = emitted tokens per second of verification, B * mean
+    (accepted + 1) / call time (B / call time for plain decoding).  Verify
+    kernels only: no model forward is timed."""
+    from speculative_decoding_verification_94_b200 import sv
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    sv.lib()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    Bmax = max(SCHED_BATCHES)
+    rows, table_us, tokens = [], {}, {}
+    for k in (0,) + SCHED_KS:
+        x = inputs.qwen_chain(B=Bmax, k=max(k, 1), sigma_d=a.sigma, seed=0)
+        for B in SCHED_BATCHES:
+            per = x.target[:B].numel() * 2 + (x.draft[:B].numel() * 2 if k else 0)
+            ncopy = max(2, math.ceil(2.2 * L2_BYTES / per))
+            sets = [dict(t=x.target[:B].contiguous().to(dev), d=x.draft[:B].contiguous().to(dev),
+                         tok=x.draft_tokens[:B].contiguous().to(dev),
+                         u=x.uniforms[:B].contiguous().to(dev)) for _ in range(ncopy)]
+            zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+            out = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty(B, max(k, 1) + 1, dtype=torch.int32, device=dev))
+
+            def step(i, s=None):
+                s = s or sets[i % ncopy]
+                if k == 0:
+                    sv.sv_verify_chain_ragged(s["t"], s["d"], s["tok"], s["u"], x.temperature,
+                                              draft_len=zeros, out=out, device_status=status)
+                else:
+                    sv.sv_verify_chain(s["t"], s["d"], s["tok"], s["u"], x.temperature, out=out,
+                                       device_status=status)
+
+            us = graph_time_us(step, a.steps, dev)
+            step(0)
+            torch.cuda.synchronize(dev)
+            acc = out["accepted_len"].cpu().numpy().astype(np.float64)
+            emitted = float(np.mean(acc + 1.0))
+            table_us[(k, B)] = us
+            tokens[(k, B)] = emitted
+            rows.append(dict(k=k, B=B, call_us=us, mean_emitted=emitted,
+                             tokens_per_s=B * emitted / (us * 1e-6)))
+            print(json.dumps(rows[-1]), flush=True)
+            del sets
+    st = int(status.item())
+    assert st & sv.SV_DEV_ERROR_MASK == 0, f"device status {st:#x}"
+    cfgs = ["plain"] + [f"k={k}" for k in SCHED_KS]
+    thr = [[r["tokens_per_s"] for r in rows if r["k"] == k] for k in (0,) + SCHED_KS]
+    table = {"what": "verify-kernel cost table: emitted tokens per second of one verification "
+                     "call, per configuration (rows) and active batch (columns)",
+             "configs": cfgs, "nonspec": 0, "batches": list(SCHED_BATCHES),
+             "throughput_tokens_per_s": thr,
+             "call_us": [[table_us[(k, B)] for B in SCHED_BATCHES] for k in (0,) + SCHED_KS],
+             "mean_emitted": [[tokens[(k, B)] for B in SCHED_BATCHES] for k in (0,) + SCHED_KS],
+             "workload": dict(V=inputs.V_QWEN, input_dtype="bf16", temperature=0.7,
+                              draft_sigma=a.sigma, seed=0),
+             "command": f"python bench.py --workload sched_table --steps {a.steps} "
+                        f"--sigma {a.sigma} --table-out <path>"}
+    if a.table_out:
+        with open(a.table_out, "w") as f:
+            json.dump(table, f, indent=1)
+            f.write("\n")
+    print(json.dumps({"metric": "verify-cost table", "table": table}), flush=True)
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         return run_reference(a)
+    if a.workload == "sched_table":
+        return run_sched_table(a)
     from speculative_decoding_verification_94_b200 import sv
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -495,8 +599,8 @@ def main():
     assert st & sv.SV_DEV_ERROR_MASK == 0, f"device status {st:#x}"
 
     peak, peak_kind = load_peaks()
-    full_bytes = algo_bytes
-    algo_bytes = needed_bytes(kind, x, outs["accepted_len"].cpu().numpy())
+    need_bytes = needed_bytes(kind, x, outs["accepted_len"].cpu().numpy())
+    # algorithmic bytes: every input logit read once plus the small I/O
     achieved = algo_bytes / (ms_launch * 1e-3) / 1e9
     value = job_value(rows, world, a.steps, ms_total)
 
@@ -562,23 +666,24 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f32", "data": "synthetic",
                 "config": dict(cfg, l2=f"{ncopy} rotating input copies "
-                                       f"({ncopy * full_bytes / 2**20:.0f} MiB > 2x L2)",
+                                       f"({ncopy * algo_bytes / 2**20:.0f} MiB > 2x L2)",
                                parallelism=f"dp{world}" if world > 1 else "single"),
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                              "unit": "GB/s", "frac": achieved / peak,
-                             "traffic": traffic, "peak_kind": peak_kind,
+                             "traffic": traffic[0] if traffic else None,
+                             "traffic_from": traffic[1] if traffic else None,
+                             "peak_kind": peak_kind,
                              "algorithmic_bytes_per_launch": algo_bytes,
-                             "full_read_bytes_per_launch": full_bytes,
+                             "needed_bytes_per_launch": need_bytes,
+                             "needed_frac": need_bytes / (ms_launch * 1e-3) / 1e9 / peak,
                              "call_us": ms_launch * 1e3,
-                             "kernel": ("sv_verify_tree_sample call: tree_sample_kernel, one "
-                                        "launch" if kind == "tree_sample" else
-                                        {"tree": "sv_verify_tree_greedy", "grad": "sv_kd_grad",
-                                         "ragged": "sv_verify_chain_ragged"}.get(
-                                             kind, "sv_verify_chain") +
-                                        " call: stream_kernel + second kernel, timed together")},
+                             "kernel": KERNEL_NAME.get(kind, KERNEL_NAME["chain"])},
+                "kernels": ({("tree_sample_kernel" if kind == "tree_sample" else "chain_kernel"):
+                             {"us_per_launch": ms_launch * 1e3, "launches_per_step": 1}}
+                            if LAUNCHES.get(kind, 1) == 1 else None),
                 "hbm_gbs": achieved, "pct_of_8tbs": 100 * achieved / 8000.0,
                 "e2e": e2e,
-                "gpu_launches": (1 if kind == "tree_sample" else LAUNCHES_PER_CALL) * a.steps,
+                "gpu_launches": LAUNCHES.get(kind, 1) * a.steps,
                 "clocks": clk,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)

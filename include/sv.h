@@ -158,7 +158,8 @@ SV_API size_t sv_kd_kl_loss_workspace_size(int B, int k, int V);
  * Verification is sequential within a request: a draft after the first
  * rejection is never tested.  Rows are streamed position-major and a row whose
  * request has already rejected at an earlier position is skipped before it is
- * loaded, so the bytes read approach the rows the outcome depends on.
+ * loaded, so the bytes read approach the rows the outcome depends on.  Chains
+ * of k <= 30 drafts run as one kernel launch; longer ones as two.
  *   device_status optional int32 status word (SV_DEV_* bits).
  */
 SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
@@ -211,20 +212,23 @@ SV_API sv_status sv_verify_chain_ragged(const void* target_logits, sv_dtype t_dt
  * interface that hands over only input and output pointers, so that they
  * cannot own a workspace buffer.
  *
- *   Arguments, results and errors are those of sv_verify_chain.
+ *   Arguments, results and errors are those of sv_verify_chain, and the
+ *   argument checks run first, so a bad argument returns the same code.
  *   The scratch is a fixed array of SV_NOALLOC_MAX_BYTES per device inside
- *   libsv.  The first call on a device (with that device current) performs a
- *   one-time setup that looks up the array's device address; make that first
- *   call before any stream capture.
+ *   libsv.  Every call looks up the array's device address in the calling
+ *   thread's current context (a host-side lookup); the first call on a device
+ *   also loads the library's device code there, so make it before any stream
+ *   capture.
  *   A call whose sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0)
  *   exceeds SV_NOALLOC_MAX_BYTES returns SV_ERR_WORKSPACE and launches
- *   nothing.  At V = 151936 that allows about B*(k+1) <= 570 target rows
- *   without KD and about 90 with K = 32.
+ *   nothing.  At V = 151936 that allows about B*(k+1) <= 3500 target rows
+ *   without KD and about 700 with K = 32 (k <= 30).
  *   The array starts zero-filled and every completed call returns it to zero,
- *   so nothing needs clearing.  All calls on a device share the one array:
- *   calls that can run at the same time (on different streams, or from host
- *   threads without mutual ordering) race on it and must be ordered by the
- *   caller.
+ *   including calls whose requests fail a device check; a call that returns
+ *   SV_ERR_CUDA after a partial launch clears it with an asynchronous memset
+ *   on `stream`.  All calls on a device share the one array: calls that can
+ *   run at the same time (on different streams, or from host threads without
+ *   mutual ordering) race on it and must be ordered by the caller.
  */
 #define SV_NOALLOC_MAX_BYTES (4u << 20)
 SV_API sv_status sv_verify_chain_noalloc(const void* target_logits, sv_dtype t_dtype,
@@ -364,6 +368,41 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
                             sv_weight_mode wmode, int group, float clip, int positions, float* grad,
                             void* workspace, size_t workspace_bytes, int32_t* device_status,
                             void* stream);
+
+/*
+ * sv_set_knob -- process-wide test and tuning settings (not needed for
+ * normal use; the pages have no counterpart).  Every knob defaults to 0, the
+ * library's own choice, and a value set applies to every later call from any
+ * thread until it is set again.  Returns SV_ERR_INVALID_ARG for an unknown
+ * knob; values outside a knob's range select the default.
+ *   SV_KNOB_CLUSTER_CTAS  finishing cluster size of the two-kernel paths, 1..16
+ *   SV_KNOB_STREAM_COUNT  two-kernel streaming pass: 1 static partition,
+ *                         2 dynamic items with in-stream row completion
+ *   SV_KNOB_STREAM_W      two-kernel streaming chunk, a multiple of 1024 entries
+ *   SV_KNOB_WAIT_NS       time limit of every bounded wait of the chain kernel,
+ *                         in ns (default 1 s); a wait that runs out sets
+ *                         SV_DEV_TIMEOUT
+ *   SV_KNOB_STALL         1: the chain kernel's warp that reduces the first
+ *                         slice of request 0's first row waits on a barrier
+ *                         nothing arrives on, for a quarter of the wait limit,
+ *                         so that the wait runs out (a test of the timeout
+ *                         path: request 0 fails with SV_DEV_TIMEOUT, everything
+ *                         else completes)
+ *   SV_KNOB_STAGES        chain kernel ring stages per CTA, 2..8
+ *   SV_KNOB_ORDER         chain kernel tile order: 1 the tiles of a row
+ *                         consecutive, 2 the requests innermost
+ *   SV_KNOB_LEGACY        1: chain calls take the two-kernel path (stream pass +
+ *                         finishing clusters) that chains of k > 30 use
+ */
+#define SV_KNOB_CLUSTER_CTAS 1
+#define SV_KNOB_STREAM_COUNT 2
+#define SV_KNOB_STREAM_W 3
+#define SV_KNOB_WAIT_NS 4
+#define SV_KNOB_STALL 5
+#define SV_KNOB_STAGES 6
+#define SV_KNOB_ORDER 7
+#define SV_KNOB_LEGACY 8
+SV_API sv_status sv_set_knob(int knob, long long value);
 
 /* Map a device status word (read back by the caller) to a host status:
  * SV_OK, SV_ERR_TIMEOUT if SV_DEV_TIMEOUT is set, else SV_ERR_DEVICE_CHECK

@@ -35,7 +35,7 @@
  *         KL(p~ || q_theta); reading notes section 5 "G3 解法": w(r) = r by
  *         default, normalised and clipped in practice; GRPO group example.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent, each the plainest one the rest supports:
  *  - accept iff u*q(x) < p(x), u in [0,1) (strict: p(x)=0 always rejects);
  *  - one uniform per draft position (column i < k) plus one uniform (column k)
  *    for the single resample-or-bonus draw;

@@ -8,7 +8,7 @@ from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
 CSRC = PKG / "csrc"
-SOURCES = ["sv_api.cu"]
+SOURCES = ["sv_api.cu", "sv_chain_bf16.cu", "sv_chain_f32.cu"]
 LIB = PKG / "libsv.so"
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
@@ -34,7 +34,7 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 4) -> Path:
     for src in SOURCES:
         obj = objdir / (src + ".o")
         objs.append(obj)
-        cmd = [nvcc, *ARCH, *FLAGS, "-dc" if False else "-c", str(CSRC / src), "-o", str(obj)]
+        cmd = [nvcc, *ARCH, *FLAGS, "-c", str(CSRC / src), "-o", str(obj)]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))

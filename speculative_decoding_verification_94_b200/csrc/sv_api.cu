@@ -7,6 +7,7 @@
 
 #include <mutex>
 
+#include "sv_chain.cuh"
 #include "sv_finish.cuh"
 #include "sv_tree_sample.cuh"
 
@@ -20,13 +21,12 @@ constexpr int kMaxSmem = 200 * 1024;            // hard per-CTA limit used by pl
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int env_int(const char* name) {
-  const char* s = getenv(name);
-  return s ? atoi(s) : 0;
-}
+enum : int { kKnobClusterCtas = 1, kKnobStreamCount = 2, kKnobStreamW = 3, kKnobLegacy = 8,
+              kKnobCount = 16 };
+long long g_knobs[kKnobCount];
 
 int forced_cluster() {
-  const int c = env_int("SV_CLUSTER_CTAS");
+  const int c = (int)knob(kKnobClusterCtas);
   return (c >= 1 && c <= kMaxCluster) ? c : 0;
 }
 
@@ -85,6 +85,11 @@ std::mutex g_mu;
 
 }  // namespace
 
+long long knob(int id) {
+  if (id < 0 || id >= kKnobCount) return 0;
+  return __atomic_load_n(&g_knobs[id], __ATOMIC_RELAXED);
+}
+
 cudaError_t ensure_kernel_attrs(const void* kernel, int smem_bytes, bool nonportable) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -132,7 +137,7 @@ static cudaError_t blocks_per_sm(const void* kernel, int threads, int smem, int*
   return cudaSuccess;
 }
 
-static cudaError_t sm_count(int* out) {
+cudaError_t sm_count(int* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -154,7 +159,7 @@ static cudaError_t sm_count(int* out) {
 // keeps the tail of the dynamic schedule short.  It
 // depends on the sizes only, so workspace sizes are device independent.
 static int stream_chunk(int V, long long nrows) {
-  const int forced = env_int("SV_STREAM_W");
+  const int forced = (int)knob(kKnobStreamW);
   if (forced >= kPiece && forced % kPiece == 0) return forced;
   int w = kPiece;
   while (w < 8 * kPiece && (long long)V * nrows / (2 * w) >= 16384) w *= 2;
@@ -230,7 +235,7 @@ static StreamGeom stream_geom(int V, long long nrows, int te, int de) {
 // warps.  Otherwise the finisher completes the rows and the stream spends
 // nothing per item on counting.
 static int stream_count_policy(const StreamParams& p, long long resident_warps) {
-  const int forced = env_int("SV_STREAM_COUNT");
+  const int forced = (int)knob(kKnobStreamCount);
   if (forced == 1 || forced == 2) return forced - 1;  // 1: off, 2: on
   return (long long)p.B * p.nchunk >= 3 * resident_warps ? 1 : 0;
 }
@@ -398,10 +403,15 @@ static cudaError_t run_chain_sample(StreamParams sp, const StreamGeom& sg, Finis
 
 using namespace sv;
 
+// Chains of at most kChainMaxK drafts run as one persistent launch; longer
+// chains (or the legacy knob) take the two-kernel path.
+static bool chain_legacy(int k) { return k > kChainMaxK || knob(kKnobLegacy) != 0; }
+
 extern "C" {
 
 size_t sv_verify_chain_workspace_size(int B, int k, int V, int K) {
   if (B <= 0 || k < 1 || V < 1) return 256;
+  if (!chain_legacy(k)) return chain_ws_bytes(B, k, V, K > 0 ? K : 0);
   return ws_layout(B, B * (k + 1), record_slots(V), K > 0 ? K : 0).bytes;
 }
 size_t sv_verify_tree_workspace_size(int B, int n, int V) {
@@ -424,14 +434,15 @@ static sv_status check_workspace(void* ws, size_t bytes, size_t need) {
 
 }  // extern "C"
 
-// Chain verification, padded (draft_len == active == nullptr) or ragged.
-static sv_status verify_chain_impl(const void* target_logits, sv_dtype t_dtype, const void* draft,
-                                   sv_dtype d_dtype, sv_draft_kind d_kind,
-                                   const int32_t* draft_tokens, const float* uniforms,
-                                   const int32_t* draft_len, const int32_t* active, int B, int k,
-                                   int V, float temperature, int32_t* accepted_len,
-                                   int32_t* out_tokens, const sv_kd_args* kd, void* workspace,
-                                   size_t workspace_bytes, int32_t* device_status, void* stream) {
+// Host-side checks of a chain call, before anything touches the workspace
+// or the device (every chain entry point runs them first).
+static sv_status validate_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                                sv_dtype d_dtype, sv_draft_kind d_kind,
+                                const int32_t* draft_tokens, const float* uniforms,
+                                const int32_t* draft_len, const int32_t* active, int B, int k,
+                                int V, float temperature, int32_t* accepted_len,
+                                int32_t* out_tokens, const sv_kd_args* kd,
+                                int32_t* device_status) {
   if (B < 0 || k < 1 || k > 255 || V < 1) return SV_ERR_INVALID_ARG;
   if ((draft_len && !aligned(draft_len, 4)) || (active && !aligned(active, 4)))
     return SV_ERR_INVALID_ARG;
@@ -464,6 +475,49 @@ static sv_status verify_chain_impl(const void* target_logits, sv_dtype t_dtype, 
     if (!isfinite(kd->clip)) return SV_ERR_INVALID_ARG;
   }
   if (V > kMaxV) return SV_ERR_UNSUPPORTED;
+  if ((long long)B * (k + 1) > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
+  return SV_OK;
+}
+
+// Chain verification, padded (draft_len == active == nullptr) or ragged.
+static sv_status verify_chain_impl(const void* target_logits, sv_dtype t_dtype, const void* draft,
+                                   sv_dtype d_dtype, sv_draft_kind d_kind,
+                                   const int32_t* draft_tokens, const float* uniforms,
+                                   const int32_t* draft_len, const int32_t* active, int B, int k,
+                                   int V, float temperature, int32_t* accepted_len,
+                                   int32_t* out_tokens, const sv_kd_args* kd, void* workspace,
+                                   size_t workspace_bytes, int32_t* device_status, void* stream) {
+  sv_status vst = validate_chain(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens,
+                                 uniforms, draft_len, active, B, k, V, temperature, accepted_len,
+                                 out_tokens, kd, device_status);
+  if (vst != SV_OK || B == 0) return vst;
+  const bool greedy = temperature == 0.f;
+  if (!chain_legacy(k)) {
+    const sv_status st = check_workspace(
+        workspace, workspace_bytes, sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0));
+    if (st != SV_OK) return st;
+    ChainArgs ca;
+    ca.target = target_logits;
+    ca.t_dtype = t_dtype;
+    ca.draft = greedy ? nullptr : draft;
+    ca.d_dtype = d_dtype;
+    ca.d_kind = d_kind;
+    ca.tokens = draft_tokens;
+    ca.u = uniforms;
+    ca.klen = draft_len;
+    ca.active = active;
+    ca.B = B;
+    ca.k = k;
+    ca.V = V;
+    ca.temperature = temperature;
+    ca.accepted_len = accepted_len;
+    ca.out_tokens = out_tokens;
+    ca.kd = kd;
+    ca.workspace = workspace;
+    ca.status = device_status;
+    ca.stream = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(t_dtype == SV_BF16 ? launch_chain_bf16(ca) : launch_chain_f32(ca));
+  }
   const int P = k + 1;
   if ((long long)B * P > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
   const int K = kd ? kd->K : 0;
@@ -609,25 +663,10 @@ sv_status sv_verify_chain_ragged(const void* target_logits, sv_dtype t_dtype, co
 }
 
 // Scratch of sv_verify_chain_noalloc: one fixed, zero-initialised array per
-// device (every completed call returns it to zero), and its device address,
-// looked up once per device.
+// device (every completed call returns it to zero).  Its device address is
+// looked up on every call, in the calling thread's current context, so a
+// context created after a device reset is served correctly.
 static __device__ __align__(256) unsigned char g_noalloc_ws[SV_NOALLOC_MAX_BYTES];
-static void* g_noalloc_ptr[64];
-
-static sv_status noalloc_workspace(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SV_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return SV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || p == nullptr)
-      return SV_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
-  return SV_OK;
-}
 
 sv_status sv_verify_chain_noalloc(const void* target_logits, sv_dtype t_dtype, const void* draft,
                                   sv_dtype d_dtype, sv_draft_kind d_kind,
@@ -635,14 +674,31 @@ sv_status sv_verify_chain_noalloc(const void* target_logits, sv_dtype t_dtype, c
                                   int V, float temperature, int32_t* accepted_len,
                                   int32_t* out_tokens, const sv_kd_args* kd,
                                   int32_t* device_status, void* stream) {
+  // the same argument checks and codes as sv_verify_chain, first
+  const sv_status vst =
+      validate_chain(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens, uniforms,
+                     nullptr, nullptr, B, k, V, temperature, accepted_len, out_tokens, kd,
+                     device_status);
+  if (vst != SV_OK || B == 0) return vst;
   const size_t need = sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0);
   if (need > (size_t)SV_NOALLOC_MAX_BYTES) return SV_ERR_WORKSPACE;
   void* ws = nullptr;
-  const sv_status st = noalloc_workspace(&ws);
-  if (st != SV_OK) return st;
-  return sv_verify_chain(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens, uniforms, B,
-                         k, V, temperature, accepted_len, out_tokens, kd, ws,
-                         (size_t)SV_NOALLOC_MAX_BYTES, device_status, stream);
+  if (cudaGetSymbolAddress(&ws, g_noalloc_ws) != cudaSuccess || ws == nullptr) return SV_ERR_CUDA;
+  const sv_status st =
+      sv_verify_chain(target_logits, t_dtype, draft, d_dtype, d_kind, draft_tokens, uniforms, B, k,
+                      V, temperature, accepted_len, out_tokens, kd, ws,
+                      (size_t)SV_NOALLOC_MAX_BYTES, device_status, stream);
+  // A launch that failed part way (the two-kernel path) can leave the
+  // scratch in use: return it to zero on the same stream.
+  if (st == SV_ERR_CUDA)
+    cudaMemsetAsync(ws, 0, need, reinterpret_cast<cudaStream_t>(stream));
+  return st;
+}
+
+sv_status sv_set_knob(int knob_id, long long value) {
+  if (knob_id < 1 || knob_id >= kKnobCount) return SV_ERR_INVALID_ARG;
+  __atomic_store_n(&g_knobs[knob_id], value, __ATOMIC_RELAXED);
+  return SV_OK;
 }
 
 sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* node_tokens,
@@ -723,10 +779,7 @@ static cudaError_t run_tree_sample(FinishParams fp, int te, int de, bool bulk_ok
   const int rows_bytes = (int)sizeof(TreeShared) + 44 * fp.k;
   const int np = feasible_plans(
       fp.V, te, de,
-      [](int, int npc) {
-        const int x = npc * kThreads * 4 + kThreads * 8;
-        return x < 2 * kThreads * 4 ? 2 * kThreads * 4 : x;
-      },
+      [](int, int npc) { return npc * kThreads * 8 + kThreads * 8; },  // float64 sums, scan
       bulk_ok, rows_bytes, plans);
   if (np == 0) return cudaErrorInvalidConfiguration;
   auto kern = tree_sample_kernel<TT, DT, DKIND>;
@@ -776,6 +829,7 @@ sv_status sv_verify_tree_sample(const void* target_logits, sv_dtype t_dtype, con
   fp.V = V;
   fp.max_depth = max_depth;
   fp.c = (float)(1.4426950408889634 / (double)temperature);
+  fp.c64 = 1.4426950408889634 / (double)temperature;
   fp.accepted_len = accepted_len;
   fp.out_tokens = out_tokens;
   fp.accepted_nodes = accepted_nodes;

@@ -288,6 +288,31 @@ __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
+// 2^x in float64 to a few units in the last place: x = k + f with k the
+// nearest integer and |f| <= 1/2, 2^f = e^y with y = f ln 2 (|y| < 0.347)
+// summed as its Taylor series through y^12 (truncation below 1e-16
+// relative), then scaled by 2^k.  Results below 2^-1022 flush to 0 (every
+// caller's terms are relative to a maximum of order 1).
+__device__ __forceinline__ double exp2_f64(double x) {
+  if (!(x > -1022.0)) return 0.0;  // also -inf and NaN-free underflow
+  const double k = rint(x);
+  const double y = (x - k) * 0.693147180559945309417232121458;
+  double s = 1.0 / 479001600.0;             // 1/12!
+  s = fma(s, y, 1.0 / 39916800.0);          // 1/11!
+  s = fma(s, y, 1.0 / 3628800.0);           // 1/10!
+  s = fma(s, y, 1.0 / 362880.0);            // 1/9!
+  s = fma(s, y, 1.0 / 40320.0);             // 1/8!
+  s = fma(s, y, 1.0 / 5040.0);              // 1/7!
+  s = fma(s, y, 1.0 / 720.0);               // 1/6!
+  s = fma(s, y, 1.0 / 120.0);               // 1/5!
+  s = fma(s, y, 1.0 / 24.0);                // 1/4!
+  s = fma(s, y, 1.0 / 6.0);                 // 1/3!
+  s = fma(s, y, 0.5);                       // 1/2!
+  s = fma(s, y, 1.0);                       // 1/1!
+  s = fma(s, y, 1.0);                       // 1/0!
+  return s * __longlong_as_double((long long)((int)k + 1023) << 52);
+}
+
 // 2^x on the special-function unit (ex2.approx.ftz.f32).
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -32,6 +32,7 @@ struct FinishParams {
   int B, k, V, L, nchunk, K;
   int max_depth;
   float c;
+  double c64;  // log2(e) / T in float64 (sampling trees)
   int use_bulk;
   RowLayout lay;
   // outputs

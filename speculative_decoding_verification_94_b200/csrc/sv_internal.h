@@ -33,4 +33,37 @@ struct WsLayout {
   size_t off_glob, off_reject, off_counter, off_rec, off_part, off_cand, bytes;
 };
 
+// Process-wide test and tuning knobs (sv_set_knob; 0 = the library's choice).
+long long knob(int id);
+
+// Per-device helpers shared by the launchers (sv_api.cu).
+cudaError_t ensure_kernel_attrs(const void* kernel, int smem_bytes, bool nonportable);
+cudaError_t sm_count(int* out);
+
+// Chain verification in one persistent launch (sv_chain_*.cu): the
+// arguments of sv_verify_chain after validation, the workspace carved by
+// chain_ws_layout.
+struct ChainArgs {
+  const void* target;
+  int t_dtype;
+  const void* draft;
+  int d_dtype;
+  int d_kind;
+  const int32_t* tokens;
+  const float* u;
+  const int32_t* klen;
+  const int32_t* active;
+  int B, k, V;
+  float temperature;
+  int32_t* accepted_len;
+  int32_t* out_tokens;
+  const sv_kd_args* kd;
+  void* workspace;
+  int32_t* status;
+  cudaStream_t stream;
+};
+size_t chain_ws_bytes(int B, int k, int V, int K);
+cudaError_t launch_chain_bf16(const ChainArgs& a);
+cudaError_t launch_chain_f32(const ChainArgs& a);
+
 }  // namespace sv

@@ -48,26 +48,52 @@ struct TreeShared {
   int nkids, err, owner, tok, piece, first_thread, last_pos, pad;
 };
 
+// Residual weights max(0, p - sigma q) of 8 consecutive entries in float64:
+// p = 2^(zt c - Gt) / St, q likewise (or the given probability), with the
+// exponents, the powers and the difference in float64, so that the running
+// residual mass and the tests against it carry float64 rounding only (the
+// difference p - sigma q cancels where the two rows agree).
 template <class TT, class DT, int DKIND>
 __device__ __forceinline__ void tree_weights8(const unsigned char* tbuf, const unsigned char* dbuf,
-                                              int e, float c, float Gt, float invSt, float Gd,
-                                              float invSd, float sg, float w[8]) {
+                                              int e, double c, double Gt, double invSt,
+                                              double Gd, double invSd, double sg, double w[8]) {
   float zt[8];
   load8<TT>(tbuf, e, zt);
   float q[8];
-  if (DKIND == kDraftLogits) {
-    float zd[8];
-    load8<DT>(dbuf, e, zd);
+  if (DKIND == kDraftLogits) load8<DT>(dbuf, e, q);
+  else load8<F32>(dbuf, e, q);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) q[t] = __fmul_rn(ex2(fmaf(zd[t], c, -Gd)), invSd);
-  } else {
-    load8<F32>(dbuf, e, q);
+  for (int t = 0; t < 8; ++t) {
+    const double p = exp2_f64(fma((double)zt[t], c, -Gt)) * invSt;
+    const double qq =
+        DKIND == kDraftLogits ? exp2_f64(fma((double)q[t], c, -Gd)) * invSd : (double)q[t];
+    w[t] = fmax(fma(-sg, qq, p), 0.0);
   }
-  // p - sigma q with one rounding: exactly p at sigma = 0, and exactly 0 where
-  // p == q at sigma = 1
+}
+
+__device__ __forceinline__ double seq_sum8d(const double w[8]) {
+  double s = w[0];
 #pragma unroll
-  for (int t = 0; t < 8; ++t)
-    w[t] = fmaxf(__fmaf_rn(-sg, q[t], __fmul_rn(ex2(fmaf(zt[t], c, -Gt)), invSt)), 0.f);
+  for (int t = 1; t < 8; ++t) s += w[t];
+  return s;
+}
+
+// Per-piece totals of per-thread float64 sums sums[p * kThreads + t], in a
+// fixed order (warp butterflies, then warps in index order).  Collective.
+__device__ __forceinline__ void piece_totals_d(const double* sums, int npieces, RowShared& sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int p = 0; p < npieces; ++p) {
+    const double v = warp_sum(sums[p * kThreads + threadIdx.x]);
+    if (lane == 0) sh.wsum[w][p] = v;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < npieces) {
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < kWarps; ++q) t += sh.wsum[q][threadIdx.x];
+    sh.ptot[threadIdx.x] = t;
+  }
+  __syncthreads();
 }
 
 // Sampling tree verification: one cluster of C CTAs per request.
@@ -93,9 +119,10 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
   unsigned char* dbuf = smem + prm.lay.off_d;
   const int b = (int)(blockIdx.x / (unsigned)C);
   const ChunkGeom g = chunk_geom(rank, prm.L, V);
-  float* sums = reinterpret_cast<float*>(smem + prm.lay.off_x);
-  double* incl_arr = reinterpret_cast<double*>(sums + g.npieces * kThreads);
+  double* sums = reinterpret_cast<double*>(smem + prm.lay.off_x);
+  double* incl_arr = sums + g.npieces * kThreads;
   const float c = prm.c;
+  const double c64 = prm.c64;
   const bool use_bulk = prm.use_bulk != 0;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   pdl_wait();
@@ -158,20 +185,20 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
   // Chunk masses of the weights max(0, p - sg q) into sums[] and ts.part,
   // then the cluster total M and this CTA's share [lo, hi).  Collective over
   // the cluster.
-  auto residual_pass = [&](float sg, float Gt, float invSt, float Gd, float invSd) {
-#pragma unroll 4
+  auto residual_pass = [&](double sg, double Gt, double invSt, double Gd, double invSd) {
+#pragma unroll 2
     for (int p = 0; p < kMaxPieces; ++p) {
       if (p >= g.npieces) break;
       const int e = p * kRound + (int)threadIdx.x * kVec;
-      float s = 0.f;
+      double s = 0.0;
       if (e < g.nvec * kVec) {
-        float wv[8];
-        tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c, Gt, invSt, Gd, invSd, sg, wv);
-        s = seq_sum8(wv);
+        double wv[8];
+        tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c64, Gt, invSt, Gd, invSd, sg, wv);
+        s = seq_sum8d(wv);
       }
       sums[p * kThreads + threadIdx.x] = s;
     }
-    piece_totals(sums, g.npieces, sh);
+    piece_totals_d(sums, g.npieces, sh);
     const int slot = red & 1;
     ++red;
     if (threadIdx.x == 0) {
@@ -253,26 +280,34 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
           if (DKIND == kDraftLogits) md = fmaxf(md, max8<DT>(dbuf, e));
         }
       }
-      stat_cover(a, mt, c);
-      if (DKIND == kDraftLogits) stat_cover(d, md, c);
+      // integer references ceil(max z * c) in float64 (exact in fp32 too);
+      // the terms 2^(z c - ref) in float64
+      a.mz = mt;
+      a.ref = mt == -INFINITY ? -INFINITY : (float)ceil((double)mt * c64);
+      if (DKIND == kDraftLogits) {
+        d.mz = md;
+        d.ref = md == -INFINITY ? -INFINITY : (float)ceil((double)md * c64);
+      }
       const bool fa = a.ref != -INFINITY, fd = DKIND == kDraftLogits && d.ref != -INFINITY;
-#pragma unroll 4
+#pragma unroll 2
       for (int p = 0; p < kMaxPieces; ++p) {
         if (p >= g.npieces) break;
         const int e = p * kRound + (int)threadIdx.x * kVec;
         if (e < g.nvec * kVec) {
-          float z[8], t[8];
+          float z[8];
           if (fa) {
             load8<TT>(tbuf, e, z);
+            double t = 0.0;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t[k] = ex2(fmaf(z[k], c, -a.ref));
-            a.S += (double)(((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7])));
+            for (int k = 0; k < 8; ++k) t += exp2_f64(fma((double)z[k], c64, -(double)a.ref));
+            a.S += t;
           }
           if (fd) {
             load8<DT>(dbuf, e, z);
+            double t = 0.0;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t[k] = ex2(fmaf(z[k], c, -d.ref));
-            d.S += (double)(((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7])));
+            for (int k = 0; k < 8; ++k) t += exp2_f64(fma((double)z[k], c64, -(double)d.ref));
+            d.S += t;
           }
         }
       }
@@ -319,14 +354,14 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
 
     // c. the children's tests against the running residual (p(x) and q(x) of
     //    every child first, in parallel)
-    const float Gt = sh.Gt, Gd = sh.Gd;
-    const float invSt = (float)(1.0 / sh.St);
-    const float invSd = DKIND == kDraftLogits ? (float)(1.0 / sh.Sd) : 1.f;
+    const double Gt = (double)sh.Gt, Gd = (double)sh.Gd;
+    const double invSt = 1.0 / sh.St;
+    const double invSd = DKIND == kDraftLogits ? 1.0 / sh.Sd : 1.0;
     {
-      const double Lt = ts.Lt, Ld = ts.Ld, cd64 = (double)c;
       for (int i = threadIdx.x; i < ts.nkids; i += kThreads) {
-        kpx[i] = exp2((double)kzt[i] * cd64 - Lt);
-        kqx[i] = DKIND == kDraftLogits ? exp2((double)kzd[i] * cd64 - Ld) : (double)kzd[i];
+        kpx[i] = exp2_f64(fma((double)kzt[i], c64, -Gt)) * invSt;
+        kqx[i] = DKIND == kDraftLogits ? exp2_f64(fma((double)kzd[i], c64, -Gd)) * invSd
+                                       : (double)kzd[i];
       }
       __syncthreads();
     }
@@ -343,7 +378,7 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
         break;
       }
       sigma += M;
-      residual_pass((float)sigma, Gt, invSt, Gd, invSd);
+      residual_pass(sigma, Gt, invSt, Gd, invSd);
       M = ts.M;
       have = true;
       if (!(M > 0.0)) {  // zero residual mass: draw from the target row
@@ -365,7 +400,7 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
       sigma = 0.0;
       have = false;
     }
-    if (!have) residual_pass((float)sigma, Gt, invSt, Gd, invSd);
+    if (!have) residual_pass(sigma, Gt, invSt, Gd, invSd);
     if (threadIdx.x == 0) {
       ts.tt = (double)prm.u[(size_t)b * n] * ts.M;
       ts.owner = (ts.M > 0.0 && ts.lo <= ts.tt && ts.tt < ts.hi) ? 1 : 0;
@@ -404,28 +439,28 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
       __syncthreads();
       const int pp = ts.piece;
       if (pp >= 0) {
-        const float s = sums[pp * kThreads + threadIdx.x];
+        const double s = sums[pp * kThreads + threadIdx.x];
         double tot;
-        const double incl = block_scan_incl((double)s, sh.redd, &tot);
+        const double incl = block_scan_incl(s, sh.redd, &tot);
         incl_arr[threadIdx.x] = incl;
         if (ts.lo + incl > ts.tt) atomicMin(&ts.first_thread, (int)threadIdx.x);
-        if (s > 0.f) atomicMax(&ts.last_pos, (int)threadIdx.x);
+        if (s > 0.0) atomicMax(&ts.last_pos, (int)threadIdx.x);
         __syncthreads();
         int tsel = ts.first_thread;
         const bool fb = (tsel == kThreads);
         if (fb) tsel = ts.last_pos;
         if ((int)threadIdx.x == tsel) {
           const int e = pp * kRound + tsel * kVec;
-          float wv[8];
-          tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c, Gt, invSt, Gd, invSd, (float)sigma, wv);
+          double wv[8];
+          tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c64, Gt, invSt, Gd, invSd, sigma, wv);
           const double b0 = ts.lo + (tsel > 0 ? incl_arr[tsel - 1] : 0.0);
-          float acc = 0.f;
+          double acc = 0.0;
           int pick = -1, lastq = -1;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            acc = __fadd_rn(acc, wv[q]);
-            if (wv[q] > 0.f) lastq = q;
-            if (!fb && pick < 0 && b0 + (double)acc > ts.tt) pick = q;
+            acc += wv[q];
+            if (wv[q] > 0.0) lastq = q;
+            if (!fb && pick < 0 && b0 + acc > ts.tt) pick = q;
           }
           if (pick < 0) pick = lastq;
           ts.tok = pick < 0 ? -1 : g.j0 + e + pick;

@@ -26,7 +26,10 @@ SV_DEV_BAD_TOKEN, SV_DEV_NO_FINITE, SV_DEV_TIMEOUT, SV_DEV_BAD_TREE = 0x1, 0x2, 
 SV_DEV_BAD_INDEX, SV_DEV_BAD_LEN, SV_DEV_ERROR_MASK = 0x10, 0x20, 0xFF
 SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
-EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc",
+SV_KNOB_CLUSTER_CTAS, SV_KNOB_STREAM_COUNT, SV_KNOB_STREAM_W, SV_KNOB_WAIT_NS = 1, 2, 3, 4
+SV_KNOB_STALL, SV_KNOB_STAGES, SV_KNOB_ORDER, SV_KNOB_LEGACY = 5, 6, 7, 8
+
+EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc", "sv_set_knob",
            "sv_verify_tree_greedy", "sv_kd_grad", "sv_kd_grad_workspace_size",
            "sv_verify_tree_sample", "sv_extract_topk_kd", "sv_kd_kl_loss", "sv_sched_select",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
@@ -101,12 +104,36 @@ def lib() -> ctypes.CDLL:
             L.sv_verify_tree_sample.restype = ci
             L.sv_sched_select.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp]
             L.sv_sched_select.restype = ci
+            L.sv_set_knob.argtypes = [ci, ctypes.c_longlong]
+            L.sv_set_knob.restype = ci
             L.sv_status_string.argtypes = [ci]
             L.sv_status_string.restype = ctypes.c_char_p
             L.sv_version.argtypes = []
             L.sv_version.restype = ci
             _lib = L
     return _lib
+
+
+def sv_set_knob(knob: int, value: int) -> None:
+    """Process-wide test / tuning setting (see sv.h); 0 restores the default."""
+    _check(lib().sv_set_knob(int(knob), int(value)), "sv_set_knob")
+
+
+class knobs:
+    """Context manager: set knobs {id: value} for the block, then restore 0."""
+
+    def __init__(self, **kw):
+        self.kw = {globals()["SV_KNOB_" + k.upper()]: v for k, v in kw.items()}
+
+    def __enter__(self):
+        for k, v in self.kw.items():
+            sv_set_knob(k, v)
+        return self
+
+    def __exit__(self, *exc):
+        for k in self.kw:
+            sv_set_knob(k, 0)
+        return False
 
 
 def status_string(status: int) -> str:

@@ -96,6 +96,13 @@ def assert_kd_match(got: dict, ref: dict, k: int):
     kl = got["kl"].cpu().numpy()
     assert_close(kl[dmask], ref["kl"][dmask], ref["scale"][dmask], "kl")
     assert np.isnan(kl[~dmask]).all()
+    # the error actually reached, relative to |KL| itself (the bar's scale
+    # above is the larger of |KL| and sum p~ |ln q|)
+    r, g = ref["kl"][dmask], kl[dmask].astype(np.float64)
+    nz = np.abs(r) > 0
+    if nz.any():
+        print(f"kl: worst error {float(np.max(np.abs(g[nz] - r[nz]) / np.abs(r[nz]))):.3e} "
+              f"of |KL| over {int(nz.sum())} rows")
 
 
 def bitwise_equal(a, b) -> bool:

@@ -178,3 +178,37 @@ def test_ragged_chain_and_sampling_tree_validate(lib):
     assert tree(d=ctypes.c_void_p(0x10001)) == E  # misaligned bf16 row
     assert tree(V=600000) == sv.SV_ERR_UNSUPPORTED
     assert tree(B=0) == sv.SV_OK                 # nothing to do, nothing enqueued
+
+
+def _noalloc(lib, **kw):
+    a = dict(target=FAKE, tdt=sv.SV_BF16, draft=FAKE, ddt=sv.SV_BF16, dk=sv.SV_DRAFT_LOGITS,
+             tok=FAKE, u=FAKE, B=4, k=3, V=1024, T=1.0, acc=FAKE, out=FAKE, kd=None,
+             status=None, stream=None)
+    a.update(kw)
+    return lib.sv_verify_chain_noalloc(a["target"], a["tdt"], a["draft"], a["ddt"], a["dk"],
+                                       a["tok"], a["u"], a["B"], a["k"], a["V"], a["T"],
+                                       a["acc"], a["out"], a["kd"], a["status"], a["stream"])
+
+
+@no_gpu
+def test_noalloc_checks_arguments_like_the_workspace_call(lib):
+    """Bad arguments give sv_verify_chain's code, not a scratch-size error,
+    even where the declared sizes would also overflow the fixed scratch."""
+    big = dict(B=4096, V=151936)
+    kd = sv.sv_kd_args(1000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0, 1, 0.0, 0x10000,
+                       0x10000)
+    for kw in (dict(kd=ctypes.byref(kd)), dict(k=300), dict(k=0), dict(T=-1.0),
+               dict(dk=sv.SV_DRAFT_PROBS, ddt=sv.SV_BF16), dict(V=600000)):
+        args = dict(big, **kw)
+        want = _chain(lib, wsb=1 << 40, **args)
+        assert want != sv.SV_OK
+        assert _noalloc(lib, **args) == want, kw
+    # valid arguments beyond the scratch: the size check answers
+    assert _noalloc(lib, **big) == sv.SV_ERR_WORKSPACE
+    assert _noalloc(lib, B=0) == sv.SV_OK
+
+
+def test_knobs_validate(lib):
+    assert lib.sv_set_knob(0, 1) == sv.SV_ERR_INVALID_ARG
+    assert lib.sv_set_knob(99, 1) == sv.SV_ERR_INVALID_ARG
+    assert lib.sv_set_knob(sv.SV_KNOB_STAGES, 0) == sv.SV_OK

@@ -59,10 +59,19 @@ def _check_idle(got, act):
     assert (out[act == 0] == -1).all()
 
 
-@pytest.mark.parametrize("count", ["1", "2"])
+PATHS = {"fused": {}, "fused-order2": dict(order=2),
+         "legacy-static": dict(legacy=1, stream_count=1),
+         "legacy-dynamic": dict(legacy=1, stream_count=2)}
+
+
+@pytest.fixture(params=list(PATHS))
+def path(request):
+    with sv.knobs(**PATHS[request.param]):
+        yield request.param
+
+
 @pytest.mark.parametrize("k,sigma", [(3, 1.0), (5, 0.5)])
-def test_ragged_sampling_chain(monkeypatch, count, k, sigma):
-    monkeypatch.setenv("SV_STREAM_COUNT", count)
+def test_ragged_sampling_chain(path, k, sigma):
     x = inputs.qwen_chain(B=32, k=k, sigma_d=sigma, seed=40 + k)
     klen, act = _lengths(x.B, k, seed=k)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -78,9 +87,7 @@ def test_ragged_sampling_chain(monkeypatch, count, k, sigma):
     assert int(torch.count_nonzero(ws)) == 0
 
 
-@pytest.mark.parametrize("count", ["1", "2"])
-def test_ragged_greedy_chain(monkeypatch, count):
-    monkeypatch.setenv("SV_STREAM_COUNT", count)
+def test_ragged_greedy_chain(path):
     x = inputs.make_chain(40, 4, 70001, dtype="bf16", sigma_d=0.3, temperature=0.0, seed=12)
     klen, act = _lengths(x.B, x.k, seed=3)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -93,12 +100,10 @@ def test_ragged_greedy_chain(monkeypatch, count):
     assert len(set(ref["accepted_len"][act == 1].tolist())) > 1
 
 
-@pytest.mark.parametrize("count", ["1", "2"])
-def test_ragged_fused_kd(monkeypatch, count):
+def test_ragged_fused_kd(path):
     """Fused KD on a ragged batch: rows 0..n of each active request defined,
     no KL for the bonus row k_b, idle requests empty, loss with n < k_b for
     the first-rejected-position rule."""
-    monkeypatch.setenv("SV_STREAM_COUNT", count)
     x = inputs.kd_chain(B=48, k=4, seed=3)
     klen, act = _lengths(x.B, x.k, seed=11)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)

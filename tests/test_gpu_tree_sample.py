@@ -3,12 +3,11 @@ oracle, and its losslessness on the GPU.
 
 Integers must match exactly except for requests whose decisions lie near a
 boundary in the oracle's exact arithmetic: a child test with
-|u - r(x)/q(x)| < 1e-5, or a draw within 1e-5 of an inverse-CDF step.  The
-kernel forms the residual max(0, p - sigma q) from fp32 terms (ex2.approx,
-about 2^-22 relative each) whose total is compared with u times a mass that
-can be well below 1 after several rejections, so its decisions carry
-roughly ten times the error of the chain's; such requests are counted and
-checked for well-formed outputs only."""
+|u - r(x)/q(x)| < 1e-6, or a draw within 1e-6 of an inverse-CDF step (the
+chain's window).  The kernel forms the row statistics, p(x), q(x), the
+residual max(0, p - sigma q) and its mass in float64, so the running residual
+carries float64 rounding although p - sigma q cancels where the rows agree;
+flagged requests are counted and checked for well-formed outputs only."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +18,7 @@ from speculative_decoding_verification_94_b200 import inputs, sv
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-WINDOW = 1e-5
+WINDOW = 1e-6
 
 
 def _run(x, draft=None, kind="logits", status=None):
@@ -64,8 +63,12 @@ def test_tree_sample_full_vocabulary():
 
 
 @pytest.mark.parametrize("ctas", ["1", "2", "5", "16"])
-def test_tree_sample_cluster_sizes(monkeypatch, ctas):
-    monkeypatch.setenv("SV_CLUSTER_CTAS", ctas)
+def test_tree_sample_cluster_sizes(ctas):
+    with sv.knobs(cluster_ctas=int(ctas)):
+        _tree_cluster_case()
+
+
+def _tree_cluster_case():
     x = inputs.make_tree_sample(B=24, V=20000, depth_counts=(4, 4, 3), branching=4,
                                 sigma_d=0.7, temperature=0.9, seed=5)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)

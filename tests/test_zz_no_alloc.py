@@ -49,7 +49,7 @@ def test_noalloc_fused_kd_matches_twice_in_a_row():
 
 
 def test_noalloc_rejects_a_batch_beyond_its_scratch():
-    B, k, V = 256, 3, 151936
+    B, k, V = 1024, 3, 151936
     assert sv.sv_verify_chain_workspace_size(B, k, V, 0) > (4 << 20)
     x = inputs.make_chain(B, k, 1024, dtype="bf16", seed=13)  # small tensors, large declared V
     t = torch.zeros(B, k + 1, V, dtype=torch.bfloat16, device=DEV)
@@ -57,3 +57,25 @@ def test_noalloc_rejects_a_batch_beyond_its_scratch():
     with pytest.raises(sv.SVError) as e:
         sv.sv_verify_chain_noalloc(t, d, x.draft_tokens.to(DEV), x.uniforms.to(DEV), 0.7)
     assert e.value.status == sv.SV_ERR_WORKSPACE
+
+
+def test_noalloc_scratch_returns_to_zero_after_a_failed_request():
+    """A call whose request 1 carries an out-of-range draft token (checked on
+    the device, reported in the status word) must leave the fixed scratch as
+    zero as a clean call does: the next call matches sv_verify_chain bit for
+    bit."""
+    x = inputs.qwen_chain(B=16, k=3, sigma_d=1.0, seed=14)
+    bad = x.draft_tokens.clone()
+    bad[1, 0] = x.V  # outside [0, V)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    got = sv.sv_verify_chain_noalloc(x.target.to(DEV), x.draft.to(DEV), bad.to(DEV),
+                                     x.uniforms.to(DEV), x.temperature, device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & sv.SV_DEV_BAD_TOKEN
+    assert got["accepted_len"][1].item() == -1
+    assert (got["out_tokens"][1] == -1).all()
+    ref = _chain(sv.sv_verify_chain, x)
+    for _ in range(2):
+        good = _chain(sv.sv_verify_chain_noalloc, x)
+        assert torch.equal(good["accepted_len"], ref["accepted_len"])
+        assert torch.equal(good["out_tokens"], ref["out_tokens"])
