@@ -158,8 +158,9 @@ SV_API size_t sv_kd_kl_loss_workspace_size(int B, int k, int V);
  * Verification is sequential within a request: a draft after the first
  * rejection is never tested.  Rows are streamed position-major and a row whose
  * request has already rejected at an earlier position is skipped before it is
- * loaded, so the bytes read approach the rows the outcome depends on.  Chains
- * of k <= 30 drafts run as one kernel launch; longer ones as two.
+ * loaded, so the bytes read approach the rows the outcome depends on.  A call
+ * is two kernel launches (a streaming pass, then per-request finishing
+ * clusters); SV_KNOB_PERSISTENT makes chains of k <= 30 one persistent launch.
  *   device_status optional int32 status word (SV_DEV_* bits).
  */
 SV_API sv_status sv_verify_chain(const void* target_logits, sv_dtype t_dtype, const void* draft,
@@ -221,8 +222,9 @@ SV_API sv_status sv_verify_chain_ragged(const void* target_logits, sv_dtype t_dt
  *   capture.
  *   A call whose sv_verify_chain_workspace_size(B, k, V, kd ? kd->K : 0)
  *   exceeds SV_NOALLOC_MAX_BYTES returns SV_ERR_WORKSPACE and launches
- *   nothing.  At V = 151936 that allows about B*(k+1) <= 3500 target rows
- *   without KD and about 700 with K = 32 (k <= 30).
+ *   nothing.  At V = 151936 (k = 3) that allows about B*(k+1) <= 580 target
+ *   rows without KD and about 90 with K = 32 on the default path; about 1450
+ *   and 520 with SV_KNOB_PERSISTENT set.
  *   The array starts zero-filled and every completed call returns it to zero,
  *   including calls whose requests fail a device check; a call that returns
  *   SV_ERR_CUDA after a partial launch clears it with an asynchronous memset
@@ -391,8 +393,11 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
  *   SV_KNOB_STAGES        chain kernel ring stages per CTA, 2..8
  *   SV_KNOB_ORDER         chain kernel tile order: 1 the tiles of a row
  *                         consecutive, 2 the requests innermost
- *   SV_KNOB_LEGACY        1: chain calls take the two-kernel path (stream pass +
- *                         finishing clusters) that chains of k > 30 use
+ *   SV_KNOB_PERSISTENT    1: chain calls with k <= 30 run as one persistent
+ *                         launch (streaming, early exit, residual and bonus
+ *                         draws and request completion in one grid); 0, the
+ *                         default, the two-kernel path (stream pass, then
+ *                         finishing clusters), which is faster on B200 today
  */
 #define SV_KNOB_CLUSTER_CTAS 1
 #define SV_KNOB_STREAM_COUNT 2
@@ -401,7 +406,7 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
 #define SV_KNOB_STALL 5
 #define SV_KNOB_STAGES 6
 #define SV_KNOB_ORDER 7
-#define SV_KNOB_LEGACY 8
+#define SV_KNOB_PERSISTENT 8
 SV_API sv_status sv_set_knob(int knob, long long value);
 
 /* Map a device status word (read back by the caller) to a host status:

@@ -21,7 +21,7 @@ constexpr int kMaxSmem = 200 * 1024;            // hard per-CTA limit used by pl
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-enum : int { kKnobClusterCtas = 1, kKnobStreamCount = 2, kKnobStreamW = 3, kKnobLegacy = 8,
+enum : int { kKnobClusterCtas = 1, kKnobStreamCount = 2, kKnobStreamW = 3, kKnobPersistent = 8,
               kKnobCount = 16 };
 long long g_knobs[kKnobCount];
 
@@ -405,7 +405,7 @@ using namespace sv;
 
 // Chains of at most kChainMaxK drafts run as one persistent launch; longer
 // chains (or the legacy knob) take the two-kernel path.
-static bool chain_legacy(int k) { return k > kChainMaxK || knob(kKnobLegacy) != 0; }
+static bool chain_legacy(int k) { return k > kChainMaxK || knob(kKnobPersistent) == 0; }
 
 extern "C" {
 

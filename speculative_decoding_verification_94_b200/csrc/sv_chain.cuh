@@ -48,11 +48,19 @@ namespace sv {
 #define SV_CHAIN_CW 16
 #endif
 constexpr int kCW = SV_CHAIN_CW;             // consumer warps per CTA
-constexpr int kChainThreads = (kCW + 2) * 32;  // + the producer warp and the manager warp
+// + the producer warp, the counter warp and the completer warp
+constexpr int kChainThreads = (kCW + 3) * 32;
 constexpr int kTaskQ = 256;                  // completion tasks queued per CTA
 constexpr int kTileW = 8192;                 // vocabulary entries per tile and row
-constexpr int kSliceW = kTileW / kCW;        // entries per consumer warp
-constexpr int kVPL = kSliceW / (32 * kVec);  // 8-entry vectors per lane
+constexpr int kRowW = kCW / 2;               // warps per row when a tile holds a row pair
+constexpr int kSliceP = kTileW / kRowW;      // entries per warp, one row of a pair tile
+constexpr int kVPLP = kSliceP / (32 * kVec); // 8-entry vectors per lane for those
+constexpr int kSliceW = kTileW / kCW;        // entries per warp, target-only and draw tiles
+constexpr int kVPL = kSliceW / (32 * kVec);  // 8-entry vectors per lane for those
+#ifndef SV_CHAIN_CLAIM
+#define SV_CHAIN_CLAIM 2
+#endif
+constexpr int kClaim = SV_CHAIN_CLAIM;       // stream tiles claimed per atomic
 constexpr int kMaxStagesC = 8;
 constexpr int kChainMaxK = 30;               // drafts per request (state word: 31 rows)
 
@@ -190,6 +198,19 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ unsigned long long atom_or_acq_rel_u64(unsigned long long* p,
+                                                              unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.or.b64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void red_or_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.or.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // A 16-byte-aligned record written by another SM, read through L2.
 template <class T>
 __device__ __forceinline__ T ldcg_rec(const T* src) {
@@ -208,6 +229,19 @@ __device__ __forceinline__ uint32_t mbar_try_wait_spin(uint64_t* bar, uint32_t p
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok;
+}
+
+// Non-blocking test of phase `parity` of an mbarrier.
+__device__ __forceinline__ uint32_t mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, P;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -287,29 +321,30 @@ __device__ __forceinline__ const unsigned char* chain_row(const void* base, size
 // slice length) read as `pad`.  From shared memory (bulk path, 16-byte
 // aligned rows) or straight from global memory (scalar path).
 // ---------------------------------------------------------------------------
-template <class T>
+template <class T, int NV>
 struct Slice;
-template <>
-struct Slice<BF16> {
-  uint4 w[kVPL];
+template <int NV>
+struct Slice<BF16, NV> {
+  uint4 w[NV];
 };
-template <>
-struct Slice<F32> {
-  float4 w[2 * kVPL];
+template <int NV>
+struct Slice<F32, NV> {
+  float4 w[2 * NV];
 };
 
+template <int NV>
 __device__ __forceinline__ void slice_load(const unsigned char* src, int n, bool smem, float pad,
-                                           Slice<BF16>& R) {
+                                           Slice<BF16, NV>& R) {
   const int lane = threadIdx.x & 31;
   const uint16_t pb = (uint16_t)(__float_as_uint(pad) >> 16);
-  if (smem && n >= kSliceW) {
+  if (smem && n >= NV * 256) {
 #pragma unroll
-    for (int v = 0; v < kVPL; ++v)
+    for (int v = 0; v < NV; ++v)
       R.w[v] = *reinterpret_cast<const uint4*>(src + (size_t)(v * 32 + lane) * 16);
     return;
   }
 #pragma unroll
-  for (int v = 0; v < kVPL; ++v) {
+  for (int v = 0; v < NV; ++v) {
     const int e = (v * 32 + lane) * kVec;
     if (smem && e + kVec <= n) {
       R.w[v] = *reinterpret_cast<const uint4*>(src + (size_t)e * 2);
@@ -324,19 +359,20 @@ __device__ __forceinline__ void slice_load(const unsigned char* src, int n, bool
   }
 }
 
+template <int NV>
 __device__ __forceinline__ void slice_load(const unsigned char* src, int n, bool smem, float pad,
-                                           Slice<F32>& R) {
+                                           Slice<F32, NV>& R) {
   const int lane = threadIdx.x & 31;
-  if (smem && n >= kSliceW) {
+  if (smem && n >= NV * 256) {
 #pragma unroll
-    for (int v = 0; v < kVPL; ++v) {
+    for (int v = 0; v < NV; ++v) {
       R.w[2 * v] = *reinterpret_cast<const float4*>(src + (size_t)(v * 32 + lane) * 32);
       R.w[2 * v + 1] = *reinterpret_cast<const float4*>(src + (size_t)(v * 32 + lane) * 32 + 16);
     }
     return;
   }
 #pragma unroll
-  for (int v = 0; v < kVPL; ++v) {
+  for (int v = 0; v < NV; ++v) {
     const int e = (v * 32 + lane) * kVec;
     float h[kVec];
 #pragma unroll
@@ -347,69 +383,77 @@ __device__ __forceinline__ void slice_load(const unsigned char* src, int n, bool
   }
 }
 
-__device__ __forceinline__ float slice_elem(const Slice<BF16>& R, int v, int t) {
+template <int NV>
+__device__ __forceinline__ float slice_elem(const Slice<BF16, NV>& R, int v, int t) {
   const uint32_t w = (t >> 1) == 0 ? R.w[v].x : (t >> 1) == 1 ? R.w[v].y : (t >> 1) == 2 ? R.w[v].z
                                                                                        : R.w[v].w;
   return (t & 1) ? bf16_hi(w) : bf16_lo(w);
 }
-__device__ __forceinline__ float slice_elem(const Slice<F32>& R, int v, int t) {
+template <int NV>
+__device__ __forceinline__ float slice_elem(const Slice<F32, NV>& R, int v, int t) {
   const float4 q = R.w[2 * v + (t >> 2)];
   const int u = t & 3;
   return u == 0 ? q.x : u == 1 ? q.y : u == 2 ? q.z : q.w;
 }
 
-__device__ __forceinline__ float slice_vmax(const Slice<BF16>& R, int v) {
+template <int NV>
+__device__ __forceinline__ float slice_vmax(const Slice<BF16, NV>& R, int v) {
   const uint32_t m = bmax2(bmax2(R.w[v].x, R.w[v].y), bmax2(R.w[v].z, R.w[v].w));
   return fmaxf(bf16_lo(m), bf16_hi(m));
 }
-__device__ __forceinline__ float slice_vmax(const Slice<F32>& R, int v) {
+template <int NV>
+__device__ __forceinline__ float slice_vmax(const Slice<F32, NV>& R, int v) {
   const float4 a = R.w[2 * v], b = R.w[2 * v + 1];
   return fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(b.x, b.y), fmaxf(b.z, b.w)));
 }
-__device__ __forceinline__ float slice_max(const Slice<BF16>& R) {
+template <int NV>
+__device__ __forceinline__ float slice_max(const Slice<BF16, NV>& R) {
   uint32_t m = bmax2(bmax2(R.w[0].x, R.w[0].y), bmax2(R.w[0].z, R.w[0].w));
 #pragma unroll
-  for (int v = 1; v < kVPL; ++v)
+  for (int v = 1; v < NV; ++v)
     m = bmax2(m, bmax2(bmax2(R.w[v].x, R.w[v].y), bmax2(R.w[v].z, R.w[v].w)));
   return fmaxf(bf16_lo(m), bf16_hi(m));
 }
-__device__ __forceinline__ float slice_max(const Slice<F32>& R) {
+template <int NV>
+__device__ __forceinline__ float slice_max(const Slice<F32, NV>& R) {
   float m = slice_vmax(R, 0);
 #pragma unroll
-  for (int v = 1; v < kVPL; ++v) m = fmaxf(m, slice_vmax(R, v));
+  for (int v = 1; v < NV; ++v) m = fmaxf(m, slice_vmax(R, v));
   return m;
 }
 
 // Sum over the lane's entries of 2^(z c - ref): packed fma, two exp2, and a
 // fixed tree of packed adds.
-__device__ __forceinline__ float slice_terms(const Slice<BF16>& R, float c, float ref) {
+template <int NV>
+__device__ __forceinline__ float slice_terms(const Slice<BF16, NV>& R, float c, float ref) {
   const unsigned long long cc = f2_pack(c, c), nr = f2_pack(-ref, -ref);
-  unsigned long long e[4 * kVPL];
+  unsigned long long e[4 * NV];
 #pragma unroll
-  for (int v = 0; v < kVPL; ++v) {
+  for (int v = 0; v < NV; ++v) {
     e[4 * v + 0] = term2(bf16_lo(R.w[v].x), bf16_hi(R.w[v].x), cc, nr);
     e[4 * v + 1] = term2(bf16_lo(R.w[v].y), bf16_hi(R.w[v].y), cc, nr);
     e[4 * v + 2] = term2(bf16_lo(R.w[v].z), bf16_hi(R.w[v].z), cc, nr);
     e[4 * v + 3] = term2(bf16_lo(R.w[v].w), bf16_hi(R.w[v].w), cc, nr);
   }
 #pragma unroll
-  for (int w = 2 * kVPL; w >= 1; w >>= 1)
+  for (int w = 2 * NV; w >= 1; w >>= 1)
 #pragma unroll
     for (int t = 0; t < w; ++t) e[t] = f2_add(e[t], e[t + w]);
   float lo, hi;
   f2_unpack(e[0], lo, hi);
   return lo + hi;
 }
-__device__ __forceinline__ float slice_terms(const Slice<F32>& R, float c, float ref) {
+template <int NV>
+__device__ __forceinline__ float slice_terms(const Slice<F32, NV>& R, float c, float ref) {
   const unsigned long long cc = f2_pack(c, c), nr = f2_pack(-ref, -ref);
-  unsigned long long e[4 * kVPL];
+  unsigned long long e[4 * NV];
 #pragma unroll
-  for (int v = 0; v < 2 * kVPL; ++v) {
+  for (int v = 0; v < 2 * NV; ++v) {
     e[2 * v + 0] = term2(R.w[v].x, R.w[v].y, cc, nr);
     e[2 * v + 1] = term2(R.w[v].z, R.w[v].w, cc, nr);
   }
 #pragma unroll
-  for (int w = 2 * kVPL; w >= 1; w >>= 1)
+  for (int w = 2 * NV; w >= 1; w >>= 1)
 #pragma unroll
     for (int t = 0; t < w; ++t) e[t] = f2_add(e[t], e[t + w]);
   float lo, hi;
@@ -417,18 +461,22 @@ __device__ __forceinline__ float slice_terms(const Slice<F32>& R, float c, float
   return lo + hi;
 }
 
-// One row of a slice into a warp partial: exponent reference G (max over
-// lanes) and S = sum 2^(z c - G) (float64 across lanes).
-template <class T>
-__device__ __forceinline__ void slice_stats(const Slice<T>& R, float pm, float c, float* G,
+// One row of a slice into a warp partial, against one reference for the
+// warp: G = ceil(c * the slice maximum) (an integer, so later rescales are
+// exact powers of two) and S = sum 2^(z c - G), fp32 per lane, float64 across
+// the warp.  pm: the lane's maximum.
+template <class T, int NV>
+__device__ __forceinline__ void slice_stats(const Slice<T, NV>& R, float pm, float c, float* G,
                                             double* S) {
-  ThreadStat st;
-  stat_init(st);
-  stat_cover(st, pm, c);
-  if (pm != -INFINITY) st.S = (double)slice_terms(R, c, st.ref);
-  const float g = warp_max_redux(st.ref);
+  const float wm = warp_max_redux(pm);
+  if (wm == -INFINITY) {
+    *G = -INFINITY;
+    *S = 0.0;
+    return;
+  }
+  const float g = ceilf(wm * c);
   *G = g;
-  *S = warp_sum(rescale_pow2(st.S, st.ref, g));
+  *S = warp_sum((double)slice_terms(R, c, g));
 }
 
 // ---------------------------------------------------------------------------
@@ -665,10 +713,7 @@ __device__ __noinline__ void chain_write_outputs(const ChainParams& p, int b, in
   __syncwarp();
   for (int i = 0; i < nz; ++i) zero_row<KD>(p, b, i);
   __syncwarp();
-  if (lane == 0) {
-    fence_acq_rel_gpu();
-    atomicOr(&p.req_state[b], kFinalBit);
-  }
+  if (lane == 0) red_or_release_u64(&p.req_state[b], kFinalBit);
 }
 
 // ---------------------------------------------------------------------------
@@ -845,8 +890,8 @@ __device__ __noinline__ void chain_finish_request(const ChainParams& p, int b, i
       d.invSt = (float)(1.0 / rn.S0);
       d.invSd = (MODE == kCMSample) ? (float)(1.0 / rn.S1) : 1.f;
       p.jobs[j] = d;
-      fence_acq_rel_gpu();
     }
+    __syncwarp();  // the job record before every lane's release of an entry
     j = __shfl_sync(0xffffffffu, j, 0);
     // each tile's queue entry names the row pair, so that a producer can
     // issue the copies as soon as it sees the entry
@@ -854,10 +899,7 @@ __device__ __noinline__ void chain_finish_request(const ChainParams& p, int b, i
     for (int q = lane; q < p.NT; q += 32) st_release_u32(&p.drawq[(size_t)j * p.NT + q], flag);
   }
   __syncwarp();
-  if (lane == 0) {
-    fence_acq_rel_gpu();
-    atomicAdd(&p.glob[kGDet], 1u);
-  }
+  if (lane == 0) red_add_release_u32(&p.glob[kGDet], 1u);
 }
 
 // ---------------------------------------------------------------------------
@@ -870,6 +912,9 @@ __device__ __noinline__ void chain_complete_row(const ChainParams& p, int b, int
   const int lane = threadIdx.x & 31;
   const int r = b * p.P + i, NT = p.NT, V = p.V;
   const bool has_draft = (MODE == kCMSample) && i < kb;
+  // the loads the decision needs, issued with the records'
+  const int x = i < kb ? __ldg(&p.tokens[(size_t)b * p.k + i]) : -1;
+  const float u_i = (MODE != kCMGreedy && i < kb) ? __ldg(&p.u[(size_t)b * p.P + i]) : 0.f;
   float g0 = -INFINITY, g1 = -INFINITY, zx0 = 0.f, zx1 = 0.f;
   double s0 = 0.0, s1 = 0.0;
   int flags = 0, hx = 0;
@@ -911,7 +956,6 @@ __device__ __noinline__ void chain_complete_row(const ChainParams& p, int b, int
   rec.L0 = (double)rec.G0 + log2(rec.S0);
   rec.L1 = (double)rec.G1 + log2(rec.S1);
   rec.argmax = key_index(key);
-  const int x = i < kb ? __ldg(&p.tokens[(size_t)b * p.k + i]) : -1;
   int err = 0, code = kRowAccepted;
   if (flags & kPTimeout) err |= SV_DEV_TIMEOUT;
   if (MODE != kCMGreedy && rec.G0 == -INFINITY) err |= SV_DEV_NO_FINITE;
@@ -928,7 +972,7 @@ __device__ __noinline__ void chain_complete_row(const ChainParams& p, int b, int
             (MODE == kCMSample)
                 ? exp2((double)zx1 * cc - rec.L1)
                 : (double)__ldg(reinterpret_cast<const float*>(p.draft) + ((size_t)b * p.k + i) * V + x);
-        const double uu = (double)__ldg(&p.u[(size_t)b * p.P + i]);
+        const double uu = (double)u_i;
         code = (uu * qx < px) ? kRowAccepted : kRowRejected;
       }
     }
@@ -1010,20 +1054,19 @@ __device__ __noinline__ void chain_complete_row(const ChainParams& p, int b, int
   if (!(MODE != kCMGreedy && i == kb)) zero_tiles(p, r);
   zero_lists<KD>(p, r);
   if (lane == 0) p.pair_cnt[r] = 0u;
-  // publish the row's outcome; the OR that makes the request's outcome known
-  // names this warp its finisher
-  fence_acq_rel_gpu();
+  // publish the row's outcome (release: the row record and staged rows
+  // first; acquire: the rows published before); the OR that makes the
+  // request's outcome known names this warp its finisher
   __syncwarp();
   int before = -1, after = -1;
   unsigned long long now = 0ull;
   if (lane == 0) {
     const unsigned long long bits =
         (1ull << i) | ((code != kRowAccepted) ? (1ull << (32 + i)) : 0ull);
-    const unsigned long long old = atomicOr(&p.req_state[b], bits);
+    const unsigned long long old = atom_or_acq_rel_u64(&p.req_state[b], bits);
     now = old | bits;
     before = chain_outcome(old, kb);
     after = chain_outcome(now, kb);
-    fence_acq_rel_gpu();
   }
   before = __shfl_sync(0xffffffffu, before, 0);
   after = __shfl_sync(0xffffffffu, after, 0);
@@ -1095,6 +1138,144 @@ __device__ __noinline__ void chain_locate(const ChainParams& p, int j) {
 // ---------------------------------------------------------------------------
 // The kernel.
 // ---------------------------------------------------------------------------
+
+// Atomic add with release semantics (this thread's earlier writes, and those
+// it has observed, are visible device-wide before the add); the returned
+// value is read only when needed.
+__device__ __forceinline__ uint32_t atom_add_release(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Push a task into a shared-memory queue (one thread; waits, bounded, for
+// room).
+__device__ __forceinline__ void queue_push(TaskQueue* q, int4 task, const ChainParams& p) {
+  const int slot = atomicAdd(&q->tail, 1);
+  const uint64_t t0 = globaltimer_ns();
+  while (slot - *reinterpret_cast<volatile int*>(&q->head) >= kTaskQ) {
+    if (globaltimer_ns() - t0 > p.wait_ns) {
+      set_status(p.status, SV_DEV_TIMEOUT);
+      atomicExch(&p.glob[kGAbort], 1u);
+      break;
+    }
+    __nanosleep(128);
+  }
+  q->task[slot % kTaskQ] = task;
+  __threadfence_block();
+  *reinterpret_cast<volatile int*>(&q->ready[slot % kTaskQ]) = 1;
+}
+
+// One consumer warp's share of a stream tile: its slice of the target row or,
+// for a tile holding a row pair, of the draft row.
+template <class TT, class DT, int MODE, bool KD, int NV>
+__device__ __forceinline__ void chain_slice(const ChainParams& p, const StageDesc& sd,
+                                            const unsigned char* st, bool use_bulk, int warp,
+                                            WarpPart& wp, unsigned long long* list_out) {
+  const int lane = threadIdx.x & 31;
+  constexpr int SW = NV * 256;
+  const bool pair = (sd.flags & kSDDraft) != 0;
+  const bool drow = pair && warp >= kRowW;       // this warp reduces the draft row
+  const int wi = drow ? warp - kRowW : warp;     // slice index inside the row
+  const int e0 = wi * SW;
+  const int n = max(0, min(SW, sd.len - e0));
+  const int t0e = sd.tile * kTileW + e0;
+  const int x = sd.i < sd.kb ? __ldg(&p.tokens[(size_t)sd.b * p.k + sd.i]) : -1;
+  const bool hasx = x >= t0e && x < t0e + n;
+  if (!drow) {
+    const unsigned char* src =
+        use_bulk ? st + (size_t)e0 * TT::bytes
+                 : chain_row<TT>(p.target, (size_t)sd.row, p.V) + (size_t)t0e * TT::bytes;
+    Slice<TT, NV> R;
+    slice_load(src, n, use_bulk, -INFINITY, R);
+    const float pm = slice_max(R);
+    if (MODE != kCMGreedy) {
+      slice_stats(R, pm, p.c, &wp.G0, &wp.S0);
+    } else {
+      int bi = -1;
+      if (pm != -INFINITY) {
+#pragma unroll
+        for (int v = NV - 1; v >= 0; --v)
+#pragma unroll
+          for (int t = kVec - 1; t >= 0; --t)
+            if (slice_elem(R, v, t) == pm) bi = (v * 32 + lane) * kVec + t;
+      }
+      wp.key = warp_max_u64(bi < 0 ? kNoKey : topk_key(pm, t0e + bi));
+    }
+    if (KD) {
+      // top-K keys of the slice above the row's running threshold and the
+      // slice floor (the smallest lane maximum: every lane holds an entry at
+      // least that large, so the slice's K best are too)
+      const int K = p.K;
+      const unsigned long long rthr = ld_relaxed_u64(&p.rowthr[sd.row]);
+      const float fl = order_float(__reduce_min_sync(0xffffffffu, float_order(pm)));
+      const unsigned long long floor_key =
+          fl == -INFINITY ? kNoKey : ((unsigned long long)float_order(fl) << 32);
+      unsigned long long thr = rthr;
+      if (floor_key > 0ull && floor_key - 1ull > thr) thr = floor_key - 1ull;
+      unsigned long long list = kNoKey;
+      unsigned pmask = 0;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const float vm = slice_vmax(R, v);
+        const unsigned long long vk = ((unsigned long long)float_order(vm) << 32) | 0xffffffffull;
+        if (vm != -INFINITY && vk > thr) pmask |= 1u << v;
+      }
+      unsigned long long last = ~0ull;
+      while (__any_sync(0xffffffffu, pmask != 0)) {
+        unsigned long long cnd = kNoKey;
+        int more = 0;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          if (!(pmask & (1u << v))) continue;
+          const int ev = (v * 32 + lane) * kVec;
+#pragma unroll
+          for (int t = 0; t < kVec; ++t) {
+            if (ev + t < n) {
+              const unsigned long long kk = topk_key(slice_elem(R, v, t), t0e + ev + t);
+              if (kk > thr && kk < last) {
+                more += cnd != kNoKey;
+                if (kk > cnd) cnd = kk;
+              }
+            }
+          }
+        }
+        if (cnd == kNoKey || more == 0) pmask = 0;
+        unsigned cm = __ballot_sync(0xffffffffu, cnd != kNoKey);
+        if (!cm) break;
+        if (__popc(cm) <= 4) {
+          while (cm) {
+            const int src2 = __ffs(cm) - 1;
+            cm &= cm - 1;
+            warp_list_insert(list, __shfl_sync(0xffffffffu, cnd, src2), 0xffffffffu);
+          }
+        } else {
+          list = warp_merge_desc(list, warp_sort_desc(cnd));
+        }
+        const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
+        if (kth > thr) thr = kth;
+        if (cnd != kNoKey) last = cnd;
+      }
+      *list_out = list;
+    }
+    if (hasx && lane == 0) {
+      wp.hx = 1;
+      wp.zx0 = load1<TT>(src, x - t0e);
+    }
+  } else {
+    const unsigned char* src =
+        use_bulk ? st + p.stage_off1 + (size_t)e0 * DT::bytes
+                 : chain_row<DT>(p.draft, (size_t)sd.b * p.k + sd.i, p.V) + (size_t)t0e * DT::bytes;
+    Slice<DT, NV> R;
+    slice_load(src, n, use_bulk, -INFINITY, R);
+    slice_stats(R, slice_max(R), p.c, &wp.G1, &wp.S1);
+    if (hasx && lane == 0) {
+      wp.hx = 2;
+      wp.zx1 = load1<DT>(src, x - t0e);
+    }
+  }
+}
+
 template <class TT, class DT, int MODE, bool KD>
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_constant__ ChainParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -1107,7 +1288,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
   int* done = reinterpret_cast<int*>(smem + p.off_done);
   WarpPart* parts = reinterpret_cast<WarpPart*>(smem + p.off_parts);
   unsigned long long* lists = reinterpret_cast<unsigned long long*>(smem + p.off_lists);
-  TaskQueue* tq = reinterpret_cast<TaskQueue*>(smem + p.off_tasks);
+  TaskQueue* tq = reinterpret_cast<TaskQueue*>(smem + p.off_tasks);  // consumers -> counter
+  TaskQueue* cq = tq + 1;                                              // counter -> completer
   const bool use_bulk = p.use_bulk != 0;
   constexpr int DB = (MODE == kCMProbs) ? 4 : DT::bytes;
 
@@ -1120,8 +1302,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
     mbar_init(stall_bar, 1);
     fence_mbar_init();
     tq->tail = tq->head = tq->consumers_done = 0;
+    cq->tail = cq->head = cq->consumers_done = 0;
   }
-  for (int q = threadIdx.x; q < kTaskQ; q += blockDim.x) tq->ready[q] = 0;
+  for (int q = threadIdx.x; q < kTaskQ; q += blockDim.x) tq->ready[q] = cq->ready[q] = 0;
   __syncthreads();
   pdl_launch_dependents();
   pdl_wait();  // the previous grid on the stream (its outputs may be our inputs) is complete
@@ -1145,10 +1328,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
         }
         return true;
       };
-      // The loads that decide the next tile (this CTA's draw-queue flag, the
-      // request state of the next stream tile, the abort word) are issued one
-      // iteration ahead, so their latency overlaps the wait for a free stage;
-      // a state read one tile late only skips a little less.
+      // Stream tiles are claimed kClaim at a time, two claims ahead, so the
+      // atomic's latency overlaps the issue of the tiles before; the loads
+      // that decide the next step (the request state of the next claim, this
+      // CTA's draw-queue entry, the abort word) are issued one step ahead.  A
+      // state read a little late only skips a little less.
       auto state_of = [&](int t) -> unsigned long long {
         if (t >= p.total) return 0ull;
         int i, b, tau;
@@ -1156,17 +1340,39 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
         return ld_relaxed_u64(&p.req_state[b]);
       };
       auto draw_flag = [&](int d) -> uint32_t { return d < nd ? ld_relaxed_u32(&p.drawq[d]) : 0u; };
-      int t0 = (int)atomicAdd(&p.glob[kGNext], 1u);
-      int t1 = t0 < p.total ? (int)atomicAdd(&p.glob[kGNext], 1u) : p.total;
-      unsigned long long pf_state = state_of(t0);
-      uint32_t pf_draw = draw_flag((int)blockIdx.x);
+      // Four claims are in flight: c0 (in use, its tiles' request states
+      // loaded), c1 (its states loading), c2 and c3 (the atomics returning),
+      // so a claim's value is first used two claims after its atomic.  The
+      // draw-queue flag is read two iterations after its load and the abort
+      // word eight, so no iteration waits on a load issued in the one before.
+      int c0 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
+      int c1 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
+      int c2 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
+      int c3 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
+      int ci = 0;  // next tile of claim c0
+      unsigned long long st0[kClaim], st1[kClaim];  // request state of each tile of c0, c1
+#pragma unroll
+      for (int q = 0; q < kClaim; ++q) st0[q] = state_of(c0 + q);
+#pragma unroll
+      for (int q = 0; q < kClaim; ++q) st1[q] = state_of(c1 + q);
+      int dq_a = (int)blockIdx.x, dq_b = (int)blockIdx.x;  // entries the flags were loaded for
+      uint32_t fl_a = draw_flag(dq_a), fl_b = draw_flag(dq_b);
       uint32_t pf_abort = 0u;
+      uint32_t iter = 0;
       bool stream_done = false;
       uint64_t idle_t0 = 0;
       while (!abort) {
-        if (pf_abort) break;
+        if ((++iter & 7u) == 0u) {
+          if (pf_abort) break;
+          pf_abort = ld_relaxed_u32(&p.glob[kGAbort]);
+        }
         // 1. this CTA's next draw tile, when its job is queued
         const int dn = (int)blockIdx.x + m * G;
+        uint32_t pf_draw = dq_a == dn ? fl_a : 0u;
+        fl_a = fl_b;
+        dq_a = dq_b;
+        fl_b = draw_flag(dn);
+        dq_b = dn;
         if (dn < nd && pf_draw) {
           // the entry names the job's row pair; its record (read by the
           // consumers) was written before the entry
@@ -1175,8 +1381,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           const int db = trow / p.P, dnr = trow - db * p.P;
           p.drawq[dn] = 0u;
           ++m;
-          pf_draw = draw_flag((int)blockIdx.x + m * G);
-          pf_abort = ld_relaxed_u32(&p.glob[kGAbort]);
           const int j = fast_div(dn, p.div_NT);
           const int tau = dn - j * p.NT;
           int s;
@@ -1211,16 +1415,26 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
         }
         // 2. the next stream tile
         if (!stream_done) {
-          const int t = t0;
-          const unsigned long long stw = pf_state;
-          t0 = t1;
-          t1 = t1 < p.total ? (int)atomicAdd(&p.glob[kGNext], 1u) : p.total;
-          pf_state = state_of(t0);
-          pf_draw = draw_flag(dn);
-          pf_abort = ld_relaxed_u32(&p.glob[kGAbort]);
-          if (t >= p.total) {
+          if (c0 >= p.total) {
             stream_done = true;
             continue;
+          }
+          const int t = c0 + ci;
+          unsigned long long stw = st0[0];
+#pragma unroll
+          for (int q = 1; q < kClaim; ++q)
+            if (ci == q) stw = st0[q];
+          if (++ci == kClaim || t + 1 >= p.total) {  // the claim is used up: move to the next
+            c0 = c1;
+            c1 = c2;
+            c2 = c3;
+            ci = 0;
+            c3 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
+#pragma unroll
+            for (int q = 0; q < kClaim; ++q) {
+              st0[q] = st1[q];
+              st1[q] = state_of(c1 + q);
+            }
           }
           int i, b, tau;
           chain_decode(p, t, i, b, tau);
@@ -1228,8 +1442,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           // a row that is not needed: with the tiles of a row consecutive,
           // move the claim counter past it (never past a row's first tile)
           auto skip_row = [&]() {
+#ifndef SV_CHAIN_NOJUMP
             if (p.order == 0 && tau + 1 < p.NT)
               atomicMax(&p.glob[kGNext], (uint32_t)(t - tau + p.NT));
+#endif
           };
           if (kb < 0) {
             // an idle request, or an invalid draft count: finished by the
@@ -1306,8 +1522,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           break;
         }
         __nanosleep(64);
-        pf_draw = draw_flag(dn);
+        // idle: the flags loaded now are read at the next pass
+        fl_a = fl_b = draw_flag(dn);
+        dq_a = dq_b = dn;
         pf_abort = ld_relaxed_u32(&p.glob[kGAbort]);
+        if (pf_abort) break;
       }
       // the consumers stop at an exit stage
       int s;
@@ -1337,11 +1556,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
       }
     }
   } else if (warp == kCW + 1) {
-    // ---------------- manager: counting, row completions, draws, idle requests ----------------
-    // Tasks are taken up to 32 at a time: one fence makes the records the
-    // consumers wrote visible device-wide, then each lane counts its tile
-    // into its row (or its draw tile into its job) with one atomic, all in
-    // flight together; the completions those counts trigger run one by one.
+    // ---------------- counter: tiles into rows, draw tiles into jobs ----------------
+    // Up to 32 count tasks at a time, one release atomic per lane, all in
+    // flight together; the counts that complete a row or a job become
+    // completion tasks for the completer warp.
     int head = 0;
     uint64_t idle_t0 = 0;
     while (true) {
@@ -1360,77 +1578,100 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
         const uint64_t now = globaltimer_ns();
         if (idle_t0 == 0) idle_t0 = now;
         else if (now - idle_t0 > 8ull * p.wait_ns) break;
-        __nanosleep(128);
+        __nanosleep(32);
         continue;
       }
       idle_t0 = 0;
-      __threadfence_block();  // the tasks' records (acquire at CTA scope)
+      __threadfence_block();  // the tasks and the records they name (acquire, CTA scope)
       int4 t = make_int4(-1, 0, 0, 0);
       if (lane < n) {
         const int slot = (head + lane) % kTaskQ;
         t = tq->task[slot];
         tq->ready[slot] = 0;
       }
+      __threadfence_block();
       __syncwarp();
       head += n;
-      if (lane == 0) {
-        __threadfence_block();
-        *reinterpret_cast<volatile int*>(&tq->head) = head;
-      }
-      // release the records device-wide, then count
-      fence_acq_rel_gpu();
+      if (lane == 0) *reinterpret_cast<volatile int*>(&tq->head) = head;
       int fire = 0;
       if (t.x == kTaskTile) {
-        fire = atomicAdd(&p.pair_cnt[t.y * p.P + t.z], 1u) == (uint32_t)p.NT - 1u;
+        fire = atom_add_release(&p.pair_cnt[t.y * p.P + t.z], 1u) == (uint32_t)p.NT - 1u;
       } else if (t.x == kTaskDraw) {
-        fire = atomicAdd(&p.job_cnt[t.y], 1u) == (uint32_t)p.NT - 1u;
+        fire = atom_add_release(&p.job_cnt[t.y], 1u) == (uint32_t)p.NT - 1u;
       } else if (t.x == kTaskIdle) {
         fire = 1;
       }
       unsigned todo = __ballot_sync(0xffffffffu, fire != 0);
-      if (todo) fence_acq_rel_gpu();  // acquire: the other tiles' records
       while (todo) {
         const int src = __ffs(todo) - 1;
         todo &= todo - 1;
-        const int kind = __shfl_sync(0xffffffffu, t.x, src);
-        const int a0 = __shfl_sync(0xffffffffu, t.y, src);
-        const int a1 = __shfl_sync(0xffffffffu, t.z, src);
-        const int a2 = __shfl_sync(0xffffffffu, t.w, src);
-        if (kind == kTaskTile) {
-          chain_complete_row<TT, DT, MODE, KD>(p, a0, a1, a2);
-        } else if (kind == kTaskDraw) {
-          chain_locate<TT, DT, MODE, KD>(p, a0);
-        } else {  // an idle request, or one with an invalid draft count
-          if (a2 == -2 && lane == 0) set_status(p.status, SV_DEV_BAD_LEN);
-          chain_write_outputs<KD>(p, a0, a2, -1, -1, 0);
-          __syncwarp();
-          if (lane == 0) {
-            fence_acq_rel_gpu();
-            atomicAdd(&p.glob[kGDet], 1u);
-          }
+        if (lane == src) queue_push(cq, t, p);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      __threadfence_block();
+      *reinterpret_cast<volatile int*>(&cq->consumers_done) = 1;
+    }
+  } else if (warp == kCW + 2) {
+    // ---------------- completer: row completions, draws, idle requests ----------------
+    int head = 0;
+    uint64_t idle_t0 = 0;
+    while (true) {
+      int go = 0;
+      int4 t = make_int4(0, 0, 0, 0);
+      if (lane == 0) {
+        const int slot = head % kTaskQ;
+        if (*reinterpret_cast<volatile int*>(&cq->ready[slot])) {
+          __threadfence_block();
+          t = cq->task[slot];
+          cq->ready[slot] = 0;
+          __threadfence_block();
+          *reinterpret_cast<volatile int*>(&cq->head) = head + 1;
+          go = 1;
+        } else if (*reinterpret_cast<volatile int*>(&cq->consumers_done) != 0 &&
+                   *reinterpret_cast<volatile int*>(&cq->tail) == head) {
+          go = 2;
         }
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (go == 2) break;
+      if (go == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (idle_t0 == 0) idle_t0 = now;
+        else if (now - idle_t0 > 8ull * p.wait_ns) break;
+        __nanosleep(32);
+        continue;
+      }
+      idle_t0 = 0;
+      ++head;
+      t.x = __shfl_sync(0xffffffffu, t.x, 0);
+      t.y = __shfl_sync(0xffffffffu, t.y, 0);
+      t.z = __shfl_sync(0xffffffffu, t.z, 0);
+      t.w = __shfl_sync(0xffffffffu, t.w, 0);
+      if (t.x == kTaskTile) {
+        // the row's count is complete: acquire it (synchronising with every
+        // tile's release), then complete the row
+        const int r = t.y * p.P + t.z;
+        if (lane == 0) (void)ld_acquire_u32(&p.pair_cnt[r]);
+        __syncwarp();
+        chain_complete_row<TT, DT, MODE, KD>(p, t.y, t.z, t.w);
+      } else if (t.x == kTaskDraw) {
+        if (lane == 0) (void)ld_acquire_u32(&p.job_cnt[t.y]);
+        __syncwarp();
+        chain_locate<TT, DT, MODE, KD>(p, t.y);
+      } else {  // an idle request, or one with an invalid draft count
+        if (t.w == -2 && lane == 0) set_status(p.status, SV_DEV_BAD_LEN);
+        chain_write_outputs<KD>(p, t.y, t.w, -1, -1, 0);
+        __syncwarp();
+        if (lane == 0) red_add_release_u32(&p.glob[kGDet], 1u);
       }
     }
   } else {
     // ---------------- consumers ----------------
-    // Hand a completion task to the manager warp (lane 0; waits, bounded, for
-    // room in the queue).
+    // The warp that folds a tile hands its count to the counter warp.
     auto push_task = [&](int kind, int a, int b2, int c2) {
-      if (lane == 0) {
-        const int slot = atomicAdd(&tq->tail, 1);
-        const uint64_t t0 = globaltimer_ns();
-        while (slot - *reinterpret_cast<volatile int*>(&tq->head) >= kTaskQ) {
-          if (globaltimer_ns() - t0 > p.wait_ns) {
-            set_status(p.status, SV_DEV_TIMEOUT);
-            atomicExch(&p.glob[kGAbort], 1u);
-            break;
-          }
-          __nanosleep(128);
-        }
-        tq->task[slot % kTaskQ] = make_int4(kind, a, b2, c2);
-        __threadfence_block();
-        *reinterpret_cast<volatile int*>(&tq->ready[slot % kTaskQ]) = 1;
-      }
+      if (lane == 0) queue_push(tq, make_int4(kind, a, b2, c2), p);
       __syncwarp();
     };
     bool stalled = false;
@@ -1459,8 +1700,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
       wp.hx = 0;
       wp.tmo = ok ? 0 : 1;
       wp.key = kNoKey;
-      const int e0 = warp * kSliceW;
-      const int n = max(0, min(kSliceW, sd.len - e0));
+      unsigned long long list = kNoKey;
       if (sd.kind == kTKStream) {
         if (p.stall && !stalled && warp == 0 && sd.row == 0 && sd.tile == 0) {
           // test hook: wait on a barrier nothing arrives on, as a copy that
@@ -1469,103 +1709,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           stalled = true;
           if (!mbar_wait_limit(stall_bar, 0, p.wait_ns / 4)) wp.tmo = 1;
         }
-        const int t0e = sd.tile * kTileW + e0;
-        const unsigned char* src0 =
-            use_bulk ? st + (size_t)e0 * TT::bytes
-                     : chain_row<TT>(p.target, (size_t)sd.row, p.V) + (size_t)t0e * TT::bytes;
-        const int x = sd.i < sd.kb ? __ldg(&p.tokens[(size_t)sd.b * p.k + sd.i]) : -1;
-        const bool hasx = x >= t0e && x < t0e + n;
-        {
-          Slice<TT> R;
-          slice_load(src0, n, use_bulk, -INFINITY, R);
-          const float pm = slice_max(R);
-          if (MODE != kCMGreedy) slice_stats(R, pm, p.c, &wp.G0, &wp.S0);
-          if (MODE == kCMGreedy) {
-            int bi = -1;
-            if (pm != -INFINITY) {
-#pragma unroll
-              for (int v = kVPL - 1; v >= 0; --v)
-#pragma unroll
-                for (int t = kVec - 1; t >= 0; --t)
-                  if (slice_elem(R, v, t) == pm) bi = (v * 32 + lane) * kVec + t;
-            }
-            wp.key = warp_max_u64(bi < 0 ? kNoKey : topk_key(pm, t0e + bi));
-          }
-          if (KD) {
-            // top-K keys of the slice above the row's running threshold and
-            // the slice floor (the smallest lane maximum: every lane holds an
-            // entry at least that large, so the slice's K best are too)
-            const int K = p.K;
-            const unsigned long long rthr = ld_relaxed_u64(&p.rowthr[sd.row]);
-            const float fl = order_float(__reduce_min_sync(0xffffffffu, float_order(pm)));
-            const unsigned long long floor_key =
-                fl == -INFINITY ? kNoKey : ((unsigned long long)float_order(fl) << 32);
-            unsigned long long thr = rthr;
-            if (floor_key > 0ull && floor_key - 1ull > thr) thr = floor_key - 1ull;
-            unsigned long long list = kNoKey;
-            unsigned pmask = 0;
-#pragma unroll
-            for (int v = 0; v < kVPL; ++v) {
-              const float vm = slice_vmax(R, v);
-              const unsigned long long vk =
-                  ((unsigned long long)float_order(vm) << 32) | 0xffffffffull;
-              if (vm != -INFINITY && vk > thr) pmask |= 1u << v;
-            }
-            unsigned long long last = ~0ull;
-            while (__any_sync(0xffffffffu, pmask != 0)) {
-              unsigned long long cnd = kNoKey;
-              int more = 0;
-              for (unsigned mm = pmask; mm; mm &= mm - 1) {
-                const int v = __ffs(mm) - 1;
-                const int ev = (v * 32 + lane) * kVec;
-#pragma unroll
-                for (int t = 0; t < kVec; ++t) {
-                  if (ev + t < n) {
-                    const float val = load1<TT>(src0, ev + t);
-                    const unsigned long long kk = topk_key(val, t0e + ev + t);
-                    if (kk > thr && kk < last) {
-                      more += cnd != kNoKey;
-                      if (kk > cnd) cnd = kk;
-                    }
-                  }
-                }
-              }
-              if (cnd == kNoKey || more == 0) pmask = 0;
-              unsigned cm = __ballot_sync(0xffffffffu, cnd != kNoKey);
-              if (!cm) break;
-              if (__popc(cm) <= 4) {
-                while (cm) {
-                  const int src = __ffs(cm) - 1;
-                  cm &= cm - 1;
-                  warp_list_insert(list, __shfl_sync(0xffffffffu, cnd, src), 0xffffffffu);
-                }
-              } else {
-                list = warp_merge_desc(list, warp_sort_desc(cnd));
-              }
-              const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
-              if (kth > thr) thr = kth;
-              if (cnd != kNoKey) last = cnd;
-            }
-            if (lane < K) lists[((size_t)s * kCW + warp) * K + lane] = list;
-          }
-        }
-        if (hasx && lane == 0) {
-          wp.hx = 1;
-          wp.zx0 = load1<TT>(src0, x - t0e);
-        }
-        if (sd.flags & kSDDraft) {
-          const unsigned char* src1 =
-              use_bulk ? st + p.stage_off1 + (size_t)e0 * DT::bytes
-                       : chain_row<DT>(p.draft, (size_t)sd.b * p.k + sd.i, p.V) + (size_t)t0e * DT::bytes;
-          Slice<DT> R1;
-          slice_load(src1, n, use_bulk, -INFINITY, R1);
-          const float pm1 = slice_max(R1);
-          slice_stats(R1, pm1, p.c, &wp.G1, &wp.S1);
-          if (hasx && lane == 0) wp.zx1 = load1<DT>(src1, x - t0e);
-        }
+        if (sd.flags & kSDDraft)
+          chain_slice<TT, DT, MODE, KD, kVPLP>(p, sd, st, use_bulk, warp, wp, &list);
+        else
+          chain_slice<TT, DT, MODE, KD, kVPL>(p, sd, st, use_bulk, warp, wp, &list);
+        if (KD && lane < p.K) lists[((size_t)s * kCW + warp) * p.K + lane] = list;
       } else if (sd.kind == kTKDraw) {
         // residual mass of the slice: p and q of the row pair sd.i
         const DrawJob dj = ldcg_rec(&p.jobs[sd.row]);
+        const int e0 = warp * kSliceW;
+        const int n = max(0, min(kSliceW, sd.len - e0));
         const int t0e = sd.tile * kTileW + e0;
         const unsigned char* ts =
             use_bulk ? st + (size_t)e0 * TT::bytes
@@ -1601,28 +1754,32 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
       last = __shfl_sync(0xffffffffu, last, 0);
       if (!last) continue;
       if (sd.kind == kTKStream) {
-        const WarpPart q = lane < kCW ? parts[s * kCW + lane] : WarpPart{-INFINITY, -INFINITY, 0.0, 0.0, 0.f, 0.f, 0, 0, kNoKey};
+        const bool pair = (sd.flags & kSDDraft) != 0;
+        const WarpPart q = lane < kCW ? parts[s * kCW + lane]
+                                      : WarpPart{-INFINITY, -INFINITY, 0.0, 0.0, 0.f, 0.f, 0, 0, kNoKey};
+        // target partials from the target warps, draft partials from the draft warps
+        const bool tl_ = lane < (pair ? kRowW : kCW);
+        const float g0 = tl_ ? q.G0 : -INFINITY, g1 = tl_ ? -INFINITY : q.G1;
+        const double s0 = tl_ ? q.S0 : 0.0, s1 = tl_ ? 0.0 : q.S1;
         TileRec tr;
-        tr.G0 = warp_max(q.G0);
-        tr.G1 = warp_max(q.G1);
-        tr.S0 = warp_sum(rescale_pow2(q.S0, q.G0, tr.G0));
-        tr.S1 = warp_sum(rescale_pow2(q.S1, q.G1, tr.G1));
-        const unsigned hm = __ballot_sync(0xffffffffu, q.hx != 0);
-        tr.zx0 = tr.zx1 = 0.f;
+        tr.G0 = warp_max(g0);
+        tr.G1 = warp_max(g1);
+        tr.S0 = warp_sum(rescale_pow2(s0, g0, tr.G0));
+        tr.S1 = warp_sum(rescale_pow2(s1, g1, tr.G1));
+        const unsigned h0 = __ballot_sync(0xffffffffu, q.hx == 1);
+        const unsigned h1 = __ballot_sync(0xffffffffu, q.hx == 2);
+        tr.zx0 = h0 ? __shfl_sync(0xffffffffu, q.zx0, __ffs(h0) - 1) : 0.f;
+        tr.zx1 = h1 ? __shfl_sync(0xffffffffu, q.zx1, __ffs(h1) - 1) : 0.f;
         int fl = __any_sync(0xffffffffu, q.tmo != 0) ? kPTimeout : 0;
-        if (hm) {
-          const int src = __ffs(hm) - 1;
-          tr.zx0 = __shfl_sync(0xffffffffu, q.zx0, src);
-          tr.zx1 = __shfl_sync(0xffffffffu, q.zx1, src);
-          fl |= kPHasX;
-        }
+        if (h0) fl |= kPHasX;
         tr.flags = fl;
         tr.pad = 0;
         tr.key = warp_max_u64(q.key);
         unsigned long long tl = kNoKey;
         if (KD) {
           const int K = p.K;
-          for (int w = 0; w < kCW; ++w)
+          const int nw = pair ? kRowW : kCW;
+          for (int w = 0; w < nw; ++w)
             tl = warp_merge_desc(tl, lane < K ? lists[((size_t)s * kCW + w) * K + lane] : kNoKey);
         }
         const bool bonus = (MODE != kCMGreedy) && (sd.flags & kSDBonus);
@@ -1642,7 +1799,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           const unsigned long long kth = __shfl_sync(0xffffffffu, tl, K - 1);
           if (lane == 0 && kth != kNoKey) atomicMax(&p.rowthr[sd.row], kth);
         }
-        // the manager counts the tile into its row (the ring does not wait)
         __threadfence_block();
         __syncwarp();
         push_task(kTaskTile, sd.b, sd.i, sd.kb);

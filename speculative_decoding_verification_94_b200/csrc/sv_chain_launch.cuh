@@ -97,7 +97,7 @@ cudaError_t launch_chain_t(const ChainArgs& a) {
     f = (f + 15) / 16 * 16 + S * 4;
     f = (f + 15) / 16 * 16 + S * kCW * (int)sizeof(WarpPart);
     f = (f + 15) / 16 * 16 + (KD ? S * kCW * K * 8 : 0);
-    f = (f + 15) / 16 * 16 + (int)sizeof(TaskQueue);
+    f = (f + 15) / 16 * 16 + 2 * (int)sizeof(TaskQueue);
     return f;
   };
   int S = (int)knob(kKnobStages);
@@ -121,7 +121,7 @@ cudaError_t launch_chain_t(const ChainArgs& a) {
   p.off_lists = o;
   o = (o + (KD ? S * kCW * K * 8 : 0) + 15) / 16 * 16;
   p.off_tasks = o;
-  o += (int)sizeof(TaskQueue);
+  o += 2 * (int)sizeof(TaskQueue);
   const int smem = o;
   p.K = K > 0 ? K : 1;
   p.accepted_len = a.accepted_len;

@@ -27,7 +27,7 @@ SV_DEV_BAD_INDEX, SV_DEV_BAD_LEN, SV_DEV_ERROR_MASK = 0x10, 0x20, 0xFF
 SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
 SV_KNOB_CLUSTER_CTAS, SV_KNOB_STREAM_COUNT, SV_KNOB_STREAM_W, SV_KNOB_WAIT_NS = 1, 2, 3, 4
-SV_KNOB_STALL, SV_KNOB_STAGES, SV_KNOB_ORDER, SV_KNOB_LEGACY = 5, 6, 7, 8
+SV_KNOB_STALL, SV_KNOB_STAGES, SV_KNOB_ORDER, SV_KNOB_PERSISTENT = 5, 6, 7, 8
 
 EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc", "sv_set_knob",
            "sv_verify_tree_greedy", "sv_kd_grad", "sv_kd_grad_workspace_size",
@@ -114,25 +114,32 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+_KNOB_VALUES: dict = {}  # what this process last set, so that knobs() can restore it
+
+
 def sv_set_knob(knob: int, value: int) -> None:
     """Process-wide test / tuning setting (see sv.h); 0 restores the default."""
     _check(lib().sv_set_knob(int(knob), int(value)), "sv_set_knob")
+    _KNOB_VALUES[int(knob)] = int(value)
 
 
 class knobs:
-    """Context manager: set knobs {id: value} for the block, then restore 0."""
+    """Context manager: set knobs by name for the block, then put back the
+    values they had before it (blocks nest)."""
 
     def __init__(self, **kw):
         self.kw = {globals()["SV_KNOB_" + k.upper()]: v for k, v in kw.items()}
+        self.saved = {}
 
     def __enter__(self):
         for k, v in self.kw.items():
+            self.saved[k] = _KNOB_VALUES.get(k, 0)
             sv_set_knob(k, v)
         return self
 
     def __exit__(self, *exc):
-        for k in self.kw:
-            sv_set_knob(k, 0)
+        for k, v in self.saved.items():
+            sv_set_knob(k, v)
         return False
 
 

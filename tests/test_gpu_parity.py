@@ -42,10 +42,18 @@ def check_chain(x, max_flag_frac=0.05):
     return assert_chain_match(got, ref, x.uniforms.numpy(), x.temperature, x.k, max_flag_frac)
 
 
+@pytest.fixture(params=["two-kernel", "persistent"])
+def chain_path(request):
+    """Run the test on both chain paths: the default two-kernel path and the
+    single persistent launch."""
+    with sv.knobs(persistent=int(request.param == "persistent")):
+        yield request.param
+
+
 # --------------------------------------------------------------------------
 # Workloads
 # --------------------------------------------------------------------------
-def test_tiny_chain_fp32():
+def test_tiny_chain_fp32(chain_path):
     r = check_chain(inputs.tiny_chain(seed=0))
     assert r["flagged"] == 0
 
@@ -55,14 +63,14 @@ def qwen32():
     return inputs.qwen_chain(B=32, k=3, sigma_d=1.0, seed=0)
 
 
-def test_qwen_chain_full_size(qwen32):
+def test_qwen_chain_full_size(qwen32, chain_path):
     r = check_chain(qwen32)
     print("qwen chain", r)
 
 
 @pytest.mark.parametrize("k", [1, 3, 5, 7])
 @pytest.mark.parametrize("sigma", [0.3, 1.0, 3.0])
-def test_active_batch_sweep(k, sigma):
+def test_active_batch_sweep(k, sigma, chain_path):
     x = inputs.qwen_chain(B=32, k=k, sigma_d=sigma, seed=100 + k)
     ref = oracle_chain(x)
     for B in (1, 2, 4, 8, 16, 32):
@@ -94,7 +102,7 @@ def kd256():
 
 
 @pytest.mark.parametrize("wmode,group", [("raw", 1), ("group_norm", 16)])
-def test_fused_verify_kd_full_size(kd256, wmode, group):
+def test_fused_verify_kd_full_size(kd256, wmode, group, chain_path):
     x = kd256
     st = status_tensor()
     kd = dict(K=32, reward=x.reward.to(DEV), wmode=wmode, group=group, clip=0.0)
@@ -153,7 +161,7 @@ def test_kl_loss_standalone(qwen32, draft_kind):
 # --------------------------------------------------------------------------
 # Losslessness on the GPU itself (Leviathan): emitted tokens follow p.
 # --------------------------------------------------------------------------
-def test_gpu_losslessness_chi_square():
+def test_gpu_losslessness_chi_square(chain_path):
     import scipy.stats
     rng = np.random.default_rng(5)
     V, k, B = 8, 3, 1_000_000
@@ -187,20 +195,20 @@ def test_gpu_losslessness_chi_square():
 # --------------------------------------------------------------------------
 @pytest.mark.parametrize("V", [1, 2, 7, 8, 64, 1001, 4099, 70001, 151936])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_ragged_and_small_vocab(V, dtype):
+def test_ragged_and_small_vocab(V, dtype, chain_path):
     x = inputs.make_chain(12, 3, V, dtype=dtype, model="zipf" if V > 64 else "gauss",
                           sigma_t=2.0, sigma_d=1.0, temperature=0.9, seed=V)
     check_chain(x, max_flag_frac=0.25)
 
 
 @pytest.mark.parametrize("k", [1, 15, 30, 31, 40])
-def test_k_extremes(k):
+def test_k_extremes(k, chain_path):
     """k <= 30 runs as one persistent launch, k > 30 on the two-kernel path."""
     check_chain(inputs.make_chain(12, k, 5000, dtype="bf16", sigma_d=0.3, temperature=1.0,
                                   seed=k), max_flag_frac=0.25)
 
 
-def test_empty_batch():
+def test_empty_batch(chain_path):
     x = inputs.make_chain(1, 3, 100, dtype="f32", seed=1)
     z = torch.empty(0, 4, 100, device=DEV)
     d = torch.empty(0, 3, 100, device=DEV)
@@ -211,7 +219,7 @@ def test_empty_batch():
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_draft_probabilities(dtype):
+def test_draft_probabilities(dtype, chain_path):
     x = inputs.make_chain(16, 3, 3000, dtype=dtype, sigma_d=1.0, temperature=0.8, seed=3)
     probs = torch.softmax(x.draft.float() / x.temperature, dim=-1).contiguous()
     y = inputs.ChainInputs(x.target, probs, x.draft_tokens, x.uniforms, x.reward, x.temperature,
@@ -219,14 +227,14 @@ def test_draft_probabilities(dtype):
     check_chain(y)
 
 
-def test_identical_draft_accepts_everything_on_gpu():
+def test_identical_draft_accepts_everything_on_gpu(chain_path):
     x = inputs.make_chain(64, 4, 30000, dtype="bf16", sigma_d=0.0, temperature=0.7, seed=9)
     got = run_chain(x)
     assert (got["accepted_len"].cpu() == 4).all()
     check_chain(x)
 
 
-def test_disjoint_support_on_gpu():
+def test_disjoint_support_on_gpu(chain_path):
     V, k, B = 4096, 3, 128
     rng = np.random.default_rng(0)
     zt = rng.normal(0, 2, (k + 1, V)).astype(np.float32)
@@ -243,7 +251,7 @@ def test_disjoint_support_on_gpu():
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_greedy_chain_with_ties(dtype):
+def test_greedy_chain_with_ties(dtype, chain_path):
     rng = np.random.default_rng(7)
     B, k, V = 64, 4, 3000
     z = rng.integers(-3, 4, size=(B, k + 1, V)).astype(np.float32)
@@ -257,7 +265,7 @@ def test_greedy_chain_with_ties(dtype):
     assert np.array_equal(got["out_tokens"].cpu().numpy(), ref["out_tokens"])
 
 
-def test_greedy_chain_full_size(qwen32):
+def test_greedy_chain_full_size(qwen32, chain_path):
     x = qwen32
     tok = x.target[:, :3].float().argmax(-1).to(torch.int32)
     tok[::3, 1] = 5
@@ -287,7 +295,7 @@ def test_topk_with_massive_ties_and_small_rows():
     assert_close(got["topk_logp"].cpu().numpy(), ref["topk_logp"], 1.0, "topk_logp")
 
 
-def test_device_checks_flag_bad_inputs():
+def test_device_checks_flag_bad_inputs(chain_path):
     x = inputs.make_chain(4, 3, 500, dtype="f32", seed=2)
     tok = x.draft_tokens.clone()
     tok[1, 0] = 500  # out of range (position 0 is always verified)
@@ -320,7 +328,7 @@ def test_device_checks_flag_bad_inputs():
     assert got["accepted_len"][0].item() >= 0
 
 
-def test_zero_residual_falls_back_to_target():
+def test_zero_residual_falls_back_to_target(chain_path):
     """p == q but x outside both supports: rejected with zero residual mass."""
     V = 64
     z = np.random.default_rng(1).normal(0, 1, (4, V)).astype(np.float32)
@@ -336,7 +344,7 @@ def test_zero_residual_falls_back_to_target():
     assert_chain_match(got, ref, x.uniforms.numpy(), 1.0, 3)
 
 
-def test_deterministic_and_workspace_reuse(kd256):
+def test_deterministic_and_workspace_reuse(kd256, chain_path):
     x = kd256
     kd = dict(K=32, reward=x.reward.to(DEV), wmode="group_norm", group=16)
     a = run_chain(x, kd=kd)
@@ -362,7 +370,7 @@ def test_deterministic_and_workspace_reuse(kd256):
 @pytest.mark.parametrize("C", [1, 2, 3, 4, 8, 12, 16])
 def test_every_cluster_size(C):
     """The two-kernel path's finishing cluster size must not change any result."""
-    with sv.knobs(legacy=1, cluster_ctas=C):
+    with sv.knobs(cluster_ctas=C):
         x = inputs.make_chain(24, 3, 20000, dtype="bf16", sigma_d=1.0, temperature=0.7, seed=C)
         check_chain(x, max_flag_frac=0.2)
         got = sv.sv_extract_topk_kd(x.target.to(DEV), 32, 0.7)
@@ -370,9 +378,9 @@ def test_every_cluster_size(C):
         assert np.array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
 
 
-PATHS = {"fused": {}, "fused-order1": dict(order=1), "fused-order2-stages2": dict(order=2, stages=2),
-         "legacy-static": dict(legacy=1, stream_count=1),
-         "legacy-dynamic": dict(legacy=1, stream_count=2)}
+PATHS = {"persistent": dict(persistent=1), "persistent-order1": dict(persistent=1, order=1),
+         "persistent-order2-stages2": dict(persistent=1, order=2, stages=2),
+         "two-kernel-static": dict(stream_count=1), "two-kernel-dynamic": dict(stream_count=2)}
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -467,7 +475,7 @@ def test_kd_grad_full_vocabulary(kd256):
     _grad_check(x, acc, x.reward, ref, O.W_GROUP_NORM, 16, x.temperature)
 
 
-def test_kd_first_rejected_position(kd256):
+def test_kd_first_rejected_position(kd256, chain_path):
     """positions=1 (the Draft-OPD variant): the loss and the gradient also
     cover the first rejected position."""
     x = inputs.ChainInputs(kd256.target[:32].contiguous(), kd256.draft[:32].contiguous(),

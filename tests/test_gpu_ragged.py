@@ -59,9 +59,8 @@ def _check_idle(got, act):
     assert (out[act == 0] == -1).all()
 
 
-PATHS = {"fused": {}, "fused-order2": dict(order=2),
-         "legacy-static": dict(legacy=1, stream_count=1),
-         "legacy-dynamic": dict(legacy=1, stream_count=2)}
+PATHS = {"persistent": dict(persistent=1), "persistent-order2": dict(persistent=1, order=2),
+         "two-kernel-static": dict(stream_count=1), "two-kernel-dynamic": dict(stream_count=2)}
 
 
 @pytest.fixture(params=list(PATHS))

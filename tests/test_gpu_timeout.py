@@ -1,6 +1,6 @@
 """A bounded device wait that runs out.
 
-The chain kernel's test hook makes the warp that reduces request 0's first
+The persistent chain kernel's test hook makes the warp that reduces request 0's first
 slice wait on a barrier nothing arrives on, under a short wait limit: the wait
 gives up, the call returns, reports SV_DEV_TIMEOUT, fails request 0 only
 (accepted length -1, tokens -1), leaves the workspace all zero, and the next
@@ -27,7 +27,7 @@ def test_bounded_wait_runs_out_and_reports():
     x = inputs.qwen_chain(B=8, k=3, sigma_d=1.0, seed=21)
     ref = O.verify_chain(x.target, x.draft, x.draft_tokens, x.uniforms, x.temperature)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    with sv.knobs(wait_ns=20_000_000, stall=1):  # 20 ms limit; the stalled wait gives up at 5 ms
+    with sv.knobs(persistent=1, wait_ns=20_000_000, stall=1):  # 20 ms limit; the stalled wait gives up at 5 ms
         got = _run(x, st)
         torch.cuda.synchronize()
     word = int(st.item())
