@@ -398,6 +398,8 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
  *                         draws and request completion in one grid); 0, the
  *                         default, the two-kernel path (stream pass, then
  *                         finishing clusters), which is faster on B200 today
+ *   SV_KNOB_KERNEL_MARKS  1: bracket every kernel launch with events (see
+ *                         sv_kernel_times)
  */
 #define SV_KNOB_CLUSTER_CTAS 1
 #define SV_KNOB_STREAM_COUNT 2
@@ -407,7 +409,29 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
 #define SV_KNOB_STAGES 6
 #define SV_KNOB_ORDER 7
 #define SV_KNOB_PERSISTENT 8
+#define SV_KNOB_KERNEL_MARKS 9
 SV_API sv_status sv_set_knob(int knob, long long value);
+
+/*
+ * sv_kernel_times -- per-launch device times, for measurement.  While
+ * SV_KNOB_KERNEL_MARKS is 1, the library records an event on the call's stream
+ * before and after each kernel it launches (also inside stream capture, where
+ * the events become graph nodes and are recorded at every replay); the events
+ * are the library's own, created on the current device at the first marked
+ * launch.  This call waits for the last marked launch, writes the duration in
+ * microseconds of each launch marked since its previous call (at most the
+ * last 2048, oldest first, at most `cap`) to us[] and its kind to tags[]
+ * (SV_MARK_STREAM: a streaming pass; SV_MARK_FINISH: a finishing or
+ * reduction kernel; SV_MARK_CHAIN: the persistent chain kernel), stores the
+ * count in *n and starts a new count.  The marks add an event record between
+ * launches, so a marked call can run slightly slower than an unmarked one.
+ *   Errors: SV_ERR_INVALID_ARG for null pointers or a current device other
+ *   than the marks' own; SV_ERR_CUDA if reading an event fails.
+ */
+#define SV_MARK_STREAM 0
+#define SV_MARK_FINISH 1
+#define SV_MARK_CHAIN 2
+SV_API sv_status sv_kernel_times(float* us, int32_t* tags, int cap, int32_t* n);
 
 /* Map a device status word (read back by the caller) to a host status:
  * SV_OK, SV_ERR_TIMEOUT if SV_DEV_TIMEOUT is set, else SV_ERR_DEVICE_CHECK

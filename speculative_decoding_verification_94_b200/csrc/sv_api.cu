@@ -22,8 +22,70 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 enum : int { kKnobClusterCtas = 1, kKnobStreamCount = 2, kKnobStreamW = 3, kKnobPersistent = 8,
-              kKnobCount = 16 };
+              kKnobKernelMarks = 9, kKnobCount = 16 };
 long long g_knobs[kKnobCount];
+
+// Kernel timing marks.  With the knob set, every kernel launch of the library
+// is bracketed by two events recorded on its stream, kept in a ring, and
+// sv_kernel_times reads the durations of the launches since its last call.
+// The records are external ones, which stream capture turns into event
+// record nodes, so the calls of a captured graph are timed launch by launch
+// at every replay.
+enum : int { kMarkStream = 0, kMarkFinish = 1, kMarkChain = 2 };
+constexpr int kMarkLaunches = 2048;
+struct MarkRing {
+  cudaEvent_t ev[2 * kMarkLaunches];
+  int tag[kMarkLaunches];
+  long long pos;  // launches bracketed since the last read
+  int dev;        // device the events belong to, -1 before the first mark
+};
+MarkRing g_mark = {{}, {}, 0, -1};
+
+bool marks_on() { return knob(kKnobKernelMarks) != 0; }
+
+cudaError_t mark_events_ready() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || g_mark.dev == dev) return e;
+  if (g_mark.dev >= 0) {
+    int cur = dev;
+    cudaSetDevice(g_mark.dev);
+    for (auto& ev : g_mark.ev) cudaEventDestroy(ev);
+    cudaSetDevice(cur);
+  }
+  g_mark.dev = -1;
+  for (auto& ev : g_mark.ev)
+    if ((e = cudaEventCreate(&ev)) != cudaSuccess) return e;
+  g_mark.dev = dev;
+  g_mark.pos = 0;
+  return cudaSuccess;
+}
+
+cudaError_t mark_record(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusActive
+             ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+             : cudaEventRecord(ev, s);
+}
+
+// Event before a launch (no-op without the knob).
+cudaError_t mark_before(cudaStream_t s) {
+  if (!marks_on()) return cudaSuccess;
+  cudaError_t e = mark_events_ready();
+  if (e != cudaSuccess) return e;
+  return mark_record(g_mark.ev[2 * (g_mark.pos % kMarkLaunches)], s);
+}
+
+// Event after a launch, and the launch's tag; passes on the launch's error.
+cudaError_t mark_after(cudaStream_t s, int tag, cudaError_t launched) {
+  if (!marks_on() || launched != cudaSuccess || g_mark.dev < 0) return launched;
+  const long long q = g_mark.pos % kMarkLaunches;
+  g_mark.tag[q] = tag;
+  ++g_mark.pos;
+  return mark_record(g_mark.ev[2 * q + 1], s);
+}
 
 int forced_cluster() {
   const int c = (int)knob(kKnobClusterCtas);
@@ -266,11 +328,12 @@ static cudaError_t launch_stream(StreamParams& p, const StreamGeom& g, cudaStrea
   if (need < grid) grid = need;
   if (grid < 1) grid = 1;
   p.nwarps_eff = (int)(grid * kStreamWarps < items ? grid * kStreamWarps : items);
+  if ((e = mark_before(s)) != cudaSuccess) return e;
   if (p.count == 0)
     ks<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
   else
     kd<<<(unsigned)grid, kStreamThreads, g.smem, s>>>(p);
-  return cudaGetLastError();
+  return mark_after(s, kMarkStream, cudaGetLastError());
 }
 
 // ---------------------------------------------------------------------------
@@ -296,7 +359,8 @@ static cudaError_t launch_clusters(K kernel, const Prm& prm, const RowPlan& plan
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kernel, prm);
+  if ((e = mark_before(s)) != cudaSuccess) return e;
+  return mark_after(s, kMarkFinish, cudaLaunchKernelEx(&cfg, kernel, prm));
 }
 
 template <class K, class Prm>
@@ -313,7 +377,8 @@ static cudaError_t launch_blocks(K kernel, const Prm& prm, int blocks, int smem,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, prm);
+  if ((e = mark_before(s)) != cudaSuccess) return e;
+  return mark_after(s, kMarkFinish, cudaLaunchKernelEx(&cfg, kernel, prm));
 }
 
 // Clusters of plan.C CTAs of this kernel that the device holds at once.
@@ -516,7 +581,10 @@ static sv_status verify_chain_impl(const void* target_logits, sv_dtype t_dtype, 
     ca.workspace = workspace;
     ca.status = device_status;
     ca.stream = reinterpret_cast<cudaStream_t>(stream);
-    return cuda_status(t_dtype == SV_BF16 ? launch_chain_bf16(ca) : launch_chain_f32(ca));
+    cudaError_t e = mark_before(ca.stream);
+    if (e != cudaSuccess) return SV_ERR_CUDA;
+    return cuda_status(mark_after(ca.stream, kMarkChain,
+                                  t_dtype == SV_BF16 ? launch_chain_bf16(ca) : launch_chain_f32(ca)));
   }
   const int P = k + 1;
   if ((long long)B * P > 0x7fffffffLL / 64) return SV_ERR_UNSUPPORTED;
@@ -695,8 +763,34 @@ sv_status sv_verify_chain_noalloc(const void* target_logits, sv_dtype t_dtype, c
   return st;
 }
 
+sv_status sv_kernel_times(float* us, int32_t* tags, int cap, int32_t* n) {
+  if (n == nullptr || (cap > 0 && (us == nullptr || tags == nullptr)) || cap < 0)
+    return SV_ERR_INVALID_ARG;
+  *n = 0;
+  if (g_mark.dev < 0 || g_mark.pos == 0) return SV_OK;
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != g_mark.dev) return SV_ERR_INVALID_ARG;
+  const long long total = g_mark.pos;
+  const long long kept = total < kMarkLaunches ? total : kMarkLaunches;
+  const long long first = total - kept;
+  const long long last = (total - 1) % kMarkLaunches;
+  if (cudaEventSynchronize(g_mark.ev[2 * last + 1]) != cudaSuccess) return SV_ERR_CUDA;
+  int m = 0;
+  for (long long j = first; j < total && m < cap; ++j, ++m) {
+    const long long q = j % kMarkLaunches;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_mark.ev[2 * q], g_mark.ev[2 * q + 1]) != cudaSuccess)
+      return SV_ERR_CUDA;
+    us[m] = 1e3f * ms;
+    tags[m] = g_mark.tag[q];
+  }
+  *n = m;
+  g_mark.pos = 0;
+  return SV_OK;
+}
+
 sv_status sv_set_knob(int knob_id, long long value) {
-  if (knob_id < 1 || knob_id >= kKnobCount) return SV_ERR_INVALID_ARG;
+  if (knob_id < 1 || knob_id > kKnobKernelMarks) return SV_ERR_INVALID_ARG;
   __atomic_store_n(&g_knobs[knob_id], value, __ATOMIC_RELAXED);
   return SV_OK;
 }

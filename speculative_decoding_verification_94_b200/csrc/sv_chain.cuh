@@ -1343,8 +1343,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
       // Four claims are in flight: c0 (in use, its tiles' request states
       // loaded), c1 (its states loading), c2 and c3 (the atomics returning),
       // so a claim's value is first used two claims after its atomic.  The
-      // draw-queue flag is read two iterations after its load and the abort
-      // word eight, so no iteration waits on a load issued in the one before.
+      // draw-queue flag is read three passes after its load and the abort
+      // word eight, so no pass waits on a load issued in the one before (a
+      // register is only read, or copied, once its load is that old).
       int c0 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
       int c1 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
       int c2 = (int)atomicAdd(&p.glob[kGNext], (uint32_t)kClaim);
@@ -1355,8 +1356,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
       for (int q = 0; q < kClaim; ++q) st0[q] = state_of(c0 + q);
 #pragma unroll
       for (int q = 0; q < kClaim; ++q) st1[q] = state_of(c1 + q);
-      int dq_a = (int)blockIdx.x, dq_b = (int)blockIdx.x;  // entries the flags were loaded for
-      uint32_t fl_a = draw_flag(dq_a), fl_b = draw_flag(dq_b);
+      int dq = (int)blockIdx.x;   // the entry the flag was loaded for
+      uint32_t fl = draw_flag(dq);  // its flag (in flight until fl_age reaches 3)
+      uint32_t fl_age = 0;
       uint32_t pf_abort = 0u;
       uint32_t iter = 0;
       bool stream_done = false;
@@ -1368,11 +1370,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
         }
         // 1. this CTA's next draw tile, when its job is queued
         const int dn = (int)blockIdx.x + m * G;
-        uint32_t pf_draw = dq_a == dn ? fl_a : 0u;
-        fl_a = fl_b;
-        dq_a = dq_b;
-        fl_b = draw_flag(dn);
-        dq_b = dn;
+        uint32_t pf_draw = 0u;
+        if (++fl_age >= 3u) {
+          pf_draw = dq == dn ? fl : 0u;
+          fl = draw_flag(dn);
+          dq = dn;
+          fl_age = 0u;
+        }
         if (dn < nd && pf_draw) {
           // the entry names the job's row pair; its record (read by the
           // consumers) was written before the entry
@@ -1381,6 +1385,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           const int db = trow / p.P, dnr = trow - db * p.P;
           p.drawq[dn] = 0u;
           ++m;
+          // the next entry's flag: jobs come in bursts, so load it now
+          dq = dn + G;
+          fl = draw_flag(dq);
+          fl_age = 0u;
           const int j = fast_div(dn, p.div_NT);
           const int tau = dn - j * p.NT;
           int s;
@@ -1522,9 +1530,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           break;
         }
         __nanosleep(64);
-        // idle: the flags loaded now are read at the next pass
-        fl_a = fl_b = draw_flag(dn);
-        dq_a = dq_b = dn;
+        // idle: the flag loaded now is read at the next pass
+        fl = draw_flag(dn);
+        dq = dn;
+        fl_age = 2u;
         pf_abort = ld_relaxed_u32(&p.glob[kGAbort]);
         if (pf_abort) break;
       }

@@ -28,8 +28,12 @@ SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 
 SV_KNOB_CLUSTER_CTAS, SV_KNOB_STREAM_COUNT, SV_KNOB_STREAM_W, SV_KNOB_WAIT_NS = 1, 2, 3, 4
 SV_KNOB_STALL, SV_KNOB_STAGES, SV_KNOB_ORDER, SV_KNOB_PERSISTENT = 5, 6, 7, 8
+SV_KNOB_KERNEL_MARKS = 9
+SV_MARK_STREAM, SV_MARK_FINISH, SV_MARK_CHAIN = 0, 1, 2
+MARK_NAMES = {SV_MARK_STREAM: "stream", SV_MARK_FINISH: "finish", SV_MARK_CHAIN: "chain"}
 
 EXPORTS = ("sv_verify_chain", "sv_verify_chain_ragged", "sv_verify_chain_noalloc", "sv_set_knob",
+           "sv_kernel_times",
            "sv_verify_tree_greedy", "sv_kd_grad", "sv_kd_grad_workspace_size",
            "sv_verify_tree_sample", "sv_extract_topk_kd", "sv_kd_kl_loss", "sv_sched_select",
            "sv_verify_chain_workspace_size", "sv_verify_tree_workspace_size",
@@ -106,6 +110,8 @@ def lib() -> ctypes.CDLL:
             L.sv_sched_select.restype = ci
             L.sv_set_knob.argtypes = [ci, ctypes.c_longlong]
             L.sv_set_knob.restype = ci
+            L.sv_kernel_times.argtypes = [vp, vp, ci, vp]
+            L.sv_kernel_times.restype = ci
             L.sv_status_string.argtypes = [ci]
             L.sv_status_string.restype = ctypes.c_char_p
             L.sv_version.argtypes = []
@@ -121,6 +127,17 @@ def sv_set_knob(knob: int, value: int) -> None:
     """Process-wide test / tuning setting (see sv.h); 0 restores the default."""
     _check(lib().sv_set_knob(int(knob), int(value)), "sv_set_knob")
     _KNOB_VALUES[int(knob)] = int(value)
+
+
+def sv_kernel_times(cap: int = 2048):
+    """Durations (us) and kinds of the kernel launches marked since the last
+    read (SV_KNOB_KERNEL_MARKS): a list of (kind name, microseconds)."""
+    import ctypes
+    us = (ctypes.c_float * cap)()
+    tags = (ctypes.c_int32 * cap)()
+    n = ctypes.c_int32(0)
+    _check(lib().sv_kernel_times(us, tags, int(cap), ctypes.byref(n)), "sv_kernel_times")
+    return [(MARK_NAMES.get(tags[j], str(tags[j])), float(us[j])) for j in range(n.value)]
 
 
 class knobs:

@@ -212,3 +212,17 @@ def test_knobs_validate(lib):
     assert lib.sv_set_knob(0, 1) == sv.SV_ERR_INVALID_ARG
     assert lib.sv_set_knob(99, 1) == sv.SV_ERR_INVALID_ARG
     assert lib.sv_set_knob(sv.SV_KNOB_STAGES, 0) == sv.SV_OK
+    assert lib.sv_set_knob(sv.SV_KNOB_KERNEL_MARKS + 1, 1) == sv.SV_ERR_INVALID_ARG
+
+
+def test_kernel_times_without_marks(lib):
+    """No marked launch yet: zero launches reported, no device touched; null
+    pointers are refused."""
+    import ctypes
+    n = ctypes.c_int32(7)
+    us = (ctypes.c_float * 4)()
+    tags = (ctypes.c_int32 * 4)()
+    assert lib.sv_kernel_times(us, tags, 4, ctypes.byref(n)) == sv.SV_OK
+    assert n.value == 0
+    assert lib.sv_kernel_times(us, tags, 4, None) == sv.SV_ERR_INVALID_ARG
+    assert lib.sv_kernel_times(None, None, 4, ctypes.byref(n)) == sv.SV_ERR_INVALID_ARG

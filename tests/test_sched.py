@@ -87,3 +87,30 @@ def test_sched_select_rejects_bad_tables():
     for thr, b, ns, a in bad:
         with pytest.raises(RuntimeError):
             sv.sv_sched_select(thr, b, ns, a)
+
+
+TABLE = os.path.join(os.path.dirname(os.path.dirname(__file__)),
+                     "speculative_decoding_verification_94_b200", "data", "verify_cost_table.json")
+
+
+def test_sched_select_on_the_measured_verify_cost_table(oracle):
+    """The lookup over the measured verify-kernel cost table of this device
+    (emitted tokens per second of one verification call for plain decoding
+    and k = 1, 3, 5, 7 drafts at active batches 1..32, written by
+    `bench.py --workload sched_table`): the C ABI's choice and predicted
+    speedup equal the oracle's at every active batch, inside and outside the
+    profiled sizes."""
+    from speculative_decoding_verification_94_b200 import sv
+    with open(TABLE, encoding="utf-8") as f:
+        t = json.load(f)
+    thr = np.asarray(t["throughput_tokens_per_s"], np.float32)
+    bs = np.asarray(t["batches"], np.int32)
+    assert thr.shape == (len(t["configs"]), len(bs)) and (thr > 0).all()
+    chosen = []
+    for a in range(1, 65):
+        cfg, sp = sv.sv_sched_select(thr, bs, t["nonspec"], a)
+        ocfg, osp = oracle.sched_select(thr, bs, t["nonspec"], a)
+        assert cfg == ocfg, a
+        assert sp == pytest.approx(osp, rel=1e-6), a
+        chosen.append(t["configs"][cfg])
+    print("configuration per active batch 1..64:", chosen)
