@@ -400,6 +400,10 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
  *                         finishing clusters), which is faster on B200 today
  *   SV_KNOB_KERNEL_MARKS  1: bracket every kernel launch with events (see
  *                         sv_kernel_times)
+ *   SV_KNOB_FINISH_READ   two-kernel sampling chain, how the finishing clusters
+ *                         read the drawn row: 1 staged in shared memory, 2 read
+ *                         from global memory (default: staged when every
+ *                         cluster fits in one wave)
  */
 #define SV_KNOB_CLUSTER_CTAS 1
 #define SV_KNOB_STREAM_COUNT 2
@@ -410,6 +414,7 @@ SV_API sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int
 #define SV_KNOB_ORDER 7
 #define SV_KNOB_PERSISTENT 8
 #define SV_KNOB_KERNEL_MARKS 9
+#define SV_KNOB_FINISH_READ 10
 SV_API sv_status sv_set_knob(int knob, long long value);
 
 /*

@@ -22,7 +22,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 enum : int { kKnobClusterCtas = 1, kKnobStreamCount = 2, kKnobStreamW = 3, kKnobPersistent = 8,
-              kKnobKernelMarks = 9, kKnobCount = 16 };
+              kKnobKernelMarks = 9, kKnobFinishRead = 10, kKnobCount = 16 };
 long long g_knobs[kKnobCount];
 
 // Kernel timing marks.  With the knob set, every kernel launch of the library
@@ -423,7 +423,7 @@ static cudaError_t cluster_capacity(K kernel, const RowPlan& plan, int* out) {
 // cluster (longer chunk) wins when it keeps the grid in one wave.
 template <class K>
 static cudaError_t pick_plan(K kernel, const RowPlan* plans, int np, int nclusters,
-                             RowPlan* out) {
+                             RowPlan* out, long long* waves_out = nullptr) {
   constexpr long long kLatencyElems = 8192;
   long long best = -1;
   for (int i = 0; i < np; ++i) {
@@ -436,19 +436,35 @@ static cudaError_t pick_plan(K kernel, const RowPlan* plans, int np, int ncluste
     if (best < 0 || cost < best) {
       best = cost;
       *out = plans[i];
+      if (waves_out) *waves_out = waves;
     }
   }
   return best < 0 ? cudaErrorInvalidConfiguration : cudaSuccess;
 }
 
+// Finishing plans of the sampling chain: `staged` (the drawn row's chunk
+// copied to shared memory) while every cluster is resident in one wave, else
+// `direct` (read from global memory, little shared memory per CTA).
 template <class TT, class DT, int DKIND>
 static cudaError_t run_chain_sample(StreamParams sp, const StreamGeom& sg, FinishParams fp,
-                                    const RowPlan* plans, int np, bool kd, cudaStream_t s) {
+                                    const RowPlan* staged, int ns, const RowPlan* direct, int nd,
+                                    bool kd, cudaStream_t s) {
   // probability drafts are not streamed: q(x) is read directly
   constexpr int base = kFStats0 | kFGather | (DKIND == kDraftLogits ? (kFRow1 | kFStats1) : 0);
-  auto fin = kd ? chain_sample_finish<TT, DT, DKIND, true> : chain_sample_finish<TT, DT, DKIND, false>;
+  auto fin_s = kd ? chain_sample_finish<TT, DT, DKIND, true, true>
+                  : chain_sample_finish<TT, DT, DKIND, false, true>;
+  auto fin_d = kd ? chain_sample_finish<TT, DT, DKIND, true, false>
+                  : chain_sample_finish<TT, DT, DKIND, false, false>;
   RowPlan plan;
-  cudaError_t e = pick_plan(fin, plans, np, fp.B, &plan);
+  long long waves = 0;
+  const long long force = knob(kKnobFinishRead);  // 1 staged, 2 direct
+  cudaError_t e = ns > 0 && force != 2 ? pick_plan(fin_s, staged, ns, fp.B, &plan, &waves)
+                                      : cudaErrorInvalidConfiguration;
+  bool use_staged = true;
+  if (e != cudaSuccess || (waves != 1 && force != 1)) {
+    use_staged = false;
+    e = pick_plan(fin_d, direct, nd, fp.B, &plan);
+  }
   if (e != cudaSuccess) return e;
   fp.L = plan.L;
   fp.use_bulk = plan.use_bulk;
@@ -461,15 +477,16 @@ static cudaError_t run_chain_sample(StreamParams sp, const StreamGeom& sg, Finis
                : launch_stream<TT, DT, base>(sp, sg, s));
   if (e != cudaSuccess) return e;
   fp.sp = sp;
-  return launch_clusters(fin, fp, plan, fp.B, s);
+  return use_staged ? launch_clusters(fin_s, fp, plan, fp.B, s)
+                    : launch_clusters(fin_d, fp, plan, fp.B, s);
 }
 
 }  // namespace sv
 
 using namespace sv;
 
-// Chains of at most kChainMaxK drafts run as one persistent launch; longer
-// chains (or the legacy knob) take the two-kernel path.
+// Chain calls take the two-kernel path; with the persistent knob set, chains
+// of at most kChainMaxK drafts run as one persistent launch.
 static bool chain_legacy(int k) { return k > kChainMaxK || knob(kKnobPersistent) == 0; }
 
 extern "C" {
@@ -680,28 +697,29 @@ static sv_status verify_chain_impl(const void* target_logits, sv_dtype t_dtype, 
                                           : launch_blocks(chain_greedy_finish<F32>, fp, B, gsm, s));
   }
 
-  RowPlan plans[kMaxCluster];
-  const int np = feasible_plans(
-      V, te, de,
-      [](int, int npc) {
-        const int x = npc * kThreads * 4 + kThreads * 8;
-        return x < 2 * kThreads * 4 ? 2 * kThreads * 4 : x;
-      },
-      bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de), P * (int)sizeof(RowRec),
-      plans);
-  if (np == 0) return SV_ERR_UNSUPPORTED;
+  // finishing plans with staging buffers for the drawn row's chunk, and
+  // without (the chunk read from global memory)
+  const auto x_bytes = [](int, int npc) {
+    const int x = npc * kThreads * 4 + kThreads * 8;
+    return x < 2 * kThreads * 4 ? 2 * kThreads * 4 : x;
+  };
+  const bool rows_aligned = bulk_ok_row(target_logits, V, te) && bulk_ok_row(draft, V, de);
+  RowPlan plans[kMaxCluster], dplans[kMaxCluster];
+  const int np = feasible_plans(V, te, de, x_bytes, rows_aligned, P * (int)sizeof(RowRec), plans);
+  const int nd = feasible_plans(V, 0, 0, x_bytes, rows_aligned, P * (int)sizeof(RowRec), dplans);
+  if (nd == 0) return SV_ERR_UNSUPPORTED;
   cudaError_t e;
   if (d_kind == SV_DRAFT_PROBS)
-    e = t_dtype == SV_BF16 ? run_chain_sample<BF16, F32, kDraftProbs>(sp, sg, fp, plans, np, kd, s)
-                           : run_chain_sample<F32, F32, kDraftProbs>(sp, sg, fp, plans, np, kd, s);
+    e = t_dtype == SV_BF16 ? run_chain_sample<BF16, F32, kDraftProbs>(sp, sg, fp, plans, np, dplans, nd, kd, s)
+                           : run_chain_sample<F32, F32, kDraftProbs>(sp, sg, fp, plans, np, dplans, nd, kd, s);
   else if (t_dtype == SV_BF16)
     e = d_dtype == SV_BF16
-            ? run_chain_sample<BF16, BF16, kDraftLogits>(sp, sg, fp, plans, np, kd, s)
-            : run_chain_sample<BF16, F32, kDraftLogits>(sp, sg, fp, plans, np, kd, s);
+            ? run_chain_sample<BF16, BF16, kDraftLogits>(sp, sg, fp, plans, np, dplans, nd, kd, s)
+            : run_chain_sample<BF16, F32, kDraftLogits>(sp, sg, fp, plans, np, dplans, nd, kd, s);
   else
     e = d_dtype == SV_BF16
-            ? run_chain_sample<F32, BF16, kDraftLogits>(sp, sg, fp, plans, np, kd, s)
-            : run_chain_sample<F32, F32, kDraftLogits>(sp, sg, fp, plans, np, kd, s);
+            ? run_chain_sample<F32, BF16, kDraftLogits>(sp, sg, fp, plans, np, dplans, nd, kd, s)
+            : run_chain_sample<F32, F32, kDraftLogits>(sp, sg, fp, plans, np, dplans, nd, kd, s);
   return cuda_status(e);
 }
 
@@ -790,7 +808,7 @@ sv_status sv_kernel_times(float* us, int32_t* tags, int cap, int32_t* n) {
 }
 
 sv_status sv_set_knob(int knob_id, long long value) {
-  if (knob_id < 1 || knob_id > kKnobKernelMarks) return SV_ERR_INVALID_ARG;
+  if (knob_id < 1 || knob_id > kKnobFinishRead) return SV_ERR_INVALID_ARG;
   __atomic_store_n(&g_knobs[knob_id], value, __ATOMIC_RELAXED);
   return SV_OK;
 }

@@ -76,12 +76,51 @@ constexpr int chain_sample_flags() {
          (KD ? kFTopk0 : 0);
 }
 
-template <class TT, class DT, int DKIND>
-__device__ __forceinline__ void weights8(const unsigned char* tbuf, const unsigned char* dbuf,
-                                         int e, int mode, float c, float Gt, float invSt,
-                                         float Gd, float invSd, float w[8]) {
-  float zt[8];
-  load8<TT>(tbuf, e, zt);
+// Eight consecutive elements j..j+7 of a row in global memory, widened to
+// fp32; elements at or past jend read as `pad`.  vec: the row base is 16-byte
+// aligned and j a multiple of 8, so a full vector is one 16-byte load (two for
+// fp32).  The rows are read-only inputs, so the loads take the read-only path.
+template <class T>
+__device__ __forceinline__ void gload8(const void* row, int j, int jend, bool vec, float pad,
+                                       float v[8]);
+
+template <>
+__device__ __forceinline__ void gload8<BF16>(const void* row, int j, int jend, bool vec, float pad,
+                                             float v[8]) {
+  const uint16_t* src = static_cast<const uint16_t*>(row) + j;
+  if (vec && j + 8 <= jend) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src));
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      v[t] = j + t < jend ? __uint_as_float((uint32_t)__ldg(src + t) << 16) : pad;
+  }
+}
+
+template <>
+__device__ __forceinline__ void gload8<F32>(const void* row, int j, int jend, bool vec, float pad,
+                                            float v[8]) {
+  const float* src = static_cast<const float*>(row) + j;
+  if (vec && j + 8 <= jend) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = j + t < jend ? __ldg(src + t) : pad;
+  }
+}
+
+// Draw weights of eight vocabulary entries from their target values zt and
+// draft values zd (draft logits, or draft probabilities): the residual
+// max(0, p - q), or p itself (mode P, where zd is not read).
+template <int DKIND>
+__device__ __forceinline__ void weights8(const float zt[8], const float zd[8], int mode, float c,
+                                         float Gt, float invSt, float Gd, float invSd,
+                                         float w[8]) {
   float p[8];
   // explicitly rounded products: p - q must be exactly 0 when p == q
 #pragma unroll
@@ -89,12 +128,11 @@ __device__ __forceinline__ void weights8(const unsigned char* tbuf, const unsign
   if (mode == kModeResidual) {
     float q[8];
     if (DKIND == kDraftLogits) {
-      float zd[8];
-      load8<DT>(dbuf, e, zd);
 #pragma unroll
       for (int t = 0; t < 8; ++t) q[t] = __fmul_rn(ex2(fmaf(zd[t], c, -Gd)), invSd);
     } else {
-      load8<F32>(dbuf, e, q);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) q[t] = zd[t];
     }
 #pragma unroll
     for (int t = 0; t < 8; ++t) w[t] = fmaxf(__fsub_rn(p[t], q[t]), 0.f);
@@ -189,8 +227,12 @@ __device__ __forceinline__ void release_rows(const FinishParams& prm, int nrows,
 //      reads it);
 //   4. the CTA that owns the drawn token writes the request's outputs (the
 //      first CTA when there is no draw: failed rows or timeouts).
-template <class TT, class DT, int DKIND, bool KD>
-__global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_constant__ FinishParams prm) {
+// STAGED: the drawn row's chunk is copied to shared memory first (one CTA per
+// SM, the registers it wants); otherwise it is read from global memory and
+// four CTAs share an SM.
+template <class TT, class DT, int DKIND, bool KD, bool STAGED>
+__global__ void __launch_bounds__(kThreads, STAGED ? 1 : 4)
+    chain_sample_finish(const __grid_constant__ FinishParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
@@ -247,32 +289,60 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
     }
   }
 
-  // 2. the draw, from row pair n (residual) or the bonus row k_b (target only)
+  // 2. the draw, from row pair n (residual) or the bonus row k_b (target only).
+  //    Staged: the chunk is copied to shared memory first.  Otherwise (when
+  //    staging would leave clusters waiting for a second wave) it is read
+  //    straight from global memory into registers and only the per-thread
+  //    piece sums are kept; the owner of the drawn token re-reads one vector.
   bool arrived = false;
   if (sh.need) {
     const bool pair = n < kb;
     const void* trow = row_ptr<TT>(prm.target, (size_t)b * P + n, V);
     const void* drow = pair ? row_ptr<DT>(prm.draft, (size_t)b * k + n, V) : nullptr;
-    if (pair)
-      stage_chunks<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, use_bulk, DKIND == kDraftProbs);
-    else
-      stage_chunks<TT, DT, false>(sh, tbuf, dbuf, trow, drow, g, use_bulk, false);
-    for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, use_bulk);
+    constexpr bool staged = STAGED;
+    if (staged) {
+      if (pair)
+        stage_chunks<TT, DT, true>(sh, tbuf, dbuf, trow, drow, g, use_bulk, DKIND == kDraftProbs);
+      else
+        stage_chunks<TT, DT, false>(sh, tbuf, dbuf, trow, drow, g, use_bulk, false);
+      for (int p = 0; p < g.npieces; ++p) wait_piece(sh, p, use_bulk);
+    } else if (threadIdx.x == 0) {
+      sh.timeouts = 0;
+    }
     __syncthreads();
+    const int jend = g.j0 + g.len;
+    const float dpad = DKIND == kDraftProbs ? 0.f : -INFINITY;
     int mode = pair ? kModeResidual : kModeP;
     const float Gt = sh.Gt, Gd = sh.Gd;
     const float invSt = (float)(1.0 / sh.St);
     const float invSd = (DKIND == kDraftLogits && pair) ? (float)(1.0 / sh.Sd) : 1.f;
+    // the weights of this thread's vector of piece p
+    auto piece_weights = [&](int p, float wv[8]) -> bool {
+      const int e = p * kRound + (int)threadIdx.x * kVec;
+      if (e >= g.nvec * kVec) return false;
+      float zt[8], zd[8];
+      if (staged) {
+        load8<TT>(tbuf, e, zt);
+        if (mode == kModeResidual) load8<DT>(dbuf, e, zd);
+      } else {
+        gload8<TT>(trow, g.j0 + e, jend, use_bulk, -INFINITY, zt);
+        if (mode == kModeResidual) gload8<DT>(drow, g.j0 + e, jend, use_bulk, dpad, zd);
+      }
+      weights8<DKIND>(zt, zd, mode, c, Gt, invSt, Gd, invSd, wv);
+      return true;
+    };
     for (int attempt = 0; attempt < 2; ++attempt) {
-      for (int p = 0; p < g.npieces; ++p) {
-        const int e = p * kRound + (int)threadIdx.x * kVec;
-        float s = 0.f;
-        if (e < g.nvec * kVec) {
+      // four pieces at a time: their loads are in flight together
+      for (int p0 = 0; p0 < g.npieces; p0 += 4) {
+        float s4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
           float wv[8];
-          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, wv);
-          s = seq_sum8(wv);
+          s4[u] = (p0 + u < g.npieces && piece_weights(p0 + u, wv)) ? seq_sum8(wv) : 0.f;
         }
-        sums[p * kThreads + threadIdx.x] = s;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (p0 + u < g.npieces) sums[(p0 + u) * kThreads + threadIdx.x] = s4[u];
       }
       piece_totals(sums, g.npieces, sh);
       if (threadIdx.x == 0) {
@@ -354,7 +424,7 @@ __global__ void __launch_bounds__(kThreads) chain_sample_finish(const __grid_con
         if ((int)threadIdx.x == ts) {
           const int e = pp * kRound + ts * kVec;
           float wv[8];
-          weights8<TT, DT, DKIND>(tbuf, dbuf, e, mode, c, Gt, invSt, Gd, invSd, wv);
+          piece_weights(pp, wv);
           const double b0 = sh.base + (ts > 0 ? incl_arr[ts - 1] : 0.0);
           float a = 0.f;
           int pick = -1, lastq = -1;

@@ -29,6 +29,7 @@ SV_DEV_RESIDUAL_ZERO, SV_DEV_TOPK_SLOW = 0x100, 0x200
 SV_KNOB_CLUSTER_CTAS, SV_KNOB_STREAM_COUNT, SV_KNOB_STREAM_W, SV_KNOB_WAIT_NS = 1, 2, 3, 4
 SV_KNOB_STALL, SV_KNOB_STAGES, SV_KNOB_ORDER, SV_KNOB_PERSISTENT = 5, 6, 7, 8
 SV_KNOB_KERNEL_MARKS = 9
+SV_KNOB_FINISH_READ = 10
 SV_MARK_STREAM, SV_MARK_FINISH, SV_MARK_CHAIN = 0, 1, 2
 MARK_NAMES = {SV_MARK_STREAM: "stream", SV_MARK_FINISH: "finish", SV_MARK_CHAIN: "chain"}
 

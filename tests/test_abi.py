@@ -212,7 +212,7 @@ def test_knobs_validate(lib):
     assert lib.sv_set_knob(0, 1) == sv.SV_ERR_INVALID_ARG
     assert lib.sv_set_knob(99, 1) == sv.SV_ERR_INVALID_ARG
     assert lib.sv_set_knob(sv.SV_KNOB_STAGES, 0) == sv.SV_OK
-    assert lib.sv_set_knob(sv.SV_KNOB_KERNEL_MARKS + 1, 1) == sv.SV_ERR_INVALID_ARG
+    assert lib.sv_set_knob(sv.SV_KNOB_FINISH_READ + 1, 1) == sv.SV_ERR_INVALID_ARG
 
 
 def test_kernel_times_without_marks(lib):

@@ -42,11 +42,16 @@ def check_chain(x, max_flag_frac=0.05):
     return assert_chain_match(got, ref, x.uniforms.numpy(), x.temperature, x.k, max_flag_frac)
 
 
-@pytest.fixture(params=["two-kernel", "persistent"])
+CHAIN_PATHS = {"two-kernel": {}, "two-kernel-direct": dict(finish_read=2),
+               "persistent": dict(persistent=1)}
+
+
+@pytest.fixture(params=list(CHAIN_PATHS))
 def chain_path(request):
-    """Run the test on both chain paths: the default two-kernel path and the
-    single persistent launch."""
-    with sv.knobs(persistent=int(request.param == "persistent")):
+    """Run the test on every chain path: the default two-kernel path (its
+    finishing clusters staging the drawn row in shared memory, or reading it
+    from global memory) and the single persistent launch."""
+    with sv.knobs(**CHAIN_PATHS[request.param]):
         yield request.param
 
 
