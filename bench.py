@@ -71,6 +71,8 @@ def parse():
     ap.add_argument("--sigma", type=float, default=1.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--min-warm-s", type=float, default=0.5,
+                    help="seconds of load before timing (0 for short profiling runs)")
     return ap.parse_args()
 
 
@@ -322,8 +324,21 @@ def cpu_baseline(kind, x, rows, min_seconds=10.0):
         dt = time.perf_counter() - t0
         if dt >= min_seconds or n >= 1000:
             break
-    return {"value": rows * n / dt, "unit": UNIT, "cores": O.max_threads(), "kind": "oracle",
-            "sample": f"{n} full batches of the same workload ({rows} rows each) in {dt:.1f} s"}
+    cores = O.max_threads()
+    out = {"value": rows * n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": f"{n} full batches of the same workload ({rows} rows each) in {dt:.1f} s"}
+    # the same oracle on one thread (run last: it leaves the oracle at one thread)
+    fn1 = oracle_step_fn(kind, x, threads=1)
+    n1, t1 = 0, time.perf_counter()
+    while True:
+        fn1()
+        n1 += 1
+        dt1 = time.perf_counter() - t1
+        if dt1 >= min_seconds / 2 or n1 >= 1000:
+            break
+    out["single_thread"] = {"value": rows * n1 / dt1, "unit": UNIT, "cores": 1,
+                            "sample": f"{n1} full batches in {dt1:.1f} s"}
+    return out
 
 
 def run_reference(a):
@@ -604,7 +619,7 @@ def main():
     for i in range(a.warmup):
         step(i)
     torch.cuda.synchronize(dev)
-    t_end = time.time() + 0.5
+    t_end = time.time() + a.min_warm_s
     i = a.warmup
     while time.time() < t_end:
         for _ in range(50):
