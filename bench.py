@@ -42,7 +42,11 @@ L2_BYTES = 126 * 1024 * 1024
 # kernel, from one capture of the current build on this workload, with the
 # profiles/ summary that holds it; absent for a workload whose kernel changed
 # since its last capture.
-NCU_TRAFFIC: dict = {}
+NCU_TRAFFIC: dict = {
+    "qwen_chain_verify": (68114688 + 557056,
+                          "profiles/stream_kernel_qwen_chain_B32_k3.md: stream_kernel, one ncu "
+                          "capture of the two-kernel path as built"),
+}
 # Kernel names of a call's launches, by the library's launch kinds (stream
 # pass, finishing kernel, persistent chain kernel).
 FINISH_NAME = {"chain": "chain_sample_finish", "kd": "chain_sample_finish",

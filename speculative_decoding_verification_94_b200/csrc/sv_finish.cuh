@@ -211,8 +211,12 @@ __device__ __forceinline__ void release_rows(const FinishParams& prm, int nrows,
   const int lane = threadIdx.x & 31;
   for (int t = t0; t < nrows; t += nt) {
     const int r = row0 + t * row_stride;
-    if (!prm.sp.count) row_zero_records(prm.sp, r, true);
-    else if (lane == 0) prm.rec[r] = RowRec{};
+    if (!prm.sp.count) {
+      row_zero_records(prm.sp, r, true);
+      if (lane == 0) prm.sp.row_counter[r] = 0u;  // the top-K floor of the row
+    } else if (lane == 0) {
+      prm.rec[r] = RowRec{};
+    }
   }
 }
 

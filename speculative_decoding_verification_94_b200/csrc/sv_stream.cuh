@@ -896,6 +896,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   unsigned long long thr_floor = kNoKey;  // lower bound of the run's K-th best key
   float thr_val = -INFINITY;
   bool seed = false;
+  // Static schedule with top-K: the row's counter word (unused by the static
+  // schedule) holds the largest K-th-best value any warp of the row has
+  // published (order-preserving bits).  At least K elements of the row are
+  // that large, so every warp of the row may drop what is below it.
+  uint32_t pub = 0u;  // the largest value this run has published
   int run_first = -1;  // the item whose record slot the run writes
   while (cur < total) {
     const int r = fast_div(cur, prm.div_nchunk);
@@ -916,9 +921,13 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
       thr_floor = kNoKey;
       thr_val = -INFINITY;
       seed = true;
+      pub = 0u;
     }
 
     for (int p = 0; p < cur_np; ++p) {
+      // the row's shared floor, read now and used after the statistics
+      uint32_t row_floor = 0u;
+      if ((FLAGS & kFTopk0) && stat) row_floor = *reinterpret_cast<volatile uint32_t*>(&prm.row_counter[r]);
       const int s = (int)(n_consumed % kStages);
       const uint32_t ph = (n_consumed / kStages) & 1u;
       unsigned char* st = ring + (size_t)s * prm.stage_bytes;
@@ -982,6 +991,16 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
             thr_val = key_value(thr_key);
             seed = false;
           }
+          if (stat) {
+            // another warp's K-th best value of this row: a floor like the
+            // lane maxima's (equal values may still enter)
+            const unsigned long long ef = (unsigned long long)row_floor << 32;
+            if (ef > thr_floor) {
+              thr_floor = ef;
+              if (thr_floor > thr_key) thr_key = thr_floor;
+              thr_val = key_value(thr_key);
+            }
+          }
           // Candidates are found lane-parallel in registers: each round, every
           // lane offers its best key above the threshold that it has not yet
           // offered; the 32 offers are sorted and merged into the list.
@@ -1030,6 +1049,15 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
             thr_key = kth > thr_floor ? kth : thr_floor;
             thr_val = thr_key == kNoKey ? -INFINITY : key_value(thr_key);
             if (cand != kNoKey) last = cand;
+          }
+          if (stat) {
+            // publish this run's K-th best value once the list is full
+            const unsigned long long kth = __shfl_sync(0xffffffffu, list, K - 1);
+            const uint32_t kv = (uint32_t)(kth >> 32);
+            if (kth != kNoKey && kv > pub) {
+              if (lane == 0) atomicMax(&prm.row_counter[r], kv);
+              pub = kv;
+            }
           }
         }
       }
