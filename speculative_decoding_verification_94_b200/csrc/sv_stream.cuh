@@ -1009,10 +1009,12 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
           // K-th cannot enter (larger index); the floor admits equal values.
           unsigned pmask = 0;
           const bool strict = thr_key != thr_floor;
+          if (pm > thr_val || (!strict && pm == thr_val)) {  // the lane maximum first
 #pragma unroll
-          for (int v = 0; v < kLaneVecs; ++v) {
-            const float vm = vec_max(R, v);
-            if (v * 32 + lane < nv && (vm > thr_val || (!strict && vm == thr_val))) pmask |= 1u << v;
+            for (int v = 0; v < kLaneVecs; ++v) {
+              const float vm = vec_max(R, v);
+              if (v * 32 + lane < nv && (vm > thr_val || (!strict && vm == thr_val))) pmask |= 1u << v;
+            }
           }
           unsigned long long last = ~0ull;
           while (__any_sync(0xffffffffu, pmask != 0)) {
