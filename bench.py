@@ -39,11 +39,11 @@ def metric_of(kind):
 UNIT = "rows/s"
 L2_BYTES = 126 * 1024 * 1024
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
-# kernel, from one capture of the current build on this workload, with the
-# profiles/ summary that holds it; absent for a workload whose kernel changed
-# since its last capture.
+# kernel, from one capture of the current build on this workload (keyed by
+# workload, B, k), with the profiles/ summary that holds it; absent for a
+# workload whose kernel changed since its last capture.
 NCU_TRAFFIC: dict = {
-    "qwen_chain_verify": (68114688 + 557056,
+    ("qwen_chain_verify", 32, 3): (68114688 + 557056,
                           "profiles/stream_kernel_qwen_chain_B32_k3.md: stream_kernel, one ncu "
                           "capture of the two-kernel path as built"),
 }
@@ -731,7 +731,7 @@ def main():
         cpu = cpu_baseline(kind, x, rows)
 
     if rank == 0:
-        traffic = NCU_TRAFFIC.get(cfg["workload"])
+        traffic = NCU_TRAFFIC.get((cfg["workload"], cfg.get("B"), cfg.get("k")))
         line = {"metric": metric_of(kind), "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_total / a.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
