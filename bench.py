@@ -378,6 +378,23 @@ SCHED_BATCHES = (1, 2, 4, 8, 16, 32)
 SCHED_SEEDS = 6
 
 
+def dominant_kernel(kind, x, algo_bytes, kern):
+    """The kernel that moves most of the call's algorithmic bytes, and those
+    bytes: the streaming pass of a chain or greedy tree (every logit once;
+    the finisher re-reads one row pair per request, the tree walk only
+    records), the one kernel of a sampling tree or of a persistent chain call,
+    and for the KD gradient the gradient kernel (the draft rows once more and
+    the fp32 gradient; the statistics pass before it reads the draft rows)."""
+    if "chain_kernel" in kern:
+        return "chain_kernel", algo_bytes
+    if kind == "tree_sample":
+        return "tree_sample_kernel", algo_bytes
+    if kind == "grad":
+        B, k, V = x.draft.shape
+        return "kd_grad_kernel", algo_bytes - B * k * V * x.draft.element_size()
+    return "stream_kernel", algo_bytes
+
+
 def kernel_times(step, steps, dev, kind):
     """Mean device time of each kernel of a call, from the library's kernel
     marks: `steps` calls captured in a CUDA graph with the marks on, replayed
@@ -662,16 +679,14 @@ def main():
     # launch, on the launching stream) and replayed once.  The marks put an
     # event between the launches, so the sum can exceed the unmarked call.
     kern = kernel_times(step, min(a.steps, 500), dev, kind)
-    dom = max(kern, key=lambda n: kern[n]["us_per_launch"] * kern[n]["launches_per_step"])
+    dom, dom_bytes = dominant_kernel(kind, x, algo_bytes, kern)
     dom_us = kern[dom]["us_per_launch"]
     (dom_us,) = reduce_max([dom_us], dist, dev)
 
     peak, peak_kind = load_peaks()
     need_bytes = needed_bytes(kind, x, outs["accepted_len"].cpu().numpy())
-    # algorithmic bytes: every input logit read once plus the small I/O, all
-    # of it read by the dominant kernel (the streaming pass, or the one kernel
-    # of a single-launch call)
-    achieved = algo_bytes / (dom_us * 1e-6) / 1e9
+    # the dominant kernel's share of the algorithmic bytes over its own time
+    achieved = dom_bytes / (dom_us * 1e-6) / 1e9
     call_gbs = algo_bytes / (ms_launch * 1e-3) / 1e9
     value = job_value(rows, world, a.steps, ms_total)
 
@@ -741,7 +756,7 @@ def main():
                                parallelism=f"dp{world}" if world > 1 else "single"),
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                              "unit": "GB/s", "frac": achieved / peak,
-                             "kernel": dom, "kernel_us": dom_us,
+                             "kernel": dom, "kernel_us": dom_us, "kernel_bytes": dom_bytes,
                              "call_achieved": call_gbs, "call_frac": call_gbs / peak,
                              "traffic": traffic[0] if traffic else None,
                              "traffic_from": traffic[1] if traffic else None,
