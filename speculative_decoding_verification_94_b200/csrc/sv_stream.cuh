@@ -617,16 +617,67 @@ __device__ __forceinline__ unsigned long long term2(float lo, float hi, unsigned
   return f2_pack(ex2(a), ex2(b));
 }
 
+// 2^a and 2^b on the FMA pipe instead of the special-function unit, for
+// arguments a, b <= 0 (-inf allowed).  Cody-Waite reduction: n = rint(a),
+// f = a - n in [-1/2, 1/2] (exact); 2^f = e^(f ln 2) by its Taylor polynomial
+// through f^6, whose coefficients are (ln 2)^k / k! rounded to fp32
+// (truncation error below 1.7e-7 relative, about that of ex2.approx),
+// evaluated for both arguments at once with packed fp32 FMAs; then n is added
+// to the exponent field.  Results below 2^-125 are 0 (ex2.approx.ftz flushes
+// below 2^-126; the terms here are relative to a maximum of order 1).
+__device__ __forceinline__ unsigned long long ex2_fma_pair(float a, float b) {
+  a = fmaxf(a, -127.f);
+  b = fmaxf(b, -127.f);
+  const float na = rintf(a), nb = rintf(b);
+  const unsigned long long f = f2_pack(a - na, b - nb);
+  auto k2 = [](float v) { return f2_pack(v, v); };
+  unsigned long long p = k2(1.540352969e-04f);  // (ln 2)^6 / 6!
+  p = f2_fma(p, f, k2(1.333355787e-03f));        // (ln 2)^5 / 5!
+  p = f2_fma(p, f, k2(9.618128650e-03f));        // (ln 2)^4 / 4!
+  p = f2_fma(p, f, k2(5.550410971e-02f));        // (ln 2)^3 / 3!
+  p = f2_fma(p, f, k2(2.402265072e-01f));        // (ln 2)^2 / 2!
+  p = f2_fma(p, f, k2(6.931471825e-01f));        // ln 2
+  p = f2_fma(p, f, k2(1.0f));
+  float pa, pb;
+  f2_unpack(p, pa, pb);
+  const int ia = (int)na, ib = (int)nb;
+  pa = ia < -125 ? 0.f : __uint_as_float(__float_as_uint(pa) + ((unsigned)ia << 23));
+  pb = ib < -125 ? 0.f : __uint_as_float(__float_as_uint(pb) + ((unsigned)ib << 23));
+  return f2_pack(pa, pb);
+}
+
+// term2 with the two powers on the FMA pipe.
+__device__ __forceinline__ unsigned long long term2_fma(float lo, float hi, unsigned long long cc,
+                                                        unsigned long long nr) {
+  float a, b;
+  f2_unpack(f2_fma(f2_pack(lo, hi), cc, nr), a, b);
+  return ex2_fma_pair(a, b);
+}
+
+// Every SV_EXP2_FMA_EVERY-th element pair of a lane's piece takes its powers
+// on the FMA pipe (0: none), to balance the special-function unit against
+// the FMA pipe.
+#ifndef SV_EXP2_FMA_EVERY
+#define SV_EXP2_FMA_EVERY 0
+#endif
+__device__ __forceinline__ unsigned long long term2_sel(int j, float lo, float hi,
+                                                        unsigned long long cc, unsigned long long nr) {
+  if (SV_EXP2_FMA_EVERY > 0 && j % (SV_EXP2_FMA_EVERY > 0 ? SV_EXP2_FMA_EVERY : 1) ==
+                                   (SV_EXP2_FMA_EVERY > 0 ? SV_EXP2_FMA_EVERY : 1) - 1)
+    return term2_fma(lo, hi, cc, nr);
+  return term2(lo, hi, cc, nr);
+}
+
 // Sum over the lane's elements of 2^(x c - ref), by a fixed tree of packed adds.
 __device__ __forceinline__ float lane_terms(const LaneRow<BF16>& R, float c, float ref) {
   const unsigned long long cc = f2_pack(c, c), nr = f2_pack(-ref, -ref);
   unsigned long long e[4 * kLaneVecs];
 #pragma unroll
   for (int v = 0; v < kLaneVecs; ++v) {
-    e[4 * v + 0] = term2(bf16_lo(R.w[v].x), bf16_hi(R.w[v].x), cc, nr);
-    e[4 * v + 1] = term2(bf16_lo(R.w[v].y), bf16_hi(R.w[v].y), cc, nr);
-    e[4 * v + 2] = term2(bf16_lo(R.w[v].z), bf16_hi(R.w[v].z), cc, nr);
-    e[4 * v + 3] = term2(bf16_lo(R.w[v].w), bf16_hi(R.w[v].w), cc, nr);
+    e[4 * v + 0] = term2_sel(4 * v + 0, bf16_lo(R.w[v].x), bf16_hi(R.w[v].x), cc, nr);
+    e[4 * v + 1] = term2_sel(4 * v + 1, bf16_lo(R.w[v].y), bf16_hi(R.w[v].y), cc, nr);
+    e[4 * v + 2] = term2_sel(4 * v + 2, bf16_lo(R.w[v].z), bf16_hi(R.w[v].z), cc, nr);
+    e[4 * v + 3] = term2_sel(4 * v + 3, bf16_lo(R.w[v].w), bf16_hi(R.w[v].w), cc, nr);
   }
 #pragma unroll
   for (int w = 2 * kLaneVecs; w >= 1; w >>= 1)
