@@ -1183,8 +1183,26 @@ sv_status sv_kd_grad(const float* topk_logp, const int32_t* topk_idx, int B, int
   fp.rec = w.rec;
   fp.status = device_status;
   fp.sp = sp;
-  e = (d_dtype == SV_BF16) ? launch_blocks(kd_grad_kernel<BF16>, fp, B * k, kFixedBytes, s)
-                           : launch_blocks(kd_grad_kernel<F32>, fp, B * k, kFixedBytes, s);
+  // CTAs per draft row: enough items for about four waves of resident CTAs
+  // (so the last wave is nearly full), at most 8, at least 2048 entries each
+  {
+    const void* kern = d_dtype == SV_BF16 ? reinterpret_cast<const void*>(kd_grad_kernel<BF16>)
+                                          : reinterpret_cast<const void*>(kd_grad_kernel<F32>);
+    int per_sm = 0, sms = 0;
+    if ((e = ensure_kernel_attrs(kern, kFixedBytes, false)) != cudaSuccess) return SV_ERR_CUDA;
+    if ((e = blocks_per_sm(kern, kThreads, kFixedBytes, &per_sm)) != cudaSuccess) return SV_ERR_CUDA;
+    if ((e = sm_count(&sms)) != cudaSuccess) return SV_ERR_CUDA;
+    const long long rows = (long long)B * k, cap = (long long)per_sm * sms;
+    long long ns = (4 * cap + rows - 1) / rows;
+    ns = ns < 1 ? 1 : (ns > 8 ? 8 : ns);
+    const long long by_len = V / 2048 < 1 ? 1 : V / 2048;
+    if (ns > by_len) ns = by_len;
+    if (rows * ns > 0x7fffffffLL) ns = 1;
+    fp.nsplit = (int)ns;
+  }
+  e = (d_dtype == SV_BF16)
+          ? launch_blocks(kd_grad_kernel<BF16>, fp, (int)((long long)B * k * fp.nsplit), kFixedBytes, s)
+          : launch_blocks(kd_grad_kernel<F32>, fp, (int)((long long)B * k * fp.nsplit), kFixedBytes, s);
   return cuda_status(e);
 }
 

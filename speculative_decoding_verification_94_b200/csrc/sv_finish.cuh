@@ -34,6 +34,7 @@ struct FinishParams {
   float c;
   double c64;  // log2(e) / T in float64 (sampling trees)
   int use_bulk;
+  int nsplit;  // kd_grad_kernel: CTAs per draft row
   RowLayout lay;
   // outputs
   int32_t* accepted_len;
@@ -675,9 +676,14 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
   extern __shared__ __align__(128) unsigned char smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int row = (int)blockIdx.x;
+  // nsplit CTAs per draft row, each a range of whole 8-element vectors, so
+  // that the grid has enough items to fill the last wave
+  const int nsplit = prm.nsplit > 0 ? prm.nsplit : 1;
+  const int row = (int)blockIdx.x / nsplit, part = (int)blockIdx.x - row * nsplit;
   const int k = prm.k, P = k + 1, V = prm.V, K = prm.K;
   const int b = row / k, i = row - b * k;
+  const int Lp = ((V + nsplit - 1) / nsplit + kVec - 1) / kVec * kVec;
+  const int lo = min(V, part * Lp), hi = min(V, lo + Lp);
   float* g = prm.grad + (size_t)row * V;
   pdl_wait();
   if (w == 0) {
@@ -690,7 +696,22 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
     }
     // the row's statistics (every draft row was streamed)
     const RowSum st = row_combine<DT, DT, kFStats0>(prm.sp, row, -1, true);
-    row_zero_records(prm.sp, row, true);
+    // the last of the row's CTAs to have folded its records clears them
+    // (the row's counter word counts the folds and returns to zero)
+    int last = 1;
+    if (nsplit > 1) {
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();  // this CTA's reads of the records before its count
+        last = atomicAdd(&prm.sp.row_counter[row], 1u) == (uint32_t)(nsplit - 1) ? 1 : 0;
+        if (last) __threadfence();  // the other CTAs' reads before the clearing
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+    }
+    if (last) {
+      row_zero_records(prm.sp, row, true);
+      if (lane == 0 && nsplit > 1) prm.sp.row_counter[row] = 0u;
+    }
     int bad = st.G0 == -INFINITY || (st.flags & kPTimeout);
     if (active && bad && lane == 0)
       set_status(prm.status, (st.flags & kPTimeout) ? SV_DEV_TIMEOUT : SV_DEV_NO_FINITE);
@@ -730,10 +751,10 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
   // streaming stores (when the row and the gradient row are 16-byte aligned)
   const bool vec = (reinterpret_cast<uintptr_t>(z) % 16 == 0) &&
                    (reinterpret_cast<uintptr_t>(g) % 16 == 0);
-  const int nvec = vec ? V / kVec : 0;
+  const int vend = vec ? lo + (hi - lo) / kVec * kVec : lo;  // end of the vector part
   const float fill = mode == 2 ? NAN : 0.f;
 #pragma unroll 4
-  for (int t = threadIdx.x; t < nvec; t += kThreads) {
+  for (int t = lo / kVec + (int)threadIdx.x; t < vend / kVec; t += kThreads) {
     float v[8];
     if (mode == 1) {
       load8<DT>(reinterpret_cast<const unsigned char*>(z), t * kVec, v);
@@ -746,7 +767,7 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
     __stcs(reinterpret_cast<float4*>(g + (size_t)t * kVec), make_float4(v[0], v[1], v[2], v[3]));
     __stcs(reinterpret_cast<float4*>(g + (size_t)t * kVec + 4), make_float4(v[4], v[5], v[6], v[7]));
   }
-  for (int e = nvec * kVec + threadIdx.x; e < V; e += kThreads) {
+  for (int e = vend + (int)threadIdx.x; e < hi; e += kThreads) {
     float v = fill;
     if (mode == 1) {
       const float zf = load1<DT>(reinterpret_cast<const unsigned char*>(z), e);
@@ -758,10 +779,12 @@ __global__ void __launch_bounds__(kThreads) kd_grad_kernel(const __grid_constant
   if (mode == 1 && w == 0 && lane < K) {
     const unsigned long long t = sh.topk[lane];
     const int j = (int)(t >> 32);
-    const float pt = __uint_as_float((uint32_t)(t & 0xffffffffu));
-    const float zf = load1<DT>(reinterpret_cast<const unsigned char*>(z), j);
-    const float q = ex2(fmaf(zf, c, -G) - l2s);
-    g[j] = scale * (q - pt);
+    if (j >= lo && j < hi) {  // this CTA's range wrote g[j]
+      const float pt = __uint_as_float((uint32_t)(t & 0xffffffffu));
+      const float zf = load1<DT>(reinterpret_cast<const unsigned char*>(z), j);
+      const float q = ex2(fmaf(zf, c, -G) - l2s);
+      g[j] = scale * (q - pt);
+    }
   }
 }
 

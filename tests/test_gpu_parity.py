@@ -458,6 +458,9 @@ def _grad_check(x, acc, reward, ref_top, mode, group, T, positions=0):
     m = np.where((acc < x.k) & (positions != 0), acc + 1, acc)
     active = np.arange(x.k)[None, :] < m[:, None]
     assert not g[~active].any()
+    # the workspace (records and the per-row fold counts of split rows) is zero again
+    ws = sv._WS[torch.cuda.current_device()]
+    assert int(torch.count_nonzero(ws)) == 0
     return got
 
 
