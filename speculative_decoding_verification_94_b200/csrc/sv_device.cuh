@@ -214,6 +214,12 @@ __device__ __forceinline__ void bulk_g2s_plain(void* dst, const void* src, uint3
       : "memory");
 }
 
+// Bring [src, src + bytes) into L2 without a destination (src 16-byte
+// aligned, bytes a multiple of 16); the copy completes on its own.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -282,6 +282,20 @@ __global__ void __launch_bounds__(kThreads, STAGED ? 1 : 4)
   }
   __syncthreads();
   const int n = sh.fin_n;
+  // Direct reads: this CTA's chunk of the drawn row (pair) starts towards L2
+  // now, so that its latency overlaps the KD rows below and the pass's loads
+  // find it there.
+  if (!STAGED && sh.need && use_bulk && threadIdx.x == 0 && g.len > 0) {
+    const uint32_t tb = (uint32_t)(g.len * TT::bytes) & ~15u;
+    if (tb) bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(
+                                 row_ptr<TT>(prm.target, (size_t)b * P + n, V)) + (size_t)g.j0 * TT::bytes,
+                             tb);
+    const uint32_t dbytes = (uint32_t)(g.len * DT::bytes) & ~15u;
+    if (n < kb && dbytes)
+      bulk_prefetch_l2(reinterpret_cast<const unsigned char*>(
+                           row_ptr<DT>(prm.draft, (size_t)b * k + n, V)) + (size_t)g.j0 * DT::bytes,
+                       dbytes);
+  }
 
   // 1. fused KD outputs of rows 0..n (static schedule; the dynamic schedule
   //    wrote them in the stream); the other rows' lists are cleared
