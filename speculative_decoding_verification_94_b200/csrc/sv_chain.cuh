@@ -57,10 +57,7 @@ constexpr int kSliceP = kTileW / kRowW;      // entries per warp, one row of a p
 constexpr int kVPLP = kSliceP / (32 * kVec); // 8-entry vectors per lane for those
 constexpr int kSliceW = kTileW / kCW;        // entries per warp, target-only and draw tiles
 constexpr int kVPL = kSliceW / (32 * kVec);  // 8-entry vectors per lane for those
-#ifndef SV_CHAIN_CLAIM
-#define SV_CHAIN_CLAIM 2
-#endif
-constexpr int kClaim = SV_CHAIN_CLAIM;       // stream tiles claimed per atomic
+constexpr int kClaim = 4;                    // stream tiles claimed per atomic (4 measured a little faster than 2)
 constexpr int kMaxStagesC = 8;
 constexpr int kChainMaxK = 30;               // drafts per request (state word: 31 rows)
 
@@ -252,18 +249,10 @@ __device__ __forceinline__ uint32_t mbar_test(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of an mbarrier, giving up after limit_ns.
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
                                                 unsigned long long limit_ns) {
-#ifdef SV_CHAIN_SUSPEND_WAITS
-  if (mbar_try_wait(bar, parity)) return true;
-#else
   if (mbar_try_wait_spin(bar, parity)) return true;
-#endif
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#ifdef SV_CHAIN_SUSPEND_WAITS
-    if (mbar_try_wait(bar, parity)) return true;
-#else
     if (mbar_try_wait_spin(bar, parity)) return true;
-#endif
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
@@ -1450,10 +1439,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(const __grid_co
           // a row that is not needed: with the tiles of a row consecutive,
           // move the claim counter past it (never past a row's first tile)
           auto skip_row = [&]() {
-#ifndef SV_CHAIN_NOJUMP
             if (p.order == 0 && tau + 1 < p.NT)
               atomicMax(&p.glob[kGNext], (uint32_t)(t - tau + p.NT));
-#endif
           };
           if (kb < 0) {
             // an idle request, or an invalid draft count: finished by the
