@@ -748,8 +748,10 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   // Static schedule: this warp's pieces [lo, hi); an item is a run of them
   // within one row (the record slot is the run's first piece).
   const int nws = prm.nwarps_eff;
-  const long long lo = (stat && gwarp < nws) ? (long long)gwarp * total / nws : 0;
-  const long long hi = (stat && gwarp < nws) ? (long long)(gwarp + 1) * total / nws : 0;
+  // (floor_div: the exact floor by a float64 quotient and one correction,
+  // cheaper than a 64-bit integer division)
+  const long long lo = (stat && gwarp < nws) ? floor_div((long long)gwarp * total, nws) : 0;
+  const long long hi = (stat && gwarp < nws) ? floor_div((long long)(gwarp + 1) * total, nws) : 0;
   auto run_end = [&](int item) -> long long {  // static: one past the run's last piece
     const long long re = (long long)(fast_div(item, prm.div_nchunk) + 1) * nchunk;
     return re < hi ? re : hi;
@@ -833,12 +835,11 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   // row into one record.  Dynamic mode: first items g and g + NW, then the
   // stripe counters.
   int cur = stat ? (lo < hi ? (int)lo : total) : gwarp, cur_np, cur_x;
+  int cur_x0 = -1;  // lane 0: the first item's draft token, read after the first copies are issued
   {
     uint32_t rj;
-    int x;
-    if (lane == 0) prefetch(cur, rj, x);
+    if (lane == 0) prefetch(cur, rj, cur_x0);
     cur_np = pieces_of(cur, rj, 0);
-    cur_x = __shfl_sync(0xffffffffu, x, 0);
   }
   int nxt = stat ? next_run(cur) : gwarp + nwarps, nxt_np = -1, nxt_x = -1;  // nxt_x: lane 0 only
   uint32_t nxt_rj = 0u;
@@ -935,6 +936,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
   };
 
   top_up();
+  cur_x = __shfl_sync(0xffffffffu, cur_x0, 0);
   // The statistics of a run: the items merged into one record (one item in
   // dynamic mode).
   ThreadStat st0, st1;
