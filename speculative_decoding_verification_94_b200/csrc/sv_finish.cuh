@@ -297,17 +297,6 @@ __global__ void __launch_bounds__(kThreads, STAGED ? 1 : 4)
                        dbytes);
   }
 
-  // 1. fused KD outputs of rows 0..n (static schedule; the dynamic schedule
-  //    wrote them in the stream); the other rows' lists are cleared
-  if (KD && !prm.sp.count) {
-    for (int t = rank * kWarps + w; t < P; t += C * kWarps) {
-      const bool ld = t < nld;
-      row_outputs<TT, DT, RF>(prm.sp, t * B + b, t < kb ? prm.tokens[(size_t)b * k + t] : -1,
-                              ld ? rows[t].L0 : 0.0, ld ? rows[t].L1 : 0.0, 0,
-                              n >= 0 && t <= n, true);
-    }
-  }
-
   // 2. the draw, from row pair n (residual) or the bonus row k_b (target only).
   //    Staged: the chunk is copied to shared memory first.  Otherwise (when
   //    staging would leave clusters waiting for a second wave) it is read
@@ -463,10 +452,46 @@ __global__ void __launch_bounds__(kThreads, STAGED ? 1 : 4)
     cluster.sync();  // every CTA has read the rows' records
   }
 
-  // 3. the rows' stream state back to zero
+  // 3. fused KD outputs, by rank 0 after the draw, so that no CTA of the
+  //    cluster waits at the scan for them: the top-K and KL of rows 0..n
+  //    (static schedule; the dynamic schedule wrote them in the stream), the
+  //    other rows' lists cleared, the rows after the emitted position filled
+  //    as empty, and the request's loss.  The emitted position is the one the
+  //    owner reports: n unless the request failed or the draw did (the owner
+  //    rejects a located token outside [0, V) too, which a draw with positive
+  //    mass cannot produce).
+  if (KD && rank == 0) {
+    const int nf = (n >= 0 && sh.need && !sh.err) ? n : -1;
+    if (!prm.sp.count) {
+      for (int t = w; t < P; t += kWarps) {
+        const bool ld = t < nld;
+        row_outputs<TT, DT, RF>(prm.sp, t * B + b, t < kb ? prm.tokens[(size_t)b * k + t] : -1,
+                                ld ? rows[t].L0 : 0.0, ld ? rows[t].L1 : 0.0, 0,
+                                n >= 0 && t <= n, true);
+      }
+      __syncthreads();
+    }
+    // rows after the emitted position are not verified: defined as empty
+    const int first_undef = nf < 0 ? 0 : nf + 1;
+    for (int t = first_undef * prm.K + (int)threadIdx.x; t < P * prm.K; t += kThreads) {
+      prm.topk_logp[(size_t)b * P * prm.K + t] = NAN;
+      prm.topk_idx[(size_t)b * P * prm.K + t] = -1;
+    }
+    for (int t = first_undef + (int)threadIdx.x; t < P; t += kThreads)
+      prm.lse[(size_t)b * P + t] = NAN;
+    // draft rows past the request's own drafts (k_b <= k) have no KL either
+    const int kl_undef = min(first_undef, kb < 0 ? 0 : kb);
+    for (int t = kl_undef + (int)threadIdx.x; t < k; t += kThreads)
+      prm.kl[(size_t)b * k + t] = NAN;
+    __syncthreads();
+    kd_finalize(b, nf, B, k, kb, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
+                prm.positions, prm.loss, prm.total, prm.glob_counter, sh);
+  }
+
+  // 4. the rows' stream state back to zero
   release_rows(prm, P, b, B, rank * kWarps + w, C * kWarps);
 
-  // 4. outputs, by the owner of the drawn token (or the first CTA without a draw)
+  // 5. outputs, by the owner of the drawn token (or the first CTA without a draw)
   const bool writer = sh.need ? (sh.owner != 0 || (sh.err && rank == 0)) : rank == 0;
   if (writer) {
     if (threadIdx.x == 0) {
@@ -483,23 +508,6 @@ __global__ void __launch_bounds__(kThreads, STAGED ? 1 : 4)
       int v = -1;
       if (nf >= 0) v = t < nf ? prm.tokens[(size_t)b * k + t] : (t == nf ? sh.tok : -1);
       prm.out_tokens[(size_t)b * P + t] = v;
-    }
-    if (KD) {
-      // rows after the emitted position are not verified: defined as empty
-      const int first_undef = nf < 0 ? 0 : nf + 1;
-      for (int t = first_undef * prm.K + (int)threadIdx.x; t < P * prm.K; t += kThreads) {
-        prm.topk_logp[(size_t)b * P * prm.K + t] = NAN;
-        prm.topk_idx[(size_t)b * P * prm.K + t] = -1;
-      }
-      for (int t = first_undef + (int)threadIdx.x; t < P; t += kThreads)
-        prm.lse[(size_t)b * P + t] = NAN;
-      // draft rows past the request's own drafts (k_b <= k) have no KL either
-      const int kl_undef = min(first_undef, kb < 0 ? 0 : kb);
-      for (int t = kl_undef + (int)threadIdx.x; t < k; t += kThreads)
-        prm.kl[(size_t)b * k + t] = NAN;
-      __syncthreads();
-      kd_finalize(b, nf, B, k, kb, prm.kl, prm.reward, prm.wmode, prm.group, prm.clip,
-                  prm.positions, prm.loss, prm.total, prm.glob_counter, sh);
     }
   }
   if (arrived) cluster_wait_acquire();  // keep this CTA's shared memory until all have read it
