@@ -420,26 +420,30 @@ static cudaError_t cluster_capacity(K kernel, const RowPlan& plan, int* out) {
 // Cluster size for `nclusters` requests: the plan minimising
 // waves * (chunk + a fixed latency worth of elements), where waves is the
 // number of rounds of co-resident clusters the grid needs.  A smaller
-// cluster (longer chunk) wins when it keeps the grid in one wave.
+// cluster (longer chunk) wins when it keeps the grid in one wave.  With
+// `fractional`, a partial last wave counts by its share (the clusters of a
+// multi-wave grid start as others finish).
 template <class K>
 static cudaError_t pick_plan(K kernel, const RowPlan* plans, int np, int nclusters,
-                             RowPlan* out, long long* waves_out = nullptr) {
+                             RowPlan* out, long long* waves_out = nullptr,
+                             bool fractional = false) {
   constexpr long long kLatencyElems = 8192;
-  long long best = -1;
+  double best = -1.0;
   for (int i = 0; i < np; ++i) {
     int cap = 0;
     cudaError_t e = cluster_capacity(kernel, plans[i], &cap);
     if (e != cudaSuccess) return e;
     if (cap < 1) continue;
     const long long waves = (nclusters + cap - 1) / cap;
-    const long long cost = waves * (plans[i].L + kLatencyElems);
-    if (best < 0 || cost < best) {
+    const double w = fractional ? (double)nclusters / cap : (double)waves;
+    const double cost = w * (double)(plans[i].L + kLatencyElems);
+    if (best < 0.0 || cost < best) {
       best = cost;
       *out = plans[i];
       if (waves_out) *waves_out = waves;
     }
   }
-  return best < 0 ? cudaErrorInvalidConfiguration : cudaSuccess;
+  return best < 0.0 ? cudaErrorInvalidConfiguration : cudaSuccess;
 }
 
 // Finishing plans of the sampling chain: `staged` (the drawn row's chunk
@@ -463,7 +467,7 @@ static cudaError_t run_chain_sample(StreamParams sp, const StreamGeom& sg, Finis
   bool use_staged = true;
   if (e != cudaSuccess || (waves != 1 && force != 1)) {
     use_staged = false;
-    e = pick_plan(fin_d, direct, nd, fp.B, &plan);
+    e = pick_plan(fin_d, direct, nd, fp.B, &plan, nullptr, true);
   }
   if (e != cudaSuccess) return e;
   fp.L = plan.L;
