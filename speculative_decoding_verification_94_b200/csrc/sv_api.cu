@@ -882,8 +882,13 @@ sv_status sv_verify_tree_greedy(const void* logits, sv_dtype dt, const int32_t* 
   fp.status = device_status;
   fp.sp = sp;
   const int tsm = kFixedBytes + n * (int)sizeof(RowRec) + 4 * n * 4;
-  return cuda_status(dt == SV_BF16 ? launch_blocks(tree_finish<BF16>, fp, B, tsm, s)
-                                   : launch_blocks(tree_finish<F32>, fp, B, tsm, s));
+  // blocks per tree: one warp per node row folds in parallel (at most 16)
+  fp.nsplit = n > kWarps ? (n + kWarps - 1) / kWarps : 1;
+  if (fp.nsplit > 16) fp.nsplit = 16;
+  if ((long long)B * fp.nsplit > 0x7fffffffLL) fp.nsplit = 1;
+  const int nb = B * fp.nsplit;
+  return cuda_status(dt == SV_BF16 ? launch_blocks(tree_finish<BF16>, fp, nb, tsm, s)
+                                   : launch_blocks(tree_finish<F32>, fp, nb, tsm, s));
 }
 
 }  // extern "C"

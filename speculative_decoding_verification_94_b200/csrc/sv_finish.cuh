@@ -552,14 +552,50 @@ __global__ void __launch_bounds__(kThreads) tree_finish(const __grid_constant__ 
   extern __shared__ __align__(128) unsigned char smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
   const int n = prm.k, V = prm.V;
-  const int b = (int)blockIdx.x;
+  // nsplit blocks per tree: each folds its share of the node rows (a warp a
+  // row) into the row records in global memory; the last to finish walks
+  // the tree.  One block folds every row itself.
+  const int S = prm.nsplit > 1 ? prm.nsplit : 1;
+  const int b = (int)blockIdx.x / S, s = (int)blockIdx.x - b * S;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   RowRec* rows = reinterpret_cast<RowRec*>(smem + kFixedBytes);
   int* garg = reinterpret_cast<int*>(smem + kFixedBytes + (size_t)n * sizeof(RowRec));
   int* par = garg + n;
   int* tok = par + n;
   int* dep = tok + n;
   pdl_wait();
-  load_rows<T, T, kFArgmax0>(prm, rows, n, b * n, 1, nullptr, 0, true);
+  if (S == 1) {
+    load_rows<T, T, kFArgmax0>(prm, rows, n, b * n, 1, nullptr, 0, true);
+  } else {
+    for (int t = s * kWarps + w; t < n; t += S * kWarps) {
+      const int r = b * n + t;
+      const RowSum rs = row_combine<T, T, kFArgmax0>(prm.sp, r, -1, true);
+      int err = 0;
+      const RowRec rr = row_decide<kFArgmax0>(prm.sp, r, -1, rs, &err);
+      if (err && lane == 0) set_status(prm.status, err);
+      row_zero_records(prm.sp, r, true);
+      if (lane == 0) prm.rec[r] = rr;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();  // this block's row records before its arrival
+      const int last = atomicAdd(&prm.req_reject[b], 1u) == (uint32_t)(S - 1) ? 1 : 0;
+      if (last) __threadfence();  // the other blocks' records before the reads below
+      sh.owner = last;
+    }
+    __syncthreads();
+    if (!sh.owner) return;
+    for (int t = threadIdx.x; t < n; t += kThreads) {
+      const uint4* src = reinterpret_cast<const uint4*>(prm.rec + (size_t)b * n + t);
+      uint4 q[3];
+      q[0] = __ldcg(src);
+      q[1] = __ldcg(src + 1);
+      q[2] = __ldcg(src + 2);
+      memcpy(&rows[t], q, sizeof(RowRec));
+      prm.rec[(size_t)b * n + t] = RowRec{};  // the workspace back to zero
+    }
+    if (threadIdx.x == 0) prm.req_reject[b] = 0u;
+  }
   __syncthreads();
   int err_any = 0;
   for (int t = threadIdx.x; t < n; t += kThreads) {
@@ -615,7 +651,7 @@ __global__ void __launch_bounds__(kThreads) tree_finish(const __grid_constant__ 
       ot[Lb] = garg[best];
     }
   }
-  release_rows(prm, n, b * n, 1, threadIdx.x >> 5, kWarps);
+  if (S == 1) release_rows(prm, n, b * n, 1, threadIdx.x >> 5, kWarps);
 }
 
 // KD loss: one block per request, one warp per draft row (b, i < k).  Draft

@@ -99,6 +99,41 @@ def test_tree_greedy_full_size():
     for key in ("accepted_len", "out_tokens", "accepted_nodes"):
         assert np.array_equal(got[key].cpu().numpy(), ref[key]), key
     assert len(set(ref["accepted_len"].tolist())) > 1
+    # the workspace (stream records, row records, arrival counts) is zero again
+    assert int(torch.count_nonzero(sv._WS[torch.cuda.current_device()])) == 0
+
+
+@pytest.mark.parametrize("n,depth", [(8, 3), (9, 4), (40, 6), (130, 9)])
+def test_tree_greedy_node_counts(n, depth):
+    """Trees of fewer nodes than a block's warps (one block), just over them
+    (two blocks per tree) and of several blocks per tree, against path
+    enumeration in the oracle; the workspace is zero afterwards."""
+    rng = np.random.default_rng(n)
+    B, V = 6, 3001
+    par = np.full((B, n), -1, np.int32)
+    for b in range(B):
+        depth_of = [0]
+        for j in range(1, n):
+            cand = [i for i in range(j) if depth_of[i] < depth]
+            p = int(rng.choice(cand))
+            par[b, j] = p
+            depth_of.append(depth_of[p] + 1)
+    logits = torch.from_numpy(rng.normal(0, 2, (B, n, V)).astype(np.float32))
+    am = logits.argmax(-1).numpy()
+    tok = rng.integers(0, V, (B, n)).astype(np.int32)
+    for b in range(B):  # plant argmax children so that paths of several depths are accepted
+        for j in range(1, n):
+            if rng.random() < 0.6:
+                tok[b, j] = am[b, par[b, j]]
+    st = status_tensor()
+    got = sv.sv_verify_tree_greedy(logits.to(DEV), torch.from_numpy(tok).to(DEV),
+                                   torch.from_numpy(par).to(DEV), depth, device_status=st)
+    ref = O.tree_greedy(logits, torch.from_numpy(tok), torch.from_numpy(par), depth)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for key in ("accepted_len", "out_tokens", "accepted_nodes"):
+        assert np.array_equal(got[key].cpu().numpy(), ref[key]), key
+    assert int(torch.count_nonzero(sv._WS[torch.cuda.current_device()])) == 0
 
 
 @pytest.fixture(scope="module")
