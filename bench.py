@@ -75,6 +75,8 @@ def parse():
     ap.add_argument("--sigma", type=float, default=1.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--knob", action="append", default=[], metavar="NAME=VALUE",
+                    help="library setting for the run (sv_set_knob), e.g. persistent=1")
     ap.add_argument("--min-warm-s", type=float, default=0.5,
                     help="seconds of load before timing (0 for short profiling runs)")
     return ap.parse_args()
@@ -553,8 +555,15 @@ def main():
                                 device_id=dev)
     sv.lib()
     assert a.warmup >= 3, "at least 3 warm-up steps"
+    knobs = {}
+    for kv in a.knob:
+        name, value = kv.split("=", 1)
+        sv.sv_set_knob(getattr(sv, "SV_KNOB_" + name.upper()), int(value))
+        knobs[name] = int(value)
 
     kind, x, cfg = make_workload(a, rank)
+    if knobs:
+        cfg = dict(cfg, knobs=knobs)
     rows, algo_bytes = rows_and_bytes(kind, x)
     # input copies rotated so that the set exceeds 2x L2: every step reads HBM
     ncopy = max(2, math.ceil(2.2 * L2_BYTES / algo_bytes))
