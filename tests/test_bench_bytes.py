@@ -70,3 +70,30 @@ def test_ragged_lengths_cover_every_length():
     assert kl.dtype == torch.int32 and act.dtype == torch.int32
     assert set(kl.tolist()) == {0, 1, 2, 3} and (act[:4] == 1).all()
     assert ((kl >= 0) & (kl <= 3)).all() and 0 < int(act.sum()) <= 32
+
+
+def test_dominant_kernel_and_its_bytes():
+    """The roofline's kernel: the streaming pass carries every logit of a chain
+    or greedy tree; the gradient kernel carries all but the statistics pass's
+    read of the draft rows; a sampling tree or a persistent call has one
+    kernel."""
+    x = inputs.make_chain(3, 3, 257, dtype="bf16", seed=1)
+    _, full = bench.rows_and_bytes("chain", x)
+    two = {"stream_kernel": {}, "chain_sample_finish": {}}
+    assert bench.dominant_kernel("chain", x, full, two) == ("stream_kernel", full)
+    assert bench.dominant_kernel("chain", x, full, {"chain_kernel": {}}) == ("chain_kernel", full)
+    _, gfull = bench.rows_and_bytes("grad", x)
+    name, by = bench.dominant_kernel("grad", x, gfull, {"stream_kernel": {}, "kd_grad_kernel": {}})
+    assert name == "kd_grad_kernel"
+    assert by == gfull - _nbytes(x.draft)
+    assert bench.kernel_names("tree")["finish"] == "tree_finish"
+    assert bench.kernel_names("kd")["stream"] == "stream_kernel"
+
+
+def test_peaks_fallback_and_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_peaks() == (6650.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6545.3, "bf16_tflops": 1590}')
+    assert bench.load_peaks() == (6545.3, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"HBM_copy_GBps": 6400}')
+    assert bench.load_peaks() == (6400.0, "measured")
