@@ -319,6 +319,28 @@ __device__ __forceinline__ double exp2_f64(double x) {
   return s * __longlong_as_double((long long)((int)k + 1023) << 52);
 }
 
+// 2^x in float64 with a shorter chain: x = k/16 + f with k = rint(16 x) and
+// |f| <= 1/32, so 2^x = 2^(k div 16) * t16[k mod 16] * e^(f ln 2), where
+// t16[j] = 2^(j/16) (filled by the caller, e.g. with exp2_f64) and e^y for
+// |y| <= ln(2)/32 is its Taylor series through y^6 (truncation below 5e-16
+// relative).  Results below 2^-1022 flush to 0.
+__device__ __forceinline__ double exp2_f64_tab(double x, const double* t16) {
+  if (!(x > -1022.0)) return 0.0;
+  const double k16 = rint(x * 16.0);
+  const double y = fma(-k16, 0.0625, x) * 0.693147180559945309417232121458;
+  double s = 1.0 / 720.0;                   // 1/6!
+  s = fma(s, y, 1.0 / 120.0);               // 1/5!
+  s = fma(s, y, 1.0 / 24.0);                // 1/4!
+  s = fma(s, y, 1.0 / 6.0);                 // 1/3!
+  s = fma(s, y, 0.5);                       // 1/2!
+  s = fma(s, y, 1.0);                       // 1/1!
+  s = fma(s, y, 1.0);                       // 1/0!
+  const long long ki = (long long)k16;
+  const int j = (int)(ki & 15);
+  const int n = (int)((ki - j) >> 4);       // floor(k / 16)
+  return s * t16[j] * __longlong_as_double((long long)(n + 1023) << 52);
+}
+
 // 2^x on the special-function unit (ex2.approx.ftz.f32).
 __device__ __forceinline__ float ex2(float x) {
   float y;

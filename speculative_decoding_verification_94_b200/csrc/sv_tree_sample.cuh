@@ -45,6 +45,7 @@ struct TreeShared {
   double Lt, Ld;     // log2-partitions of the staged rows
   double M, lo, hi;  // residual mass of the cluster, this CTA's share [lo, hi)
   double tt;         // the draw's target in [0, M)
+  double t16[16];    // 2^(j/16), j = 0..15, for exp2_f64_tab
   int nkids, err, owner, tok, piece, first_thread, last_pos, pad;
 };
 
@@ -56,7 +57,8 @@ struct TreeShared {
 template <class TT, class DT, int DKIND>
 __device__ __forceinline__ void tree_weights8(const unsigned char* tbuf, const unsigned char* dbuf,
                                               int e, double c, double Gt, double invSt,
-                                              double Gd, double invSd, double sg, double w[8]) {
+                                              double Gd, double invSd, double sg,
+                                              const double* t16, double w[8]) {
   float zt[8];
   load8<TT>(tbuf, e, zt);
   float q[8];
@@ -64,9 +66,9 @@ __device__ __forceinline__ void tree_weights8(const unsigned char* tbuf, const u
   else load8<F32>(dbuf, e, q);
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
-    const double p = exp2_f64(fma((double)zt[t], c, -Gt)) * invSt;
+    const double p = exp2_f64_tab(fma((double)zt[t], c, -Gt), t16) * invSt;
     const double qq =
-        DKIND == kDraftLogits ? exp2_f64(fma((double)q[t], c, -Gd)) * invSd : (double)q[t];
+        DKIND == kDraftLogits ? exp2_f64_tab(fma((double)q[t], c, -Gd), t16) * invSd : (double)q[t];
     w[t] = fmax(fma(-sg, qq, p), 0.0);
   }
 }
@@ -136,7 +138,10 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
       issue_item_copies<TT, DT, true>(sh, tbuf, dbuf, root_t, root_d, g, policy_evict_first());
   }
 
-  // 0. the tree, checked the same way in every CTA
+  if (threadIdx.x < 16) ts.t16[threadIdx.x] = exp2_f64((double)threadIdx.x * 0.0625);
+
+  // 0. the tree, checked the same way in every CTA (its barriers also
+  //    publish the table above)
   int bad_tree = 0, bad_tok = 0;
   for (int t = threadIdx.x; t < n; t += kThreads) {
     const int pj = prm.parents[(size_t)b * n + t];
@@ -193,7 +198,7 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
       double s = 0.0;
       if (e < g.nvec * kVec) {
         double wv[8];
-        tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c64, Gt, invSt, Gd, invSd, sg, wv);
+        tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c64, Gt, invSt, Gd, invSd, sg, ts.t16, wv);
         s = seq_sum8d(wv);
       }
       sums[p * kThreads + threadIdx.x] = s;
@@ -299,14 +304,14 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
             load8<TT>(tbuf, e, z);
             double t = 0.0;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t += exp2_f64(fma((double)z[k], c64, -(double)a.ref));
+            for (int k = 0; k < 8; ++k) t += exp2_f64_tab(fma((double)z[k], c64, -(double)a.ref), ts.t16);
             a.S += t;
           }
           if (fd) {
             load8<DT>(dbuf, e, z);
             double t = 0.0;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t += exp2_f64(fma((double)z[k], c64, -(double)d.ref));
+            for (int k = 0; k < 8; ++k) t += exp2_f64_tab(fma((double)z[k], c64, -(double)d.ref), ts.t16);
             d.S += t;
           }
         }
@@ -359,8 +364,8 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
     const double invSd = DKIND == kDraftLogits ? 1.0 / sh.Sd : 1.0;
     {
       for (int i = threadIdx.x; i < ts.nkids; i += kThreads) {
-        kpx[i] = exp2_f64(fma((double)kzt[i], c64, -Gt)) * invSt;
-        kqx[i] = DKIND == kDraftLogits ? exp2_f64(fma((double)kzd[i], c64, -Gd)) * invSd
+        kpx[i] = exp2_f64_tab(fma((double)kzt[i], c64, -Gt), ts.t16) * invSt;
+        kqx[i] = DKIND == kDraftLogits ? exp2_f64_tab(fma((double)kzd[i], c64, -Gd), ts.t16) * invSd
                                        : (double)kzd[i];
       }
       __syncthreads();
@@ -452,7 +457,7 @@ __global__ void __launch_bounds__(kThreads) tree_sample_kernel(const __grid_cons
         if ((int)threadIdx.x == tsel) {
           const int e = pp * kRound + tsel * kVec;
           double wv[8];
-          tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c64, Gt, invSt, Gd, invSd, sigma, wv);
+          tree_weights8<TT, DT, DKIND>(tbuf, dbuf, e, c64, Gt, invSt, Gd, invSd, sigma, ts.t16, wv);
           const double b0 = ts.lo + (tsel > 0 ? incl_arr[tsel - 1] : 0.0);
           double acc = 0.0;
           int pick = -1, lastq = -1;

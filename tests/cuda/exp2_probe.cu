@@ -23,3 +23,21 @@ extern "C" int exp2_probe(const float* x, float* y_fma, float* y_sfu, int n) {
   exp2_probe_kernel<<<(pairs + 255) / 256, 256>>>(x, y_fma, y_sfu, n);
   return (int)cudaDeviceSynchronize();
 }
+
+// The float64 powers of the sampling-tree kernel: the Taylor form and the
+// table-assisted form (table filled as the kernel fills it).
+__global__ void exp2d_probe_kernel(const double* x, double* y_tab, double* y_taylor, int n) {
+  __shared__ double t16[16];
+  if (threadIdx.x < 16) t16[threadIdx.x] = sv::exp2_f64((double)threadIdx.x * 0.0625);
+  __syncthreads();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  y_tab[i] = sv::exp2_f64_tab(x[i], t16);
+  y_taylor[i] = sv::exp2_f64(x[i]);
+}
+
+extern "C" int exp2d_probe(const double* x, double* y_tab, double* y_taylor, int n) {
+  if (n <= 0) return 0;
+  exp2d_probe_kernel<<<(n + 255) / 256, 256>>>(x, y_tab, y_taylor, n);
+  return (int)cudaDeviceSynchronize();
+}

@@ -57,3 +57,24 @@ def test_fma_exp2_tails(probe):
     assert yf[6] == np.float32(2.0 ** -125)
     assert abs(yf[7] / 2.0 ** -124.5 - 1) < 4e-7
     assert yf[8] == 1.0 and yf[9] == 1.0
+
+
+def test_float64_exp2_forms_match_exact_powers(probe):
+    """The sampling-tree kernel's float64 2^x, in both forms, against numpy's
+    float64 exp2 (itself within about an ulp): within 2e-15 relative over the
+    arguments the kernel uses (x <= 0), 0 below 2^-1022."""
+    probe.exp2d_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int]
+    rng = np.random.default_rng(1)
+    x = np.concatenate([-rng.uniform(0, 1000, 1 << 18), -rng.uniform(0, 1, 1 << 16),
+                        -np.arange(0, 1000, 1 / 16.0), [0.0, -1021.9, -1022.0, -1e9]])
+    xd = torch.from_numpy(x).cuda()
+    yt, yy = torch.empty_like(xd), torch.empty_like(xd)
+    assert probe.exp2d_probe(xd.data_ptr(), yt.data_ptr(), yy.data_ptr(), x.size) == 0
+    yt, yy = yt.cpu().numpy(), yy.cpu().numpy()
+    exact = np.exp2(x)
+    live = x > -1022.0
+    for y in (yt, yy):
+        rel = np.abs(y[live] - exact[live]) / exact[live]
+        print(f"float64 exp2: max relative error {rel.max():.3e}")
+        assert rel.max() < 2e-15
+        assert np.all(y[~live] == 0.0)
