@@ -1077,14 +1077,22 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
               const int vi = (__ffs(mm) - 1) * 32 + lane;
               float xs[8];
               load8<T0>(st, vi * kVec, xs);  // (the stage is still this piece's)
+              // the elements whose value can give a key above the threshold
+              // (a value below thr_val cannot); keys only for those
+              unsigned em = 0;
 #pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                if (vi * kVec + t < n) {
-                  const unsigned long long key = topk_key(xs[t], e0 + vi * kVec + t);
-                  if (key > thr_key && key < last) {
-                    more += cand != kNoKey;
-                    if (key > cand) cand = key;
-                  }
+              for (int t = 0; t < 8; ++t)
+                if (vi * kVec + t < n && !(xs[t] < thr_val)) em |= 1u << t;
+              for (; em; em &= em - 1) {
+                const int t = __ffs(em) - 1;
+                float xv = xs[0];
+#pragma unroll
+                for (int q = 1; q < 8; ++q)
+                  if (t == q) xv = xs[q];
+                const unsigned long long key = topk_key(xv, e0 + vi * kVec + t);
+                if (key > thr_key && key < last) {
+                  more += cand != kNoKey;
+                  if (key > cand) cand = key;
                 }
               }
             }
