@@ -43,9 +43,10 @@ L2_BYTES = 126 * 1024 * 1024
 # workload, B, k), with the profiles/ summary that holds it; absent for a
 # workload whose kernel changed since its last capture.
 NCU_TRAFFIC: dict = {
-    ("qwen_chain_verify", 32, 3): (68114688 + 557056,
-                          "profiles/stream_kernel_qwen_chain_B32_k3.md: stream_kernel, one ncu "
-                          "capture of the two-kernel path as built"),
+    ("qwen_chain_verify", 32, 3): (68115200 + 218112,
+                                   "profiles/stream_kernel_qwen_chain_B32_k3.md: stream_kernel, "
+                                   "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch "
+                                   "at commit d7ff710"),
 }
 # Kernel names of a call's launches, by the library's launch kinds (stream
 # pass, finishing kernel, persistent chain kernel).
