@@ -1099,7 +1099,7 @@ __global__ void __launch_bounds__(kStreamThreads, 3) stream_kernel(const __grid_
             if (cand == kNoKey || more == 0) pmask = 0;  // nothing left after this offer
             unsigned cm = __ballot_sync(0xffffffffu, cand != kNoKey);
             if (!cm) break;
-            if (__popc(cm) <= 4) {  // few offers: insert them one by one
+            if (__popc(cm) <= 12) {  // few offers: one by one (a sort costs about ten inserts)
               while (cm) {
                 const int src = __ffs(cm) - 1;
                 cm &= cm - 1;
