@@ -508,6 +508,18 @@ def test_kd_grad_small_and_ragged():
     _grad_check(x, acc, x.reward, ref, O.W_RAW, 1, 1.0)
 
 
+def test_kd_grad_split_rows_with_unaligned_tails():
+    """V = 8193: each draft row is split over several CTAs (the last one
+    ragged), odd rows start off a 16-byte boundary (scalar path) and the
+    last vector of a row is partial."""
+    x = inputs.make_chain(8, 3, 8193, dtype="bf16", sigma_d=1.0, temperature=0.9, seed=23)
+    ref = O.verify_kd(x.target, x.draft, x.draft_tokens, x.uniforms, x.reward, 0.9, 32,
+                      mode=O.W_GROUP_NORM, group=4)
+    acc = ref["accepted_len"].astype(np.int32)
+    acc[0] = 3
+    _grad_check(x, acc, x.reward, ref, O.W_GROUP_NORM, 4, 0.9)
+
+
 def test_kd_grad_full_vocabulary(kd256):
     x = inputs.ChainInputs(kd256.target[:32].contiguous(), kd256.draft[:32].contiguous(),
                            kd256.draft_tokens[:32].contiguous(), kd256.uniforms[:32].contiguous(),
