@@ -375,7 +375,8 @@ def run_reference(a):
             "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * dt / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": cfg,
+            "data": "synthetic",
+            "config": dict(cfg, parallelism=f"dp{a.gpus}" if a.gpus > 1 else "single"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.max_threads(),
                              "kind": "oracle",
                              "sample": f"{a.steps} timed full batches ({rows} rows each)"},
